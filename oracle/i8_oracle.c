@@ -1,0 +1,210 @@
+/*
+ * i8_oracle.c -- plain, slow CPU oracle for the LLM.int8() decomposed linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or call this
+ * file: only the test-suite, the smoke check and the CPU-baseline leg of the benchmark
+ * do.  It shares no code, header, table or helper with the CUDA library.
+ *
+ * Sources (all from the pages "A Gentle Introduction to 8-bit Matrix Multiplication for
+ * transformers at scale" (Hugging Face blog, Chinese translation), its summary on
+ * agentlenshq.com, and the LLM.int8() abstract):
+ *   - absmax quantisation: scale = 127 / max|x|, code = round(x * scale)
+ *     ("absmax 量化", the [1.2, -0.5, ..., 5.4] worked example);
+ *   - vector-wise quantisation: one absmax per row of the hidden states and one per
+ *     output channel of the weight, dequantised by the outer product of the two absmax
+ *     vectors ("absmax 量化", the A*B=C paragraph; "内部的 MatMul");
+ *   - the three-step decomposition: outlier columns of the hidden states are found with
+ *     a threshold, multiplied in fp16, the rest in int8, and the two results are added
+ *     ("LLM.int8() 的总结"; "内部的 MatMul": magnitude 6 or larger);
+ *   - weight recovery for the outlier product: CB * SCB / 127 ("用法", the printout
+ *     after .to(0)).
+ *
+ * Readings taken where the pages are silent (each listed in the design notes):
+ *   - an element is an outlier when |x| >= threshold ("6 or larger");
+ *   - a column is an outlier column when any row of the call has an outlier in it;
+ *   - the row absmax of X runs over the non-outlier columns only; the weight absmax
+ *     runs over the whole output row (per output channel);
+ *   - rounding is half away from zero (C99 roundf), applied to the fp32 product
+ *     x * fl32(127 / absmax); a zero absmax gives scale 0 and all-zero codes;
+ *   - the reference output is formed in fp64 (no fp16 rounding of the result).
+ *
+ * Build: gcc -O2 -std=c11 -fopenmp -ffp-contract=off -fPIC -shared (see build.py).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* IEEE 754 binary16 -> binary32 by the format's definition: 1 sign bit, 5 exponent
+ * bits (bias 15), 10 fraction bits; exponent 0 is zero/subnormal (value f * 2^-24),
+ * exponent 31 is inf/NaN.  Every binary16 value is exact in binary32. */
+float oracle_half_to_float(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int f = h & 0x3ff;
+    float v;
+    if (e == 0) {
+        v = ldexpf((float)f, -24);
+    } else if (e == 31) {
+        v = (f == 0) ? INFINITY : NAN;
+    } else {
+        v = ldexpf((float)(f + 1024), e - 25);
+    }
+    return sign ? -v : v;
+}
+
+/* Step 1 -- outlier column scan.  is_outlier[k] = 1 when some row t has
+ * |X[t,k]| >= threshold.  idx receives the outlier columns in ascending order and
+ * *n_o their count.  mask_words (nullable) receives the same set packed 32 columns per
+ * word, column k at bit (k % 32) of word k / 32. */
+void oracle_outlier_scan(const uint16_t *X, int64_t T, int64_t K, float threshold,
+                         uint8_t *is_outlier, uint32_t *mask_words,
+                         int32_t *idx, int32_t *n_o)
+{
+    for (int64_t k = 0; k < K; ++k)
+        is_outlier[k] = 0;
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t k = 0; k < K; ++k)
+            if (fabsf(oracle_half_to_float(X[t * K + k])) >= threshold)
+                is_outlier[k] = 1;
+    int32_t count = 0;
+    for (int64_t k = 0; k < K; ++k)
+        if (is_outlier[k])
+            idx[count++] = (int32_t)k;
+    *n_o = count;
+    if (mask_words) {
+        int64_t words = (K + 31) / 32;
+        for (int64_t w = 0; w < words; ++w)
+            mask_words[w] = 0;
+        for (int64_t k = 0; k < K; ++k)
+            if (is_outlier[k])
+                mask_words[k / 32] |= (uint32_t)1 << (k % 32);
+    }
+}
+
+/* Steps 2 and 3 -- row-wise absmax quantisation of an fp16 matrix A [R,K].
+ * skip (nullable) marks columns excluded from the absmax and coded as 0 (the outlier
+ * columns of the hidden states; NULL for the weight, whose scale covers the whole
+ * output row).  scale[r] = max |A[r,k]| over the kept columns, as fp32;
+ * q[r,k] = round_half_away(fl32(A[r,k] * fl32(127 / scale[r]))). */
+void oracle_absmax_quantize_rows(const uint16_t *A, int64_t R, int64_t K,
+                                 const uint8_t *skip, int8_t *q, float *scale)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r) {
+        const uint16_t *row = A + r * K;
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            if (skip && skip[k])
+                continue;
+            float a = fabsf(oracle_half_to_float(row[k]));
+            if (a > amax)
+                amax = a;
+        }
+        scale[r] = amax;
+        int8_t *qr = q + r * K;
+        if (amax == 0.0f) {
+            for (int64_t k = 0; k < K; ++k)
+                qr[k] = 0;
+            continue;
+        }
+        float s = 127.0f / amax;
+        for (int64_t k = 0; k < K; ++k) {
+            if (skip && skip[k]) {
+                qr[k] = 0;
+                continue;
+            }
+            float v = oracle_half_to_float(row[k]) * s;
+            float c = roundf(v);
+            if (c > 127.0f) c = 127.0f;
+            if (c < -127.0f) c = -127.0f;
+            qr[k] = (int8_t)c;
+        }
+    }
+}
+
+/* Step 4 -- integer matmul acc[i,n] = sum_k A[rows[i],k] * B[n,k] (B in the
+ * [out,in] layout), accumulated in int64 and returned as int32.  rows (nullable)
+ * selects a subset of A's rows; otherwise rows 0..nrows-1.  Returns the number of
+ * results that do not fit in int32 (0 at every size the layer admits). */
+int64_t oracle_int_matmul(const int8_t *A, const int8_t *B, int64_t nrows,
+                          const int64_t *rows, int64_t N, int64_t K, int32_t *acc)
+{
+    int64_t overflow = 0;
+    #pragma omp parallel for collapse(2) schedule(static) reduction(+:overflow)
+    for (int64_t i = 0; i < nrows; ++i) {
+        for (int64_t n = 0; n < N; ++n) {
+            const int8_t *a = A + (rows ? rows[i] : i) * K;
+            const int8_t *b = B + n * K;
+            int64_t s = 0;
+            for (int64_t k = 0; k < K; ++k)
+                s += (int64_t)a[k] * (int64_t)b[k];
+            if (s > INT32_MAX || s < INT32_MIN)
+                ++overflow;
+            acc[i * N + n] = (int32_t)s;
+        }
+    }
+    return overflow;
+}
+
+/* Steps 5 and 6 -- the decomposed product for the selected rows, in fp64:
+ *   C[i,n] = acc[i,n] * SCx[t] * SCB[n] / 127^2                  (int8 part, dequantised)
+ *          + sum_{j < n_o} X[t, idx[j]] * CB[n, idx[j]] * SCB[n] / 127   (fp16 outlier part)
+ *          + bias[n]                                               (bias nullable)
+ * with t = rows[i].  acc holds the int8 products of exactly those rows. */
+void oracle_decomposed_output(const uint16_t *X, int64_t K, const int64_t *rows,
+                              int64_t nrows, const int32_t *acc, const float *SCx,
+                              const int8_t *CB, const float *SCB, const uint16_t *bias,
+                              int64_t N, const int32_t *idx, int32_t n_o, double *C)
+{
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t i = 0; i < nrows; ++i) {
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t t = rows ? rows[i] : i;
+            double int_part = (double)acc[i * N + n] * (double)SCx[t] * (double)SCB[n]
+                              / (127.0 * 127.0);
+            double out_part = 0.0;
+            for (int32_t j = 0; j < n_o; ++j) {
+                int64_t k = idx[j];
+                double w = (double)CB[n * K + k] * (double)SCB[n] / 127.0;
+                out_part += (double)oracle_half_to_float(X[t * K + k]) * w;
+            }
+            double b = bias ? (double)oracle_half_to_float(bias[n]) : 0.0;
+            C[i * N + n] = int_part + out_part + b;
+        }
+    }
+}
+
+/* The whole forward for a subset of rows: steps 1 and 2 over ALL rows of X (the
+ * column mask depends on every row of the call), then steps 4-6 for the selected rows
+ * against an already-quantised weight (CB, SCB).  All outputs are caller-owned:
+ * mask_words [ceil(K/32)], idx [K], n_o [1], Xq [T,K], SCx [T],
+ * acc [nrows,N], C [nrows,N]. */
+int64_t oracle_linear_forward_rows(const uint16_t *X, int64_t T, int64_t K,
+                                   const int8_t *CB, const float *SCB,
+                                   const uint16_t *bias, int64_t N, float threshold,
+                                   const int64_t *rows, int64_t nrows,
+                                   uint32_t *mask_words, int32_t *idx, int32_t *n_o,
+                                   int8_t *Xq, float *SCx, int32_t *acc, double *C)
+{
+    uint8_t *is_outlier = (uint8_t *)malloc((size_t)(K > 0 ? K : 1));
+    if (!is_outlier)
+        return -1;
+    oracle_outlier_scan(X, T, K, threshold, is_outlier, mask_words, idx, n_o);
+    oracle_absmax_quantize_rows(X, T, K, is_outlier, Xq, SCx);
+    int64_t overflow = oracle_int_matmul(Xq, CB, nrows, rows, N, K, acc);
+    oracle_decomposed_output(X, K, rows, nrows, acc, SCx, CB, SCB, bias, N, idx, *n_o, C);
+    free(is_outlier);
+    return overflow;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

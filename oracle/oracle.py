@@ -1,0 +1,160 @@
+"""ctypes view of the plain-C oracle (i8_oracle.c) -- test infrastructure only.
+
+Each function takes and returns numpy arrays; fp16 data is passed as its raw bits.
+The arithmetic lives entirely in i8_oracle.c; this file only marshals arguments.
+"""
+import ctypes
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+_override = None
+
+
+class use_library:
+    """Context manager: route every call to another build of i8_oracle.c (a copy with a
+    planted mistake, compiled by a test) and restore the normal build afterwards."""
+
+    def __init__(self, path):
+        self.path = path
+
+    def __enter__(self):
+        global _override
+        self._saved = _override
+        _override = _load(self.path)
+        return self
+
+    def __exit__(self, *exc):
+        global _override
+        _override = self._saved
+        return False
+
+
+def lib():
+    global _lib
+    if _override is not None:
+        return _override
+    if _lib is None:
+        _lib = _load(_build.build())
+    return _lib
+
+
+def _load(path):
+    L = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    i64 = ctypes.c_int64
+    L.oracle_half_to_float.argtypes = [ctypes.c_uint16]
+    L.oracle_half_to_float.restype = ctypes.c_float
+    L.oracle_outlier_scan.argtypes = [P, i64, i64, ctypes.c_float, P, P, P, P]
+    L.oracle_outlier_scan.restype = None
+    L.oracle_absmax_quantize_rows.argtypes = [P, i64, i64, P, P, P]
+    L.oracle_absmax_quantize_rows.restype = None
+    L.oracle_int_matmul.argtypes = [P, P, i64, P, i64, i64, P]
+    L.oracle_int_matmul.restype = i64
+    L.oracle_decomposed_output.argtypes = [P, i64, P, i64, P, P, P, P, P, i64, P,
+                                           ctypes.c_int32, P]
+    L.oracle_decomposed_output.restype = None
+    L.oracle_linear_forward_rows.argtypes = [P, i64, i64, P, P, P, i64, ctypes.c_float,
+                                             P, i64, P, P, P, P, P, P, P]
+    L.oracle_linear_forward_rows.restype = i64
+    L.oracle_num_threads.argtypes = []
+    L.oracle_num_threads.restype = ctypes.c_int
+    return L
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def _bits(a):
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.float16:
+        return a.view(np.uint16)
+    assert a.dtype == np.uint16, a.dtype
+    return a
+
+
+def num_threads() -> int:
+    return lib().oracle_num_threads()
+
+
+def half_to_float(bits: int) -> float:
+    return lib().oracle_half_to_float(int(bits))
+
+
+def outlier_scan(X, threshold):
+    """Step 1: returns (is_outlier uint8 [K], mask_words uint32 [ceil(K/32)], idx int32 [n_o])."""
+    Xb = _bits(X)
+    T, K = Xb.shape
+    flags = np.zeros(K, np.uint8)
+    words = np.zeros((K + 31) // 32, np.uint32)
+    idx = np.zeros(max(K, 1), np.int32)
+    n_o = np.zeros(1, np.int32)
+    lib().oracle_outlier_scan(_ptr(Xb), T, K, float(threshold), _ptr(flags), _ptr(words),
+                              _ptr(idx), _ptr(n_o))
+    return flags, words, idx[: int(n_o[0])].copy()
+
+
+def absmax_quantize_rows(A, skip=None):
+    """Steps 2/3: returns (codes int8 [R,K], scale float32 [R])."""
+    Ab = _bits(A)
+    R, K = Ab.shape
+    q = np.zeros((R, K), np.int8)
+    s = np.zeros(R, np.float32)
+    sk = None if skip is None else np.ascontiguousarray(skip, dtype=np.uint8)
+    lib().oracle_absmax_quantize_rows(_ptr(Ab), R, K, _ptr(sk), _ptr(q), _ptr(s))
+    return q, s
+
+
+def quantize_weight(W):
+    """Step 3: per-output-channel quantisation of W [N,K] -> (CB int8 [N,K], SCB float32 [N])."""
+    return absmax_quantize_rows(W, None)
+
+
+def int_matmul(A, B, rows=None):
+    """Step 4: acc int32 [len(rows) or A.shape[0], N]; raises on int32 overflow."""
+    A = np.ascontiguousarray(A, np.int8)
+    B = np.ascontiguousarray(B, np.int8)
+    K = A.shape[1]
+    assert B.shape[1] == K
+    r = None if rows is None else np.ascontiguousarray(rows, np.int64)
+    nrows = A.shape[0] if r is None else r.shape[0]
+    N = B.shape[0]
+    acc = np.zeros((nrows, N), np.int32)
+    ov = lib().oracle_int_matmul(_ptr(A), _ptr(B), nrows, _ptr(r), N, K, _ptr(acc))
+    if ov:
+        raise OverflowError("int32 accumulator overflow in %d results" % ov)
+    return acc
+
+
+def linear_forward(X, CB, SCB, bias, threshold, rows=None):
+    """Whole forward (steps 1,2 over all rows; 4-6 for `rows`, default all rows).
+
+    Returns a dict with mask_words, idx, n_o, Xq, SCx, acc (rows) and C (fp64, rows).
+    """
+    Xb = _bits(X)
+    T, K = Xb.shape
+    CB = np.ascontiguousarray(CB, np.int8)
+    SCB = np.ascontiguousarray(SCB, np.float32)
+    N = CB.shape[0]
+    bb = None if bias is None else _bits(bias)
+    r = None if rows is None else np.ascontiguousarray(rows, np.int64)
+    nrows = T if r is None else r.shape[0]
+    words = np.zeros((K + 31) // 32, np.uint32)
+    idx = np.zeros(max(K, 1), np.int32)
+    n_o = np.zeros(1, np.int32)
+    Xq = np.zeros((T, K), np.int8)
+    SCx = np.zeros(T, np.float32)
+    acc = np.zeros((nrows, N), np.int32)
+    C = np.zeros((nrows, N), np.float64)
+    ov = lib().oracle_linear_forward_rows(_ptr(Xb), T, K, _ptr(CB), _ptr(SCB), _ptr(bb), N,
+                                          float(threshold), _ptr(r), nrows, _ptr(words),
+                                          _ptr(idx), _ptr(n_o), _ptr(Xq), _ptr(SCx),
+                                          _ptr(acc), _ptr(C))
+    if ov < 0:
+        raise MemoryError("oracle allocation failed")
+    if ov:
+        raise OverflowError("int32 accumulator overflow in %d results" % ov)
+    n = int(n_o[0])
+    return dict(mask_words=words, idx=idx[:n].copy(), n_o=n, Xq=Xq, SCx=SCx, acc=acc, C=C)

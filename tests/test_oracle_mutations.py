@@ -1,0 +1,60 @@
+"""Planted mistakes in the oracle (on the CPU): each plausible slip, compiled into a copy
+of i8_oracle.c, must make at least one pin fail.  Shows the pins are not self-confirming."""
+import os
+import subprocess
+
+import pytest
+
+from oracle import oracle as O
+from tests import oracle_pins
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                   "oracle", "i8_oracle.c")
+
+# (name, exact text in the oracle, replacement)
+MUTATIONS = [
+    ("round_half_even", "float c = roundf(v);", "float c = rintf(v);"),
+    ("truncate", "float c = roundf(v);", "float c = truncf(v);"),
+    ("strict_threshold", ">= threshold)", "> threshold)"),
+    ("scale_128", "float s = 127.0f / amax;", "float s = 128.0f / amax;"),
+    ("absmax_includes_outliers",
+     "            if (skip && skip[k])\n                continue;\n            float a",
+     "            float a"),
+    ("outlier_part_dropped", "out_part += (double)", "out_part += 0.0 * (double)"),
+    ("recovery_over_128", "* (double)SCB[n] / 127.0;", "* (double)SCB[n] / 128.0;"),
+    ("dequant_missing_weight_scale",
+     "(double)acc[i * N + n] * (double)SCx[t] * (double)SCB[n]",
+     "(double)acc[i * N + n] * (double)SCx[t]"),
+    ("transposed_weight_index", "const int8_t *b = B + n * K;",
+     "const int8_t *b = B + (n * K) % (K * N > 0 ? K : 1);"),
+    ("bias_sign", "C[i * N + n] = int_part + out_part + b;",
+     "C[i * N + n] = int_part + out_part - b;"),
+    ("mask_bit_order", "mask_words[k / 32] |= (uint32_t)1 << (k % 32);",
+     "mask_words[k / 32] |= (uint32_t)1 << (31 - k % 32);"),
+    ("subnormal_decode", "v = ldexpf((float)f, -24);", "v = ldexpf((float)f, -25);"),
+]
+
+
+def _build_mutant(tmp_path, name, old, new):
+    src = open(SRC, encoding="utf-8").read()
+    assert src.count(old) >= 1, "mutation anchor not found: %s" % name
+    mut = src.replace(old, new)
+    c = tmp_path / ("%s.c" % name)
+    so = tmp_path / ("lib%s.so" % name)
+    c.write_text(mut, encoding="utf-8")
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off",
+                           "-fPIC", "-shared", str(c), "-o", str(so), "-lm"])
+    return str(so)
+
+
+@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_planted_mistake_is_caught(tmp_path, name, old, new):
+    so = _build_mutant(tmp_path, name, old, new)
+    failed = []
+    with O.use_library(so):
+        for pin in oracle_pins.ALL_PINS:
+            try:
+                pin()
+            except (AssertionError, OverflowError, ValueError, IndexError):
+                failed.append(pin.__name__)
+    assert failed, "no pin caught the planted mistake %r" % name
