@@ -1,0 +1,182 @@
+"""Thin Python binding of libi8linear (include/i8linear.h): same names as the C ABI.
+
+Argument marshalling only -- every step of the layer runs in the library's CUDA kernels.
+Tensors are torch tensors on the current CUDA device (PyTorch provides device memory and
+streams); their data pointers, sizes and the current stream go straight to the C calls.
+A missing or unloadable library raises; nothing here falls back to another computation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libi8linear.so")
+
+STATUS = {0: "I8_OK", 1: "I8_ERR_INVALID_ARG", 2: "I8_ERR_UNSUPPORTED", 3: "I8_ERR_CUDA",
+          4: "I8_ERR_TIMEOUT", 5: "I8_ERR_DEVICE"}
+
+# every symbol the header declares, with (restype, argtypes)
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+_ST = ctypes.c_int
+SIGNATURES = {
+    "i8_status_string": (ctypes.c_char_p, [_ST]),
+    "i8_quantize_weight": (_ST, [_P, _I64, _I64, _P, _P, _P]),
+    "i8_outlier_scan": (_ST, [_P, _I64, _I64, _F, _P, _P, _P, _P]),
+    "i8_outlier_slice_elems": (_SZ, [_I64, _I64]),
+    "i8_quantize_act": (_ST, [_P, _I64, _I64, _P, _P, _P, _P, _P, _P, _P]),
+    "i8_linear_workspace_size": (_SZ, [_I64, _I64, _I64]),
+    "i8_linear_forward": (_ST, [_P, _I64, _I64, _P, _P, _P, _I64, _F, _P, _P, _SZ, _P]),
+    "i8_igemm_s32": (_ST, [_P, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
+    "i8_sync_status": (_ST, [_P]),
+    "i8_set_profile_events": (_ST, [_P, _P]),
+    "i8_selftest_bounded_wait": (_ST, [_I64, _P]),
+}
+
+
+class I8Error(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__("%s returned %s" % (fn, STATUS.get(code, code)))
+        self.code = code
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libi8linear.so (raises OSError when it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise OSError("libi8linear.so not built: run python -m bit_matmul_decomposition_b200.build")
+        L = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(fn, code):
+    if code != 0:
+        raise I8Error(fn, code)
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+# ----------------------------------------------------------------- the C calls
+def i8_quantize_weight(W, CB, SCB, stream=None):
+    N, K = W.shape
+    _check("i8_quantize_weight",
+           load().i8_quantize_weight(_ptr(W), N, K, _ptr(CB), _ptr(SCB), _stream(stream)))
+
+
+def i8_outlier_scan(X, threshold, col_mask, outlier_idx, n_outliers, stream=None):
+    T, K = X.shape
+    _check("i8_outlier_scan",
+           load().i8_outlier_scan(_ptr(X), T, K, float(threshold), _ptr(col_mask),
+                                  _ptr(outlier_idx), _ptr(n_outliers), _stream(stream)))
+
+
+def i8_outlier_slice_elems(rows, K) -> int:
+    return int(load().i8_outlier_slice_elems(rows, K))
+
+
+def i8_quantize_act(X, col_mask, outlier_idx, n_outliers, Xq, SCx, X_o, stream=None):
+    T, K = X.shape
+    _check("i8_quantize_act",
+           load().i8_quantize_act(_ptr(X), T, K, _ptr(col_mask), _ptr(outlier_idx),
+                                  _ptr(n_outliers), _ptr(Xq), _ptr(SCx), _ptr(X_o),
+                                  _stream(stream)))
+
+
+def i8_linear_workspace_size(T, N, K) -> int:
+    return int(load().i8_linear_workspace_size(T, N, K))
+
+
+def i8_linear_forward(X, CB, SCB, bias, threshold, C, workspace, stream=None):
+    T, K = X.shape
+    N = CB.shape[0]
+    _check("i8_linear_forward",
+           load().i8_linear_forward(_ptr(X), T, K, _ptr(CB), _ptr(SCB), _ptr(bias), N,
+                                    float(threshold), _ptr(C), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(),
+                                    _stream(stream)))
+
+
+def i8_igemm_s32(A, B, acc, workspace, stream=None):
+    T, K = A.shape
+    N = B.shape[0]
+    _check("i8_igemm_s32",
+           load().i8_igemm_s32(_ptr(A), T, K, _ptr(B), N, _ptr(acc), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def i8_sync_status(stream=None) -> int:
+    """Returns the raw status code (0 = I8_OK); see STATUS."""
+    return int(load().i8_sync_status(_stream(stream)))
+
+
+def i8_set_profile_events(start=None, stop=None):
+    s = None if start is None else start.cuda_event
+    e = None if stop is None else stop.cuda_event
+    _check("i8_set_profile_events", load().i8_set_profile_events(s, e))
+
+
+def i8_selftest_bounded_wait(limit_ns, stream=None):
+    _check("i8_selftest_bounded_wait",
+           load().i8_selftest_bounded_wait(int(limit_ns), _stream(stream)))
+
+
+# ----------------------------------------------------------------- allocating helpers
+class Linear8bit:
+    """A decomposed int8 linear layer holding CB/SCB/bias and a workspace (device memory
+    from PyTorch); forward() is one i8_linear_forward call."""
+
+    def __init__(self, W, bias=None, threshold: float = 6.0, stream=None):
+        import torch
+        N, K = W.shape
+        self.N, self.K = N, K
+        self.threshold = float(threshold)
+        self.CB = torch.empty((N, K), dtype=torch.int8, device=W.device)
+        self.SCB = torch.empty((N,), dtype=torch.float32, device=W.device)
+        self.bias = bias
+        i8_quantize_weight(W, self.CB, self.SCB, stream)
+        self._ws = None
+        self._ws_T = -1
+
+    def workspace(self, T):
+        import torch
+        need = i8_linear_workspace_size(T, self.N, self.K)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty((need,), dtype=torch.uint8, device=self.CB.device)
+        return self._ws
+
+    def forward(self, X, out=None, stream=None):
+        import torch
+        T = X.shape[0]
+        if out is None:
+            out = torch.empty((T, self.N), dtype=torch.float16, device=X.device)
+        i8_linear_forward(X, self.CB, self.SCB, self.bias, self.threshold, out,
+                          self.workspace(T), stream)
+        return out

@@ -1,0 +1,458 @@
+// api.cu -- the C ABI of libi8linear (declared in include/i8linear.h): argument checks,
+// workspace layout, TMA descriptors and kernel launches.  One translation unit holds every
+// kernel, so the per-device error word is a single module global.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "../../include/i8linear.h"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "gemv.cuh"
+#include "quant.cuh"
+
+namespace {
+
+using namespace i8;
+
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s for every device-side wait
+constexpr int64_t kDecodeMaxT = 16;               // T <= 16 takes the decode GEMV path
+constexpr int kMaxDevices = 64;
+
+// ------------------------------------------------------------------ device info
+struct DeviceInfo {
+  bool init = false;
+  bool sm100 = false;
+  int sms = 0;
+  bool gemm_attr = false;
+};
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+cudaEvent_t g_prof_start = nullptr;
+cudaEvent_t g_prof_stop = nullptr;
+
+i8_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return I8_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return I8_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    cudaDeviceProp p;
+    if (cudaGetDeviceProperties(&p, dev) != cudaSuccess) return I8_ERR_CUDA;
+    d.sm100 = (p.major == 10 && p.minor == 0);
+    d.sms = p.multiProcessorCount;
+    d.init = true;
+  }
+  if (!d.sm100) return I8_ERR_UNSUPPORTED;
+  if (!d.gemm_attr) {
+    const int bytes = static_cast<int>(gemm::SMEM_BYTES);
+    if (cudaFuncSetAttribute(gemm::i8_gemm_tcgen05_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(gemm::i8_gemm_tcgen05_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+      return I8_ERR_CUDA;
+    d.gemm_attr = true;
+  }
+  *out = &d;
+  return I8_OK;
+}
+
+// ------------------------------------------------------------------ checks
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool shape_ok(int64_t T, int64_t K) {
+  return T > 0 && K > 0 && (K % 16) == 0 && T <= 0x7fffffffLL && K <= 0x7fffffffLL;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+i8_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? I8_OK : I8_ERR_CUDA;
+}
+
+size_t slice_elems(int64_t rows, int64_t K) {
+  return static_cast<size_t>((K + 63) / 64) * static_cast<size_t>(rows) * 64u;
+}
+
+// ------------------------------------------------------------------ workspace layout
+struct Workspace {
+  size_t mask, idx, n_o, scx, xq, xo, cbo, part, total;
+};
+
+Workspace layout(int64_t T, int64_t N, int64_t K) {
+  Workspace w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  w.mask = take(static_cast<size_t>((K + 31) / 32) * 4);
+  w.idx = take(static_cast<size_t>(K) * 4);
+  w.n_o = take(16);
+  w.scx = take(static_cast<size_t>(T) * 4);
+  w.xq = take(static_cast<size_t>(T) * static_cast<size_t>(K));
+  w.xo = take(slice_elems(T, K) * 2);
+  if (T > kDecodeMaxT) {
+    w.cbo = take(slice_elems(N, K) * 2);
+    w.part = 0;
+  } else {
+    w.cbo = 0;
+    w.part = take(static_cast<size_t>(gemv::num_slices(K)) * static_cast<size_t>(T) *
+                  static_cast<size_t>(N) * 4);
+  }
+  w.total = off;
+  return w;
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major [outer, inner] tensor, 128-byte-swizzled box [box_outer, box_inner].
+bool map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
+            uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Chunk-major outlier slice [chunks][rows][64] fp16; box [1][box_rows][64].
+bool map_slice(CUtensorMap* m, const void* base, uint64_t rows, uint64_t chunks,
+               uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {64, rows, chunks};
+  cuuint64_t strides[2] = {128, rows * 128};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ stage launchers
+i8_status run_scan(const void* X, int64_t T, int64_t K, float thr, uint32_t* mask, int32_t* idx,
+                   int32_t* n_o, const DeviceInfo& d, cudaStream_t s) {
+  const int64_t words = (K + 31) / 32;
+  if (cudaMemsetAsync(mask, 0, static_cast<size_t>(words) * 4, s) != cudaSuccess)
+    return I8_ERR_CUDA;
+  const int64_t groups = K / 8;
+  const int64_t gx = (groups + kScanThreads - 1) / kScanThreads;
+  const int64_t target = static_cast<int64_t>(d.sms) * 8;
+  int64_t gy = (target + gx - 1) / gx;
+  if (gy > T) gy = T;
+  if (gy < 1) gy = 1;
+  const int64_t rows_per_cta = (T + gy - 1) / gy;
+  gy = (T + rows_per_cta - 1) / rows_per_cta;
+  if (gx > 0x7fffffffLL || gy > 65535) return I8_ERR_INVALID_ARG;
+  outlier_scan_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), kScanThreads,
+                        0, s>>>(static_cast<const __half*>(X), T, K, thr, rows_per_cta, mask);
+  if (launch_status() != I8_OK) return I8_ERR_CUDA;
+  compact_kernel<<<1, kCompactThreads, 0, s>>>(mask, words, idx, n_o);
+  return launch_status();
+}
+
+i8_status run_quant_rows(const void* A, int64_t R, int64_t K, const uint32_t* mask, int8_t* Q,
+                         float* scale, const int32_t* idx, const int32_t* n_o, void* A_o,
+                         cudaStream_t s) {
+  quantize_rows_kernel<<<static_cast<unsigned>(R), kQuantThreads, 0, s>>>(
+      static_cast<const __half*>(A), R, K, mask, Q, scale, idx, n_o, static_cast<__half*>(A_o));
+  return launch_status();
+}
+
+// tcgen05 GEMM; raw=true writes the int32 accumulator (no outlier phase).
+i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t* B, int64_t N,
+                   const void* A_o, const void* B_o, const int32_t* n_o, const float* SCx,
+                   const float* SCB, const void* bias, void* C, int32_t* acc,
+                   const DeviceInfo& d, cudaStream_t s) {
+  CUtensorMap tA, tB, tAo, tBo;
+  if (!map_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, T, K, gemm::BK, gemm::BM) ||
+      !map_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, K, gemm::BK, gemm::BN))
+    return I8_ERR_CUDA;
+  if (raw) {
+    tAo = tA;
+    tBo = tB;
+  } else {
+    const uint64_t chunks = static_cast<uint64_t>((K + 63) / 64);
+    if (!map_slice(&tAo, A_o, T, chunks, gemm::BM) || !map_slice(&tBo, B_o, N, chunks, gemm::BN))
+      return I8_ERR_CUDA;
+  }
+  gemm::Args a;
+  a.T = static_cast<int>(T);
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.m_tiles = static_cast<int>((T + gemm::BM - 1) / gemm::BM);
+  a.n_tiles = static_cast<int>((N + gemm::BN - 1) / gemm::BN);
+  a.k_blocks = static_cast<int>((K + gemm::BK - 1) / gemm::BK);
+  a.n_outliers = raw ? nullptr : n_o;
+  a.SCx = SCx;
+  a.SCB = SCB;
+  a.bias = static_cast<const __half*>(bias);
+  a.C = static_cast<__half*>(C);
+  a.acc_out = acc;
+  a.wait_limit_ns = kWaitLimitNs;
+  const int64_t tiles = static_cast<int64_t>(a.m_tiles) * a.n_tiles;
+  const int grid = static_cast<int>(tiles < d.sms ? tiles : d.sms);
+  if (raw)
+    gemm::i8_gemm_tcgen05_kernel<true><<<grid, gemm::THREADS, gemm::SMEM_BYTES, s>>>(tA, tB, tAo,
+                                                                                    tBo, a);
+  else
+    gemm::i8_gemm_tcgen05_kernel<false><<<grid, gemm::THREADS, gemm::SMEM_BYTES, s>>>(tA, tB, tAo,
+                                                                                     tBo, a);
+  return launch_status();
+}
+
+// decode GEMV partials; the caller then runs the finalize kernel
+i8_status run_gemv_partial(const int8_t* A, int64_t T, int64_t K, const int8_t* B, int64_t N,
+                           int32_t* P, const DeviceInfo& d, cudaStream_t s) {
+  const int nt = T <= 8 ? 1 : 2;
+  const size_t smem = gemv::smem_bytes(nt, K);
+  if (smem > 200 * 1024) return I8_ERR_INVALID_ARG;
+  const int S = static_cast<int>(gemv::num_slices(K));
+  int per_sm = 0;
+  cudaError_t e;
+  if (nt == 1) {
+    e = cudaFuncSetAttribute(gemv::gemv_partial_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv::gemv_partial_kernel<1>,
+                                                        gemv::THREADS, smem);
+  } else {
+    e = cudaFuncSetAttribute(gemv::gemv_partial_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv::gemv_partial_kernel<2>,
+                                                        gemv::THREADS, smem);
+  }
+  if (e != cudaSuccess) return I8_ERR_CUDA;
+  if (per_sm < 1) per_sm = 1;
+  const int64_t tiles = (N + gemv::ROWS - 1) / gemv::ROWS;
+  int64_t grid = static_cast<int64_t>(d.sms) * per_sm;
+  grid = (grid / S) * S;
+  if (grid < S) grid = S;
+  if (grid > tiles * S) grid = tiles * S;
+  if (nt == 1)
+    gemv::gemv_partial_kernel<1><<<static_cast<unsigned>(grid), gemv::THREADS, smem, s>>>(
+        A, B, static_cast<int>(T), N, K, P);
+  else
+    gemv::gemv_partial_kernel<2><<<static_cast<unsigned>(grid), gemv::THREADS, smem, s>>>(
+        A, B, static_cast<int>(T), N, K, P);
+  return launch_status();
+}
+
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // nothing ever arrives on `bar`: the wait must give up after limit_ns and flag it
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0u, &abort_flag, limit_ns);
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+const char* i8_status_string(i8_status s) {
+  switch (s) {
+    case I8_OK: return "I8_OK";
+    case I8_ERR_INVALID_ARG: return "I8_ERR_INVALID_ARG";
+    case I8_ERR_UNSUPPORTED: return "I8_ERR_UNSUPPORTED";
+    case I8_ERR_CUDA: return "I8_ERR_CUDA";
+    case I8_ERR_TIMEOUT: return "I8_ERR_TIMEOUT";
+    case I8_ERR_DEVICE: return "I8_ERR_DEVICE";
+  }
+  return "I8_UNKNOWN_STATUS";
+}
+
+size_t i8_outlier_slice_elems(int64_t rows, int64_t K) {
+  if (rows <= 0 || K <= 0) return 0;
+  return slice_elems(rows, K);
+}
+
+size_t i8_linear_workspace_size(int64_t T, int64_t N, int64_t K) {
+  if (!shape_ok(T, K) || N <= 0 || N > 0x7fffffffLL) return 0;
+  return layout(T, N, K).total;
+}
+
+i8_status i8_quantize_weight(const void* W, int64_t N, int64_t K, int8_t* CB, float* SCB,
+                             void* stream) {
+  if (!W || !CB || !SCB || !aligned16(W) || !aligned16(CB) || !aligned16(SCB)) return I8_ERR_INVALID_ARG;
+  if (!shape_ok(N, K)) return I8_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  i8_status st = device_info(&d);
+  if (st != I8_OK) return st;
+  return run_quant_rows(W, N, K, nullptr, CB, SCB, nullptr, nullptr, nullptr,
+                        static_cast<cudaStream_t>(stream));
+}
+
+i8_status i8_outlier_scan(const void* X, int64_t T, int64_t K, float threshold, uint32_t* col_mask,
+                          int32_t* outlier_idx, int32_t* n_outliers, void* stream) {
+  if (!X || !col_mask || !outlier_idx || !n_outliers || !aligned16(X) || !aligned16(col_mask) ||
+      !aligned16(outlier_idx) || !aligned16(n_outliers))
+    return I8_ERR_INVALID_ARG;
+  if (!shape_ok(T, K) || threshold != threshold) return I8_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  i8_status st = device_info(&d);
+  if (st != I8_OK) return st;
+  return run_scan(X, T, K, threshold, col_mask, outlier_idx, n_outliers, *d,
+                  static_cast<cudaStream_t>(stream));
+}
+
+i8_status i8_quantize_act(const void* X, int64_t T, int64_t K, const uint32_t* col_mask,
+                          const int32_t* outlier_idx, const int32_t* n_outliers, int8_t* Xq,
+                          float* SCx, void* X_o, void* stream) {
+  if (!X || !col_mask || !outlier_idx || !n_outliers || !Xq || !SCx || !X_o)
+    return I8_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(col_mask) || !aligned16(outlier_idx) || !aligned16(Xq) ||
+      !aligned16(SCx) || !aligned16(X_o) || !aligned16(n_outliers))
+    return I8_ERR_INVALID_ARG;
+  if (!shape_ok(T, K)) return I8_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  i8_status st = device_info(&d);
+  if (st != I8_OK) return st;
+  return run_quant_rows(X, T, K, col_mask, Xq, SCx, outlier_idx, n_outliers, X_o,
+                        static_cast<cudaStream_t>(stream));
+}
+
+i8_status i8_linear_forward(const void* X, int64_t T, int64_t K, const int8_t* CB,
+                            const float* SCB, const void* bias, int64_t N, float threshold,
+                            void* C, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!X || !CB || !SCB || !C || !workspace) return I8_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(CB) || !aligned16(SCB) || !aligned16(C) ||
+      !aligned16(workspace) || (bias && !aligned16(bias)))
+    return I8_ERR_INVALID_ARG;
+  if (!shape_ok(T, K) || N <= 0 || N > 0x7fffffffLL || threshold != threshold)
+    return I8_ERR_INVALID_ARG;
+  const Workspace w = layout(T, N, K);
+  if (workspace_bytes < w.total) return I8_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  i8_status st = device_info(&d);
+  if (st != I8_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* mask = reinterpret_cast<uint32_t*>(ws + w.mask);
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + w.idx);
+  int32_t* n_o = reinterpret_cast<int32_t*>(ws + w.n_o);
+  float* SCx = reinterpret_cast<float*>(ws + w.scx);
+  int8_t* Xq = reinterpret_cast<int8_t*>(ws + w.xq);
+  void* X_o = ws + w.xo;
+
+  st = run_scan(X, T, K, threshold, mask, idx, n_o, *d, s);
+  if (st != I8_OK) return st;
+  st = run_quant_rows(X, T, K, mask, Xq, SCx, idx, n_o, X_o, s);
+  if (st != I8_OK) return st;
+
+  const bool prof = g_prof_start != nullptr && g_prof_stop != nullptr;
+  if (T > kDecodeMaxT) {
+    void* CB_o = ws + w.cbo;
+    const int64_t blocks = static_cast<int64_t>(d->sms) * 8;
+    gather_outlier_weights_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+        CB, N, K, idx, n_o, static_cast<__half*>(CB_o));
+    if (launch_status() != I8_OK) return I8_ERR_CUDA;
+    if (prof && cudaEventRecord(g_prof_start, s) != cudaSuccess) return I8_ERR_CUDA;
+    st = run_gemm(false, Xq, T, K, CB, N, X_o, CB_o, n_o, SCx, SCB, bias, C, nullptr, *d, s);
+    if (st != I8_OK) return st;
+    if (prof && cudaEventRecord(g_prof_stop, s) != cudaSuccess) return I8_ERR_CUDA;
+    return I8_OK;
+  }
+  int32_t* P = reinterpret_cast<int32_t*>(ws + w.part);
+  if (prof && cudaEventRecord(g_prof_start, s) != cudaSuccess) return I8_ERR_CUDA;
+  st = run_gemv_partial(Xq, T, K, CB, N, P, *d, s);
+  if (st != I8_OK) return st;
+  if (prof && cudaEventRecord(g_prof_stop, s) != cudaSuccess) return I8_ERR_CUDA;
+  const int S = static_cast<int>(gemv::num_slices(K));
+  gemv::gemv_finalize_kernel<false><<<static_cast<unsigned>((N + 255) / 256), 256, 0, s>>>(
+      P, S, static_cast<int>(T), N, K, SCx, SCB, static_cast<const __half*>(bias), CB, idx, n_o,
+      static_cast<const __half*>(X_o), static_cast<__half*>(C), nullptr);
+  return launch_status();
+}
+
+i8_status i8_igemm_s32(const int8_t* A, int64_t T, int64_t K, const int8_t* B, int64_t N,
+                       int32_t* acc, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!A || !B || !acc || !workspace || !aligned16(A) || !aligned16(B) || !aligned16(acc) ||
+      !aligned16(workspace))
+    return I8_ERR_INVALID_ARG;
+  if (!shape_ok(T, K) || N <= 0 || N > 0x7fffffffLL || K > 133144) return I8_ERR_INVALID_ARG;
+  const Workspace w = layout(T, N, K);
+  if (workspace_bytes < w.total) return I8_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  i8_status st = device_info(&d);
+  if (st != I8_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (T > kDecodeMaxT)
+    return run_gemm(true, A, T, K, B, N, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                    nullptr, acc, *d, s);
+  int32_t* P = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + w.part);
+  st = run_gemv_partial(A, T, K, B, N, P, *d, s);
+  if (st != I8_OK) return st;
+  const int S = static_cast<int>(gemv::num_slices(K));
+  gemv::gemv_finalize_kernel<true><<<static_cast<unsigned>((N + 255) / 256), 256, 0, s>>>(
+      P, S, static_cast<int>(T), N, K, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+      nullptr, nullptr, acc);
+  return launch_status();
+}
+
+i8_status i8_sync_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return I8_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, i8::g_error_word, sizeof(word)) != cudaSuccess)
+    return I8_ERR_CUDA;
+  if (word == 0) return I8_OK;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(i8::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return I8_ERR_CUDA;
+  if (word & i8::kErrWaitTimeout) return I8_ERR_TIMEOUT;
+  return I8_ERR_DEVICE;
+}
+
+i8_status i8_set_profile_events(void* start_event, void* stop_event) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_prof_start = static_cast<cudaEvent_t>(start_event);
+  g_prof_stop = static_cast<cudaEvent_t>(stop_event);
+  return I8_OK;
+}
+
+i8_status i8_selftest_bounded_wait(int64_t limit_ns, void* stream) {
+  if (limit_ns < 1000 || limit_ns > 10000000000LL) return I8_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  i8_status st = device_info(&d);
+  if (st != I8_OK) return st;
+  bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(limit_ns));
+  return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,177 @@
+/*
+ * i8linear.h -- C ABI of libi8linear: the LLM.int8() mixed-precision decomposed linear
+ * layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer, as the pages describe it ("A Gentle Introduction to 8-bit Matrix
+ * Multiplication for transformers at scale", Hugging Face blog; sections
+ * "LLM.int8() 的总结" and "内部的 MatMul"):
+ *   1. find the outlier feature columns of the fp16 hidden states X (magnitude >= 6);
+ *   2. quantise the remaining columns of X row-wise (one absmax per token);
+ *   3. quantise the weight W once per output channel into int8 codes CB and scales SCB;
+ *   4. multiply the int8 parts with an int32 accumulator;
+ *   5. dequantise by the outer product of the two absmax vectors;
+ *   6. multiply the outlier columns in fp16 against the recovered weights CB*SCB/127,
+ *      add both parts and the bias, and return fp16.
+ *
+ * Conventions for every call
+ *   - fp16 means IEEE 754 binary16; it is passed as `const void*` / `void*`.
+ *   - All tensors are dense and row-major.  X is [T, K] (T tokens, K input features);
+ *     W and CB are [N, K] (the nn.Linear [out, in] layout); C is [T, N].
+ *   - Every pointer is a DEVICE pointer, owned and allocated by the caller (for example
+ *     by PyTorch), 16-byte aligned.  The library allocates no device memory.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls only enqueue
+ *     work; they return before the GPU finishes and never synchronise, except
+ *     i8_sync_status().
+ *   - Arguments are validated on the host before anything is launched; a violation
+ *     returns I8_ERR_INVALID_ARG and enqueues nothing.  Shapes: T, N, K > 0 and
+ *     K % 16 == 0 (the int8 row pitch must be a multiple of 16 bytes for TMA).
+ *   - The calls need an sm_100 device (B200); another device gives I8_ERR_UNSUPPORTED.
+ *   - Every device-side wait is bounded (about one second); a wait that runs out, or a
+ *     failed device-side check, sets a per-device error word that i8_sync_status()
+ *     reports and clears.  The kernels never trap.
+ *   - Calls are safe from several host threads on distinct buffers; the error word and
+ *     the profiling events below are process-wide.
+ */
+#ifndef I8LINEAR_H_
+#define I8LINEAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum i8_status {
+  I8_OK = 0,
+  I8_ERR_INVALID_ARG = 1,  /* bad pointer, shape, threshold or workspace size   */
+  I8_ERR_UNSUPPORTED = 2,  /* the current device is not sm_100                  */
+  I8_ERR_CUDA = 3,         /* a CUDA runtime call or a launch failed            */
+  I8_ERR_TIMEOUT = 4,      /* a bounded device-side wait ran out (sync_status)  */
+  I8_ERR_DEVICE = 5        /* a device-side consistency check failed            */
+} i8_status;
+
+/* Human-readable name of a status code (static storage). */
+const char* i8_status_string(i8_status s);
+
+/*
+ * Step 3 -- per-output-channel weight quantisation, run once per weight.
+ * Source: "用法" (usage) section -- the weight is quantised when the module moves to the
+ * GPU, the codes lie in [-127, 127], and CB * SCB / 127 recovers the fp16 weight; the
+ * 64x64 printout there has one absmax per output row.  "内部的 MatMul": the weight is
+ * quantised column-wise in the A*B orientation, i.e. per output channel.
+ *   W   [N, K] fp16 (read)
+ *   CB  [N, K] int8 (written): CB[n,k] = round_half_away(fl32(W[n,k] * fl32(127/SCB[n])))
+ *   SCB [N]    fp32 (written): SCB[n]  = max_k |W[n,k]|   (0 for an all-zero row: codes 0)
+ * A pure function of W: calling it again on the same W rewrites the same bytes (there is
+ * no "quantise twice" state).
+ */
+i8_status i8_quantize_weight(const void* W, int64_t N, int64_t K, int8_t* CB, float* SCB,
+                             void* stream);
+
+/*
+ * Step 1 -- outlier column scan.
+ * Source: "LLM.int8() 的总结" (outliers are taken column-wise from the hidden states) and
+ * "内部的 MatMul" (all outliers of magnitude 6 or larger).
+ *   X           [T, K] fp16 (read)
+ *   threshold   fp32, not NaN.  Column k is an outlier column when |X[t,k]| >= threshold
+ *               for some row t.  threshold <= 0 marks every column; +inf marks only
+ *               columns holding an infinity.
+ *   col_mask    [ceil(K/32)] uint32 (written; cleared by the call first): column k at
+ *               bit k % 32 of word k / 32.
+ *   outlier_idx [K] int32 (written): the outlier columns in ascending order, first n_o.
+ *   n_outliers  [1] int32 (written): n_o.  Stays on the device; no host copy is made.
+ */
+i8_status i8_outlier_scan(const void* X, int64_t T, int64_t K, float threshold,
+                          uint32_t* col_mask, int32_t* outlier_idx, int32_t* n_outliers,
+                          void* stream);
+
+/* Number of fp16 elements of an outlier slice buffer holding `rows` rows:
+ * ceil(K/64) * rows * 64.  The slice is stored chunk-major: element (row r, outlier j)
+ * sits at ((j / 64) * rows + r) * 64 + j % 64, and entries j >= n_o of the last
+ * 64-wide chunk are zero. */
+size_t i8_outlier_slice_elems(int64_t rows, int64_t K);
+
+/*
+ * Step 2 -- row-wise absmax quantisation of the non-outlier columns of X, and the fp16
+ * outlier slice of X.  Source: "absmax 量化" (scale 127/absmax, then multiply and round;
+ * the [1.2, -0.5, ..., 5.4] example) and "内部的 MatMul" (hidden states quantised per row).
+ *   X           [T, K] fp16 (read)
+ *   col_mask, outlier_idx, n_outliers: as written by i8_outlier_scan (read)
+ *   Xq          [T, K] int8 (written): outlier columns are 0, the others
+ *               round_half_away(fl32(X[t,k] * fl32(127/SCx[t]))) in [-127, 127]
+ *   SCx         [T] fp32 (written): max |X[t,k]| over the non-outlier columns (0 if none
+ *               is nonzero; then the row's codes are 0)
+ *   X_o         fp16 outlier slice, i8_outlier_slice_elems(T, K) elements (written):
+ *               X_o(t, j) = X[t, outlier_idx[j]]
+ */
+i8_status i8_quantize_act(const void* X, int64_t T, int64_t K, const uint32_t* col_mask,
+                          const int32_t* outlier_idx, const int32_t* n_outliers, int8_t* Xq,
+                          float* SCx, void* X_o, void* stream);
+
+/* Device workspace bytes that i8_linear_forward and i8_igemm_s32 need for these sizes
+ * (worst case over the outlier count, which is only known on the device).  0 when a size
+ * is invalid. */
+size_t i8_linear_workspace_size(int64_t T, int64_t N, int64_t K);
+
+/*
+ * Steps 1, 2, 4, 5 and 6 -- the whole forward of the decomposed linear layer.
+ * Sources: "LLM.int8() 的总结" (three steps), "内部的 MatMul" (threshold 6, fp16 outlier
+ * product, row/column vector-wise int8 product, dequantise and add), "absmax 量化"
+ * (outer-product dequantisation), "用法" (fp16 weights recovered as CB * SCB / 127).
+ *   X          [T, K] fp16 (read)         CB [N, K] int8, SCB [N] fp32 (read; from
+ *                                         i8_quantize_weight)
+ *   bias       [N] fp16 or NULL (read)    threshold: as in i8_outlier_scan
+ *   C          [T, N] fp16 (written):
+ *     C[t,n] = fp16_rn( (acc[t,n] * SCx[t] / 127 + sum_j X[t,idx_j] * CB[n,idx_j]) * SCB[n] / 127
+ *                       + bias[n] )
+ *     with acc the exact int32 product of Xq and CB; the outlier sum uses the fp16
+ *     operands with fp32 accumulation, and the epilogue runs in fp32.
+ *   workspace  device buffer of at least i8_linear_workspace_size(T, N, K) bytes, owned by
+ *              the caller; its contents need no initialisation and are scratch after the
+ *              call (calls sharing one workspace must be ordered on one stream).
+ * T <= 16 runs the decode path (warp-level int8 tensor-core GEMV, split over K);
+ * larger T runs the tcgen05 kind::i8 GEMM with the fused outlier/dequant epilogue.
+ */
+i8_status i8_linear_forward(const void* X, int64_t T, int64_t K, const int8_t* CB,
+                            const float* SCB, const void* bias, int64_t N, float threshold,
+                            void* C, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Step 4 alone -- acc[T, N] int32 = A[T, K] int8 * B[N, K]^T int8, on the same kernels
+ * as i8_linear_forward (the tcgen05 GEMM for T > 16, the decode GEMV for T <= 16), with
+ * the epilogue writing the raw accumulator.  Source: "内部的 MatMul" (the 8-bit matrix
+ * multiplication).  Exact: |acc| <= K * 127^2 must fit in int32 (K <= 133144).
+ *   workspace: at least i8_linear_workspace_size(T, N, K) bytes.
+ */
+i8_status i8_igemm_s32(const int8_t* A, int64_t T, int64_t K, const int8_t* B, int64_t N,
+                       int32_t* acc, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronise `stream`, then read and clear the per-device error word.
+ * Returns I8_ERR_CUDA if the stream reports an error, I8_ERR_TIMEOUT if a bounded wait
+ * ran out, I8_ERR_DEVICE if a device-side check failed, else I8_OK.
+ */
+i8_status i8_sync_status(void* stream);
+
+/*
+ * Benchmark hook: when both are non-NULL cudaEvent_t handles, every following
+ * i8_linear_forward records `start` just before and `stop` just after its dominant
+ * kernel (the GEMM or the decode GEMV), on the call's stream.  NULL, NULL turns it off.
+ * Process-wide; meant for single-threaded benchmarking.
+ */
+i8_status i8_set_profile_events(void* start_event, void* stop_event);
+
+/*
+ * Failure-path self test: launch one thread that waits on a device barrier nothing will
+ * complete, with a wait limit of `limit_ns` nanoseconds (1e3 .. 1e10).  The wait runs
+ * out, the error word is set, and the kernel returns; a following i8_sync_status()
+ * must give I8_ERR_TIMEOUT.  Faults nothing and leaves the context usable.
+ */
+i8_status i8_selftest_bounded_wait(int64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* I8LINEAR_H_ */
