@@ -1,0 +1,449 @@
+"""Benchmark of the LLM.int8() decomposed linear layer on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one i8_linear_forward over one batch (outlier scan, activation quantisation,
+int8 tcgen05 GEMM with the fused fp16 outlier product, dequantisation and bias).  The
+weight is quantised once before timing (i8_quantize_weight; timed separately and reported
+under "weight_quant").  Inputs are synthetic (numpy PCG64, see synth.py) with the shape of
+the named workload; the default is the OPT-6.7B FFN up-projection prefill,
+X [2048, 4096] x W [16384, 4096] with 6 fixed outlier columns.
+
+Timing: W untimed warm-up steps; then K timed steps, each bracketed by CUDA events on the
+launching stream, with a 256 MiB buffer written between steps (outside the events) to
+flush the 126 MB L2; barrier + synchronize around the loop; value = total effective
+ops of all ranks / the slowest rank's summed step time.  Multi-GPU: one process per GPU
+(torchrun), each rank owns a disjoint block of output channels of a layer N*world wide
+(column-parallel, no collective on the data path): weak scaling.
+
+--impl reference times the CPU oracle (oracle/, plain C) on this host's cores on the
+same workload, each step a bounded row sample, and prints the same line with
+"impl": "reference".  Only rank 0 runs it.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_matmul_decomposition_b200 import synth  # noqa: E402
+
+METRIC = "int8 decomposed linear: effective TOPS & HBM GB/s, % of sm_100a roofline"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def workloads():
+    w = {"opt_ffn_up": synth.opt_ffn_up_prefill(), "bloom_qkv": synth.bloom_qkv_prefill(),
+         "tiny": synth.tiny()}
+    for T in (1, 8, 16):
+        w["bloom_decode_%d" % T] = synth.bloom_ffn_decode(T)
+    for c in (0, 8, 64, 256):
+        for thr in (6.0, math.inf):
+            w["opt175b_cols%d_thr%s" % (c, "inf" if math.isinf(thr) else "6")] = \
+                synth.opt175b_sweep(c, thr)
+    return w
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sus=float(p["bf16_tflops_sustained"]), source="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+def rank_workload(w, rank):
+    """Weak scaling: rank r owns the r-th block of output channels (its own weight shard);
+    the hidden states are replicated."""
+    if rank == 0:
+        return w, w
+    import dataclasses
+    return w, dataclasses.replace(w, seed=w.seed * 1000 + rank)
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid=None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = os.path.join("/tmp", "i8bench_clocks_%d.csv" % os.getpid())
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                if self.uuid and parts[1] != self.uuid:
+                    continue
+                rows.append(parts)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return None
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[6:10]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][3]) if rows[0][3].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[4]) for r in rows if r[4].replace(".", "").isdigit())}
+
+
+# ----------------------------------------------------------------------------- helpers
+def work_counts(T, N, K, n_o):
+    """Algorithmic work and bytes of one forward."""
+    i8_ops = 2.0 * T * N * (K - n_o)
+    f16_flops = 2.0 * T * N * n_o
+    eff_ops = 2.0 * T * N * K
+    # X read twice (scan, quantise), Xq written and read, CB read, SCB/bias, C written,
+    # the fp16 outlier slices written and read
+    bytes_ = (2 * 2 * T * K + 2 * T * K + N * K + 4 * N + 2 * N + 2 * T * N
+              + 2 * (2 * T * n_o + 2 * N * n_o))
+    return i8_ops, f16_flops, eff_ops, bytes_
+
+
+def traffic_record(kernel):
+    """DRAM bytes per launch from the committed ncu summary (profiles/dram_traffic.txt), if
+    it was taken on the current CUDA sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    try:
+        with open(path) as f:
+            lines = [l.split(None, 4) for l in f if l.strip() and not l.startswith("#")]
+    except OSError:
+        return None
+    for parts in lines:
+        if len(parts) >= 3 and parts[0] == kernel and parts[2] == source_hash():
+            return {"dram_bytes_per_launch": int(parts[1]),
+                    "note": parts[4].strip() if len(parts) > 4 else ""}
+    return None
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for f in ("api.cu", "common.cuh", "quant.cuh", "gemm.cuh", "gemv.cuh"):
+        with open(os.path.join(ROOT, "bit_matmul_decomposition_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def fp16_tensor(a, device):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.float16).to(device)
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample(w, X, CB, SCB, b, budget_s):
+    """Time the oracle on a row sample of the workload: the whole scan + row quantisation
+    (the mask needs every row) and the int8 product/dequant/outlier/bias for `rows` rows,
+    sized to take about budget_s.  Returns (seconds, rows, effective ops)."""
+    from oracle import oracle as O
+    T = X.shape[0]
+    t0 = time.perf_counter()
+    O.linear_forward(X, CB, SCB, b, w.threshold, rows=np.arange(1))
+    one = time.perf_counter() - t0
+    rows = int(max(1, min(T, budget_s / max(one, 1e-4))))
+    sel = np.linspace(0, T - 1, rows).astype(np.int64)
+    t0 = time.perf_counter()
+    O.linear_forward(X, CB, SCB, b, w.threshold, rows=sel)
+    dt = time.perf_counter() - t0
+    return dt, rows, 2.0 * rows * w.N * w.K
+
+
+def run_reference(args, w):
+    """--impl reference: the oracle on the host cores, same workload, per-step row sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from oracle import oracle as O
+    X, W, b = synth.make_x(w), synth.make_w(w), synth.make_bias(w)
+    CB, SCB = O.quantize_weight(W)
+    per_step = max(0.05, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
+    t0 = time.perf_counter()
+    O.linear_forward(X, CB, SCB, b, w.threshold, rows=np.arange(1))
+    one = time.perf_counter() - t0
+    rows = int(max(1, min(w.T, per_step / max(one, 1e-4))))
+    sel = np.linspace(0, w.T - 1, rows).astype(np.int64)
+    for _ in range(args.warmup):
+        O.linear_forward(X, CB, SCB, b, w.threshold, rows=sel)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.linear_forward(X, CB, SCB, b, w.threshold, rows=sel)
+    dt = time.perf_counter() - t0
+    ops = 2.0 * rows * w.N * w.K * args.steps
+    val = ops / dt / 1e12
+    sample = ("per step: scan + row quantisation of all %d rows, then int8 product, "
+              "dequant, fp64 outlier part and bias for %d of %d rows" % (w.T, rows, w.T))
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TOPS",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": dict(w.describe(), sample_rows=rows),
+            "cpu_baseline": {"value": val, "unit": "TOPS", "cores": O.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": val, "unit": "TOPS", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_gpu(args, w0):
+    import torch
+    import torch.distributed as dist
+
+    from bit_matmul_decomposition_b200 import abi
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    _, w = rank_workload(w0, rank)
+    X = synth.make_x(w0)                      # replicated hidden states
+    W = synth.make_w(w)
+    b = synth.make_bias(w)
+    T, K, N = w.T, w.K, w.N
+    abi.load()
+    stream = torch.cuda.current_stream()
+
+    X_d, W_d = fp16_tensor(X, dev), fp16_tensor(W, dev)
+    b_d = None if b is None else fp16_tensor(b, dev)
+    CB = torch.empty((N, K), dtype=torch.int8, device=dev)
+    SCB = torch.empty((N,), dtype=torch.float32, device=dev)
+
+    # weight quantisation (once per weight): timed on its own
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    abi.i8_quantize_weight(W_d, CB, SCB)
+    torch.cuda.synchronize()
+    reps = 5
+    ev[0].record(stream)
+    for _ in range(reps):
+        abi.i8_quantize_weight(W_d, CB, SCB)
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    wq_ms = ev[0].elapsed_time(ev[1]) / reps
+    del W_d
+
+    ws = torch.empty((abi.i8_linear_workspace_size(T, N, K),), dtype=torch.uint8, device=dev)
+    C = torch.empty((T, N), dtype=torch.float16, device=dev)
+    flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=dev)
+
+    def step():
+        abi.i8_linear_forward(X_d, CB, SCB, b_d, w.threshold, C, ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    st = abi.i8_sync_status()
+    if st != 0:
+        raise RuntimeError("device error during warm-up: %s" % abi.STATUS.get(st, st))
+    # outlier count of this input (the scan's device scalar), for the work accounting
+    mask = torch.empty(((K + 31) // 32,), dtype=torch.int32, device=dev)
+    idx = torch.empty((K,), dtype=torch.int32, device=dev)
+    n_o_d = torch.empty((4,), dtype=torch.int32, device=dev)
+    abi.i8_outlier_scan(X_d, w.threshold, mask, idx, n_o_d)
+    n_o = int(n_o_d[0].item())
+
+    K_steps = args.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K_steps)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K_steps)]
+    kv_s = [torch.cuda.Event(enable_timing=True) for _ in range(K_steps)]
+    kv_e = [torch.cuda.Event(enable_timing=True) for _ in range(K_steps)]
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        pass
+    for e in kv_s + kv_e:          # torch creates the CUDA event on its first record
+        e.record(stream)
+    clocks = ClockSampler(uuid)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(K_steps):
+        flush.zero_()
+        abi.i8_set_profile_events(kv_s[i], kv_e[i])
+        ev_s[i].record(stream)
+        step()
+        ev_e[i].record(stream)
+    abi.i8_set_profile_events(None, None)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    st = abi.i8_sync_status()
+    if st != 0:
+        raise RuntimeError("device error in the timed loop: %s" % abi.STATUS.get(st, st))
+
+    step_ms = sum(ev_s[i].elapsed_time(ev_e[i]) for i in range(K_steps))
+    kern_ms = sum(kv_s[i].elapsed_time(kv_e[i]) for i in range(K_steps))
+    t_local = torch.tensor([step_ms, kern_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
+    step_ms, kern_ms = float(t_local[0]), float(t_local[1])
+
+    i8_ops, f16_flops, eff_ops, bytes_ = work_counts(T, N, K, n_o)
+    ms_per_step = step_ms / K_steps
+    value = world * eff_ops / (ms_per_step * 1e-3) / 1e12
+    hbm_gbs = bytes_ / (ms_per_step * 1e-3) / 1e9
+
+    # ---------------------------------------------------------------- end to end
+    e2e_steps = max(3, min(K_steps, 50))
+    X_h = torch.from_numpy(np.ascontiguousarray(X).view(np.int16)).view(torch.float16).pin_memory()
+    C_h = torch.empty((T, N), dtype=torch.float16).pin_memory()
+    X_in = torch.empty_like(X_d)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(2):
+        X_in.copy_(X_h, non_blocking=True)
+        abi.i8_linear_forward(X_in, CB, SCB, b_d, w.threshold, C, ws)
+        C_h.copy_(C, non_blocking=True)
+    barrier()
+    torch.cuda.synchronize()
+    e2e_ms = 0.0
+    for _ in range(e2e_steps):
+        flush.zero_()
+        e0.record(stream)
+        X_in.copy_(X_h, non_blocking=True)
+        abi.i8_linear_forward(X_in, CB, SCB, b_d, w.threshold, C, ws)
+        C_h.copy_(C, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms += e0.elapsed_time(e1)
+    t_e2e = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_e2e, op=dist.ReduceOp.MAX)
+    e2e_per = float(t_e2e[0]) / e2e_steps
+    e2e_value = world * eff_ops / (e2e_per * 1e-3) / 1e12
+    st = abi.i8_sync_status()
+    if st != 0:
+        raise RuntimeError("device error in the e2e loop: %s" % abi.STATUS.get(st, st))
+
+    decode = T <= 16
+    pk = peaks()
+    kern_per = kern_ms / K_steps
+    if decode:
+        # dominant kernel: the K-sliced GEMV streaming CB once
+        gemv_bytes = N * K + T * K + 4 * 4 * T * N
+        achieved = gemv_bytes / (kern_per * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                "frac": achieved / pk["hbm"], "kernel": "gemv_partial_kernel",
+                "algorithmic_bytes_per_launch": gemv_bytes}
+        tr = traffic_record("gemv_partial_kernel")
+    else:
+        # dominant kernel: the tcgen05 GEMM; int8 ops plus fp16 flops counted at the int8
+        # rate x 2 (the nominal fp16 : int8 tensor rate is 1 : 2)
+        equiv = i8_ops + 2.0 * f16_flops
+        achieved = equiv / (kern_per * 1e-3) / 1e12
+        peak_i8 = 2.0 * pk["bf16_sus"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak_i8, "unit": "TOPS",
+                "frac": achieved / peak_i8, "kernel": "i8_gemm_tcgen05_kernel",
+                "peak_basis": "%s sustained bf16 %.1f TF/s x 2 (nominal int8:bf16 ratio)"
+                              % (pk["source"], pk["bf16_sus"]),
+                "frac_of_burst_peak": achieved / (2.0 * pk["bf16"]),
+                "algorithmic_ops_per_launch": equiv}
+        tr = traffic_record("i8_gemm_tcgen05_kernel")
+    roof["kernel_ms"] = kern_per
+    roof["traffic"] = None if tr is None else tr["dram_bytes_per_launch"]
+    if tr is not None:
+        roof["traffic_note"] = tr.get("note", "")
+
+    line = {"metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+            "steps": K_steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8", "data": "synthetic",
+            "config": dict(w0.describe(), n_outliers=n_o,
+                           parallelism="column-parallel x%d (own output-channel block per GPU)"
+                                       % world,
+                           l2="256 MiB buffer written between timed steps (outside the events)"),
+            "hbm_gbs": hbm_gbs * world, "hbm_frac": hbm_gbs / pk["hbm"],
+            "roofline": roof,
+            "weight_quant": {"ms": wq_ms, "gbs": 3.0 * N * K / (wq_ms * 1e-3) / 1e9,
+                             "frac_hbm": 3.0 * N * K / (wq_ms * 1e-3) / 1e9 / pk["hbm"]},
+            "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": 2 * T * K,
+                    "d2h_bytes_per_step": 2 * T * N, "ms_per_step": e2e_per},
+            "gpu_launches": K_steps * (5 if not decode else 5),
+            "clocks": clk}
+
+    # CPU baseline: the oracle on this host, rank 0 at N = 1 only
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import oracle as O
+        CB_h = CB.cpu().numpy()
+        SCB_h = SCB.cpu().numpy()
+        dt, rows, ops = oracle_sample(w, X, CB_h, SCB_h, b, args.cpu_budget)
+        line["cpu_baseline"] = {
+            "value": ops / dt / 1e12, "unit": "TOPS", "cores": O.num_threads(),
+            "kind": "oracle",
+            "sample": "scan + row quantisation of all %d rows, then int8 product, dequant, "
+                      "fp64 outlier part and bias for %d evenly spaced rows x all %d outputs "
+                      "(%.1f s)" % (T, rows, N, dt)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="opt_ffn_up", choices=sorted(workloads()))
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    w = workloads()[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

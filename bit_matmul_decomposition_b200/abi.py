@@ -140,6 +140,9 @@ def i8_sync_status(stream=None) -> int:
 def i8_set_profile_events(start=None, stop=None):
     s = None if start is None else start.cuda_event
     e = None if stop is None else stop.cuda_event
+    if (start is not None and not s) or (stop is not None and not e):
+        raise ValueError("record a torch.cuda.Event once before passing it: torch creates "
+                         "the CUDA event lazily")
     _check("i8_set_profile_events", load().i8_set_profile_events(s, e))
 
 
