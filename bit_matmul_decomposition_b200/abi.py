@@ -32,6 +32,7 @@ SIGNATURES = {
     "i8_linear_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "i8_linear_forward": (_ST, [_P, _I64, _I64, _P, _P, _P, _I64, _F, _P, _P, _SZ, _P]),
     "i8_igemm_s32": (_ST, [_P, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
+    "i8_linear_forward_noalloc": (_ST, [_P, _I64, _I64, _P, _P, _P, _I64, _F, _P, _P]),
     "i8_sync_status": (_ST, [_P]),
     "i8_set_profile_events": (_ST, [_P, _P]),
     "i8_selftest_bounded_wait": (_ST, [_I64, _P]),
@@ -122,6 +123,15 @@ def i8_linear_forward(X, CB, SCB, bias, threshold, C, workspace, stream=None):
                                     float(threshold), _ptr(C), _ptr(workspace),
                                     workspace.numel() * workspace.element_size(),
                                     _stream(stream)))
+
+
+def i8_linear_forward_noalloc(X, CB, SCB, bias, threshold, C, stream=None):
+    """i8_linear_forward with the library's fixed 32 MiB device scratch (no workspace)."""
+    T, K = X.shape
+    N = CB.shape[0]
+    _check("i8_linear_forward_noalloc",
+           load().i8_linear_forward_noalloc(_ptr(X), T, K, _ptr(CB), _ptr(SCB), _ptr(bias), N,
+                                            float(threshold), _ptr(C), _stream(stream)))
 
 
 def i8_igemm_s32(A, B, acc, workspace, stream=None):

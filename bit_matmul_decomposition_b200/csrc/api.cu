@@ -281,6 +281,32 @@ __global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
   if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0u, &abort_flag, limit_ns);
 }
 
+// ------------------------------------------------------------------ fixed scratch
+// Scratch for i8_linear_forward_noalloc: a file-scope device array, so that entry point
+// needs no allocation.  Every GPU that loads this library holds these bytes until the
+// process exits.  In host code the symbol is only a stand-in for the array; its device
+// address comes from cudaGetSymbolAddress, once per device, on that device.
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;  // 32 MiB
+__device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+void* g_static_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device (looked up on first use).
+i8_status static_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return I8_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return I8_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_static_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr)
+      return I8_ERR_CUDA;
+    g_static_scratch_addr[dev] = p;
+  }
+  *out = g_static_scratch_addr[dev];
+  return I8_OK;
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -454,5 +480,22 @@ i8_status i8_selftest_bounded_wait(int64_t limit_ns, void* stream) {
       static_cast<uint64_t>(limit_ns));
   return launch_status();
 }
+
+i8_status i8_linear_forward_noalloc(const void* X, int64_t T, int64_t K, const int8_t* CB,
+                                    const float* SCB, const void* bias, int64_t N,
+                                    float threshold, void* C, void* stream) {
+  if (!X || !CB || !SCB || !C) return I8_ERR_INVALID_ARG;
+  if (!shape_ok(T, K) || N <= 0 || N > 0x7fffffffLL) return I8_ERR_INVALID_ARG;
+  if (layout(T, N, K).total > kStaticScratchBytes) return I8_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  i8_status st = device_info(&d);
+  if (st != I8_OK) return st;
+  void* scratch = nullptr;
+  st = static_scratch_address(&scratch);
+  if (st != I8_OK) return st;
+  return i8_linear_forward(X, T, K, CB, SCB, bias, N, threshold, C, scratch,
+                           kStaticScratchBytes, stream);
+}
+
 
 }  // extern "C"

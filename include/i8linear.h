@@ -18,7 +18,8 @@
  *   - All tensors are dense and row-major.  X is [T, K] (T tokens, K input features);
  *     W and CB are [N, K] (the nn.Linear [out, in] layout); C is [T, N].
  *   - Every pointer is a DEVICE pointer, owned and allocated by the caller (for example
- *     by PyTorch), 16-byte aligned.  The library allocates no device memory.
+ *     by PyTorch), 16-byte aligned.  No call allocates device memory; the only device
+ *     memory the library holds is the fixed scratch array of i8_linear_forward_noalloc.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls only enqueue
  *     work; they return before the GPU finishes and never synchronise, except
  *     i8_sync_status().
@@ -136,6 +137,29 @@ size_t i8_linear_workspace_size(int64_t T, int64_t N, int64_t K);
 i8_status i8_linear_forward(const void* X, int64_t T, int64_t K, const int8_t* CB,
                             const float* SCB, const void* bias, int64_t N, float threshold,
                             void* C, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * i8_linear_forward without a workspace argument: the same forward as i8_linear_forward,
+ * with its scratch taken from a fixed 32 MiB array that the library itself holds in
+ * device memory.  The pages have no counterpart to this call; it exists for callers that
+ * cannot allocate device memory and have none to lend -- for example a plugin inside a
+ * host application that owns every device allocation and hands its plugins no scratch,
+ * or a serving loop that must never call cudaMalloc/cudaFree, because those calls can
+ * synchronise the whole device and stall other work.  This call allocates nothing.
+ *   X, T, K, CB, SCB, bias, N, threshold, C, stream: exactly as in i8_linear_forward.
+ * Limit: sizes whose i8_linear_workspace_size(T, N, K) exceeds 32 MiB are rejected with
+ * I8_ERR_INVALID_ARG before anything is launched (decode batches of large layers, e.g.
+ * T <= 16 with N = 57344, K = 14336, fit; large prefill shapes do not).
+ * Every GPU that loads the library holds the 32 MiB until the process exits.  The first
+ * call on a device looks up the array's device address (once per device, with that
+ * device current); make that first call before any stream capture.  All calls share the
+ * one array and it keeps the last call's contents; nothing in it needs to start at zero
+ * (each call clears what it uses).  Calls that overlap on the GPU -- on different
+ * streams, or from different host threads -- race on the array: order them on one stream.
+ */
+i8_status i8_linear_forward_noalloc(const void* X, int64_t T, int64_t K, const int8_t* CB,
+                                    const float* SCB, const void* bias, int64_t N,
+                                    float threshold, void* C, void* stream);
 
 /*
  * Step 4 alone -- acc[T, N] int32 = A[T, K] int8 * B[N, K]^T int8, on the same kernels
