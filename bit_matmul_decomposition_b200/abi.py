@@ -29,6 +29,7 @@ SIGNATURES = {
     "i8_outlier_scan": (_ST, [_P, _I64, _I64, _F, _P, _P, _P, _P]),
     "i8_outlier_slice_elems": (_SZ, [_I64, _I64]),
     "i8_quantize_act": (_ST, [_P, _I64, _I64, _P, _P, _P, _P, _P, _P, _P]),
+    "i8_prepare_act": (_ST, [_P, _I64, _I64, _F, _P, _P, _P, _P, _P, _P, _P]),
     "i8_linear_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "i8_linear_forward": (_ST, [_P, _I64, _I64, _P, _P, _P, _I64, _F, _P, _P, _SZ, _P]),
     "i8_igemm_s32": (_ST, [_P, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
@@ -109,6 +110,15 @@ def i8_quantize_act(X, col_mask, outlier_idx, n_outliers, Xq, SCx, X_o, stream=N
            load().i8_quantize_act(_ptr(X), T, K, _ptr(col_mask), _ptr(outlier_idx),
                                   _ptr(n_outliers), _ptr(Xq), _ptr(SCx), _ptr(X_o),
                                   _stream(stream)))
+
+
+def i8_prepare_act(X, threshold, col_mask, outlier_idx, n_outliers, Xq, SCx, X_o, stream=None):
+    """col_mask needs ceil(K/32) + 1 words (the last is scratch)."""
+    T, K = X.shape
+    _check("i8_prepare_act",
+           load().i8_prepare_act(_ptr(X), T, K, float(threshold), _ptr(col_mask),
+                                 _ptr(outlier_idx), _ptr(n_outliers), _ptr(Xq), _ptr(SCx),
+                                 _ptr(X_o), _stream(stream)))
 
 
 def i8_linear_workspace_size(T, N, K) -> int:

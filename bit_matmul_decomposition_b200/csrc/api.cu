@@ -26,12 +26,21 @@ struct DeviceInfo {
   bool sm100 = false;
   int sms = 0;
   bool gemm_attr = false;
+  int gemm_clusters = 0;  // co-resident CTA pairs of the GEMM kernel
+  int prep_smem_max = 0;  // dynamic shared memory granted to prepare_kernel
 };
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
 
 cudaEvent_t g_prof_start = nullptr;
 cudaEvent_t g_prof_stop = nullptr;
+
+size_t p_smem_optin(int dev) {
+  int v = 0;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return 0;
+  return static_cast<size_t>(v);
+}
 
 i8_status device_info(DeviceInfo** out) {
   int dev = 0;
@@ -54,6 +63,25 @@ i8_status device_info(DeviceInfo** out) {
         cudaFuncSetAttribute(gemm::i8_gemm_tcgen05_kernel<true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
       return I8_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * d.sms, 1, 1);
+    cfg.blockDim = dim3(gemm::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = gemm::SMEM_BYTES;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, gemm::i8_gemm_tcgen05_kernel<false>, &cfg) !=
+            cudaSuccess ||
+        clusters < 1)
+      return I8_ERR_CUDA;
+    d.gemm_clusters = clusters;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, prepare_kernel) != cudaSuccess) return I8_ERR_CUDA;
+    const int prep_max =
+        static_cast<int>(p_smem_optin(dev)) - static_cast<int>(fa.sharedSizeBytes) - 1024;
+    if (prep_max < 32 * 1024 ||
+        cudaFuncSetAttribute(prepare_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             prep_max) != cudaSuccess)
+      return I8_ERR_CUDA;
+    d.prep_smem_max = prep_max;
     d.gemm_attr = true;
   }
   *out = &d;
@@ -90,7 +118,7 @@ Workspace layout(int64_t T, int64_t N, int64_t K) {
     off = align_up(off + bytes, 256);
     return o;
   };
-  w.mask = take(static_cast<size_t>((K + 31) / 32) * 4);
+  w.mask = take(static_cast<size_t>((K + 31) / 32 + 1) * 4);  // mask + barrier word
   w.idx = take(static_cast<size_t>(K) * 4);
   w.n_o = take(16);
   w.scx = take(static_cast<size_t>(T) * 4);
@@ -188,29 +216,79 @@ i8_status run_quant_rows(const void* A, int64_t R, int64_t K, const uint32_t* ma
   return launch_status();
 }
 
-// tcgen05 GEMM; raw=true writes the int32 accumulator (no outlier phase).
+// Fused steps 1 + 2 (+ the fp16 outlier slices): one cooperative launch.
+// mask must hold ceil(K/32) + 1 words; the last one is the grid-barrier counter.
+i8_status run_prepare(const void* X, int64_t T, int64_t K, float thr, uint32_t* mask,
+                      int32_t* idx, int32_t* n_o, int8_t* Xq, float* SCx, void* X_o,
+                      const int8_t* CB, int64_t N, void* CB_o, const DeviceInfo& d,
+                      cudaStream_t s) {
+  const int64_t words = (K + 31) / 32;
+  if (cudaMemsetAsync(mask, 0, static_cast<size_t>(words + 1) * 4, s) != cudaSuccess)
+    return I8_ERR_CUDA;
+  const int64_t G0 = d.sms;
+  const int64_t rows_per_cta = (T + G0 - 1) / G0;
+  const size_t head = prepare_smem_bytes(K, 0, rows_per_cta);
+  const size_t budget = static_cast<size_t>(d.prep_smem_max);
+  if (head + 16 > budget) return I8_ERR_INVALID_ARG;
+  int64_t cache_rows = static_cast<int64_t>((budget - head) / (static_cast<size_t>(K) * 2));
+  if (cache_rows > rows_per_cta) cache_rows = rows_per_cta;
+  if (cache_rows * K * 2 > static_cast<int64_t>(kPrepChunk) * kPrepMaxChunks)
+    cache_rows = static_cast<int64_t>(kPrepChunk) * kPrepMaxChunks / (K * 2);
+  const size_t smem = prepare_smem_bytes(K, cache_rows, rows_per_cta);
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prepare_kernel, kPrepThreads,
+                                                    smem) != cudaSuccess ||
+      per_sm < 1)
+    return I8_ERR_CUDA;
+  const int grid = d.sms;  // one CTA per SM: every CTA is resident for the grid barrier
+  PrepArgs a;
+  a.X = static_cast<const __half*>(X);
+  a.T = T;
+  a.K = K;
+  a.thr = thr;
+  a.mask = mask;
+  a.idx_out = idx;
+  a.n_o_out = n_o;
+  a.Xq = Xq;
+  a.SCx = SCx;
+  a.X_o = static_cast<__half*>(X_o);
+  a.CB = CB;
+  a.N = N;
+  a.CB_o = static_cast<__half*>(CB_o);
+  a.rows_per_cta = rows_per_cta;
+  a.cache_rows = cache_rows;
+  a.cache_bytes_all = cache_rows * K * 2;
+  a.wait_limit_ns = kWaitLimitNs;
+  void* params[] = {&a};
+  if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(prepare_kernel), dim3(grid),
+                                  dim3(kPrepThreads), params, smem, s) != cudaSuccess)
+    return I8_ERR_CUDA;
+  return launch_status();
+}
+
+// tcgen05 GEMM (pairs of CTAs, 256 x 256 tiles); raw=true writes the int32 accumulator.
 i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t* B, int64_t N,
                    const void* A_o, const void* B_o, const int32_t* n_o, const float* SCx,
                    const float* SCB, const void* bias, void* C, int32_t* acc,
                    const DeviceInfo& d, cudaStream_t s) {
   CUtensorMap tA, tB, tAo, tBo;
-  if (!map_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, T, K, gemm::BK, gemm::BM) ||
-      !map_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, K, gemm::BK, gemm::BN))
+  if (!map_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, T, K, gemm::BK, gemm::HM) ||
+      !map_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, K, gemm::BK, gemm::HN))
     return I8_ERR_CUDA;
   if (raw) {
     tAo = tA;
     tBo = tB;
   } else {
     const uint64_t chunks = static_cast<uint64_t>((K + 63) / 64);
-    if (!map_slice(&tAo, A_o, T, chunks, gemm::BM) || !map_slice(&tBo, B_o, N, chunks, gemm::BN))
+    if (!map_slice(&tAo, A_o, T, chunks, gemm::HM) || !map_slice(&tBo, B_o, N, chunks, gemm::HN))
       return I8_ERR_CUDA;
   }
   gemm::Args a;
   a.T = static_cast<int>(T);
   a.N = static_cast<int>(N);
   a.K = static_cast<int>(K);
-  a.m_tiles = static_cast<int>((T + gemm::BM - 1) / gemm::BM);
-  a.n_tiles = static_cast<int>((N + gemm::BN - 1) / gemm::BN);
+  a.m_tiles = static_cast<int>((T + gemm::TM - 1) / gemm::TM);
+  a.n_tiles = static_cast<int>((N + gemm::TN - 1) / gemm::TN);
   a.k_blocks = static_cast<int>((K + gemm::BK - 1) / gemm::BK);
   a.n_outliers = raw ? nullptr : n_o;
   a.SCx = SCx;
@@ -220,13 +298,13 @@ i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t
   a.acc_out = acc;
   a.wait_limit_ns = kWaitLimitNs;
   const int64_t tiles = static_cast<int64_t>(a.m_tiles) * a.n_tiles;
-  const int grid = static_cast<int>(tiles < d.sms ? tiles : d.sms);
+  const int clusters = static_cast<int>(tiles < d.gemm_clusters ? tiles : d.gemm_clusters);
   if (raw)
-    gemm::i8_gemm_tcgen05_kernel<true><<<grid, gemm::THREADS, gemm::SMEM_BYTES, s>>>(tA, tB, tAo,
-                                                                                    tBo, a);
+    gemm::i8_gemm_tcgen05_kernel<true><<<2 * clusters, gemm::THREADS, gemm::SMEM_BYTES, s>>>(
+        tA, tB, tAo, tBo, a);
   else
-    gemm::i8_gemm_tcgen05_kernel<false><<<grid, gemm::THREADS, gemm::SMEM_BYTES, s>>>(tA, tB, tAo,
-                                                                                     tBo, a);
+    gemm::i8_gemm_tcgen05_kernel<false><<<2 * clusters, gemm::THREADS, gemm::SMEM_BYTES, s>>>(
+        tA, tB, tAo, tBo, a);
   return launch_status();
 }
 
@@ -374,6 +452,22 @@ i8_status i8_quantize_act(const void* X, int64_t T, int64_t K, const uint32_t* c
                         static_cast<cudaStream_t>(stream));
 }
 
+i8_status i8_prepare_act(const void* X, int64_t T, int64_t K, float threshold,
+                         uint32_t* col_mask, int32_t* outlier_idx, int32_t* n_outliers,
+                         int8_t* Xq, float* SCx, void* X_o, void* stream) {
+  if (!X || !col_mask || !outlier_idx || !n_outliers || !Xq || !SCx || !X_o)
+    return I8_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(col_mask) || !aligned16(outlier_idx) || !aligned16(Xq) ||
+      !aligned16(SCx) || !aligned16(X_o) || !aligned16(n_outliers))
+    return I8_ERR_INVALID_ARG;
+  if (!shape_ok(T, K) || threshold != threshold) return I8_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  i8_status st = device_info(&d);
+  if (st != I8_OK) return st;
+  return run_prepare(X, T, K, threshold, col_mask, outlier_idx, n_outliers, Xq, SCx, X_o,
+                     nullptr, 0, nullptr, *d, static_cast<cudaStream_t>(stream));
+}
+
 i8_status i8_linear_forward(const void* X, int64_t T, int64_t K, const int8_t* CB,
                             const float* SCB, const void* bias, int64_t N, float threshold,
                             void* C, void* workspace, size_t workspace_bytes, void* stream) {
@@ -397,31 +491,27 @@ i8_status i8_linear_forward(const void* X, int64_t T, int64_t K, const int8_t* C
   int8_t* Xq = reinterpret_cast<int8_t*>(ws + w.xq);
   void* X_o = ws + w.xo;
 
-  st = run_scan(X, T, K, threshold, mask, idx, n_o, *d, s);
-  if (st != I8_OK) return st;
-  st = run_quant_rows(X, T, K, mask, Xq, SCx, idx, n_o, X_o, s);
-  if (st != I8_OK) return st;
-
   const bool prof = g_prof_start != nullptr && g_prof_stop != nullptr;
   if (T > kDecodeMaxT) {
     void* CB_o = ws + w.cbo;
-    const int64_t blocks = static_cast<int64_t>(d->sms) * 8;
-    gather_outlier_weights_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-        CB, N, K, idx, n_o, static_cast<__half*>(CB_o));
-    if (launch_status() != I8_OK) return I8_ERR_CUDA;
+    st = run_prepare(X, T, K, threshold, mask, idx, n_o, Xq, SCx, X_o, CB, N, CB_o, *d, s);
+    if (st != I8_OK) return st;
     if (prof && cudaEventRecord(g_prof_start, s) != cudaSuccess) return I8_ERR_CUDA;
     st = run_gemm(false, Xq, T, K, CB, N, X_o, CB_o, n_o, SCx, SCB, bias, C, nullptr, *d, s);
     if (st != I8_OK) return st;
     if (prof && cudaEventRecord(g_prof_stop, s) != cudaSuccess) return I8_ERR_CUDA;
     return I8_OK;
   }
+  st = run_prepare(X, T, K, threshold, mask, idx, n_o, Xq, SCx, X_o, nullptr, N, nullptr, *d, s);
+  if (st != I8_OK) return st;
   int32_t* P = reinterpret_cast<int32_t*>(ws + w.part);
   if (prof && cudaEventRecord(g_prof_start, s) != cudaSuccess) return I8_ERR_CUDA;
   st = run_gemv_partial(Xq, T, K, CB, N, P, *d, s);
   if (st != I8_OK) return st;
   if (prof && cudaEventRecord(g_prof_stop, s) != cudaSuccess) return I8_ERR_CUDA;
   const int S = static_cast<int>(gemv::num_slices(K));
-  gemv::gemv_finalize_kernel<false><<<static_cast<unsigned>((N + 255) / 256), 256, 0, s>>>(
+  gemv::gemv_finalize_kernel<false>
+      <<<dim3(static_cast<unsigned>((N + 255) / 256), static_cast<unsigned>(T)), 256, 0, s>>>(
       P, S, static_cast<int>(T), N, K, SCx, SCB, static_cast<const __half*>(bias), CB, idx, n_o,
       static_cast<const __half*>(X_o), static_cast<__half*>(C), nullptr);
   return launch_status();
@@ -446,7 +536,8 @@ i8_status i8_igemm_s32(const int8_t* A, int64_t T, int64_t K, const int8_t* B, i
   st = run_gemv_partial(A, T, K, B, N, P, *d, s);
   if (st != I8_OK) return st;
   const int S = static_cast<int>(gemv::num_slices(K));
-  gemv::gemv_finalize_kernel<true><<<static_cast<unsigned>((N + 255) / 256), 256, 0, s>>>(
+  gemv::gemv_finalize_kernel<true>
+      <<<dim3(static_cast<unsigned>((N + 255) / 256), static_cast<unsigned>(T)), 256, 0, s>>>(
       P, S, static_cast<int>(T), N, K, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
       nullptr, nullptr, acc);
   return launch_status();

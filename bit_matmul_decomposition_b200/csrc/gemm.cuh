@@ -1,8 +1,9 @@
 // gemm.cuh -- steps 4, 5 and 6 for prefill shapes on the 5th-generation tensor cores.
 //
-//   acc[t,n]   = sum_k Xq[t,k] * CB[n,k]              tcgen05.mma kind::i8 -> int32 in TMEM
-//   acc_o[t,n] = sum_j X_o[t,j] * CB_o[n,j]            tcgen05.mma kind::f16 -> fp32 in TMEM
-//   C[t,n]     = fp16((acc * SCx[t]/127 + acc_o) * SCB[n]/127 + bias[n])   (epilogue)
+//   acc[t,n]  = sum_k Xq[t,k] * CB[n,k]                     tcgen05.mma kind::i8 (int32, TMEM)
+//   D[t,n]    = acc[t,n] * SCx[t]/127                       epilogue, written back to TMEM (fp32)
+//   D[t,n]   += sum_j X_o[t,j] * CB_o[n,j]                  tcgen05.mma kind::f16 on top of D
+//   C[t,n]    = fp16(D[t,n] * SCB[n]/127 + bias[n])         epilogue
 //
 // Source: "A Gentle Introduction to 8-bit Matrix Multiplication for transformers at
 // scale" (Hugging Face blog), "内部的 MatMul": the int8 product of row-quantised hidden
@@ -10,17 +11,19 @@
 // outlier columns; "absmax 量化": dequantisation by the outer product of the absmax
 // vectors; "用法": the fp16 weights of the outlier product are CB * SCB / 127.
 //
-// Design (sm_100a, one CTA per SM, persistent over 128 x 256 output tiles):
-//   warp 0      TMA producer: Xq/CB tiles (128 B of K per stage, 128-byte swizzle), then
-//               the X_o/CB_o outlier chunks (64 fp16 per stage), into a 4-stage ring.
-//   warp 1      TMEM allocator and MMA issuer (one thread): 4 MMAs of K=32 bytes per
-//               stage; commits free the ring slot and, per tile, hand the accumulator
-//               to the epilogue.
-//   warps 2..5  epilogue: tcgen05.ld of 32 columns at a time, the fp32 dequant / outlier
-//               add / bias, fp16 stores.  Warp w reads TMEM lanes 32*(w%4)..+31.
-// TMEM (512 columns): with no outliers, two int32 accumulators of 256 columns alternate
-// so the epilogue of tile i overlaps the MMAs of tile i+1; with outliers, one int32
-// accumulator [0,256) and one fp32 outlier accumulator [256,512).
+// Design (sm_100a): persistent clusters of two CTAs on an SM pair, 256 x 256 output tiles,
+// tcgen05.mma.cta_group::2 (M = 256: each CTA holds 128 rows of A and 128 rows of B in its
+// own shared memory, and 128 rows x 256 columns of the accumulator in its own TMEM).
+//   warp 0      TMA producer (both CTAs): 128 B of K per stage, 128-byte swizzle, no
+//               multicast; both CTAs' loads complete on the leader CTA's barrier.
+//   warp 1      TMEM allocation (both CTAs); the leader's lane 0 issues every MMA and
+//               commits with multicast to both CTAs' barriers.
+//   warps 2..5  epilogue (both CTAs): tcgen05.ld / tcgen05.st, per-column scales staged in
+//               shared memory, fp16 stores.  Warp w reads TMEM lanes 32*(w%4)..+31.
+// TMEM holds two 256-column accumulators, so the epilogue of one tile always overlaps the
+// MMAs of the next.  With outlier columns, the int32 accumulator of tile i is converted in
+// place to fp32 (times SCx/127) by the epilogue, and the fp16 outlier MMAs of tile i,
+// issued after the first few K-blocks of tile i+1, accumulate on top of it.
 #pragma once
 
 #include "common.cuh"
@@ -28,22 +31,28 @@
 namespace i8 {
 namespace gemm {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int BK = 128;  // bytes of K per stage
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK;
-constexpr int B_BYTES = BN * BK;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TM = 256;        // cluster tile rows (tokens)
+constexpr int TN = 256;        // cluster tile columns (output features)
+constexpr int HM = TM / 2;     // rows of A per CTA
+constexpr int HN = TN / 2;     // rows of B per CTA
+constexpr int BK = 128;        // bytes of K per stage
+constexpr int STAGES = 6;
+constexpr int A_BYTES = HM * BK;
+constexpr int B_BYTES = HN * BK;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // per CTA
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t IDESC_I8 = idesc_s8_s32(BM, BN);
-constexpr uint32_t IDESC_F16 = idesc_f16_f32(BM, BN);
+constexpr uint32_t IDESC_I8 = idesc_s8_s32(TM, TN);
+constexpr uint32_t IDESC_F16 = idesc_f16_f32(TM, TN);
+constexpr int INSERT_AT = 8;    // K-blocks of tile i+1 issued before the outlier MMAs of tile i
+constexpr int GROUP_M = 16;     // m-tiles per raster group (L2 reuse of Xq)
+constexpr int COL_BYTES = 2 * 2 * TN * 4;        // SCB/127 and bias as fp32, two buffers
 constexpr int BAR_BYTES = 256;
-constexpr size_t SMEM_BYTES = static_cast<size_t>(STAGES) * STAGE_BYTES + BAR_BYTES + 1024;
+constexpr size_t SMEM_BYTES =
+    static_cast<size_t>(STAGES) * STAGE_BYTES + COL_BYTES + BAR_BYTES + 1024;
+constexpr uint16_t PAIR_MASK = 0x3;
 
-static_assert(BM == 128 && BN % 16 == 0 && BN <= 256, "UMMA M=128 shape");
-static_assert(THREADS == 192, "warp roles assume 6 warps");
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
 struct Args {
   int T, N, K;
@@ -58,15 +67,124 @@ struct Args {
 };
 
 struct SmemBars {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
-  uint64_t tmem_full[2];
-  uint64_t tmem_empty[2];
-  uint64_t drain;
+  uint64_t full[STAGES];     // leader: TMA bytes of both CTAs landed
+  uint64_t empty[STAGES];    // both: MMAs reading the slot are done
+  uint64_t int_full[2];      // both: int8 MMAs of the buffer's tile are done
+  uint64_t tmem_full[2];     // both: the buffer's tile is final
+  uint64_t converted[2];     // leader: both epilogues converted the buffer to fp32
+  uint64_t tmem_empty[2];    // leader: both epilogues released the buffer
+  uint64_t drain;            // leader: every issued MMA is done
   uint32_t tmem_base;
   int abort_flag;
 };
 static_assert(sizeof(SmemBars) <= BAR_BYTES, "barrier block");
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+
+// shared::cluster address of the same offset in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* m,
+                                                 uint32_t leader_bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(leader_bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* m,
+                                                 uint32_t leader_bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(leader_bar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void umma_i8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive once on the barrier at `bar` in both CTAs of the pair when every tcgen05 op
+// issued so far by this thread is done.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"(PAIR_MASK)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void epilogue_bar() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
 
 // Stores 32 consecutive fp16 outputs of one row (c0 = first column of the chunk).
 __device__ __forceinline__ void store_row32_f16(__half* crow, int c0, int N, const float (&v)[32],
@@ -93,8 +211,36 @@ __device__ __forceinline__ void store_row32_f16(__half* crow, int c0, int N, con
   }
 }
 
+// The order in which both the producer and the MMA issuer walk the shared-memory ring:
+// for each local tile, its int8 K-blocks; the outlier chunks of the previous tile are
+// slotted in after INSERT_AT K-blocks (or after the last one), and those of the final
+// tile come last.  `visit(kind, tile_slot, idx)` is called per ring stage with kind 0 =
+// int8 K-block idx of local tile tile_slot, kind 1 = outlier chunk idx of tile_slot, and
+// kind 2 / 3 marking the start / end of a tile's int8 phase (no ring stage).
+template <class F>
+__device__ __forceinline__ bool walk_schedule(int L, int KB, int OC, F&& visit) {
+  const int ins = KB < INSERT_AT ? KB : INSERT_AT;
+  for (int it = 0; it < L; ++it) {
+    if (!visit(2, it, 0)) return false;
+    for (int kb = 0; kb < KB; ++kb) {
+      if (OC > 0 && it > 0 && kb == ins)
+        for (int c = 0; c < OC; ++c)
+          if (!visit(1, it - 1, c)) return false;
+      if (!visit(0, it, kb)) return false;
+    }
+    if (OC > 0 && it > 0 && ins >= KB)
+      for (int c = 0; c < OC; ++c)
+        if (!visit(1, it - 1, c)) return false;
+    if (!visit(3, it, 0)) return false;
+  }
+  if (OC > 0 && L > 0)
+    for (int c = 0; c < OC; ++c)
+      if (!visit(1, L - 1, c)) return false;
+  return true;
+}
+
 template <bool kRaw>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     i8_gemm_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmAo,
@@ -104,10 +250,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
   const uint32_t ring = raw_s + pad;  // 1024-aligned shared address of stage 0
-  SmemBars* bars = reinterpret_cast<SmemBars*>(smem + static_cast<size_t>(STAGES) * STAGE_BYTES);
+  float* colbuf = reinterpret_cast<float*>(smem + static_cast<size_t>(STAGES) * STAGE_BYTES);
+  SmemBars* bars = reinterpret_cast<SmemBars*>(smem + static_cast<size_t>(STAGES) * STAGE_BYTES +
+                                               COL_BYTES);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
   volatile int* abort_flag = &bars->abort_flag;
 
   if (threadIdx.x == 0) {
@@ -116,8 +265,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(smem_u32(&bars->empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&bars->int_full[b]), 1);
       mbar_init(smem_u32(&bars->tmem_full[b]), 1);
-      mbar_init(smem_u32(&bars->tmem_empty[b]), 128);
+      mbar_init(smem_u32(&bars->converted[b]), 8);   // 4 epilogue warps x 2 CTAs
+      mbar_init(smem_u32(&bars->tmem_empty[b]), 8);
     }
     mbar_init(smem_u32(&bars->drain), 1);
     bars->abort_flag = 0;
@@ -130,56 +281,88 @@ __global__ void __launch_bounds__(THREADS, 1)
     tma_prefetch_desc(&tmBo);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(&bars->tmem_base), TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(&bars->tmem_base), TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = bars->tmem_base;
 
   const int n_o = (a.n_outliers != nullptr) ? max(0, __ldg(a.n_outliers)) : 0;
-  const int o_chunks = (n_o + 63) >> 6;
-  const int nbuf = (o_chunks == 0) ? 2 : 1;
+  const int OC = (n_o + 63) >> 6;
+  const int KB = a.k_blocks;
   const int num_tiles = a.m_tiles * a.n_tiles;
-  const int steps_per_tile = a.k_blocks + o_chunks;
+  const int cluster_id = blockIdx.x >> 1;
+  const int num_clusters = gridDim.x >> 1;
+  const int L = cluster_id < num_tiles ? (num_tiles - 1 - cluster_id) / num_clusters + 1 : 0;
   const uint64_t lim = a.wait_limit_ns;
+
+  // Grouped raster: consecutive tiles walk GROUP_M m-tiles, then the next n-tile, so the
+  // tiles in flight share a block of Xq rows and a few CB row blocks that fit in L2.
+  const int G = a.m_tiles < GROUP_M ? a.m_tiles : GROUP_M;
+  auto tile_mn = [&](int it, int& m0, int& n0) {
+    const int t = cluster_id + it * num_clusters;
+    const int group = t / (G * a.n_tiles);
+    const int r = t - group * (G * a.n_tiles);
+    const int mb = group * G;
+    const int rows = (a.m_tiles - mb) < G ? (a.m_tiles - mb) : G;
+    m0 = (mb + r % rows) * TM;
+    n0 = (r / rows) * TN;
+  };
+  auto tile_m0 = [&](int it) {
+    int m0, n0;
+    tile_mn(it, m0, n0);
+    return m0;
+  };
+  auto tile_n0 = [&](int it) {
+    int m0, n0;
+    tile_mn(it, m0, n0);
+    return n0;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ TMA producer
+      // Tile coordinates are computed once per tile (the ring only ever refers to the
+      // current tile and the one before it), so a stage costs a handful of instructions.
       int s = 0;
       uint32_t ph = 0;
       uint32_t issued = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m0 = (tile % a.m_tiles) * BM;
-        const int n0 = (tile / a.m_tiles) * BN;
-        for (int kb = 0; kb < steps_per_tile; ++kb) {
-          if (!mbar_wait(smem_u32(&bars->empty[s]), ph ^ 1u, abort_flag, lim)) {
-            ok = false;
-            break;
-          }
-          const uint32_t sa = ring + s * STAGE_BYTES;
-          const uint32_t sb = sa + A_BYTES;
-          const uint32_t fb = smem_u32(&bars->full[s]);
-          mbar_arrive_expect_tx(fb, STAGE_BYTES);
-          if (kb < a.k_blocks) {
-            tma_load_2d(sa, &tmA, fb, kb * BK, m0);
-            tma_load_2d(sb, &tmB, fb, kb * BK, n0);
-          } else {
-            const int c = kb - a.k_blocks;
-            tma_load_3d(sa, &tmAo, fb, 0, m0, c);
-            tma_load_3d(sb, &tmBo, fb, 0, n0, c);
-          }
-          ++issued;
-          if (++s == STAGES) {
-            s = 0;
-            ph ^= 1u;
-          }
+      int coord_it[2] = {-1, -1};
+      int coord_a[2] = {0, 0}, coord_b[2] = {0, 0};
+      const uint32_t full_leader0 = map_to_rank(smem_u32(&bars->full[0]), 0);
+      const bool ok = walk_schedule(L, KB, OC, [&](int kind, int it, int idx) -> bool {
+        if (kind >= 2) return true;
+        const int slot = it & 1;
+        if (coord_it[slot] != it) {
+          int m0, n0;
+          tile_mn(it, m0, n0);
+          coord_a[slot] = m0 + static_cast<int>(rank) * HM;
+          coord_b[slot] = n0 + static_cast<int>(rank) * HN;
+          coord_it[slot] = it;
         }
-      }
-      if (!ok) {
+        if (!mbar_wait(smem_u32(&bars->empty[s]), ph ^ 1u, abort_flag, lim)) return false;
+        const uint32_t sa = ring + s * STAGE_BYTES;
+        const uint32_t sb = sa + A_BYTES;
+        if (rank == 0) mbar_arrive_expect_tx(smem_u32(&bars->full[s]), 2 * STAGE_BYTES);
+        const uint32_t fb = full_leader0 + static_cast<uint32_t>(s) * 8u;
+        if (kind == 0) {
+          tma_load_2d_pair(sa, &tmA, fb, idx * BK, coord_a[slot]);
+          tma_load_2d_pair(sb, &tmB, fb, idx * BK, coord_b[slot]);
+        } else {
+          tma_load_3d_pair(sa, &tmAo, fb, 0, coord_a[slot], idx);
+          tma_load_3d_pair(sb, &tmBo, fb, 0, coord_b[slot], idx);
+        }
+        ++issued;
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+        return true;
+      });
+      if (!ok && rank == 0) {
         // wind down: wait (bounded, ignoring the abort flag) for the copies in flight
         int no_abort = 0;
         const uint32_t inflight = issued < STAGES ? issued : STAGES;
@@ -190,82 +373,124 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && rank == 0) {
+      // ------------------------------------------------------------ MMA issuer (leader)
       int s = 0;
       uint32_t ph = 0;
-      bool ok = true;
-      int it = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
-        const int b = (nbuf == 2) ? (it & 1) : 0;
-        const uint32_t use = (nbuf == 2) ? static_cast<uint32_t>(it >> 1) : static_cast<uint32_t>(it);
-        if (!mbar_wait(smem_u32(&bars->tmem_empty[b]), (use & 1u) ^ 1u, abort_flag, lim)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_int = tmem_base + static_cast<uint32_t>(b * BN);
-        const uint32_t d_out = tmem_base + static_cast<uint32_t>(BN);
-        for (int kb = 0; kb < steps_per_tile; ++kb) {
-          if (!mbar_wait(smem_u32(&bars->full[s]), ph, abort_flag, lim)) {
-            ok = false;
-            break;
-          }
+      int conv_wait_done = -1;  // last tile whose conversion barrier was consumed
+      walk_schedule(L, KB, OC, [&](int kind, int it, int idx) -> bool {
+        const int b = it & 1;
+        const uint32_t use = static_cast<uint32_t>(it >> 1);
+        if (kind == 2) {  // start of tile it's int8 phase: its buffer must be free
+          if (!mbar_wait(smem_u32(&bars->tmem_empty[b]), (use & 1u) ^ 1u, abort_flag, lim))
+            return false;
           tc_fence_after();
-          const uint32_t sa = ring + s * STAGE_BYTES;
-          const uint32_t sb = sa + A_BYTES;
-          if (kb < a.k_blocks) {
-#pragma unroll
-            for (int kk = 0; kk < BK / 32; ++kk)
-              umma_i8(d_int, sdesc_k_sw128(sa + kk * 32), sdesc_k_sw128(sb + kk * 32), IDESC_I8,
-                      (kb | kk) != 0);
-          } else {
-            const int c = kb - a.k_blocks;
-#pragma unroll
-            for (int kk = 0; kk < BK / 32; ++kk)
-              umma_f16(d_out, sdesc_k_sw128(sa + kk * 32), sdesc_k_sw128(sb + kk * 32),
-                       IDESC_F16, (c | kk) != 0);
-          }
-          umma_commit(smem_u32(&bars->empty[s]));
-          if (++s == STAGES) {
-            s = 0;
-            ph ^= 1u;
-          }
+          return true;
         }
-        if (!ok) break;
-        umma_commit(smem_u32(&bars->tmem_full[b]));
-      }
+        if (kind == 3) {  // end of tile it's int8 phase
+          umma_commit_pair(smem_u32(OC > 0 ? &bars->int_full[b] : &bars->tmem_full[b]));
+          return true;
+        }
+        if (kind == 1 && conv_wait_done != it) {  // first outlier chunk of tile it
+          if (!mbar_wait(smem_u32(&bars->converted[b]), use & 1u, abort_flag, lim)) return false;
+          tc_fence_after();
+          conv_wait_done = it;
+        }
+        if (!mbar_wait(smem_u32(&bars->full[s]), ph, abort_flag, lim)) return false;
+        tc_fence_after();
+        const uint32_t sa = ring + s * STAGE_BYTES;
+        const uint32_t sb = sa + A_BYTES;
+        const uint32_t d = tmem_base + static_cast<uint32_t>(b * TN);
+        if (kind == 0) {
+#pragma unroll
+          for (int kk = 0; kk < BK / 32; ++kk)
+            umma_i8_pair(d, sdesc_k_sw128(sa + kk * 32), sdesc_k_sw128(sb + kk * 32), IDESC_I8,
+                         (idx | kk) != 0);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < BK / 32; ++kk)
+            umma_f16_pair(d, sdesc_k_sw128(sa + kk * 32), sdesc_k_sw128(sb + kk * 32), IDESC_F16,
+                          1u);
+        }
+        umma_commit_pair(smem_u32(&bars->empty[s]));
+        if (kind == 1 && idx == OC - 1) umma_commit_pair(smem_u32(&bars->tmem_full[b]));
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+        return true;
+      });
       // every MMA issued by this thread completes before TMEM is released
       int no_abort = 0;
-      umma_commit(smem_u32(&bars->drain));
+      umma_commit_pair(smem_u32(&bars->drain));
       mbar_wait(smem_u32(&bars->drain), 0u, &no_abort, lim);
     }
   } else {
     // -------------------------------------------------------------- epilogue warps
     const int q = warp & 3;
     const int row = q * 32 + lane;
+    const int et = threadIdx.x - 64;  // 0..127 among the epilogue threads
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     const bool vec_ok = (a.N % 8) == 0;
-    int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
-      const int b = (nbuf == 2) ? (it & 1) : 0;
-      const uint32_t use = (nbuf == 2) ? static_cast<uint32_t>(it >> 1) : static_cast<uint32_t>(it);
-      // all 32 lanes must take the same branch: tcgen05.ld below is warp-collective
-      const bool got = mbar_wait(smem_u32(&bars->tmem_full[b]), use & 1u, abort_flag, lim);
-      if (!__all_sync(0xffffffffu, got)) break;
-      tc_fence_after();
-      const int m0 = (tile % a.m_tiles) * BM;
-      const int n0 = (tile / a.m_tiles) * BN;
-      const int t = m0 + row;
+    // A warp that gives up on a wait keeps walking the tiles (it must still meet the
+    // other epilogue warps at every named barrier) but touches TMEM no more.
+    bool dead = false;
+    for (int it = 0; it < L; ++it) {
+      const int b = it & 1;
+      const uint32_t use = static_cast<uint32_t>(it >> 1);
+      const int m0 = tile_m0(it);
+      const int n0 = tile_n0(it);
+      const int t = m0 + static_cast<int>(rank) * HM + row;
       const bool row_ok = t < a.T;
-      float sx = 0.0f;
-      if (!kRaw && row_ok) sx = __ldg(a.SCx + t) * (1.0f / 127.0f);
+      float* ws = colbuf + b * (2 * TN);
+      float* bs = ws + TN;
+      if (!kRaw) {
+        for (int j = et; j < TN; j += 128) {
+          const int n = n0 + j;
+          ws[j] = n < a.N ? __ldg(a.SCB + n) * (1.0f / 127.0f) : 0.0f;
+          bs[j] = (n < a.N && a.bias) ? __half2float(a.bias[n]) : 0.0f;
+        }
+      }
+      epilogue_bar();
+      if (dead) continue;
+      const float sx = (!kRaw && row_ok) ? __ldg(a.SCx + t) * (1.0f / 127.0f) : 0.0f;
+      const uint32_t tb = lane_base + static_cast<uint32_t>(b * TN);
+
+      if (!kRaw && OC > 0) {
+        // int32 -> fp32 * SCx/127 in place; the outlier MMAs then add on top
+        bool got = mbar_wait(smem_u32(&bars->int_full[b]), use & 1u, abort_flag, lim);
+        if (!__all_sync(0xffffffffu, got)) {
+          dead = true;
+          continue;
+        }
+        tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < TN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tb + static_cast<uint32_t>(c * 32), r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            r[j] = __float_as_uint(static_cast<float>(static_cast<int32_t>(r[j])) * sx);
+          tmem_st_32x32b_x32(tb + static_cast<uint32_t>(c * 32), r);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(map_to_rank(smem_u32(&bars->converted[b]), 0));
+      }
+      {
+        bool got = mbar_wait(smem_u32(&bars->tmem_full[b]), use & 1u, abort_flag, lim);
+        if (!__all_sync(0xffffffffu, got)) {
+          dead = true;
+          continue;
+        }
+      }
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < TN / 32; ++c) {
         uint32_t r[32];
-        uint32_t o[32];
-        tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>(b * BN + c * 32), r);
-        if (!kRaw && nbuf == 1) tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>(BN + c * 32), o);
+        tmem_ld_32x32b_x32(tb + static_cast<uint32_t>(c * 32), r);
         tmem_ld_wait();
         const int c0 = n0 + c * 32;
         if (row_ok && c0 < a.N) {
@@ -283,30 +508,34 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
           } else {
             float v[32];
+            const float* wsc = ws + c * 32;
+            const float* bsc = bs + c * 32;
+            if (OC > 0) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int n = min(c0 + j, a.N - 1);
-              const float ws = __ldg(a.SCB + n) * (1.0f / 127.0f);
-              const float bn = a.bias ? __half2float(a.bias[n]) : 0.0f;
-              const float oj = (nbuf == 1) ? __uint_as_float(o[j]) : 0.0f;
-              const float part = fmaf(static_cast<float>(static_cast<int32_t>(r[j])), sx, oj);
-              v[j] = fmaf(part, ws, bn);
+              for (int j = 0; j < 32; ++j) v[j] = fmaf(__uint_as_float(r[j]), wsc[j], bsc[j]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                v[j] = fmaf(static_cast<float>(static_cast<int32_t>(r[j])) * sx, wsc[j], bsc[j]);
             }
             store_row32_f16(a.C + static_cast<int64_t>(t) * a.N, c0, a.N, v, vec_ok);
           }
         }
       }
       tc_fence_before();
-      mbar_arrive(smem_u32(&bars->tmem_empty[b]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(map_to_rank(smem_u32(&bars->tmem_empty[b]), 0));
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
+  cluster_sync();
 }
 
 }  // namespace gemm

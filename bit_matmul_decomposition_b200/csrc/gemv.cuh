@@ -147,8 +147,9 @@ __global__ void __launch_bounds__(THREADS)
   }
 }
 
-// One thread per output column n: sum the slices, then dequantise, add the outlier part
-// (read straight from CB with the index list) and the bias.  kRaw writes the int32 sum.
+// One thread per output (t, n) -- grid.y is the token: sum the K-slice partials (exact
+// int32), then dequantise, add the outlier part (CB read straight through the index list,
+// 8 loads in flight) and the bias.  kRaw writes the int32 sum.
 template <bool kRaw>
 __global__ void __launch_bounds__(256)
     gemv_finalize_kernel(const int32_t* __restrict__ P, int S, int T, int64_t N, int64_t K,
@@ -158,25 +159,35 @@ __global__ void __launch_bounds__(256)
                          const __half* __restrict__ X_o, __half* __restrict__ C,
                          int32_t* __restrict__ acc_out) {
   const int64_t n = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int t = blockIdx.y;
   if (n >= N) return;
-  const int n_o = (kRaw || n_o_ptr == nullptr) ? 0 : *n_o_ptr;
-  const float ws = kRaw ? 0.0f : __ldg(SCB + n) * (1.0f / 127.0f);
-  const float bn = (!kRaw && bias) ? __half2float(bias[n]) : 0.0f;
-  for (int t = 0; t < T; ++t) {
-    int32_t acc = 0;
-    for (int s = 0; s < S; ++s) acc += P[(static_cast<int64_t>(s) * T + t) * N + n];
-    if (kRaw) {
-      acc_out[static_cast<int64_t>(t) * N + n] = acc;
-      continue;
-    }
-    float o = 0.0f;
-    for (int j = 0; j < n_o; ++j) {
-      const float xo = __half2float(X_o[(static_cast<int64_t>(j >> 6) * T + t) * 64 + (j & 63)]);
-      o = fmaf(xo, static_cast<float>(CB[n * K + idx[j]]), o);
-    }
-    const float part = fmaf(static_cast<float>(acc), __ldg(SCx + t) * (1.0f / 127.0f), o);
-    C[static_cast<int64_t>(t) * N + n] = __float2half_rn(fmaf(part, ws, bn));
+  int32_t acc = 0;
+  for (int s = 0; s < S; ++s) acc += __ldcs(P + (static_cast<int64_t>(s) * T + t) * N + n);
+  if (kRaw) {
+    acc_out[static_cast<int64_t>(t) * N + n] = acc;
+    return;
   }
+  const int n_o = (n_o_ptr == nullptr) ? 0 : *n_o_ptr;
+  float o = 0.0f;
+  for (int j0 = 0; j0 < n_o; j0 += 8) {
+    float cb[8], xo[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u;
+      cb[u] = 0.0f;
+      xo[u] = 0.0f;
+      if (j < n_o) {
+        cb[u] = static_cast<float>(CB[n * K + __ldg(idx + j)]);
+        xo[u] = __half2float(X_o[(static_cast<int64_t>(j >> 6) * T + t) * 64 + (j & 63)]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) o = fmaf(xo[u], cb[u], o);
+  }
+  const float ws = __ldg(SCB + n) * (1.0f / 127.0f);
+  const float bn = bias ? __half2float(bias[n]) : 0.0f;
+  const float part = fmaf(static_cast<float>(acc), __ldg(SCx + t) * (1.0f / 127.0f), o);
+  C[static_cast<int64_t>(t) * N + n] = __float2half_rn(fmaf(part, ws, bn));
 }
 
 }  // namespace gemv

@@ -3,7 +3,8 @@
 //   compact_kernel         step 1: mask -> ascending outlier index list + count
 //   quantize_rows_kernel   steps 2/3: row absmax (over the non-outlier columns) and int8
 //                          codes; for the hidden states also the fp16 outlier slice X_o
-//   gather_outlier_weights_kernel  step 6 operand: CB[:, idx] as exact fp16, chunk-major
+//   prepare_kernel         steps 1 and 2 fused (one read of X), plus the fp16 outlier
+//                          slices of X and of CB for step 6
 // Source: "A Gentle Introduction to 8-bit Matrix Multiplication for transformers at
 // scale" (Hugging Face blog), sections "absmax 量化", "LLM.int8() 的总结", "内部的 MatMul".
 #pragma once
@@ -218,28 +219,433 @@ __global__ void __launch_bounds__(kQuantThreads)
   }
 }
 
-// ------------------------------------------------------------------ step 6 operand
-// CB_o(n, j) = (fp16) CB[n, idx[j]] (exact: |CB| <= 127), chunk-major [ceil(n_o/64)][N][64],
-// zero for j >= n_o.  One warp per (chunk, row); each lane writes two adjacent halves.
-__global__ void __launch_bounds__(256)
-    gather_outlier_weights_kernel(const int8_t* __restrict__ CB, int64_t N, int64_t K,
-                                  const int32_t* __restrict__ idx,
-                                  const int32_t* __restrict__ n_o_ptr,
-                                  __half* __restrict__ CB_o) {
-  const int n_o = *n_o_ptr;
-  const int64_t chunks = (n_o + 63) >> 6;
-  const int64_t items = chunks * N;
-  const int lane = threadIdx.x & 31;
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t it = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-       it < items; it += nwarps) {
-    const int64_t c = it / N, n = it - c * N;
-    const int64_t j0 = c * 64 + 2 * lane;
-    float v0 = 0.0f, v1 = 0.0f;
-    if (j0 < n_o) v0 = static_cast<float>(CB[n * K + idx[j0]]);
-    if (j0 + 1 < n_o) v1 = static_cast<float>(CB[n * K + idx[j0 + 1]]);
-    reinterpret_cast<__half2*>(CB_o + (c * N + n) * 64)[lane] = __floats2half2_rn(v0, v1);
+
+// ====================================================================== fused pass
+// prepare_kernel: steps 1 and 2 in one launch, reading X from HBM once when the rows of
+// each CTA fit in its shared memory (re-reading, mostly from L2, the rows that do not):
+//   phase 1  each CTA pulls its block of rows into shared memory with bulk (TMA) copies,
+//            scans it, and ORs its column bits into the global mask;
+//   barrier  one grid-wide barrier (every CTA is resident: one CTA per SM; the wait is
+//            bounded like every other wait in this library);
+//   phase 2  every CTA reads the final mask and builds the ascending outlier index list
+//            in its own shared memory; CTA 0 also writes it (and n_o) to global memory;
+//   phase 3  all threads of the CTA walk its rows together: absmax over the non-outlier
+//            columns, int8 codes, the fp16 outlier slice X_o;
+//   phase 4  (GEMM path) the fp16 outlier slice of the weight, CB_o, for all N rows.
+// The caller clears mask[0 .. words] (the last word is the barrier counter) beforehand.
+constexpr int kPrepThreads = 512;
+constexpr int kPrepWarps = kPrepThreads / 32;
+constexpr int kPrepChunk = 32768;   // bytes per bulk copy of the row cache
+constexpr int kPrepMaxChunks = 8;
+
+struct PrepArgs {
+  const __half* X;
+  int64_t T, K;
+  float thr;
+  uint32_t* mask;         // [words + 1]: mask, then the barrier counter
+  int32_t* idx_out;       // [K]
+  int32_t* n_o_out;       // [1]
+  int8_t* Xq;
+  float* SCx;
+  __half* X_o;            // chunk-major slice [ceil(K/64)][T][64]
+  const int8_t* CB;       // [N, K] (phase 4) or NULL
+  int64_t N;
+  __half* CB_o;           // chunk-major slice [ceil(K/64)][N][64] or NULL
+  int64_t rows_per_cta;
+  int64_t cache_rows;     // rows of its block each CTA keeps in shared memory
+  int64_t cache_bytes_all; // size of the row-cache region (reused by phase 4)
+  uint64_t wait_limit_ns;
+};
+
+__host__ __device__ inline int g32_of(int64_t K) { return static_cast<int>(K / 16); }
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// fast absmax of 8 fp16 values when none of them is excluded (exact in fp16)
+__device__ __forceinline__ float absmax8_all(const uint4 v) {
+  __half2 a = __habs2(*reinterpret_cast<const __half2*>(&v.x));
+  __half2 b = __habs2(*reinterpret_cast<const __half2*>(&v.y));
+  __half2 c = __habs2(*reinterpret_cast<const __half2*>(&v.z));
+  __half2 d = __habs2(*reinterpret_cast<const __half2*>(&v.w));
+  const __half2 m = __hmax2(__hmax2(a, b), __hmax2(c, d));
+  return fmaxf(__low2float(m), __high2float(m));
+}
+
+__device__ __forceinline__ uint32_t scan_bits(const uint32_t* smask, int64_t g) {
+  return (smask[g >> 2] >> (8 * (g & 3))) & 0xffu;
+}
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+// 16-byte group v of a row held in shared memory (kShared, `base` a shared address) or in
+// global memory (`gbase`).
+template <bool kShared>
+__device__ __forceinline__ uint4 row_vec(uint32_t base, const uint4* gbase, int v) {
+  if (kShared) return lds_v4(base + static_cast<uint32_t>(v) * 16u);
+  return ldg_v4(gbase + v);
+}
+
+// Max |x| over the non-outlier columns of groups start, start+step, ... of one row.
+template <bool kShared>
+__device__ __forceinline__ float row_absmax(uint32_t base, const uint4* gbase, int gpr, int start,
+                                            int step, const uint32_t* smask) {
+  float m0 = 0.0f, m1 = 0.0f, m2 = 0.0f, m3 = 0.0f;
+  int v = start;
+  for (; v + 3 * step < gpr; v += 4 * step) {
+    const uint4 x0 = row_vec<kShared>(base, gbase, v);
+    const uint4 x1 = row_vec<kShared>(base, gbase, v + step);
+    const uint4 x2 = row_vec<kShared>(base, gbase, v + 2 * step);
+    const uint4 x3 = row_vec<kShared>(base, gbase, v + 3 * step);
+    const uint32_t k0 = scan_bits(smask, v), k1 = scan_bits(smask, v + step);
+    const uint32_t k2 = scan_bits(smask, v + 2 * step), k3 = scan_bits(smask, v + 3 * step);
+    m0 = fmaxf(m0, k0 ? absmax8(x0, k0) : absmax8_all(x0));
+    m1 = fmaxf(m1, k1 ? absmax8(x1, k1) : absmax8_all(x1));
+    m2 = fmaxf(m2, k2 ? absmax8(x2, k2) : absmax8_all(x2));
+    m3 = fmaxf(m3, k3 ? absmax8(x3, k3) : absmax8_all(x3));
   }
+  for (; v < gpr; v += step) {
+    const uint32_t k = scan_bits(smask, v);
+    const uint4 x = row_vec<kShared>(base, gbase, v);
+    m0 = fmaxf(m0, k ? absmax8(x, k) : absmax8_all(x));
+  }
+  return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+}
+
+// int8 codes of groups start, start+step, ... of one row.
+template <bool kShared>
+__device__ __forceinline__ void row_codes(uint32_t base, const uint4* gbase, uint2* q, int gpr,
+                                          int start, int step, const uint32_t* smask, float s) {
+  int v = start;
+  for (; v + 3 * step < gpr; v += 4 * step) {
+    const uint4 x0 = row_vec<kShared>(base, gbase, v);
+    const uint4 x1 = row_vec<kShared>(base, gbase, v + step);
+    const uint4 x2 = row_vec<kShared>(base, gbase, v + 2 * step);
+    const uint4 x3 = row_vec<kShared>(base, gbase, v + 3 * step);
+    q[v] = codes8(x0, scan_bits(smask, v), s);
+    q[v + step] = codes8(x1, scan_bits(smask, v + step), s);
+    q[v + 2 * step] = codes8(x2, scan_bits(smask, v + 2 * step), s);
+    q[v + 3 * step] = codes8(x3, scan_bits(smask, v + 3 * step), s);
+  }
+  for (; v < gpr; v += step) q[v] = codes8(row_vec<kShared>(base, gbase, v), scan_bits(smask, v), s);
+}
+
+__global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs p) {
+  extern __shared__ __align__(128) uint8_t psm[];
+  const int64_t K = p.K;
+  const int64_t words = (K + 31) / 32;
+  const int64_t gpr = K / 8;  // 16-byte groups per row
+  // shared memory: [row cache][mask words][prefix words + 1][idx K][row scales]
+  const size_t cache_bytes = static_cast<size_t>(p.cache_rows) * static_cast<size_t>(K) * 2;
+  uint4* cache = reinterpret_cast<uint4*>(psm);
+  uint32_t* smask = reinterpret_cast<uint32_t*>(psm + cache_bytes);
+  int32_t* spre = reinterpret_cast<int32_t*>(smask + words);
+  int32_t* sidx = spre + words + 1;
+  float* samax = reinterpret_cast<float*>(sidx + K);   // [rows_per_cta]
+  __shared__ __align__(8) uint64_t s_bar[kPrepMaxChunks];
+  __shared__ int s_fail;
+  __shared__ int s_wsum[kPrepWarps];
+  __shared__ float s_red[kPrepWarps];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * p.rows_per_cta;
+  const int64_t r1 = min(p.T, r0 + p.rows_per_cta);
+  const int64_t nrows = r1 > r0 ? r1 - r0 : 0;
+  const int64_t ncached = min(nrows, p.cache_rows);
+  const int64_t cbytes = ncached * K * 2;
+  const int nchunks = static_cast<int>((cbytes + kPrepChunk - 1) / kPrepChunk);
+
+  // ------------------------------------------------ phase 1: scan (and cache) the rows
+  if (tid == 0) {
+    s_fail = 0;
+    for (int c = 0; c < nchunks; ++c) mbar_init(smem_u32(&s_bar[c]), 1);
+    fence_mbar_init();
+  }
+  for (int64_t w = tid; w < words; w += kPrepThreads) smask[w] = 0u;
+  __syncthreads();
+  if (tid == 0) {
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(p.X + r0 * K);
+    for (int c = 0; c < nchunks; ++c) {
+      const int64_t off = static_cast<int64_t>(c) * kPrepChunk;
+      const uint32_t bytes = static_cast<uint32_t>(min(static_cast<int64_t>(kPrepChunk), cbytes - off));
+      mbar_arrive_expect_tx(smem_u32(&s_bar[c]), bytes);
+      bulk_load(smem_u32(psm + off), src + off, bytes, smem_u32(&s_bar[c]));
+    }
+  }
+  // rows beyond the cache: scanned straight from global memory while the copies land
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(p.X + (r0 + ncached) * K);
+    const int64_t nvec = (nrows - ncached) * gpr;
+    int64_t v = tid;
+    for (; v + 3 * kPrepThreads < nvec; v += 4 * kPrepThreads) {
+      uint4 x[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) x[u] = ldg_v4(src + v + u * kPrepThreads);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t f = outlier_bits8(x[u], p.thr);
+        if (f) {
+          const int64_t g = (v + u * kPrepThreads) % gpr;
+          atomicOr(smask + (g >> 2), f << (8 * (g & 3)));
+        }
+      }
+    }
+    for (; v < nvec; v += kPrepThreads) {
+      const uint32_t f = outlier_bits8(ldg_v4(src + v), p.thr);
+      if (f) {
+        const int64_t g = v % gpr;
+        atomicOr(smask + (g >> 2), f << (8 * (g & 3)));
+      }
+    }
+  }
+  // cached rows: scan each chunk as it lands
+  {
+    int no_abort = 0;
+    for (int c = 0; c < nchunks; ++c) {
+      const bool got = mbar_wait(smem_u32(&s_bar[c]), 0u, &no_abort, p.wait_limit_ns);
+      if (!got) s_fail = 1;
+      const int64_t v0 = static_cast<int64_t>(c) * (kPrepChunk / 16);
+      const int64_t v1 = min(v0 + static_cast<int64_t>(kPrepChunk / 16), cbytes / 16);
+      for (int64_t v = v0 + tid; v < v1; v += kPrepThreads) {
+        const uint32_t f = got ? outlier_bits8(cache[v], p.thr) : 0u;
+        if (f) {
+          const int64_t g = v % gpr;
+          atomicOr(smask + (g >> 2), f << (8 * (g & 3)));
+        }
+      }
+    }
+  }
+  __syncthreads();
+  for (int64_t w = tid; w < words; w += kPrepThreads)
+    if (smask[w]) atomicOr(p.mask + w, smask[w]);
+
+  // ------------------------------------------------ grid barrier (bounded)
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t* counter = p.mask + words;
+    __threadfence();
+    atomicAdd(counter, 1u);
+    const uint32_t target = gridDim.x;
+    if (ld_acquire_gpu(counter) < target) {
+      const uint64_t t0 = globaltimer_ns();
+      for (uint32_t it = 1;; ++it) {
+        if (ld_acquire_gpu(counter) >= target) break;
+        if ((it & 63u) == 0u && globaltimer_ns() - t0 > p.wait_limit_ns) {
+          raise_error(kErrWaitTimeout);
+          s_fail = 1;
+          break;
+        }
+      }
+    }
+    __threadfence();
+  }
+  __syncthreads();
+  if (s_fail) {
+    if (tid == 0) {
+      raise_error(kErrWaitTimeout);
+      int no_abort = 0;  // let the copies in flight land before the CTA exits (bounded)
+      for (int c = 0; c < nchunks; ++c)
+        mbar_wait(smem_u32(&s_bar[c]), 0u, &no_abort, p.wait_limit_ns);
+    }
+    __syncthreads();
+    return;
+  }
+
+  // ------------------------------------------------ phase 2: final mask, index list
+  // exclusive prefix of the per-word popcounts, blocks of kPrepThreads words at a time
+  int carry = 0;
+  for (int64_t base = 0; base < words; base += kPrepThreads) {
+    const int64_t w = base + tid;
+    uint32_t m = 0u;
+    if (w < words) {
+      m = __ldcg(p.mask + w);
+      smask[w] = m;
+    }
+    const int c = __popc(m);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w2 = 0; w2 < kPrepWarps; ++w2) {
+      const int x = s_wsum[w2];
+      before += (w2 < warp) ? x : 0;
+      total += x;
+    }
+    if (w < words) spre[w] = carry + before + incl - c;
+    carry += total;
+    __syncthreads();
+  }
+  if (tid == 0) spre[words] = carry;
+  const int n_o = carry;
+  for (int64_t w = tid; w < words; w += kPrepThreads) {
+    uint32_t m = smask[w];
+    int pos = spre[w];
+    while (m) {
+      const int b = __ffs(m) - 1;
+      sidx[pos++] = static_cast<int32_t>(w * 32 + b);
+      m &= m - 1u;
+    }
+  }
+  for (int64_t i = tid; i < nrows; i += kPrepThreads) samax[i] = 0.0f;
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    for (int j = tid; j < n_o; j += kPrepThreads) p.idx_out[j] = sidx[j];
+    if (tid == 0) *p.n_o_out = n_o;
+  }
+
+  // ------------------------------------------------ phase 3: quantise
+  // Rows go in rounds of (16 / wpr) rows with wpr warps per row (wpr = 1 when the CTA owns
+  // 16 rows or more; up to 16 when it owns one, as in decode batches).  Every warp walks
+  // the same rounds, so the block barriers of the cross-warp reduction are uniform.
+  {
+    const int padded = (n_o + 63) & ~63;
+    int wpr = 1;
+    while (wpr < kPrepWarps && wpr * 2 * nrows <= kPrepWarps) wpr *= 2;
+    const int rows_per_round = kPrepWarps / wpr;
+    const int sub = warp % wpr;
+    const int rr = warp / wpr;
+    const int start = sub * 32 + lane, step = 32 * wpr;
+    const int g32 = static_cast<int>(gpr);
+    const uint32_t cache_s = smem_u32(cache);
+    const int64_t rounds = (nrows + rows_per_round - 1) / rows_per_round;
+    for (int64_t round = 0; round < rounds; ++round) {
+      const int64_t i = round * rows_per_round + rr;
+      const bool have = i < nrows;
+      const bool cached = have && i < ncached;
+      const int64_t t = r0 + i;
+      const uint32_t sbase = cache_s + static_cast<uint32_t>(i * gpr * 16);
+      const uint4* gbase = reinterpret_cast<const uint4*>(p.X + t * K);
+      float amax = 0.0f;
+      if (cached)
+        amax = row_absmax<true>(sbase, gbase, g32, start, step, smask);
+      else if (have)
+        amax = row_absmax<false>(sbase, gbase, g32, start, step, smask);
+      amax = warp_max(amax);
+      if (wpr > 1) {
+        __syncthreads();
+        if (lane == 0) s_red[warp] = amax;
+        __syncthreads();
+        for (int w2 = 0; w2 < wpr; ++w2) amax = fmaxf(amax, s_red[rr * wpr + w2]);
+      }
+      if (!have) continue;
+      const float sc = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+      uint2* qrow = reinterpret_cast<uint2*>(p.Xq + t * K);
+      if (cached)
+        row_codes<true>(sbase, gbase, qrow, g32, start, step, smask, sc);
+      else
+        row_codes<false>(sbase, gbase, qrow, g32, start, step, smask, sc);
+      if (sub == 0 && lane == 0) p.SCx[t] = amax;
+      for (int j = start; j < padded; j += step) {
+        __half v = __float2half_rn(0.0f);
+        if (j < n_o) {
+          const int64_t k = sidx[j];
+          v = cached ? reinterpret_cast<const __half*>(cache + i * gpr)[k] : p.X[t * K + k];
+        }
+        p.X_o[(static_cast<int64_t>(j >> 6) * p.T + t) * 64 + (j & 63)] = v;
+      }
+    }
+  }
+  __syncthreads();   // the row cache is free from here on (phase 4 may reuse it)
+
+  // ------------------------------------------------ phase 4: fp16 outlier slice of CB
+  if (p.CB_o != nullptr && n_o > 0) {
+    const int64_t chunks = (n_o + 63) >> 6;
+    const int64_t nbuf = min(static_cast<int64_t>(kPrepWarps), p.cache_bytes_all / K);
+    if (static_cast<int64_t>(n_o) * 32 >= K && nbuf > 0) {
+      // Many outlier columns: stream whole CB rows (coalesced) into a per-warp buffer in
+      // the freed row cache and pick the outlier columns there.
+      if (warp < nbuf) {
+        uint8_t* rowbuf = psm + static_cast<size_t>(warp) * static_cast<size_t>(K);
+        const int64_t nw = static_cast<int64_t>(gridDim.x) * nbuf;
+        for (int64_t n = static_cast<int64_t>(blockIdx.x) * nbuf + warp; n < p.N; n += nw) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.CB + n * K);
+          int v = lane;
+          for (; v + 96 < g32_of(K); v += 128) {
+            uint4 x0 = ldg_stream_v4(src + v), x1 = ldg_stream_v4(src + v + 32);
+            uint4 x2 = ldg_stream_v4(src + v + 64), x3 = ldg_stream_v4(src + v + 96);
+            reinterpret_cast<uint4*>(rowbuf)[v] = x0;
+            reinterpret_cast<uint4*>(rowbuf)[v + 32] = x1;
+            reinterpret_cast<uint4*>(rowbuf)[v + 64] = x2;
+            reinterpret_cast<uint4*>(rowbuf)[v + 96] = x3;
+          }
+          for (; v < g32_of(K); v += 32) reinterpret_cast<uint4*>(rowbuf)[v] = ldg_stream_v4(src + v);
+          __syncwarp();
+          for (int64_t c = 0; c < chunks; ++c) {
+            const int64_t j0 = c * 64 + 2 * lane;
+            float v0 = 0.0f, v1 = 0.0f;
+            if (j0 < n_o) v0 = static_cast<float>(static_cast<int8_t>(rowbuf[sidx[j0]]));
+            if (j0 + 1 < n_o) v1 = static_cast<float>(static_cast<int8_t>(rowbuf[sidx[j0 + 1]]));
+            reinterpret_cast<__half2*>(p.CB_o + (c * p.N + n) * 64)[lane] =
+                __floats2half2_rn(v0, v1);
+          }
+          __syncwarp();
+        }
+      }
+    } else {
+      // Few outlier columns: one warp per (chunk, row) item, 8 items in flight per warp
+      // (the loads are scattered bytes of CB, so latency sets the pace).
+      constexpr int U = 8;
+      const int64_t items = chunks * p.N;
+      const int64_t nw = static_cast<int64_t>(gridDim.x) * kPrepWarps;
+      for (int64_t it0 = (static_cast<int64_t>(blockIdx.x) * kPrepWarps + warp) * U; it0 < items;
+           it0 += nw * U) {
+        float v0[U], v1[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int64_t it = it0 + u;
+          v0[u] = 0.0f;
+          v1[u] = 0.0f;
+          if (it < items) {
+            const int64_t c = it / p.N, n = it - c * p.N;
+            const int64_t j0 = c * 64 + 2 * lane;
+            if (j0 < n_o) v0[u] = static_cast<float>(p.CB[n * K + sidx[j0]]);
+            if (j0 + 1 < n_o) v1[u] = static_cast<float>(p.CB[n * K + sidx[j0 + 1]]);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int64_t it = it0 + u;
+          if (it < items) {
+            const int64_t c = it / p.N, n = it - c * p.N;
+            reinterpret_cast<__half2*>(p.CB_o + (c * p.N + n) * 64)[lane] =
+                __floats2half2_rn(v0[u], v1[u]);
+          }
+        }
+      }
+    }
+  }
+}
+
+// Dynamic shared memory of prepare_kernel: a row cache of `cache_rows` rows, the mask,
+// its prefix, the index list and one scale per row of the CTA's block.
+__host__ inline size_t prepare_smem_bytes(int64_t K, int64_t cache_rows, int64_t rows_per_cta) {
+  const int64_t words = (K + 31) / 32;
+  return static_cast<size_t>(cache_rows) * static_cast<size_t>(K) * 2 +
+         static_cast<size_t>(2 * words + 1 + K + rows_per_cta) * 4;
 }
 
 }  // namespace i8

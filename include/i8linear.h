@@ -110,6 +110,23 @@ i8_status i8_quantize_act(const void* X, int64_t T, int64_t K, const uint32_t* c
                           const int32_t* outlier_idx, const int32_t* n_outliers, int8_t* Xq,
                           float* SCx, void* X_o, void* stream);
 
+/*
+ * Steps 1 and 2 fused: the outlier column scan, the row-wise absmax quantisation and the
+ * fp16 outlier slice in ONE launch that reads X from HBM once (each CTA keeps its rows in
+ * shared memory across a bounded grid-wide barrier; rows that do not fit are re-read).
+ * Sources: as i8_outlier_scan and i8_quantize_act.  Results are identical to
+ * i8_outlier_scan followed by i8_quantize_act.
+ *   X           [T, K] fp16 (read)            threshold: as in i8_outlier_scan
+ *   col_mask    [ceil(K/32) + 1] uint32 (written): the packed mask, then one word of
+ *               scratch (the grid barrier); cleared by the call first
+ *   outlier_idx [K] int32, n_outliers [1] int32, Xq [T, K] int8, SCx [T] fp32,
+ *   X_o         i8_outlier_slice_elems(T, K) fp16: all written, as in the two calls above
+ * Uses a cooperative launch of one CTA per SM.
+ */
+i8_status i8_prepare_act(const void* X, int64_t T, int64_t K, float threshold,
+                         uint32_t* col_mask, int32_t* outlier_idx, int32_t* n_outliers,
+                         int8_t* Xq, float* SCx, void* X_o, void* stream);
+
 /* Device workspace bytes that i8_linear_forward and i8_igemm_s32 need for these sizes
  * (worst case over the outlier count, which is only known on the device).  0 when a size
  * is invalid. */

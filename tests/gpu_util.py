@@ -61,6 +61,21 @@ def gpu_quantize_act(X_d, mask, idx, n_o):
     return Xq, SCx, X_o
 
 
+def gpu_prepare(X_d, thr):
+    """The fused one-pass scan + quantisation (i8_prepare_act)."""
+    T, K = X_d.shape
+    words = (K + 31) // 32
+    mask = torch.empty((words + 1,), dtype=torch.int32, device=DEV)
+    idx = torch.empty((K,), dtype=torch.int32, device=DEV)
+    n_o = torch.empty((4,), dtype=torch.int32, device=DEV)
+    Xq = torch.empty((T, K), dtype=torch.int8, device=DEV)
+    SCx = torch.empty((T,), dtype=torch.float32, device=DEV)
+    X_o = torch.full((abi.i8_outlier_slice_elems(T, K),), float("nan"), dtype=torch.float16,
+                     device=DEV)
+    abi.i8_prepare_act(X_d, thr, mask, idx, n_o, Xq, SCx, X_o)
+    return mask[:words], idx, n_o, Xq, SCx, X_o
+
+
 def gpu_forward(X_d, CB, SCB, bias_d, thr):
     T, K = X_d.shape
     N = CB.shape[0]

@@ -14,8 +14,9 @@ import torch
 
 from bit_matmul_decomposition_b200 import abi, synth
 from oracle import oracle as O
-from tests.gpu_util import (check_output, dev, gpu_forward, gpu_igemm, gpu_quantize_act,
-                            gpu_quantize_weight, gpu_scan, host, slice_to_matrix, sync_ok)
+from tests.gpu_util import (check_output, dev, gpu_forward, gpu_igemm, gpu_prepare,
+                            gpu_quantize_act, gpu_quantize_weight, gpu_scan, host,
+                            slice_to_matrix, sync_ok)
 
 pytestmark = pytest.mark.gpu
 
@@ -59,15 +60,21 @@ SCAN_CASES = [
     (33, 96, (1,), 0.0, -1.0),
     (33, 96, (1, 2), 0.0, math.inf),
     (4100, 1040, (7, 1039), 1e-4, 6.0),
+    (3000, 16384, (0, 9000, 16383), 0.0, 6.0),    # rows beyond the per-CTA cache
+    (16, 14336, (100, 14000), 0.0, 6.0),
 ]
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["two_pass", "fused"])
 @pytest.mark.parametrize("T,K,cols,frac,thr", SCAN_CASES)
-def test_scan_and_quantize_act_bitexact(T, K, cols, frac, thr):
+def test_scan_and_quantize_act_bitexact(T, K, cols, frac, thr, fused):
     w, X, _, _ = _case(T, K, 8, seed=T + K, cols=cols, random_frac=frac)
     X_d = dev(X)
-    mask, idx, n_o = gpu_scan(X_d, thr)
-    Xq, SCx, X_o = gpu_quantize_act(X_d, mask, idx, n_o)
+    if fused:
+        mask, idx, n_o, Xq, SCx, X_o = gpu_prepare(X_d, thr)
+    else:
+        mask, idx, n_o = gpu_scan(X_d, thr)
+        Xq, SCx, X_o = gpu_quantize_act(X_d, mask, idx, n_o)
     sync_ok()
     flags, words, idx_r = O.outlier_scan(X, thr)
     n = int(host(n_o)[0])
