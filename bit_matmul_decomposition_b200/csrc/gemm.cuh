@@ -40,7 +40,7 @@ constexpr int STAGES = 6;
 constexpr int A_BYTES = HM * BK;
 constexpr int B_BYTES = HN * BK;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // per CTA
-constexpr int THREADS = 192;
+constexpr int THREADS = 224;     // warps 0,6 TMA (A, B); 1 MMA; 2..5 epilogue
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC_I8 = idesc_s8_s32(TM, TN);
 constexpr uint32_t IDESC_F16 = idesc_f16_f32(TM, TN);
@@ -53,6 +53,7 @@ constexpr size_t SMEM_BYTES =
 constexpr uint16_t PAIR_MASK = 0x3;
 
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+static_assert(THREADS == 224, "warp roles assume 7 warps");
 
 struct Args {
   int T, N, K;
@@ -322,39 +323,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     return n0;
   };
 
-  if (warp == 0) {
+  if (warp == 0 || warp == 6) {
     if (lane == 0) {
-      // ------------------------------------------------------------ TMA producer
-      // Tile coordinates are computed once per tile (the ring only ever refers to the
-      // current tile and the one before it), so a stage costs a handful of instructions.
+      // ------------------------------------------------------------ TMA producers
+      // Warp 0 loads the A (Xq / X_o) half of every stage and arms the leader's barrier
+      // for both halves; warp 6 loads the B (CB / CB_o) half.  Splitting the issue over
+      // two warps halves the per-stage latency chain of each issuing thread.
+      const bool loads_a = (warp == 0);
       int s = 0;
       uint32_t ph = 0;
       uint32_t issued = 0;
       int coord_it[2] = {-1, -1};
-      int coord_a[2] = {0, 0}, coord_b[2] = {0, 0};
+      int coord[2] = {0, 0};
       const uint32_t full_leader0 = map_to_rank(smem_u32(&bars->full[0]), 0);
+      const CUtensorMap* map_i = loads_a ? &tmA : &tmB;
+      const CUtensorMap* map_o = loads_a ? &tmAo : &tmBo;
+      const uint32_t half_off = loads_a ? 0u : static_cast<uint32_t>(A_BYTES);
       const bool ok = walk_schedule(L, KB, OC, [&](int kind, int it, int idx) -> bool {
         if (kind >= 2) return true;
         const int slot = it & 1;
         if (coord_it[slot] != it) {
           int m0, n0;
           tile_mn(it, m0, n0);
-          coord_a[slot] = m0 + static_cast<int>(rank) * HM;
-          coord_b[slot] = n0 + static_cast<int>(rank) * HN;
+          coord[slot] = (loads_a ? m0 : n0) + static_cast<int>(rank) * (loads_a ? HM : HN);
           coord_it[slot] = it;
         }
         if (!mbar_wait(smem_u32(&bars->empty[s]), ph ^ 1u, abort_flag, lim)) return false;
-        const uint32_t sa = ring + s * STAGE_BYTES;
-        const uint32_t sb = sa + A_BYTES;
-        if (rank == 0) mbar_arrive_expect_tx(smem_u32(&bars->full[s]), 2 * STAGE_BYTES);
+        const uint32_t dst = ring + s * STAGE_BYTES + half_off;
+        if (loads_a && rank == 0) mbar_arrive_expect_tx(smem_u32(&bars->full[s]), 2 * STAGE_BYTES);
         const uint32_t fb = full_leader0 + static_cast<uint32_t>(s) * 8u;
-        if (kind == 0) {
-          tma_load_2d_pair(sa, &tmA, fb, idx * BK, coord_a[slot]);
-          tma_load_2d_pair(sb, &tmB, fb, idx * BK, coord_b[slot]);
-        } else {
-          tma_load_3d_pair(sa, &tmAo, fb, 0, coord_a[slot], idx);
-          tma_load_3d_pair(sb, &tmBo, fb, 0, coord_b[slot], idx);
-        }
+        if (kind == 0)
+          tma_load_2d_pair(dst, map_i, fb, idx * BK, coord[slot]);
+        else
+          tma_load_3d_pair(dst, map_o, fb, 0, coord[slot], idx);
         ++issued;
         if (++s == STAGES) {
           s = 0;
@@ -362,7 +363,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         return true;
       });
-      if (!ok && rank == 0) {
+      if (!ok && loads_a && rank == 0) {
         // wind down: wait (bounded, ignoring the abort flag) for the copies in flight
         int no_abort = 0;
         const uint32_t inflight = issued < STAGES ? issued : STAGES;
@@ -425,7 +426,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       umma_commit_pair(smem_u32(&bars->drain));
       mbar_wait(smem_u32(&bars->drain), 0u, &no_abort, lim);
     }
-  } else {
+  } else if (warp >= 2 && warp <= 5) {
     // -------------------------------------------------------------- epilogue warps
     const int q = warp & 3;
     const int row = q * 32 + lane;
