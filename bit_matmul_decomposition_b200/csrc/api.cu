@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <utility>
 
 #include "../../include/i8linear.h"
 #include "common.cuh"
@@ -86,6 +87,25 @@ i8_status device_info(DeviceInfo** out) {
   }
   *out = &d;
   return I8_OK;
+}
+
+// ------------------------------------------------------------------ launches
+// Launch with programmatic stream serialization: the kernel may begin while the previous
+// kernel on the stream drains, and waits (griddepcontrol.wait) before reading its output.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_overlapped(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // ------------------------------------------------------------------ checks
@@ -299,13 +319,14 @@ i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t
   a.wait_limit_ns = kWaitLimitNs;
   const int64_t tiles = static_cast<int64_t>(a.m_tiles) * a.n_tiles;
   const int clusters = static_cast<int>(tiles < d.gemm_clusters ? tiles : d.gemm_clusters);
+  cudaError_t e;
   if (raw)
-    gemm::i8_gemm_tcgen05_kernel<true><<<2 * clusters, gemm::THREADS, gemm::SMEM_BYTES, s>>>(
-        tA, tB, tAo, tBo, a);
+    e = launch_overlapped(gemm::i8_gemm_tcgen05_kernel<true>, dim3(2 * clusters),
+                          dim3(gemm::THREADS), gemm::SMEM_BYTES, s, tA, tB, tAo, tBo, a);
   else
-    gemm::i8_gemm_tcgen05_kernel<false><<<2 * clusters, gemm::THREADS, gemm::SMEM_BYTES, s>>>(
-        tA, tB, tAo, tBo, a);
-  return launch_status();
+    e = launch_overlapped(gemm::i8_gemm_tcgen05_kernel<false>, dim3(2 * clusters),
+                          dim3(gemm::THREADS), gemm::SMEM_BYTES, s, tA, tB, tAo, tBo, a);
+  return e == cudaSuccess ? launch_status() : I8_ERR_CUDA;
 }
 
 // decode GEMV partials; the caller then runs the finalize kernel
@@ -337,13 +358,14 @@ i8_status run_gemv_partial(const int8_t* A, int64_t T, int64_t K, const int8_t* 
   grid = (grid / S) * S;
   if (grid < S) grid = S;
   if (grid > tiles * S) grid = tiles * S;
+  const int Ti = static_cast<int>(T);
   if (nt == 1)
-    gemv::gemv_partial_kernel<1><<<static_cast<unsigned>(grid), gemv::THREADS, smem, s>>>(
-        A, B, static_cast<int>(T), N, K, P);
+    e = launch_overlapped(gemv::gemv_partial_kernel<1>, dim3(static_cast<unsigned>(grid)),
+                          dim3(gemv::THREADS), smem, s, A, B, Ti, N, K, P);
   else
-    gemv::gemv_partial_kernel<2><<<static_cast<unsigned>(grid), gemv::THREADS, smem, s>>>(
-        A, B, static_cast<int>(T), N, K, P);
-  return launch_status();
+    e = launch_overlapped(gemv::gemv_partial_kernel<2>, dim3(static_cast<unsigned>(grid)),
+                          dim3(gemv::THREADS), smem, s, A, B, Ti, N, K, P);
+  return e == cudaSuccess ? launch_status() : I8_ERR_CUDA;
 }
 
 __global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
@@ -510,11 +532,14 @@ i8_status i8_linear_forward(const void* X, int64_t T, int64_t K, const int8_t* C
   if (st != I8_OK) return st;
   if (prof && cudaEventRecord(g_prof_stop, s) != cudaSuccess) return I8_ERR_CUDA;
   const int S = static_cast<int>(gemv::num_slices(K));
-  gemv::gemv_finalize_kernel<false>
-      <<<dim3(static_cast<unsigned>((N + 255) / 256), static_cast<unsigned>(T)), 256, 0, s>>>(
-      P, S, static_cast<int>(T), N, K, SCx, SCB, static_cast<const __half*>(bias), CB, idx, n_o,
-      static_cast<const __half*>(X_o), static_cast<__half*>(C), nullptr);
-  return launch_status();
+  const cudaError_t e = launch_overlapped(
+      gemv::gemv_finalize_kernel<false>,
+      dim3(static_cast<unsigned>((N + 255) / 256), static_cast<unsigned>(T)), dim3(256), 0, s,
+      static_cast<const int32_t*>(P), S, static_cast<int>(T), N, K, static_cast<const float*>(SCx),
+      SCB, static_cast<const __half*>(bias), CB, static_cast<const int32_t*>(idx),
+      static_cast<const int32_t*>(n_o), static_cast<const __half*>(X_o), static_cast<__half*>(C),
+      static_cast<int32_t*>(nullptr));
+  return e == cudaSuccess ? launch_status() : I8_ERR_CUDA;
 }
 
 i8_status i8_igemm_s32(const int8_t* A, int64_t T, int64_t K, const int8_t* B, int64_t N,
@@ -536,11 +561,15 @@ i8_status i8_igemm_s32(const int8_t* A, int64_t T, int64_t K, const int8_t* B, i
   st = run_gemv_partial(A, T, K, B, N, P, *d, s);
   if (st != I8_OK) return st;
   const int S = static_cast<int>(gemv::num_slices(K));
-  gemv::gemv_finalize_kernel<true>
-      <<<dim3(static_cast<unsigned>((N + 255) / 256), static_cast<unsigned>(T)), 256, 0, s>>>(
-      P, S, static_cast<int>(T), N, K, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
-      nullptr, nullptr, acc);
-  return launch_status();
+  const cudaError_t e = launch_overlapped(
+      gemv::gemv_finalize_kernel<true>,
+      dim3(static_cast<unsigned>((N + 255) / 256), static_cast<unsigned>(T)), dim3(256), 0, s,
+      static_cast<const int32_t*>(P), S, static_cast<int>(T), N, K,
+      static_cast<const float*>(nullptr), static_cast<const float*>(nullptr),
+      static_cast<const __half*>(nullptr), static_cast<const int8_t*>(nullptr),
+      static_cast<const int32_t*>(nullptr), static_cast<const int32_t*>(nullptr),
+      static_cast<const __half*>(nullptr), static_cast<__half*>(nullptr), acc);
+  return e == cudaSuccess ? launch_status() : I8_ERR_CUDA;
 }
 
 i8_status i8_sync_status(void* stream) {

@@ -218,6 +218,20 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// ------------------------------------------------------------------ launch overlap
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while its predecessor drains; it must call grid_dep_wait()
+// before touching anything the predecessor writes (the wait returns once the
+// predecessor has completed and its writes are visible; it is a no-op without the
+// launch attribute).  grid_dep_launch() lets the successor start launching early.
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ small helpers
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll

@@ -290,6 +290,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = bars->tmem_base;
+  // everything above overlaps the previous kernel; its outputs are read from here on
+  grid_dep_wait();
 
   const int n_o = (a.n_outliers != nullptr) ? max(0, __ldg(a.n_outliers)) : 0;
   const int OC = (n_o + 63) >> 6;

@@ -71,6 +71,8 @@ __global__ void __launch_bounds__(THREADS)
   const int cta_in_slice = blockIdx.x / S;
   const int ctas_in_slice = (static_cast<int>(gridDim.x) - slice + S - 1) / S;
   const int64_t k0 = static_cast<int64_t>(slice) * KS;
+  grid_dep_wait();    // Xq comes from the previous kernel
+  grid_dep_launch();  // the finalize kernel may start launching
 
   // stage Xq[:, k0 : k0+KS] (tokens >= T and columns >= K are zero)
   const int64_t vec_per_row = KS / 16;
@@ -160,6 +162,7 @@ __global__ void __launch_bounds__(256)
                          int32_t* __restrict__ acc_out) {
   const int64_t n = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int t = blockIdx.y;
+  grid_dep_wait();    // the partial sums come from the previous kernel
   if (n >= N) return;
   int32_t acc = 0;
   for (int s = 0; s < S; ++s) acc += __ldcs(P + (static_cast<int64_t>(s) * T + t) * N + n);

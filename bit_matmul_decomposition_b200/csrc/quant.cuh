@@ -436,6 +436,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
   __syncthreads();
   for (int64_t w = tid; w < words; w += kPrepThreads)
     if (smask[w]) atomicOr(p.mask + w, smask[w]);
+  grid_dep_launch();  // the GEMM / GEMV may start launching (it waits for our writes)
 
   // ------------------------------------------------ grid barrier (bounded)
   __syncthreads();

@@ -1,0 +1,95 @@
+"""Host logic of bench.py on the CPU: the max-over-ranks reduction across two gloo ranks,
+the per-rank output-channel sharding (weak scaling), and the JSON contract of the
+reference arm (the CPU oracle timed on this host)."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+from bit_matmul_decomposition_b200 import synth  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        got = bench.max_over_ranks([rank + 1.0, 10.0 - rank, 0.5 * rank])
+        out[rank] = got
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_two_gloo_ranks():
+    world = 2
+    port = _free_port()
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
+    for r in range(world):
+        assert out[r] == [2.0, 10.0, 0.5]
+
+
+def test_max_over_ranks_without_process_group_is_identity():
+    assert bench.max_over_ranks([1.5, 2.5]) == [1.5, 2.5]
+
+
+def test_each_rank_owns_its_own_output_channels():
+    w = synth.Workload("t", 8, 64, 32, seed=7)
+    w0, r0 = bench.rank_workload(w, 0)
+    _, r1 = bench.rank_workload(w, 1)
+    # the hidden states are replicated (same seed for X on every rank) ...
+    assert np.array_equal(synth.make_x(w0), synth.make_x(w))
+    # ... while every rank draws a different weight block
+    assert r0.seed == w.seed and r1.seed != w.seed
+    assert not np.array_equal(synth.make_w(r0), synth.make_w(r1))
+
+
+REQUIRED = ["metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+            "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config"]
+
+
+def _run_ref(extra_env=None, *args):
+    env = dict(os.environ, **(extra_env or {}))
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                           "--workload", "tiny", "--steps", "2", "--warmup", "3", *args],
+                          capture_output=True, text=True, env=env, timeout=600)
+
+
+def test_reference_arm_prints_one_contract_line():
+    r = _run_ref()
+    assert r.returncode == 0, r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in REQUIRED:
+        assert k in d, k
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "TOPS"
+    assert d["higher_is_better"] is True and d["scaling"] == "weak"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "TOPS", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    assert d["config"]["workload"].startswith("tiny")
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    r = _run_ref({"RANK": "1", "WORLD_SIZE": "2"})
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == ""
