@@ -191,6 +191,21 @@ bool map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t i
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D row-major uint8 tensor without swizzle (box inner extent up to 256 bytes).
+bool map_2d_plain(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                  uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Chunk-major outlier slice [chunks][rows][64] fp16; box [1][box_rows][64].
 bool map_slice(CUtensorMap* m, const void* base, uint64_t rows, uint64_t chunks,
                uint32_t box_rows) {
@@ -329,42 +344,31 @@ i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t
   return e == cudaSuccess ? launch_status() : I8_ERR_CUDA;
 }
 
-// decode GEMV partials; the caller then runs the finalize kernel
+// decode GEMV partials (TMA-streamed CB); the caller then runs the finalize kernel
 i8_status run_gemv_partial(const int8_t* A, int64_t T, int64_t K, const int8_t* B, int64_t N,
                            int32_t* P, const DeviceInfo& d, cudaStream_t s) {
   const int nt = T <= 8 ? 1 : 2;
-  const size_t smem = gemv::smem_bytes(nt, K);
-  if (smem > 200 * 1024) return I8_ERR_INVALID_ARG;
+  const size_t smem = gemv::stream_smem_bytes(nt, K);
+  if (smem > static_cast<size_t>(d.prep_smem_max)) return I8_ERR_INVALID_ARG;
+  CUtensorMap tCB;
+  if (!map_2d_plain(&tCB, B, K, N, K, gemv::BOXW, gemv::ROWS)) return I8_ERR_CUDA;
   const int S = static_cast<int>(gemv::num_slices(K));
-  int per_sm = 0;
-  cudaError_t e;
-  if (nt == 1) {
-    e = cudaFuncSetAttribute(gemv::gemv_partial_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv::gemv_partial_kernel<1>,
-                                                        gemv::THREADS, smem);
-  } else {
-    e = cudaFuncSetAttribute(gemv::gemv_partial_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv::gemv_partial_kernel<2>,
-                                                        gemv::THREADS, smem);
-  }
+  cudaError_t e = nt == 1 ? cudaFuncSetAttribute(gemv::gemv_stream_kernel<1>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(smem))
+                          : cudaFuncSetAttribute(gemv::gemv_stream_kernel<2>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(smem));
   if (e != cudaSuccess) return I8_ERR_CUDA;
-  if (per_sm < 1) per_sm = 1;
-  const int64_t tiles = (N + gemv::ROWS - 1) / gemv::ROWS;
-  int64_t grid = static_cast<int64_t>(d.sms) * per_sm;
-  grid = (grid / S) * S;
+  int grid = (d.sms / S) * S;  // one CTA per SM, the same number of CTAs on every slice
   if (grid < S) grid = S;
-  if (grid > tiles * S) grid = tiles * S;
   const int Ti = static_cast<int>(T);
   if (nt == 1)
-    e = launch_overlapped(gemv::gemv_partial_kernel<1>, dim3(static_cast<unsigned>(grid)),
-                          dim3(gemv::THREADS), smem, s, A, B, Ti, N, K, P);
+    e = launch_overlapped(gemv::gemv_stream_kernel<1>, dim3(static_cast<unsigned>(grid)),
+                          dim3(gemv::STREAM_THREADS), smem, s, tCB, A, Ti, N, K, P, kWaitLimitNs);
   else
-    e = launch_overlapped(gemv::gemv_partial_kernel<2>, dim3(static_cast<unsigned>(grid)),
-                          dim3(gemv::THREADS), smem, s, A, B, Ti, N, K, P);
+    e = launch_overlapped(gemv::gemv_stream_kernel<2>, dim3(static_cast<unsigned>(grid)),
+                          dim3(gemv::STREAM_THREADS), smem, s, tCB, A, Ti, N, K, P, kWaitLimitNs);
   return e == cudaSuccess ? launch_status() : I8_ERR_CUDA;
 }
 

@@ -59,94 +59,178 @@ __device__ __forceinline__ void mma_s8_16816(int (&c)[4], uint32_t a0, uint32_t 
 }
 
 // P[slice][t][n] = sum over k in the slice of Xq[t,k] * CB[n,k]   (t < T only)
+//
+// Warp CW (one thread) streams CB through a ring of STAGES stages, each 16 rows x CH
+// bytes of K, loaded as 2-D TMA boxes of 256 B x 16 rows (no swizzle: the widest box TMA
+// takes, which streams HBM best -- ~6 TB/s measured on B200 for this layout).  The CW
+// compute warps each own one 64-byte MMA step of every stage, accumulate their
+// 16 x (8*NT) int32 partials in registers over the tile's stages, and only at the tile's
+// end reduce across warps (a named barrier among the compute warps); the producer keeps
+// the ring full meanwhile.
+constexpr int BOXW = 256;                   // bytes of K per TMA box
+constexpr int CW = 8;                       // compute warps, one 64-byte step each
+constexpr int STREAM_THREADS = (CW + 1) * 32;
+constexpr int CH = 64 * CW;                 // bytes of K per stage per row
+constexpr int BOXES = CH / BOXW;            // TMA boxes per stage
+constexpr int STAGES = 16;
+constexpr int STAGE_BYTES = ROWS * CH;      // 8 KB
+
+static_assert(CH % BOXW == 0, "whole boxes per stage");
+
+__host__ inline size_t stream_smem_bytes(int nt, int64_t K) {
+  return 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES +
+         static_cast<size_t>(nt * 8) * static_cast<size_t>(slice_bytes(K) + 16) +
+         static_cast<size_t>(CW) * ROWS * nt * 8 * sizeof(int32_t) + 2 * STAGES * 8;
+}
+
 template <int NT>
-__global__ void __launch_bounds__(THREADS)
-    gemv_partial_kernel(const int8_t* __restrict__ Xq, const int8_t* __restrict__ CB, int T,
-                        int64_t N, int64_t K, int32_t* __restrict__ P) {
-  extern __shared__ __align__(16) uint8_t sm[];
+__global__ void __launch_bounds__(STREAM_THREADS, 1)
+    gemv_stream_kernel(const __grid_constant__ CUtensorMap tmCB, const int8_t* __restrict__ Xq,
+                       int T, int64_t N, int64_t K, int32_t* __restrict__ P, uint64_t lim) {
+  extern __shared__ uint8_t smraw[];
+  const uint32_t raw_s = smem_u32(smraw);
+  const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
+  uint8_t* sm = smraw + pad;
+  const uint32_t ring = raw_s + pad;
   const int64_t KS = slice_bytes(K);
   const int S = static_cast<int>(num_slices(K));
   const int64_t pitch = KS + 16;
+  uint8_t* xs = sm + static_cast<size_t>(STAGES) * STAGE_BYTES;
+  int32_t* red = reinterpret_cast<int32_t*>(xs + NT * 8 * pitch);
+  uint64_t* full = reinterpret_cast<uint64_t*>(red + CW * ROWS * NT * 8);
+  uint64_t* empty = full + STAGES;
+  __shared__ int s_abort;
+
   const int slice = blockIdx.x % S;
   const int cta_in_slice = blockIdx.x / S;
   const int ctas_in_slice = (static_cast<int>(gridDim.x) - slice + S - 1) / S;
   const int64_t k0 = static_cast<int64_t>(slice) * KS;
+  const int64_t klen = min(KS, K - k0);
+  const int spt = static_cast<int>((klen + CH - 1) / CH);   // stages per tile
+  const int64_t n_tiles = (N + ROWS - 1) / ROWS;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(smem_u32(full + i), 1);
+      mbar_init(smem_u32(empty + i), CW);
+    }
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == CW && lane == 0) tma_prefetch_desc(&tmCB);
   grid_dep_wait();    // Xq comes from the previous kernel
   grid_dep_launch();  // the finalize kernel may start launching
-
   // stage Xq[:, k0 : k0+KS] (tokens >= T and columns >= K are zero)
   const int64_t vec_per_row = KS / 16;
-  for (int64_t i = threadIdx.x; i < NT * 8 * vec_per_row; i += THREADS) {
+  for (int64_t i = threadIdx.x; i < NT * 8 * vec_per_row; i += STREAM_THREADS) {
     const int tok = static_cast<int>(i / vec_per_row);
     const int64_t c16 = i - tok * vec_per_row;
     const int64_t k = k0 + c16 * 16;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (tok < T && k < K) v = ldg_v4(Xq + static_cast<int64_t>(tok) * K + k);
-    *reinterpret_cast<uint4*>(sm + tok * pitch + c16 * 16) = v;
+    *reinterpret_cast<uint4*>(xs + tok * pitch + c16 * 16) = v;
   }
   __syncthreads();
+  volatile int* abort_flag = &s_abort;
 
-  int32_t* red = reinterpret_cast<int32_t*>(sm + NT * 8 * pitch);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, q = lane & 3;
-  const int64_t kw = KS / WARPS;
-  const int steps = static_cast<int>(kw / 64);
-  const int64_t n_tiles = (N + ROWS - 1) / ROWS;
-
-  for (int64_t tile = cta_in_slice; tile < n_tiles; tile += ctas_in_slice) {
-    const int64_t n0 = tile * ROWS;
-    const int64_t ra = n0 + g, rb = n0 + g + 8;
-    const int8_t* pa = CB + ra * K;
-    const int8_t* pb = CB + rb * K;
-    const bool va = ra < N, vb = rb < N;
-    int c[NT][4];
+  if (warp == CW) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      uint32_t issued = 0;
+      bool ok = true;
+      for (int64_t tile = cta_in_slice; tile < n_tiles && ok; tile += ctas_in_slice) {
+        const int y = static_cast<int>(tile * ROWS);
+        for (int st = 0; st < spt; ++st) {
+          if (!mbar_wait(smem_u32(empty + s), ph ^ 1u, abort_flag, lim)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(full + s);
+          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          const int x = static_cast<int>(k0 + static_cast<int64_t>(st) * CH);
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) c[nt][0] = c[nt][1] = c[nt][2] = c[nt][3] = 0;
-
-    constexpr int U = 4;  // steps in flight
-    for (int st0 = 0; st0 < steps; st0 += U) {
-      uint4 A0[U], A1[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int64_t ks = static_cast<int64_t>(warp) * kw + (st0 + u) * 64 + q * 16;
-        const int64_t k = k0 + ks;
-        const bool in = (st0 + u < steps) && (k < K);
-        A0[u] = (in && va) ? ldg_stream_v4(pa + k) : make_uint4(0u, 0u, 0u, 0u);
-        A1[u] = (in && vb) ? ldg_stream_v4(pb + k) : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        if (st0 + u < steps) {
-          const int64_t ks = static_cast<int64_t>(warp) * kw + (st0 + u) * 64 + q * 16;
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const uint4 B = *reinterpret_cast<const uint4*>(sm + (nt * 8 + g) * pitch + ks);
-            mma_s8_16816(c[nt], A0[u].x, A1[u].x, A0[u].y, A1[u].y, B.x, B.y);
-            mma_s8_16816(c[nt], A0[u].z, A1[u].z, A0[u].w, A1[u].w, B.z, B.w);
+          for (int c = 0; c < BOXES; ++c)
+            tma_load_2d(ring + s * STAGE_BYTES + c * (ROWS * BOXW), &tmCB, fb, x + c * BOXW, y);
+          ++issued;
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
           }
         }
       }
+      if (!ok) {
+        // wind down: let the copies in flight land (bounded) before the CTA exits
+        int no_abort = 0;
+        const uint32_t inflight = issued < STAGES ? issued : STAGES;
+        for (uint32_t i = 0; i < inflight; ++i) {
+          const uint32_t u = issued - 1 - i;
+          mbar_wait(smem_u32(full + u % STAGES), (u / STAGES) & 1u, &no_abort, lim);
+        }
+      }
     }
-    // c[nt][0..3] = (row g, tok nt*8+2q), (row g, tok +1), (row g+8, tok), (row g+8, tok+1)
+  } else {
+    // ------------------------------------------------------------ compute warps
+    const int g = lane >> 2, q = lane & 3;
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int64_t tile = cta_in_slice; tile < n_tiles; tile += ctas_in_slice) {
+      int c[NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      int32_t* rw = red + (warp * ROWS) * (NT * 8);
-      rw[g * (NT * 8) + nt * 8 + 2 * q] = c[nt][0];
-      rw[g * (NT * 8) + nt * 8 + 2 * q + 1] = c[nt][1];
-      rw[(g + 8) * (NT * 8) + nt * 8 + 2 * q] = c[nt][2];
-      rw[(g + 8) * (NT * 8) + nt * 8 + 2 * q + 1] = c[nt][3];
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < ROWS * NT * 8; i += THREADS) {
-      const int rr = i / (NT * 8), tok = i - rr * (NT * 8);
-      int32_t sum = 0;
+      for (int nt = 0; nt < NT; ++nt) c[nt][0] = c[nt][1] = c[nt][2] = c[nt][3] = 0;
+      for (int st = 0; st < spt; ++st) {
+        if (ok) {
+          const bool got = mbar_wait(smem_u32(full + s), ph, abort_flag, lim);
+          ok = __all_sync(0xffffffffu, got);
+        }
+        if (ok) {
+          // this warp's 64-byte step of the stage: box warp / 4, bytes 64 * (warp % 4) of
+          // each 256-byte row; k offset within the slice = stage * CH + 64 * warp
+          const uint32_t rowbase = ring + s * STAGE_BYTES + (warp >> 2) * (ROWS * BOXW) +
+                                   (warp & 3) * 64 + q * 16;
+          const int64_t kx = static_cast<int64_t>(st) * CH + 64 * warp + 16 * q;
+          const uint4 A0 = lds_v4(rowbase + g * BOXW);
+          const uint4 A1 = lds_v4(rowbase + (g + 8) * BOXW);
 #pragma unroll
-      for (int w = 0; w < WARPS; ++w) sum += red[(w * ROWS + rr) * (NT * 8) + tok];
-      const int64_t n = n0 + rr;
-      if (tok < T && n < N) P[(static_cast<int64_t>(slice) * T + tok) * N + n] = sum;
+          for (int nt = 0; nt < NT; ++nt) {
+            const uint4 B = *reinterpret_cast<const uint4*>(xs + (nt * 8 + g) * pitch + kx);
+            mma_s8_16816(c[nt], A0.x, A1.x, A0.y, A1.y, B.x, B.y);
+            mma_s8_16816(c[nt], A0.z, A1.z, A0.w, A1.w, B.z, B.w);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(empty + s));
+        }
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      // reduce the CW warps' partials of this tile; write P
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        int32_t* rw = red + (warp * ROWS) * (NT * 8);
+        rw[g * (NT * 8) + nt * 8 + 2 * q] = c[nt][0];
+        rw[g * (NT * 8) + nt * 8 + 2 * q + 1] = c[nt][1];
+        rw[(g + 8) * (NT * 8) + nt * 8 + 2 * q] = c[nt][2];
+        rw[(g + 8) * (NT * 8) + nt * 8 + 2 * q + 1] = c[nt][3];
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(CW * 32) : "memory");
+      const int64_t n0 = tile * ROWS;
+      for (int i = threadIdx.x; i < ROWS * NT * 8; i += CW * 32) {
+        const int rr = i / (NT * 8), tok = i - rr * (NT * 8);
+        int32_t sum = 0;
+#pragma unroll
+        for (int w = 0; w < CW; ++w) sum += red[(w * ROWS + rr) * (NT * 8) + tok];
+        const int64_t n = n0 + rr;
+        if (tok < T && n < N) P[(static_cast<int64_t>(slice) * T + tok) * N + n] = sum;
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(CW * 32) : "memory");
     }
-    __syncthreads();
   }
+  __syncthreads();
 }
 
 // One thread per output (t, n) -- grid.y is the token: sum the K-slice partials (exact
