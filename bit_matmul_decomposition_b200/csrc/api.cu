@@ -128,8 +128,11 @@ size_t slice_elems(int64_t rows, int64_t K) {
 // ------------------------------------------------------------------ workspace layout
 struct Workspace {
   size_t mask, idx, n_o, scx, xq, xo, cbo, part, total;
+  int64_t zero_words;  // words from `mask` on that must be zero when a forward starts
 };
 
+// The first region holds the packed outlier mask and the grid-barrier word of the fused
+// prepare pass; one memset clears both at the start of every forward.
 Workspace layout(int64_t T, int64_t N, int64_t K) {
   Workspace w{};
   size_t off = 0;
@@ -138,17 +141,18 @@ Workspace layout(int64_t T, int64_t N, int64_t K) {
     off = align_up(off + bytes, 256);
     return o;
   };
-  w.mask = take(static_cast<size_t>((K + 31) / 32 + 1) * 4);  // mask + barrier word
+  const int64_t words = (K + 31) / 32;
+  const bool decode = T <= kDecodeMaxT;
+  w.zero_words = words + 1;
+  w.mask = take(static_cast<size_t>(w.zero_words) * 4);
   w.idx = take(static_cast<size_t>(K) * 4);
   w.n_o = take(16);
   w.scx = take(static_cast<size_t>(T) * 4);
   w.xq = take(static_cast<size_t>(T) * static_cast<size_t>(K));
   w.xo = take(slice_elems(T, K) * 2);
-  if (T > kDecodeMaxT) {
+  if (!decode) {
     w.cbo = take(slice_elems(N, K) * 2);
-    w.part = 0;
   } else {
-    w.cbo = 0;
     w.part = take(static_cast<size_t>(gemv::num_slices(K)) * static_cast<size_t>(T) *
                   static_cast<size_t>(N) * 4);
   }
@@ -253,12 +257,13 @@ i8_status run_quant_rows(const void* A, int64_t R, int64_t K, const uint32_t* ma
 
 // Fused steps 1 + 2 (+ the fp16 outlier slices): one cooperative launch.
 // mask must hold ceil(K/32) + 1 words; the last one is the grid-barrier counter.
+// `zero_words` words from `mask` on are cleared first (at least the mask and the barrier
+// word, ceil(K/32) + 1).
 i8_status run_prepare(const void* X, int64_t T, int64_t K, float thr, uint32_t* mask,
-                      int32_t* idx, int32_t* n_o, int8_t* Xq, float* SCx, void* X_o,
-                      const int8_t* CB, int64_t N, void* CB_o, const DeviceInfo& d,
+                      int64_t zero_words, int32_t* idx, int32_t* n_o, int8_t* Xq, float* SCx,
+                      void* X_o, const int8_t* CB, int64_t N, void* CB_o, const DeviceInfo& d,
                       cudaStream_t s) {
-  const int64_t words = (K + 31) / 32;
-  if (cudaMemsetAsync(mask, 0, static_cast<size_t>(words + 1) * 4, s) != cudaSuccess)
+  if (cudaMemsetAsync(mask, 0, static_cast<size_t>(zero_words) * 4, s) != cudaSuccess)
     return I8_ERR_CUDA;
   const int64_t G0 = d.sms;
   const int64_t rows_per_cta = (T + G0 - 1) / G0;
@@ -344,31 +349,47 @@ i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t
   return e == cudaSuccess ? launch_status() : I8_ERR_CUDA;
 }
 
-// decode GEMV partials (TMA-streamed CB); the caller then runs the finalize kernel
-i8_status run_gemv_partial(const int8_t* A, int64_t T, int64_t K, const int8_t* B, int64_t N,
-                           int32_t* P, const DeviceInfo& d, cudaStream_t s) {
+// decode: TMA-streamed int8 partials, then the finalize pass (slice sums, outlier
+// product, epilogue)
+i8_status run_gemv(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t* B, int64_t N,
+                   int32_t* P, const int32_t* idx, const int32_t* n_o, const void* X_o,
+                   const float* SCx, const float* SCB, const void* bias, void* C, int32_t* acc,
+                   const DeviceInfo& d, cudaStream_t s, cudaEvent_t ev_stop) {
   const int nt = T <= 8 ? 1 : 2;
   const size_t smem = gemv::stream_smem_bytes(nt, K);
   if (smem > static_cast<size_t>(d.prep_smem_max)) return I8_ERR_INVALID_ARG;
   CUtensorMap tCB;
   if (!map_2d_plain(&tCB, B, K, N, K, gemv::BOXW, gemv::ROWS)) return I8_ERR_CUDA;
   const int S = static_cast<int>(gemv::num_slices(K));
-  cudaError_t e = nt == 1 ? cudaFuncSetAttribute(gemv::gemv_stream_kernel<1>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(smem))
-                          : cudaFuncSetAttribute(gemv::gemv_stream_kernel<2>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(smem));
-  if (e != cudaSuccess) return I8_ERR_CUDA;
   int grid = (d.sms / S) * S;  // one CTA per SM, the same number of CTAs on every slice
   if (grid < S) grid = S;
   const int Ti = static_cast<int>(T);
-  if (nt == 1)
-    e = launch_overlapped(gemv::gemv_stream_kernel<1>, dim3(static_cast<unsigned>(grid)),
-                          dim3(gemv::STREAM_THREADS), smem, s, tCB, A, Ti, N, K, P, kWaitLimitNs);
+  auto go = [&](auto kernel) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    return launch_overlapped(kernel, dim3(static_cast<unsigned>(grid)),
+                             dim3(gemv::STREAM_THREADS), smem, s, tCB, A, Ti, N, K, P,
+                             kWaitLimitNs);
+  };
+  cudaError_t e = nt == 1 ? go(gemv::gemv_stream_kernel<1>) : go(gemv::gemv_stream_kernel<2>);
+  if (e != cudaSuccess || launch_status() != I8_OK) return I8_ERR_CUDA;
+  if (ev_stop && cudaEventRecord(ev_stop, s) != cudaSuccess) return I8_ERR_CUDA;
+  const dim3 fgrid(static_cast<unsigned>((N + gemv::FIN_THREADS - 1) / gemv::FIN_THREADS),
+                   static_cast<unsigned>((T + gemv::TG - 1) / gemv::TG));
+  const int32_t* Pc = P;
+  if (raw)
+    e = launch_overlapped(gemv::gemv_finalize_kernel<true>, fgrid, dim3(gemv::FIN_THREADS), 0, s,
+                          Pc, S, Ti, N, K, static_cast<const float*>(nullptr),
+                          static_cast<const float*>(nullptr), static_cast<const __half*>(nullptr),
+                          static_cast<const int8_t*>(nullptr), static_cast<const int32_t*>(nullptr),
+                          static_cast<const int32_t*>(nullptr), static_cast<const __half*>(nullptr),
+                          static_cast<__half*>(nullptr), acc);
   else
-    e = launch_overlapped(gemv::gemv_stream_kernel<2>, dim3(static_cast<unsigned>(grid)),
-                          dim3(gemv::STREAM_THREADS), smem, s, tCB, A, Ti, N, K, P, kWaitLimitNs);
+    e = launch_overlapped(gemv::gemv_finalize_kernel<false>, fgrid, dim3(gemv::FIN_THREADS), 0,
+                          s, Pc, S, Ti, N, K, SCx, SCB, static_cast<const __half*>(bias), B, idx,
+                          n_o, static_cast<const __half*>(X_o), static_cast<__half*>(C),
+                          static_cast<int32_t*>(nullptr));
   return e == cudaSuccess ? launch_status() : I8_ERR_CUDA;
 }
 
@@ -490,8 +511,8 @@ i8_status i8_prepare_act(const void* X, int64_t T, int64_t K, float threshold,
   DeviceInfo* d;
   i8_status st = device_info(&d);
   if (st != I8_OK) return st;
-  return run_prepare(X, T, K, threshold, col_mask, outlier_idx, n_outliers, Xq, SCx, X_o,
-                     nullptr, 0, nullptr, *d, static_cast<cudaStream_t>(stream));
+  return run_prepare(X, T, K, threshold, col_mask, (K + 31) / 32 + 1, outlier_idx, n_outliers,
+                     Xq, SCx, X_o, nullptr, 0, nullptr, *d, static_cast<cudaStream_t>(stream));
 }
 
 i8_status i8_linear_forward(const void* X, int64_t T, int64_t K, const int8_t* CB,
@@ -520,7 +541,8 @@ i8_status i8_linear_forward(const void* X, int64_t T, int64_t K, const int8_t* C
   const bool prof = g_prof_start != nullptr && g_prof_stop != nullptr;
   if (T > kDecodeMaxT) {
     void* CB_o = ws + w.cbo;
-    st = run_prepare(X, T, K, threshold, mask, idx, n_o, Xq, SCx, X_o, CB, N, CB_o, *d, s);
+    st = run_prepare(X, T, K, threshold, mask, w.zero_words, idx, n_o, Xq, SCx, X_o, CB, N, CB_o,
+                     *d, s);
     if (st != I8_OK) return st;
     if (prof && cudaEventRecord(g_prof_start, s) != cudaSuccess) return I8_ERR_CUDA;
     st = run_gemm(false, Xq, T, K, CB, N, X_o, CB_o, n_o, SCx, SCB, bias, C, nullptr, *d, s);
@@ -528,22 +550,12 @@ i8_status i8_linear_forward(const void* X, int64_t T, int64_t K, const int8_t* C
     if (prof && cudaEventRecord(g_prof_stop, s) != cudaSuccess) return I8_ERR_CUDA;
     return I8_OK;
   }
-  st = run_prepare(X, T, K, threshold, mask, idx, n_o, Xq, SCx, X_o, nullptr, N, nullptr, *d, s);
+  st = run_prepare(X, T, K, threshold, mask, w.zero_words, idx, n_o, Xq, SCx, X_o, nullptr, N,
+                   nullptr, *d, s);
   if (st != I8_OK) return st;
-  int32_t* P = reinterpret_cast<int32_t*>(ws + w.part);
   if (prof && cudaEventRecord(g_prof_start, s) != cudaSuccess) return I8_ERR_CUDA;
-  st = run_gemv_partial(Xq, T, K, CB, N, P, *d, s);
-  if (st != I8_OK) return st;
-  if (prof && cudaEventRecord(g_prof_stop, s) != cudaSuccess) return I8_ERR_CUDA;
-  const int S = static_cast<int>(gemv::num_slices(K));
-  const cudaError_t e = launch_overlapped(
-      gemv::gemv_finalize_kernel<false>,
-      dim3(static_cast<unsigned>((N + 255) / 256), static_cast<unsigned>(T)), dim3(256), 0, s,
-      static_cast<const int32_t*>(P), S, static_cast<int>(T), N, K, static_cast<const float*>(SCx),
-      SCB, static_cast<const __half*>(bias), CB, static_cast<const int32_t*>(idx),
-      static_cast<const int32_t*>(n_o), static_cast<const __half*>(X_o), static_cast<__half*>(C),
-      static_cast<int32_t*>(nullptr));
-  return e == cudaSuccess ? launch_status() : I8_ERR_CUDA;
+  return run_gemv(false, Xq, T, K, CB, N, reinterpret_cast<int32_t*>(ws + w.part), idx, n_o,
+                  X_o, SCx, SCB, bias, C, nullptr, *d, s, prof ? g_prof_stop : nullptr);
 }
 
 i8_status i8_igemm_s32(const int8_t* A, int64_t T, int64_t K, const int8_t* B, int64_t N,
@@ -561,19 +573,9 @@ i8_status i8_igemm_s32(const int8_t* A, int64_t T, int64_t K, const int8_t* B, i
   if (T > kDecodeMaxT)
     return run_gemm(true, A, T, K, B, N, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                     nullptr, acc, *d, s);
-  int32_t* P = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + w.part);
-  st = run_gemv_partial(A, T, K, B, N, P, *d, s);
-  if (st != I8_OK) return st;
-  const int S = static_cast<int>(gemv::num_slices(K));
-  const cudaError_t e = launch_overlapped(
-      gemv::gemv_finalize_kernel<true>,
-      dim3(static_cast<unsigned>((N + 255) / 256), static_cast<unsigned>(T)), dim3(256), 0, s,
-      static_cast<const int32_t*>(P), S, static_cast<int>(T), N, K,
-      static_cast<const float*>(nullptr), static_cast<const float*>(nullptr),
-      static_cast<const __half*>(nullptr), static_cast<const int8_t*>(nullptr),
-      static_cast<const int32_t*>(nullptr), static_cast<const int32_t*>(nullptr),
-      static_cast<const __half*>(nullptr), static_cast<__half*>(nullptr), acc);
-  return e == cudaSuccess ? launch_status() : I8_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  return run_gemv(true, A, T, K, B, N, reinterpret_cast<int32_t*>(ws + w.part), nullptr, nullptr,
+                  nullptr, nullptr, nullptr, nullptr, nullptr, acc, *d, s, nullptr);
 }
 
 i8_status i8_sync_status(void* stream) {

@@ -1,23 +1,17 @@
 // gemv.cuh -- steps 4, 5 and 6 for decode batches (T <= 16), where the layer is a stream
 // of CB through HBM: each CB byte is used by at most 16 tokens, so the bound is memory,
-// not the tensor pipe.
-//
-//   gemv_partial_kernel   int8 x int8 -> int32 partial sums over one K-slice, with the
-//                         warp-level tensor-core MMA m16n8k32 (16 CB rows x 8 tokens):
-//                         CB streams from HBM in 16-byte loads (no L1 allocation),
-//                         the slice of Xq sits in shared memory.
-//   gemv_finalize_kernel  sums the K-slice partials (exact int32), then the same
-//                         epilogue as the GEMM: (acc*SCx/127 + sum_j X_o*CB_o)*SCB/127 + bias.
+// not the tensor pipe.  gemv_stream_kernel computes the int8 K-slice partial sums;
+// gemv_finalize_kernel adds them up and applies the fp16 outlier product, the
+// dequantisation and the bias.
 //
 // Source: "A Gentle Introduction to 8-bit Matrix Multiplication for transformers at
 // scale" (Hugging Face blog), "内部的 MatMul" (int8 product, dequantisation, fp16
 // outlier product); "改进范围" notes that small-batch inference was the slow case.
 //
-// K-slicing keeps the Xq slice resident in shared memory while the CTA streams many
-// 16-row tiles of CB; partial sums are written once each (no atomics), so the result is
-// deterministic.  Within one 64-byte step a thread loads 16 contiguous CB bytes of rows
-// g and g+8 and the 16 matching Xq bytes of token g; two MMAs consume them.  The k
-// order inside the step is permuted identically for A and B, which leaves each dot
+// K-slicing keeps the Xq slice resident in shared memory while a CTA streams many 16-row
+// tiles of CB.  Within one 64-byte step a thread takes 16 contiguous CB bytes of rows g
+// and g+8 and the 16 matching Xq bytes of token g; two m16n8k32 MMAs consume them.  The
+// k order inside the step is permuted identically for A and B, which leaves each dot
 // product unchanged.
 #pragma once
 
@@ -27,8 +21,7 @@
 namespace i8 {
 namespace gemv {
 
-constexpr int THREADS = 256;
-constexpr int WARPS = THREADS / 32;
+constexpr int WARPS = 8;             // slice lengths are whole multiples of WARPS * 64 bytes
 constexpr int ROWS = 16;          // CB rows per tile (MMA M)
 constexpr int SLICE_TARGET = 3584;  // bytes of K per slice (before rounding)
 
@@ -44,10 +37,6 @@ __host__ __device__ inline int64_t num_slices(int64_t K) {
   return (K + ks - 1) / ks;
 }
 
-__host__ inline size_t smem_bytes(int nt, int64_t K) {
-  return static_cast<size_t>(nt * 8) * static_cast<size_t>(slice_bytes(K) + 16) +
-         static_cast<size_t>(WARPS) * ROWS * nt * 8 * sizeof(int32_t);
-}
 
 __device__ __forceinline__ void mma_s8_16816(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                              uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -58,15 +47,23 @@ __device__ __forceinline__ void mma_s8_16816(int (&c)[4], uint32_t a0, uint32_t 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// P[slice][t][n] = sum over k in the slice of Xq[t,k] * CB[n,k]   (t < T only)
+// Decode kernels (steps 4, 5 and 6 for T <= 16), two launches after the fused prepare.
 //
-// Warp CW (one thread) streams CB through a ring of STAGES stages, each 16 rows x CH
-// bytes of K, loaded as 2-D TMA boxes of 256 B x 16 rows (no swizzle: the widest box TMA
-// takes, which streams HBM best -- ~6 TB/s measured on B200 for this layout).  The CW
-// compute warps each own one 64-byte MMA step of every stage, accumulate their
-// 16 x (8*NT) int32 partials in registers over the tile's stages, and only at the tile's
-// end reduce across warps (a named barrier among the compute warps); the producer keeps
-// the ring full meanwhile.
+// gemv_stream_kernel: warp CW (one thread) streams CB through a ring of STAGES stages,
+// each 16 rows x CH bytes of K, loaded as 2-D TMA boxes of 256 B x 16 rows (no swizzle:
+// the widest box TMA takes, which streams HBM best -- ~6 TB/s measured on B200 for this
+// layout).  The CW compute warps each own one 64-byte MMA step of every stage and
+// accumulate, over the tile's stages of their CTA's K-slice,
+//   P[slice][t][n] = sum_{k in slice} Xq[t,k] * CB[n,k]     (int32, mma.sync m16n8k32)
+// in registers; at the tile's end the warps' partials are reduced in a fixed order.
+// The loop carries nothing but the int8 product: the outlier columns are a handful, and
+// any per-column work inside it lands on the same warp in every tile and holds up the
+// tile-end barrier.
+//
+// gemv_finalize_kernel: one thread per output channel n and group of TG tokens sums the
+// slice partials (exact int32) and gathers the n_o outlier bytes CB[n, idx[j]] once,
+// applying each to the group's tokens (fp32), then writes
+//   C[t,n] = fp16((P[t,n] * SCx[t]/127 + sum_j X_o[t,j] * CB[n,idx[j]]) * SCB[n]/127 + bias[n]).
 constexpr int BOXW = 256;                   // bytes of K per TMA box
 constexpr int CW = 8;                       // compute warps, one 64-byte step each
 constexpr int STREAM_THREADS = (CW + 1) * 32;
@@ -74,13 +71,19 @@ constexpr int CH = 64 * CW;                 // bytes of K per stage per row
 constexpr int BOXES = CH / BOXW;            // TMA boxes per stage
 constexpr int STAGES = 16;
 constexpr int STAGE_BYTES = ROWS * CH;      // 8 KB
+constexpr int RP = ROWS + 4;                // row pitch of the reduction buffer (in words):
+                                            // fragment stores and the row-fastest reads
+                                            // then fall on (nearly) distinct banks
+constexpr int TG = 4;                       // tokens per finalize thread
+constexpr int FIN_THREADS = 128;
 
 static_assert(CH % BOXW == 0, "whole boxes per stage");
+static_assert(SLICE_TARGET % CH == 0 && (WARPS * 64) % CH == 0, "slices hold whole stages");
 
 __host__ inline size_t stream_smem_bytes(int nt, int64_t K) {
   return 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES +
          static_cast<size_t>(nt * 8) * static_cast<size_t>(slice_bytes(K) + 16) +
-         static_cast<size_t>(CW) * ROWS * nt * 8 * sizeof(int32_t) + 2 * STAGES * 8;
+         static_cast<size_t>(CW) * RP * nt * 8 * 4 + 2 * STAGES * 8;
 }
 
 template <int NT>
@@ -97,7 +100,7 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1)
   const int64_t pitch = KS + 16;
   uint8_t* xs = sm + static_cast<size_t>(STAGES) * STAGE_BYTES;
   int32_t* red = reinterpret_cast<int32_t*>(xs + NT * 8 * pitch);
-  uint64_t* full = reinterpret_cast<uint64_t*>(red + CW * ROWS * NT * 8);
+  uint64_t* full = reinterpret_cast<uint64_t*>(red + CW * RP * NT * 8);
   uint64_t* empty = full + STAGES;
   __shared__ int s_abort;
 
@@ -208,22 +211,23 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1)
           ph ^= 1u;
         }
       }
-      // reduce the CW warps' partials of this tile; write P
+      // ---- reduce the warps' partials of this tile (fixed order) and write P;
+      // the buffer is [warp][token][row] with row pitch RP
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        int32_t* rw = red + (warp * ROWS) * (NT * 8);
-        rw[g * (NT * 8) + nt * 8 + 2 * q] = c[nt][0];
-        rw[g * (NT * 8) + nt * 8 + 2 * q + 1] = c[nt][1];
-        rw[(g + 8) * (NT * 8) + nt * 8 + 2 * q] = c[nt][2];
-        rw[(g + 8) * (NT * 8) + nt * 8 + 2 * q + 1] = c[nt][3];
+        const int i0 = (warp * (NT * 8) + nt * 8 + 2 * q) * RP + g;
+        red[i0] = c[nt][0];
+        red[i0 + RP] = c[nt][1];
+        red[i0 + 8] = c[nt][2];
+        red[i0 + RP + 8] = c[nt][3];
       }
       asm volatile("bar.sync 1, %0;" ::"n"(CW * 32) : "memory");
       const int64_t n0 = tile * ROWS;
       for (int i = threadIdx.x; i < ROWS * NT * 8; i += CW * 32) {
-        const int rr = i / (NT * 8), tok = i - rr * (NT * 8);
+        const int tok = i / ROWS, rr = i - tok * ROWS;   // consecutive threads: consecutive n
         int32_t sum = 0;
 #pragma unroll
-        for (int w = 0; w < CW; ++w) sum += red[(w * ROWS + rr) * (NT * 8) + tok];
+        for (int w = 0; w < CW; ++w) sum += red[(w * (NT * 8) + tok) * RP + rr];
         const int64_t n = n0 + rr;
         if (tok < T && n < N) P[(static_cast<int64_t>(slice) * T + tok) * N + n] = sum;
       }
@@ -233,11 +237,13 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1)
   __syncthreads();
 }
 
-// One thread per output (t, n) -- grid.y is the token: sum the K-slice partials (exact
-// int32), then dequantise, add the outlier part (CB read straight through the index list,
-// 8 loads in flight) and the bias.  kRaw writes the int32 sum.
+// One thread per output channel n (consecutive threads on consecutive n) and group of TG
+// tokens (grid.y): the outlier bytes CB[n, idx[j]] are gathered once per group (8 loads in
+// flight; later groups find them in L2) and applied to the group's tokens in fp32, column
+// order j = 0 .. n_o-1; the slice partials are summed exactly (int32, slice order).
+// kRaw writes the int32 sums.
 template <bool kRaw>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(FIN_THREADS)
     gemv_finalize_kernel(const int32_t* __restrict__ P, int S, int T, int64_t N, int64_t K,
                          const float* __restrict__ SCx, const float* __restrict__ SCB,
                          const __half* __restrict__ bias, const int8_t* __restrict__ CB,
@@ -245,36 +251,55 @@ __global__ void __launch_bounds__(256)
                          const __half* __restrict__ X_o, __half* __restrict__ C,
                          int32_t* __restrict__ acc_out) {
   const int64_t n = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int t = blockIdx.y;
+  const int t0 = blockIdx.y * TG;
+  const int tn = min(TG, T - t0);
   grid_dep_wait();    // the partial sums come from the previous kernel
   if (n >= N) return;
-  int32_t acc = 0;
-  for (int s = 0; s < S; ++s) acc += __ldcs(P + (static_cast<int64_t>(s) * T + t) * N + n);
+  int32_t acc[TG];
+#pragma unroll
+  for (int u = 0; u < TG; ++u) acc[u] = 0;
+  for (int sl = 0; sl < S; ++sl) {
+    const int32_t* p = P + (static_cast<int64_t>(sl) * T + t0) * N + n;
+#pragma unroll
+    for (int u = 0; u < TG; ++u)
+      if (u < tn) acc[u] += __ldcs(p + u * N);
+  }
   if (kRaw) {
-    acc_out[static_cast<int64_t>(t) * N + n] = acc;
+#pragma unroll
+    for (int u = 0; u < TG; ++u)
+      if (u < tn) acc_out[static_cast<int64_t>(t0 + u) * N + n] = acc[u];
     return;
   }
-  const int n_o = (n_o_ptr == nullptr) ? 0 : *n_o_ptr;
-  float o = 0.0f;
+  float o[TG];
+#pragma unroll
+  for (int u = 0; u < TG; ++u) o[u] = 0.0f;
+  const int n_o = n_o_ptr == nullptr ? 0 : __ldg(n_o_ptr);
+  const int8_t* cbrow = CB + n * K;
   for (int j0 = 0; j0 < n_o; j0 += 8) {
-    float cb[8], xo[8];
+    float cb[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int j = j0 + u;
-      cb[u] = 0.0f;
-      xo[u] = 0.0f;
-      if (j < n_o) {
-        cb[u] = static_cast<float>(CB[n * K + __ldg(idx + j)]);
-        xo[u] = __half2float(X_o[(static_cast<int64_t>(j >> 6) * T + t) * 64 + (j & 63)]);
-      }
+    for (int v = 0; v < 8; ++v)
+      cb[v] = j0 + v < n_o ? static_cast<float>(cbrow[__ldg(idx + j0 + v)]) : 0.0f;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const int j = j0 + v;
+      if (j >= n_o) break;
+      const __half* xo = X_o + (static_cast<int64_t>(j >> 6) * T + t0) * 64 + (j & 63);
+#pragma unroll
+      for (int u = 0; u < TG; ++u)
+        if (u < tn) o[u] = fmaf(__half2float(xo[u * 64]), cb[v], o[u]);
     }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) o = fmaf(xo[u], cb[u], o);
   }
   const float ws = __ldg(SCB + n) * (1.0f / 127.0f);
   const float bn = bias ? __half2float(bias[n]) : 0.0f;
-  const float part = fmaf(static_cast<float>(acc), __ldg(SCx + t) * (1.0f / 127.0f), o);
-  C[static_cast<int64_t>(t) * N + n] = __float2half_rn(fmaf(part, ws, bn));
+#pragma unroll
+  for (int u = 0; u < TG; ++u) {
+    if (u < tn) {
+      const float part =
+          fmaf(static_cast<float>(acc[u]), __ldg(SCx + t0 + u) * (1.0f / 127.0f), o[u]);
+      C[static_cast<int64_t>(t0 + u) * N + n] = __float2half_rn(fmaf(part, ws, bn));
+    }
+  }
 }
 
 }  // namespace gemv
