@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 #include <utility>
 
@@ -18,7 +19,7 @@ namespace {
 using namespace i8;
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s for every device-side wait
-constexpr int64_t kDecodeMaxT = 16;               // T <= 16 takes the decode GEMV path
+constexpr int64_t kDecodeMaxT = 16;               // T <= 16 takes the decode kernel
 constexpr int kMaxDevices = 64;
 
 // ------------------------------------------------------------------ device info
@@ -29,6 +30,7 @@ struct DeviceInfo {
   bool gemm_attr = false;
   int gemm_clusters = 0;  // co-resident CTA pairs of the GEMM kernel
   int prep_smem_max = 0;  // dynamic shared memory granted to prepare_kernel
+  int smem_optin = 0;     // largest dynamic shared memory a kernel may opt in to
 };
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
@@ -83,6 +85,7 @@ i8_status device_info(DeviceInfo** out) {
                              prep_max) != cudaSuccess)
       return I8_ERR_CUDA;
     d.prep_smem_max = prep_max;
+    d.smem_optin = static_cast<int>(p_smem_optin(dev));
     d.gemm_attr = true;
   }
   *out = &d;
@@ -126,13 +129,19 @@ size_t slice_elems(int64_t rows, int64_t K) {
 }
 
 // ------------------------------------------------------------------ workspace layout
+// Decode batches (T <= 16, K <= 65536) run as one kernel: small T, and each CTA keeps what it
+// needs in shared memory.
+bool use_decode(int64_t T, int64_t K) { return T <= kDecodeMaxT && K <= gemv::MAX_K; }
+
 struct Workspace {
-  size_t mask, idx, n_o, scx, xq, xo, cbo, part, total;
+  size_t mask, idx, n_o, scx, xq, xo, cbo, rec, cnt, gmask, gscx, gbar, total;
   int64_t zero_words;  // words from `mask` on that must be zero when a forward starts
 };
 
-// The first region holds the packed outlier mask and the grid-barrier word of the fused
-// prepare pass; one memset clears both at the start of every forward.
+// GEMM path: the first region holds the packed outlier mask and the grid-barrier word of
+// the fused prepare pass; one memset clears both at the start of every forward.
+// Decode path: the slice records of every 32-row tile, the tiles' arrival counters and the
+// words of the cooperative prologue (none needs clearing: they carry the launch's epoch).
 Workspace layout(int64_t T, int64_t N, int64_t K) {
   Workspace w{};
   size_t off = 0;
@@ -141,8 +150,19 @@ Workspace layout(int64_t T, int64_t N, int64_t K) {
     off = align_up(off + bytes, 256);
     return o;
   };
+  if (use_decode(T, K)) {
+    const size_t n_tiles = static_cast<size_t>((N + gemv::ROWS - 1) / gemv::ROWS);
+    w.rec = take(n_tiles * static_cast<size_t>(gemv::num_slices(K)) *
+                 static_cast<size_t>(gemv::rec_bytes(T)));
+    w.cnt = take(n_tiles * 8);
+    w.gmask = take(static_cast<size_t>((K + 31) / 32) * 8);
+    w.gscx = take(static_cast<size_t>(T) * 8);
+    w.gbar = take(24);
+    w.xq = take(static_cast<size_t>(T) * static_cast<size_t>(K));
+    w.total = off;
+    return w;
+  }
   const int64_t words = (K + 31) / 32;
-  const bool decode = T <= kDecodeMaxT;
   w.zero_words = words + 1;
   w.mask = take(static_cast<size_t>(w.zero_words) * 4);
   w.idx = take(static_cast<size_t>(K) * 4);
@@ -150,12 +170,7 @@ Workspace layout(int64_t T, int64_t N, int64_t K) {
   w.scx = take(static_cast<size_t>(T) * 4);
   w.xq = take(static_cast<size_t>(T) * static_cast<size_t>(K));
   w.xo = take(slice_elems(T, K) * 2);
-  if (!decode) {
-    w.cbo = take(slice_elems(N, K) * 2);
-  } else {
-    w.part = take(static_cast<size_t>(gemv::num_slices(K)) * static_cast<size_t>(T) *
-                  static_cast<size_t>(N) * 4);
-  }
+  w.cbo = take(slice_elems(N, K) * 2);
   w.total = off;
   return w;
 }
@@ -349,47 +364,76 @@ i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t
   return e == cudaSuccess ? launch_status() : I8_ERR_CUDA;
 }
 
-// decode: TMA-streamed int8 partials, then the finalize pass (slice sums, outlier
-// product, epilogue)
-i8_status run_gemv(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t* B, int64_t N,
-                   int32_t* P, const int32_t* idx, const int32_t* n_o, const void* X_o,
-                   const float* SCx, const float* SCB, const void* bias, void* C, int32_t* acc,
-                   const DeviceInfo& d, cudaStream_t s, cudaEvent_t ev_stop) {
+// decode: one launch of the decode kernel (forward from X, or the raw product of codes)
+std::atomic<unsigned long long> g_epoch{0};
+
+// The prologue of the forward reads all of X in every CTA when X fits two ring stages;
+// beyond that the CTAs split it (cooperative launch, three grid barriers).
+bool decode_coop(bool raw, int64_t T, int64_t K) {
+  return !raw && T * K * 2 > 2 * static_cast<int64_t>(gemv::STAGE_BYTES);
+}
+
+i8_status run_decode(bool raw, const void* X, const int8_t* Xq, int64_t T, int64_t K,
+                     const int8_t* CB, int64_t N, float thr, const float* SCB, const void* bias,
+                     void* C, int32_t* acc, uint8_t* ws, const Workspace& w,
+                     const DeviceInfo& d, cudaStream_t s) {
   const int nt = T <= 8 ? 1 : 2;
-  const size_t smem = gemv::stream_smem_bytes(nt, K);
-  if (smem > static_cast<size_t>(d.prep_smem_max)) return I8_ERR_INVALID_ARG;
+  const size_t smem = gemv::smem_bytes(nt, K);
+  if (smem > static_cast<size_t>(d.smem_optin)) return I8_ERR_INVALID_ARG;
   CUtensorMap tCB;
-  if (!map_2d_plain(&tCB, B, K, N, K, gemv::BOXW, gemv::ROWS)) return I8_ERR_CUDA;
+  if (!map_2d_plain(&tCB, CB, K, N, K, gemv::BOXW, gemv::ROWS)) return I8_ERR_CUDA;
   const int S = static_cast<int>(gemv::num_slices(K));
   int grid = (d.sms / S) * S;  // one CTA per SM, the same number of CTAs on every slice
+  if (grid > 255) grid = (255 / S) * S;  // arrival counts are 8-bit
   if (grid < S) grid = S;
-  const int Ti = static_cast<int>(T);
+  gemv::Args a;
+  a.X = static_cast<const __half*>(X);
+  a.Xq = Xq;
+  a.T = static_cast<int>(T);
+  a.N = N;
+  a.K = K;
+  a.thr = thr;
+  a.CB = CB;
+  a.SCB = SCB;
+  a.bias = static_cast<const __half*>(bias);
+  a.C = static_cast<__half*>(C);
+  a.acc = acc;
+  a.rec = ws + w.rec;
+  a.cnt = reinterpret_cast<unsigned long long*>(ws + w.cnt);
+  a.epoch = g_epoch.fetch_add(1) % 0xffffffffull + 1;  // 1 .. 2^32 - 1
+  a.lim = kWaitLimitNs;
+  a.coop = decode_coop(raw, T, K);
+  a.gmask = reinterpret_cast<unsigned long long*>(ws + w.gmask);
+  a.gscx = reinterpret_cast<unsigned long long*>(ws + w.gscx);
+  a.gbar = reinterpret_cast<unsigned long long*>(ws + w.gbar);
+  a.xq = reinterpret_cast<int8_t*>(ws + w.xq);
   auto go = [&](auto kernel) -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    return launch_overlapped(kernel, dim3(static_cast<unsigned>(grid)),
-                             dim3(gemv::STREAM_THREADS), smem, s, tCB, A, Ti, N, K, P,
-                             kWaitLimitNs);
+    if (!a.coop)
+      return launch_overlapped(kernel, dim3(static_cast<unsigned>(grid)), dim3(gemv::THREADS),
+                               smem, s, tCB, a);
+    // every CTA must be resident for the grid barriers
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(gemv::THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeCooperative;
+    at[0].val.cooperative = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kernel, tCB, a);
   };
-  cudaError_t e = nt == 1 ? go(gemv::gemv_stream_kernel<1>) : go(gemv::gemv_stream_kernel<2>);
-  if (e != cudaSuccess || launch_status() != I8_OK) return I8_ERR_CUDA;
-  if (ev_stop && cudaEventRecord(ev_stop, s) != cudaSuccess) return I8_ERR_CUDA;
-  const dim3 fgrid(static_cast<unsigned>((N + gemv::FIN_THREADS - 1) / gemv::FIN_THREADS),
-                   static_cast<unsigned>((T + gemv::TG - 1) / gemv::TG));
-  const int32_t* Pc = P;
-  if (raw)
-    e = launch_overlapped(gemv::gemv_finalize_kernel<true>, fgrid, dim3(gemv::FIN_THREADS), 0, s,
-                          Pc, S, Ti, N, K, static_cast<const float*>(nullptr),
-                          static_cast<const float*>(nullptr), static_cast<const __half*>(nullptr),
-                          static_cast<const int8_t*>(nullptr), static_cast<const int32_t*>(nullptr),
-                          static_cast<const int32_t*>(nullptr), static_cast<const __half*>(nullptr),
-                          static_cast<__half*>(nullptr), acc);
+  cudaError_t e;
+  if (nt == 1)
+    e = raw ? go(gemv::decode_kernel<1, true>) : go(gemv::decode_kernel<1, false>);
   else
-    e = launch_overlapped(gemv::gemv_finalize_kernel<false>, fgrid, dim3(gemv::FIN_THREADS), 0,
-                          s, Pc, S, Ti, N, K, SCx, SCB, static_cast<const __half*>(bias), B, idx,
-                          n_o, static_cast<const __half*>(X_o), static_cast<__half*>(C),
-                          static_cast<int32_t*>(nullptr));
+    e = raw ? go(gemv::decode_kernel<2, true>) : go(gemv::decode_kernel<2, false>);
   return e == cudaSuccess ? launch_status() : I8_ERR_CUDA;
 }
 
@@ -531,31 +575,30 @@ i8_status i8_linear_forward(const void* X, int64_t T, int64_t K, const int8_t* C
   if (st != I8_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const bool prof = g_prof_start != nullptr && g_prof_stop != nullptr;
+  if (use_decode(T, K)) {
+    if (prof && cudaEventRecord(g_prof_start, s) != cudaSuccess) return I8_ERR_CUDA;
+    st = run_decode(false, X, nullptr, T, K, CB, N, threshold, SCB, bias, C, nullptr, ws, w, *d,
+                    s);
+    if (st != I8_OK) return st;
+    if (prof && cudaEventRecord(g_prof_stop, s) != cudaSuccess) return I8_ERR_CUDA;
+    return I8_OK;
+  }
   uint32_t* mask = reinterpret_cast<uint32_t*>(ws + w.mask);
   int32_t* idx = reinterpret_cast<int32_t*>(ws + w.idx);
   int32_t* n_o = reinterpret_cast<int32_t*>(ws + w.n_o);
   float* SCx = reinterpret_cast<float*>(ws + w.scx);
   int8_t* Xq = reinterpret_cast<int8_t*>(ws + w.xq);
   void* X_o = ws + w.xo;
-
-  const bool prof = g_prof_start != nullptr && g_prof_stop != nullptr;
-  if (T > kDecodeMaxT) {
-    void* CB_o = ws + w.cbo;
-    st = run_prepare(X, T, K, threshold, mask, w.zero_words, idx, n_o, Xq, SCx, X_o, CB, N, CB_o,
-                     *d, s);
-    if (st != I8_OK) return st;
-    if (prof && cudaEventRecord(g_prof_start, s) != cudaSuccess) return I8_ERR_CUDA;
-    st = run_gemm(false, Xq, T, K, CB, N, X_o, CB_o, n_o, SCx, SCB, bias, C, nullptr, *d, s);
-    if (st != I8_OK) return st;
-    if (prof && cudaEventRecord(g_prof_stop, s) != cudaSuccess) return I8_ERR_CUDA;
-    return I8_OK;
-  }
-  st = run_prepare(X, T, K, threshold, mask, w.zero_words, idx, n_o, Xq, SCx, X_o, nullptr, N,
-                   nullptr, *d, s);
+  void* CB_o = ws + w.cbo;
+  st = run_prepare(X, T, K, threshold, mask, w.zero_words, idx, n_o, Xq, SCx, X_o, CB, N, CB_o,
+                   *d, s);
   if (st != I8_OK) return st;
   if (prof && cudaEventRecord(g_prof_start, s) != cudaSuccess) return I8_ERR_CUDA;
-  return run_gemv(false, Xq, T, K, CB, N, reinterpret_cast<int32_t*>(ws + w.part), idx, n_o,
-                  X_o, SCx, SCB, bias, C, nullptr, *d, s, prof ? g_prof_stop : nullptr);
+  st = run_gemm(false, Xq, T, K, CB, N, X_o, CB_o, n_o, SCx, SCB, bias, C, nullptr, *d, s);
+  if (st != I8_OK) return st;
+  if (prof && cudaEventRecord(g_prof_stop, s) != cudaSuccess) return I8_ERR_CUDA;
+  return I8_OK;
 }
 
 i8_status i8_igemm_s32(const int8_t* A, int64_t T, int64_t K, const int8_t* B, int64_t N,
@@ -570,12 +613,11 @@ i8_status i8_igemm_s32(const int8_t* A, int64_t T, int64_t K, const int8_t* B, i
   i8_status st = device_info(&d);
   if (st != I8_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (T > kDecodeMaxT)
+  if (!use_decode(T, K))
     return run_gemm(true, A, T, K, B, N, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                     nullptr, acc, *d, s);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  return run_gemv(true, A, T, K, B, N, reinterpret_cast<int32_t*>(ws + w.part), nullptr, nullptr,
-                  nullptr, nullptr, nullptr, nullptr, nullptr, acc, *d, s, nullptr);
+  return run_decode(true, nullptr, A, T, K, B, N, 0.0f, nullptr, nullptr, nullptr, acc,
+                    static_cast<uint8_t*>(workspace), w, *d, s);
 }
 
 i8_status i8_sync_status(void* stream) {

@@ -1,18 +1,51 @@
-// gemv.cuh -- steps 4, 5 and 6 for decode batches (T <= 16), where the layer is a stream
-// of CB through HBM: each CB byte is used by at most 16 tokens, so the bound is memory,
-// not the tensor pipe.  gemv_stream_kernel computes the int8 K-slice partial sums;
-// gemv_finalize_kernel adds them up and applies the fp16 outlier product, the
-// dequantisation and the bias.
+// gemv.cuh -- the whole layer for decode batches (T <= 16) in one kernel.  With at most
+// 16 tokens each CB byte feeds at most 16 multiply-adds, so the layer is a stream of CB
+// through HBM and the bound is memory bandwidth, not the tensor pipe.
 //
 // Source: "A Gentle Introduction to 8-bit Matrix Multiplication for transformers at
-// scale" (Hugging Face blog), "内部的 MatMul" (int8 product, dequantisation, fp16
-// outlier product); "改进范围" notes that small-batch inference was the slow case.
+// scale" (Hugging Face blog): "LLM.int8() 的总结" (outlier columns, row-wise absmax of the
+// hidden states), "内部的 MatMul" (int8 product, dequantisation by the outer product of
+// the scales, fp16 product of the outlier columns); "改进范围" notes that small-batch
+// inference was the slow case of the original implementation.
 //
-// K-slicing keeps the Xq slice resident in shared memory while a CTA streams many 16-row
-// tiles of CB.  Within one 64-byte step a thread takes 16 contiguous CB bytes of rows g
-// and g+8 and the 16 matching Xq bytes of token g; two m16n8k32 MMAs consume them.  The
-// k order inside the step is permuted identically for A and B, which leaves each dot
-// product unchanged.
+// decode_kernel: one CTA per SM; CTA b works on K-slice b % S (KS bytes of K) and on the
+// 32-row tiles b / S, b / S + G, ... of CB (G CTAs per slice).  Warp roles:
+//
+//   producer (1 thread)  a ring of STAGES 16 KB stages filled by TMA (96 KB in flight per SM
+//                        covers the HBM latency; a deeper ring only lengthens the queues
+//                        every other load waits in): first (forward only)
+//                        all of X in 16 KB pieces, then this slice of every row of X, then
+//                        the CTA's CB tiles, 32 rows x 512 B per stage (2-D boxes of
+//                        32 rows x 256 B).
+//   compute (8 warps)    the prologue, from the X pieces (every CTA reads all of X when it
+//                        fits two stages; otherwise the CTAs split the scan of X, combine
+//                        mask and row maxima in global memory and meet at two grid
+//                        barriers of a cooperative launch):
+//                          step 1: mask bit k = some row has |x| >= threshold, and the
+//                          largest |x| of every (row, 512-column block);
+//                          SCx[t] = max |x| over the non-outlier columns of row t (a block
+//                          free of outlier columns contributes its maximum, the others are
+//                          re-read without them), the ascending outlier list;
+//                          step 2 on the slice rows: Xq = round(x * fl32(127/SCx)) (half
+//                          away from zero), outlier columns 0, into shared memory;
+//                        then per CB stage each warp one 64-byte step of K for all 32 rows
+//                        (mma.sync m16n8k32 s8: two 16-row groups x 8 tokens), copying out
+//                        the CB bytes of the slice's outlier columns as they pass; at a
+//                        tile's end the partials go into one of EW reduction buffers
+//                        (shared-memory integer adds).
+//   epilogue (4 warps)   warp e drains buffer e (the CTA's tiles e, e+4, ...) into the
+//                        tile's slice record in global memory,
+//                          P_s[t,n] = acc_s[t,n] * SCx[t]/127 + sum_{j in slice s}
+//                                     X[t,idx_j] * CB[n,idx_j]          (fp32)
+//                        (the exact int32 acc_s for the raw product), and counts the
+//                        arrival on the tile's counter; the CTA that completes a tile sums
+//                        the S records in slice order and writes
+//                          C[t,n] = fp16((sum_s P_s[t,n]) * SCB[n]/127 + bias[n]).
+//
+// The tile counters and the words of the cooperative prologue carry the launch's epoch in
+// their upper 32 bits: a word of an earlier launch (or uninitialised memory) is claimed
+// afresh by the first update, and every word is put back to (epoch, 0) before the launch
+// ends, so the workspace needs no clearing between calls, graph replays included.
 #pragma once
 
 #include "common.cuh"
@@ -21,15 +54,39 @@
 namespace i8 {
 namespace gemv {
 
-constexpr int WARPS = 8;             // slice lengths are whole multiples of WARPS * 64 bytes
-constexpr int ROWS = 16;          // CB rows per tile (MMA M)
-constexpr int SLICE_TARGET = 3584;  // bytes of K per slice (before rounding)
+constexpr int ROWS = 32;                    // CB rows per tile
+constexpr int CW = 8;                       // compute warps
+constexpr int EW = 4;                       // epilogue warps, one reduction buffer each
+constexpr int PRODUCER = CW;                // warp index of the TMA producer
+constexpr int EPI0 = CW + 1;                // first epilogue warp
+constexpr int THREADS = (CW + 1 + EW) * 32;
+constexpr int PRO_THREADS = (CW + EW) * 32;  // the warps that meet at the prologue's end
+constexpr int SLICE_TARGET = 3584;          // bytes of K per slice (before rounding)
+constexpr int BOXW = 256;                   // bytes of K per TMA box
+constexpr int CH = 64 * CW;                 // bytes of K per stage per row
+constexpr int BOXES = CH / BOXW;            // TMA boxes per stage
+constexpr int STAGES = 6;
+constexpr int STAGE_BYTES = ROWS * CH;      // 16 KB
+constexpr int RP = ROWS + 4;                // token pitch of a reduction buffer (words):
+                                            // the fragment adds fall on distinct banks
+constexpr int MAXO = 128;                   // outlier columns kept in shared memory
+constexpr int MAXOS = 32;                   // outlier columns per slice copied from CB (the
+                                            // rest are read from CB when a tile completes)
+constexpr int XB = 512;                     // columns per block of the prologue's maxima
+constexpr int64_t MAX_K = 65536;            // larger K take the GEMM path
+constexpr int MAX_S = 32;                   // slices at MAX_K: 19
 
+static_assert(CH % BOXW == 0, "whole boxes per stage");
+static_assert(SLICE_TARGET % CH == 0, "slices hold whole stages");
+static_assert(EW == 4, "tile i of a CTA goes to epilogue warp i % 4");
+static_assert(2 * SLICE_TARGET <= STAGE_BYTES, "a slice row of X fits one stage");
+static_assert(XB == 512, "a block is 64 groups of 8 columns: two per lane");
+
+// bytes of K per slice: K split evenly, rounded up to whole stages
 __host__ __device__ inline int64_t slice_bytes(int64_t K) {
-  // rounded to WARPS * 64 so that every warp owns a whole number of 64-byte steps
   const int64_t S = (K + SLICE_TARGET - 1) / SLICE_TARGET;
   const int64_t per = (K + S - 1) / S;
-  return ((per + WARPS * 64 - 1) / (WARPS * 64)) * (WARPS * 64);
+  return ((per + CH - 1) / CH) * CH;
 }
 
 __host__ __device__ inline int64_t num_slices(int64_t K) {
@@ -37,6 +94,82 @@ __host__ __device__ inline int64_t num_slices(int64_t K) {
   return (K + ks - 1) / ks;
 }
 
+// One slice record of a tile in global memory: [T][32 rows] values (a warp's access to one
+// token is 128 contiguous bytes), fp32 partial outputs (forward) or int32 partial sums
+// (raw product).
+__host__ __device__ inline int64_t rec_bytes(int64_t T) { return T * ROWS * 4; }
+
+__host__ __device__ inline int64_t mask_words_smem(int64_t K) {
+  const int64_t a = num_slices(K) * (slice_bytes(K) / 32);
+  const int64_t b = (XB / 32) * ((K + XB - 1) / XB);
+  return (a > b ? a : b) + 2;
+}
+
+// Dynamic shared memory, offsets from a 1024-byte aligned base.
+struct Smem {
+  uint32_t ring, xs, red, cbo, mask, spre, bm, dl, rmx, idx, jinfo, xo, scx, scale, jbase, misc,
+      bars, total;
+};
+
+__host__ __device__ inline uint32_t smem_take(uint32_t& off, uint64_t bytes, uint32_t align) {
+  off = (off + align - 1) / align * align;
+  const uint32_t o = off;
+  off += static_cast<uint32_t>(bytes);
+  return o;
+}
+
+__host__ __device__ inline Smem smem_layout(int NT, int64_t K) {
+  Smem s;
+  uint32_t off = 0;
+  const int TP = NT * 8;                    // token rows held (padded)
+  const int64_t KS = slice_bytes(K);
+  s.ring = smem_take(off, static_cast<uint64_t>(STAGES) * STAGE_BYTES, 1024);
+  s.xs = smem_take(off, static_cast<uint64_t>(TP) * (KS + 16), 16);
+  s.red = smem_take(off, static_cast<uint64_t>(EW) * TP * RP * 4, 16);
+  s.cbo = smem_take(off, static_cast<uint64_t>(EW) * MAXOS * ROWS, 16);
+  s.mask = smem_take(off, static_cast<uint64_t>(mask_words_smem(K)) * 4, 16);
+  s.spre = smem_take(off, static_cast<uint64_t>(KS / 32) * 4, 16);
+  s.bm = smem_take(off, static_cast<uint64_t>(TP) * ((K + XB - 1) / XB) * 4, 16);
+  s.dl = smem_take(off, static_cast<uint64_t>((K + XB - 1) / XB) * 4, 16);
+  s.rmx = smem_take(off, TP * 4, 16);
+  s.idx = smem_take(off, MAXO * 4, 16);
+  s.jinfo = smem_take(off, MAXO * 4, 16);
+  s.xo = smem_take(off, static_cast<uint64_t>(TP) * MAXO * 2, 16);
+  s.scx = smem_take(off, TP * 4, 16);
+  s.scale = smem_take(off, TP * 4, 16);
+  s.jbase = smem_take(off, (MAX_S + 1) * 4, 16);
+  s.misc = smem_take(off, 16, 16);
+  s.bars = smem_take(off, (2 * STAGES + 2 * EW + 1) * 8, 16);
+  s.total = off;
+  return s;
+}
+
+// bytes of dynamic shared memory to request (the base is aligned up to 1024 in-kernel)
+__host__ inline size_t smem_bytes(int NT, int64_t K) { return smem_layout(NT, K).total + 1024; }
+
+struct Args {
+  const __half* X;           // forward: hidden states [T, K]
+  const int8_t* Xq;          // raw product (i8_igemm_s32): codes [T, K]
+  int T;
+  int64_t N, K;
+  float thr;
+  const int8_t* CB;          // [N, K] (outlier bytes beyond the copied ones are read here)
+  const float* SCB;          // [N]
+  const __half* bias;        // [N] or NULL
+  __half* C;                 // forward output [T, N]
+  int32_t* acc;              // raw output [T, N]
+  uint8_t* rec;              // [n_tiles][S][T][32] slice records (fp32 or int32)
+  unsigned long long* cnt;   // [n_tiles] arrival counters (epoch << 32 | arrivals)
+  unsigned long long epoch;  // this launch's epoch, 1 .. 2^32 - 1
+  uint64_t lim;              // bound of every wait, ns
+  // cooperative prologue (larger X): the CTAs split the scan of X and meet at two grid
+  // barriers; the words carry the epoch in their upper 32 bits
+  bool coop;
+  unsigned long long* gmask;  // [ceil(K/32)] outlier mask words
+  unsigned long long* gscx;   // [T] row maxima (fp32 bit patterns)
+  unsigned long long* gbar;   // [3] barrier counters (epoch << 32 | arrivals)
+  int8_t* xq;                 // [T, K] codes, written in shares and read back per slice
+};
 
 __device__ __forceinline__ void mma_s8_16816(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                              uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -47,69 +180,567 @@ __device__ __forceinline__ void mma_s8_16816(int (&c)[4], uint32_t a0, uint32_t 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Decode kernels (steps 4, 5 and 6 for T <= 16), two launches after the fused prepare.
-//
-// gemv_stream_kernel: warp CW (one thread) streams CB through a ring of STAGES stages,
-// each 16 rows x CH bytes of K, loaded as 2-D TMA boxes of 256 B x 16 rows (no swizzle:
-// the widest box TMA takes, which streams HBM best -- ~6 TB/s measured on B200 for this
-// layout).  The CW compute warps each own one 64-byte MMA step of every stage and
-// accumulate, over the tile's stages of their CTA's K-slice,
-//   P[slice][t][n] = sum_{k in slice} Xq[t,k] * CB[n,k]     (int32, mma.sync m16n8k32)
-// in registers; at the tile's end the warps' partials are reduced in a fixed order.
-// The loop carries nothing but the int8 product: the outlier columns are a handful, and
-// any per-column work inside it lands on the same warp in every tile and holds up the
-// tile-end barrier.
-//
-// gemv_finalize_kernel: one thread per output channel n and group of TG tokens sums the
-// slice partials (exact int32) and gathers the n_o outlier bytes CB[n, idx[j]] once,
-// applying each to the group's tokens (fp32), then writes
-//   C[t,n] = fp16((P[t,n] * SCx[t]/127 + sum_j X_o[t,j] * CB[n,idx[j]]) * SCB[n]/127 + bias[n]).
-constexpr int BOXW = 256;                   // bytes of K per TMA box
-constexpr int CW = 8;                       // compute warps, one 64-byte step each
-constexpr int STREAM_THREADS = (CW + 1) * 32;
-constexpr int CH = 64 * CW;                 // bytes of K per stage per row
-constexpr int BOXES = CH / BOXW;            // TMA boxes per stage
-constexpr int STAGES = 16;
-constexpr int STAGE_BYTES = ROWS * CH;      // 8 KB
-constexpr int RP = ROWS + 4;                // row pitch of the reduction buffer (in words):
-                                            // fragment stores and the row-fastest reads
-                                            // then fall on (nearly) distinct banks
-constexpr int TG = 4;                       // tokens per finalize thread
-constexpr int FIN_THREADS = 128;
-
-static_assert(CH % BOXW == 0, "whole boxes per stage");
-static_assert(SLICE_TARGET % CH == 0 && (WARPS * 64) % CH == 0, "slices hold whole stages");
-
-__host__ inline size_t stream_smem_bytes(int nt, int64_t K) {
-  return 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES +
-         static_cast<size_t>(nt * 8) * static_cast<size_t>(slice_bytes(K) + 16) +
-         static_cast<size_t>(CW) * RP * nt * 8 * 4 + 2 * STAGES * 8;
+__device__ __forceinline__ void all_sync() {   // compute + epilogue warps
+  asm volatile("bar.sync 1, %0;" ::"n"(PRO_THREADS) : "memory");
 }
 
+__device__ __forceinline__ void compute_sync() {   // compute warps
+  asm volatile("bar.sync 2, %0;" ::"n"(CW * 32) : "memory");
+}
+
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
+// max |x| of 8 fp16 values as the bit pattern of the fp16 absolute value (the patterns of
+// non-negative fp16 numbers order like the numbers)
+__device__ __forceinline__ uint32_t absmax8_bits(const uint4 v) {
+  const __half2 a = __habs2(*reinterpret_cast<const __half2*>(&v.x));
+  const __half2 b = __habs2(*reinterpret_cast<const __half2*>(&v.y));
+  const __half2 c = __habs2(*reinterpret_cast<const __half2*>(&v.z));
+  const __half2 d = __habs2(*reinterpret_cast<const __half2*>(&v.w));
+  const __half2 m = __hmax2(__hmax2(a, b), __hmax2(c, d));
+  const uint32_t u = *reinterpret_cast<const uint32_t*>(&m);
+  const uint32_t lo = u & 0xffffu, hi = u >> 16;
+  return lo > hi ? lo : hi;
+}
+
+__device__ __forceinline__ float half_bits_to_float(uint32_t b) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(b)));
+}
+
+// Epoch-tagged words: the upper 32 bits hold the epoch of the launch that last claimed the
+// word, and a word of another epoch reads as zero.  The first update in a launch claims
+// the word with one compare-and-swap (a late claim finds it changed and fails harmlessly),
+// after which plain atomics apply -- no retry loops, however many CTAs update it.
+__device__ __forceinline__ void tag_claim(unsigned long long* w, uint32_t e) {
+  const unsigned long long v = __ldcg(w);
+  if (static_cast<uint32_t>(v >> 32) != e) atomicCAS(w, v, static_cast<unsigned long long>(e) << 32);
+}
+
+__device__ __forceinline__ uint32_t tagged_get(const unsigned long long* w, uint32_t e) {
+  const unsigned long long v = __ldcg(w);
+  return static_cast<uint32_t>(v >> 32) == e ? static_cast<uint32_t>(v) : 0u;
+}
+
+// Arrival on a tile counter: the number of arrivals of this epoch including this one.
+__device__ __forceinline__ int tile_arrive(unsigned long long* c, uint32_t e) {
+  tag_claim(c, e);
+  return static_cast<int>(static_cast<uint32_t>(atomicAdd(c, 1ull))) + 1;
+}
+
+// Grid barrier of the cooperative launch (one thread per CTA).  The counter only grows
+// within an epoch (a replay of the same launch starts the next generation of `target`
+// arrivals).  Bounded: false after `lim` ns (the error word records it).
+__device__ __forceinline__ bool grid_sync(unsigned long long* ctr, uint32_t e, uint32_t target,
+                                          uint64_t lim) {
+  fence_acq_rel_gpu();  // this CTA's writes before its arrival
+  tag_claim(ctr, e);
+  const uint32_t c = static_cast<uint32_t>(atomicAdd(ctr, 1ull));
+  const uint32_t goal = (c / target + 1) * target;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    const unsigned long long v = __ldcg(ctr);
+    if (static_cast<uint32_t>(v >> 32) == e && static_cast<uint32_t>(v) >= goal) break;
+    if ((it & 15u) == 15u && globaltimer_ns() - t0 > lim) {
+      raise_error(kErrWaitTimeout);
+      return false;
+    }
+  }
+  fence_acq_rel_gpu();
+  return true;
+}
+
+// Consumer side of the ring: wait for stage s (phase ph), then advance.
+struct Ring {
+  uint32_t full, empty;  // shared addresses of the first full / empty barrier
+  int s = 0;
+  uint32_t ph = 0;
+  __device__ __forceinline__ uint32_t full_bar() const { return full + 8u * s; }
+  __device__ __forceinline__ uint32_t empty_bar() const { return empty + 8u * s; }
+  __device__ __forceinline__ void advance() {
+    if (++s == STAGES) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+};
+
+// ---------------------------------------------------------------------- forward prologue
+// Run by the compute warps (ct = thread index among them).  Consumes the X stages of the
+// ring in the producer's order: (unless a.coop) the ceil(2TK / STAGE_BYTES) pieces of the
+// flat X starting at piece blockIdx.x (mod their count), then the T slice rows starting at
+// row blockIdx.x / S (mod T) -- the CTAs start at different places, which spreads their
+// reads of X over the L2 slices.  Leaves the slice of Xq in xs, the mask, ranks, SCx and
+// the outlier tables in shared memory.  Returns false when a wait gave up.
 template <int NT>
-__global__ void __launch_bounds__(STREAM_THREADS, 1)
-    gemv_stream_kernel(const __grid_constant__ CUtensorMap tmCB, const int8_t* __restrict__ Xq,
-                       int T, int64_t N, int64_t K, int32_t* __restrict__ P, uint64_t lim) {
+__device__ __forceinline__ bool forward_prologue(
+    const Args& a, const int ct, const int slice, const int64_t KS, const int S, Ring& rg,
+    const uint8_t* ring_p, uint8_t* xs, const int64_t pitch, uint32_t* maskall, int32_t* spre,
+    uint32_t* bm, int32_t* dl, uint32_t* rmx, int32_t* idx_s, uint32_t* jinfo, __half* xo_s,
+    float* scx, float* scale, int32_t* jbase, int* misc, uint64_t* xq_bar,
+    volatile int* abort_flag) {
+  const int T = a.T;
+  const int64_t K = a.K;
+  const __half* __restrict__ X = a.X;
+  const float thr = a.thr;
+  const int64_t KW = (K + 31) / 32;
+  const int64_t NBK = (K + XB - 1) / XB;
+  const int64_t G = K / 8;  // 16-byte groups of 8 columns per row
+  const int w = ct >> 5, lane = ct & 31;
+  constexpr int GPB = XB / 8;  // groups per block
+
+  bool ok = true;
+  if (!a.coop) {
+    // (a) step 1 and the block maxima, piece by piece
+    const int64_t xbytes = static_cast<int64_t>(T) * K * 2;
+    const int64_t pieces = (xbytes + STAGE_BYTES - 1) / STAGE_BYTES;
+    for (int64_t pc = 0; pc < pieces; ++pc) {
+      if (ok) {
+        const bool got = mbar_wait(rg.full_bar(), rg.ph, abort_flag, a.lim);
+        ok = __all_sync(0xffffffffu, got);
+      }
+      if (ok) {
+        const int p = static_cast<int>((pc + blockIdx.x) % pieces);
+        const uint4* sp = reinterpret_cast<const uint4*>(ring_p + rg.s * STAGE_BYTES);
+        const int64_t left = xbytes - static_cast<int64_t>(p) * STAGE_BYTES;
+        const int nvec = static_cast<int>(min(static_cast<int64_t>(STAGE_BYTES), left) / 16);
+        const int Gi = static_cast<int>(G);
+        if ((Gi & 31) == 0) {
+          // the 32 groups of a warp lie in one row and one block (rows are whole multiples
+          // of 32 groups, blocks of 64)
+          for (int i0 = w * 32; i0 < nvec; i0 += CW * 32) {
+            const int f0 = p * (STAGE_BYTES / 16) + i0;  // flat group index of lane 0
+            const int t = f0 / Gi;
+            const int g = f0 - t * Gi + lane;
+            const uint4 v = sp[i0 + lane];
+            const uint32_t m = absmax8_bits(v);
+            if (half_bits_to_float(m) >= thr) {  // rare: an outlier in this group
+              const uint32_t bits = outlier_bits8(v, thr);
+              if (bits) atomicOr(&maskall[g >> 2], bits << (8 * (g & 3)));
+            }
+            const uint32_t mx = __reduce_max_sync(0xffffffffu, m);
+            if (lane == 0) atomicMax(&bm[t * NBK + g / GPB], mx);
+          }
+        } else {
+          for (int i0 = w * 32; i0 < nvec; i0 += CW * 32) {
+            const int i = i0 + lane;
+            const bool valid = i < nvec;
+            uint32_t m = 0u, key = 0xffffffffu;
+            if (valid) {
+              const uint4 v = sp[i];
+              const int gf = p * (STAGE_BYTES / 16) + i;  // group index in the flat X
+              const int t = gf / Gi, g = gf - t * Gi;
+              m = absmax8_bits(v);
+              if (half_bits_to_float(m) >= thr) {
+                const uint32_t bits = outlier_bits8(v, thr);
+                if (bits) atomicOr(&maskall[g >> 2], bits << (8 * (g & 3)));
+              }
+              key = static_cast<uint32_t>(t * NBK + g / GPB);
+            }
+            const uint32_t peers = __match_any_sync(0xffffffffu, key);
+            const uint32_t mx = __reduce_max_sync(peers, m);
+            if (valid && lane == __ffs(peers) - 1) atomicMax(&bm[key], mx);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(rg.empty_bar());
+      }
+      rg.advance();
+    }
+    compute_sync();
+
+  } else {
+    // (a') the CTAs split X into shares of 16-byte groups.  Step 1: each ORs the outlier
+    // bits of its share into the global mask; grid barrier; each takes the masked maxima
+    // of its share into the global row maxima; grid barrier; step 2 on its share into the
+    // global codes; grid barrier; then this CTA's slice of the codes is copied into xs.
+    const uint32_t e = static_cast<uint32_t>(a.epoch);
+    const int64_t TG = static_cast<int64_t>(T) * G;
+    const int64_t f_lo = TG * blockIdx.x / gridDim.x, f_hi = TG * (blockIdx.x + 1) / gridDim.x;
+    for (int64_t f = f_lo + ct; f < f_hi; f += CW * 32) {
+      const int64_t t = f / G, g = f - t * G;
+      const uint4 v = ldg_v4(X + t * K + g * 8);
+      if (half_bits_to_float(absmax8_bits(v)) >= thr) {
+        const uint32_t bits = outlier_bits8(v, thr);
+        if (bits) {
+          tag_claim(a.gmask + (g >> 2), e);
+          atomicOr(a.gmask + (g >> 2), static_cast<unsigned long long>(bits << (8 * (g & 3))));
+        }
+      }
+    }
+    compute_sync();
+    if (ct == 0 && !grid_sync(a.gbar, e, gridDim.x, a.lim)) *abort_flag = 1;
+    compute_sync();
+    ok = *abort_flag == 0;
+    for (int64_t x = ct; x < KW; x += CW * 32) maskall[x] = ok ? tagged_get(a.gmask + x, e) : 0u;
+    compute_sync();
+    for (int64_t f = f_lo + ct; f < f_hi && ok; f += CW * 32) {
+      const int64_t t = f / G, g = f - t * G;
+      const uint4 v = ldg_v4(X + t * K + g * 8);
+      const uint32_t skip = (maskall[g >> 2] >> (8 * (g & 3))) & 0xffu;
+      atomicMax(&rmx[t], __float_as_uint(absmax8(v, skip)));
+    }
+    compute_sync();
+    for (int t = ct; t < T && ok; t += CW * 32) {
+      if (rmx[t] != 0u) {
+        tag_claim(a.gscx + t, e);
+        atomicMax(a.gscx + t, (static_cast<unsigned long long>(e) << 32) | rmx[t]);
+      }
+    }
+    compute_sync();
+    if (ct == 0 && ok && !grid_sync(a.gbar + 1, e, gridDim.x, a.lim)) *abort_flag = 1;
+    compute_sync();
+    ok = *abort_flag == 0;
+    for (int t = ct; t < T; t += CW * 32) {
+      const float m = ok ? __uint_as_float(tagged_get(a.gscx + t, e)) : 0.0f;
+      scx[t] = m;
+      scale[t] = m > 0.0f ? __fdiv_rn(127.0f, m) : 0.0f;
+    }
+    compute_sync();
+    for (int64_t f = f_lo + ct; f < f_hi && ok; f += CW * 32) {
+      const int64_t t = f / G, g = f - t * G;
+      const uint4 v = ldg_v4(X + t * K + g * 8);
+      const uint32_t skip = (maskall[g >> 2] >> (8 * (g & 3))) & 0xffu;
+      *reinterpret_cast<uint2*>(a.xq + t * K + g * 8) = codes8(v, skip, scale[t]);
+    }
+    // the codes are read back by TMA (the async proxy) in other CTAs
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    compute_sync();
+    if (ct == 0 && ok && !grid_sync(a.gbar + 2, e, gridDim.x, a.lim)) *abort_flag = 1;
+    if (ct == 0 && *abort_flag == 0) {
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      const int64_t k0 = static_cast<int64_t>(slice) * KS;
+      const int64_t klen = KS < K - k0 ? KS : K - k0;
+      mbar_arrive_expect_tx(smem_u32(xq_bar), static_cast<uint32_t>(T * klen));
+      for (int t = 0; t < T; ++t)
+        bulk_load(smem_u32(xs + t * pitch), a.xq + static_cast<int64_t>(t) * K + k0,
+                  static_cast<uint32_t>(klen), smem_u32(xq_bar));
+      // every CTA has read the mask and row maxima: CTA 0 puts them back to (epoch, 0)
+      if (blockIdx.x == 0) {
+        for (int64_t x = 0; x < KW; ++x) a.gmask[x] = static_cast<unsigned long long>(e) << 32;
+        for (int t = 0; t < T; ++t) a.gscx[t] = static_cast<unsigned long long>(e) << 32;
+      }
+    }
+    compute_sync();
+    ok = *abort_flag == 0;
+  }
+
+  // (b) ranks (warp 0: lane l takes a contiguous run of mask words)
+  const int WPS = static_cast<int>(KS / 32);  // mask words per slice
+  if (w == 0) {
+    const int KWi = static_cast<int>(KW);
+    const int cw = (KWi + 31) / 32;
+    const int wb = lane * cw;
+    const int we = wb + cw < KWi ? wb + cw : KWi;
+    int cnt = 0;
+    for (int x = wb; x < we; ++x) cnt += __popc(maskall[x]);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - cnt;
+    int nb = (wb + WPS - 1) / WPS * WPS;  // next slice boundary at or after wb
+    const int sw0 = slice * WPS;
+    for (int x = wb; x < we; ++x) {
+      if (x == nb) {
+        jbase[x / WPS] = run;
+        nb += WPS;
+      }
+      if (x >= sw0 && x < sw0 + WPS) spre[x - sw0] = run;
+      uint32_t bits = maskall[x];
+      while (bits) {
+        const int bpos = __ffs(bits) - 1;
+        bits &= bits - 1u;
+        if (run < MAXO) idx_s[run] = x * 32 + bpos;
+        ++run;
+      }
+    }
+    if (lane == 31) {
+      misc[0] = run;  // n_o
+      jbase[S] = run;
+    }
+  }
+  compute_sync();
+
+  // (c) the row scales, where each kept outlier column is found in the epilogue, and its
+  // X values
+  const int n_o = misc[0];
+  const int nf = n_o < MAXO ? n_o : MAXO;
+  // jinfo[j]: 0 when the CTAs of column idx_j's slice copy its CB bytes (rank below MAXOS
+  // in the slice), else 0x80000000 | idx_j (read from CB when the tile completes)
+  for (int j = ct; j < nf; j += CW * 32) {
+    const int c = idx_s[j];
+    const int jl = j - jbase[c / static_cast<int>(KS)];
+    jinfo[j] = jl < MAXOS ? 0u : (0x80000000u | static_cast<uint32_t>(c));
+  }
+  for (int i = ct; i < T * nf; i += CW * 32) {
+    const int t = i / nf, j = i - t * nf;
+    xo_s[t * MAXO + j] = X[static_cast<int64_t>(t) * K + idx_s[j]];
+  }
+  if (!a.coop) {
+    // blocks holding outlier columns (warp 1 lists them); the other blocks give their
+    // maxima from (a)
+    if (w == 1) {
+      int nd = 0;
+      for (int64_t b0 = 0; b0 < NBK; b0 += 32) {
+        const int64_t b = b0 + lane;
+        uint32_t o = 0u;
+        if (b < NBK) {
+#pragma unroll
+          for (int i = 0; i < XB / 32; ++i) o |= maskall[b * (XB / 32) + i];
+        }
+        const uint32_t db = __ballot_sync(0xffffffffu, o != 0u);
+        if (o != 0u) dl[nd + __popc(db & ((1u << lane) - 1u))] = static_cast<int32_t>(b);
+        nd += __popc(db);
+      }
+      if (lane == 0) misc[2] = nd;
+    }
+    for (int t = w; t < T; t += CW) {
+      float m = 0.0f;
+      for (int64_t b0 = 0; b0 < NBK; b0 += 32) {
+        const int64_t b = b0 + lane;
+        if (b < NBK) {
+          uint32_t o = 0u;
+#pragma unroll
+          for (int i = 0; i < XB / 32; ++i) o |= maskall[b * (XB / 32) + i];
+          if (o == 0u) m = fmaxf(m, half_bits_to_float(bm[t * NBK + b]));
+        }
+      }
+      m = warp_max(m);
+      if (lane == 0) rmx[t] = __float_as_uint(m);
+    }
+    compute_sync();
+    // the blocks holding outlier columns, re-read from X without them: a warp takes
+    // (row, block) pairs, two groups of 8 columns per lane, four pairs' loads in flight
+    {
+      const int nd = misc[2];
+      const int pairs = T * nd;
+      constexpr int U = 4;
+      for (int q0 = w; q0 < pairs; q0 += CW * U) {
+        uint4 v[U][2];
+        uint32_t sk[U][2];
+        int tt[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int q = q0 + u * CW;
+          tt[u] = 0;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            v[u][h] = make_uint4(0u, 0u, 0u, 0u);
+            sk[u][h] = 0xffu;
+          }
+          if (q < pairs) {
+            const int t = q / nd, d = q - t * nd;
+            tt[u] = t;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int64_t g = static_cast<int64_t>(dl[d]) * GPB + h * 32 + lane;
+              if (g < G) {
+                v[u][h] = ldg_v4(X + static_cast<int64_t>(t) * K + g * 8);
+                sk[u][h] = (maskall[g >> 2] >> (8 * (g & 3))) & 0xffu;
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          if (q0 + u * CW < pairs) {  // uniform over the warp
+            const float m = fmaxf(absmax8(v[u][0], sk[u][0]), absmax8(v[u][1], sk[u][1]));
+            const uint32_t mm = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
+            if (lane == 0) atomicMax(&rmx[tt[u]], mm);
+          }
+        }
+      }
+    }
+  }
+  compute_sync();
+  if (!a.coop) {  // (the cooperative path has SCx from (a'))
+    for (int t = ct; t < T; t += CW * 32) {
+      const float m = __uint_as_float(rmx[t]);
+      scx[t] = m;
+      scale[t] = m > 0.0f ? __fdiv_rn(127.0f, m) : 0.0f;
+    }
+  }
+  compute_sync();
+
+  // (d) step 2 on this slice: one ring stage per row of X (the cooperative path has its
+  // codes from (a') already)
+  if (!a.coop) {
+    const int64_t k0 = static_cast<int64_t>(slice) * KS;
+    const int64_t klen = KS < K - k0 ? KS : K - k0;
+    const int64_t gl = klen / 8;
+    for (int tt = 0; tt < T; ++tt) {
+      const int t = static_cast<int>((tt + blockIdx.x / S) % T);
+      if (ok) {
+        const bool got = mbar_wait(rg.full_bar(), rg.ph, abort_flag, a.lim);
+        ok = __all_sync(0xffffffffu, got);
+      }
+      if (ok) {
+        const uint4* sp = reinterpret_cast<const uint4*>(ring_p + rg.s * STAGE_BYTES);
+        const float sc = scale[t];
+        for (int64_t i = ct; i < gl; i += CW * 32) {
+          const int64_t g = k0 / 8 + i;
+          const uint32_t skip = (maskall[g >> 2] >> (8 * (g & 3))) & 0xffu;
+          *reinterpret_cast<uint2*>(xs + t * pitch + i * 8) = codes8(sp[i], skip, sc);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(rg.empty_bar());
+      }
+      rg.advance();
+    }
+  }
+  return ok;
+}
+
+// ---------------------------------------------------------------------- tile completion
+// Run by the epilogue warp of the CTA whose arrival completed `tile`: sums the S slice
+// records in slice order and writes the raw int32 sums (kRaw) or the fp16 output, adding
+// the outlier columns whose CB bytes no slice copied.  Lane r owns output channel
+// tile * 32 + r, all tokens.
+template <int NT, bool kRaw>
+__device__ __forceinline__ void finish_tile(const Args& a, const int64_t tile, const int S,
+                                            const int rb, const uint32_t* maskall,
+                                            const int32_t* idx_s, const uint32_t* jinfo,
+                                            const __half* xo_s, const int* misc) {
+  constexpr int TP = NT * 8;
+  const int lane = threadIdx.x & 31;
+  const int T = a.T;
+  const int64_t N = a.N, K = a.K;
+  const int64_t n = tile * ROWS + lane;
+  const uint8_t* tb = a.rec + tile * S * rb + lane * 4;  // this row in slice 0's record
+  if constexpr (kRaw) {
+    int32_t acc[TP];
+#pragma unroll
+    for (int t = 0; t < TP; ++t) acc[t] = 0;
+    for (int sp = 0; sp < S; sp += 2) {  // two records' loads in flight at a time
+      const int32_t* p0 = reinterpret_cast<const int32_t*>(tb + static_cast<int64_t>(sp) * rb);
+      const int32_t* p1 = reinterpret_cast<const int32_t*>(tb + static_cast<int64_t>(sp + 1) * rb);
+      const bool two = sp + 1 < S;
+      int32_t v0[TP], v1[TP];
+#pragma unroll
+      for (int t = 0; t < TP; ++t) {
+        v0[t] = t < T ? __ldcg(p0 + t * ROWS) : 0;
+        v1[t] = (two && t < T) ? __ldcg(p1 + t * ROWS) : 0;
+      }
+#pragma unroll
+      for (int t = 0; t < TP; ++t) acc[t] += v0[t] + v1[t];
+    }
+    if (n < N) {
+#pragma unroll
+      for (int t = 0; t < TP; ++t)
+        if (t < T) a.acc[static_cast<int64_t>(t) * N + n] = acc[t];
+    }
+  } else {
+    float ws = 0.0f, bn = 0.0f;
+    if (n < N) {
+      ws = __ldg(a.SCB + n) * (1.0f / 127.0f);
+      bn = a.bias ? __half2float(a.bias[n]) : 0.0f;
+    }
+    float part[TP];
+#pragma unroll
+    for (int t = 0; t < TP; ++t) part[t] = 0.0f;
+    for (int sp = 0; sp < S; sp += 2) {
+      const float* p0 = reinterpret_cast<const float*>(tb + static_cast<int64_t>(sp) * rb);
+      const float* p1 = reinterpret_cast<const float*>(tb + static_cast<int64_t>(sp + 1) * rb);
+      const bool two = sp + 1 < S;
+      float v0[TP], v1[TP];
+#pragma unroll
+      for (int t = 0; t < TP; ++t) {
+        v0[t] = t < T ? __ldcg(p0 + t * ROWS) : 0.0f;
+        v1[t] = (two && t < T) ? __ldcg(p1 + t * ROWS) : 0.0f;
+      }
+#pragma unroll
+      for (int t = 0; t < TP; ++t) part[t] = (part[t] + v0[t]) + v1[t];
+    }
+    // outlier columns whose CB bytes were not copied: the first MAXO through jinfo, the
+    // rest by walking the mask from the column after the last kept index
+    const int n_o = misc[0];
+    const int nf = n_o < MAXO ? n_o : MAXO;
+    for (int j = 0; j < nf; ++j) {
+      const uint32_t inf = jinfo[j];
+      if (inf != 0u) {
+        const float cb =
+            n < N ? static_cast<float>(__ldg(a.CB + n * K + (inf & 0x7fffffffu))) : 0.0f;
+#pragma unroll
+        for (int t = 0; t < TP; ++t)
+          if (t < T) part[t] = fmaf(__half2float(xo_s[t * MAXO + j]), cb, part[t]);
+      }
+    }
+    if (n_o > MAXO) {
+      const int64_t KW = (K + 31) / 32;
+      const int c0 = idx_s[MAXO - 1];
+      int64_t w = c0 >> 5;
+      uint32_t bits = (c0 & 31) == 31 ? 0u : (maskall[w] & ~((2u << (c0 & 31)) - 1u));
+      while (true) {
+        while (bits == 0u && w + 1 < KW) bits = maskall[++w];
+        if (bits == 0u) break;
+        const int bp = __ffs(bits) - 1;
+        bits &= bits - 1u;
+        const int64_t col = w * 32 + bp;
+        const float cb = n < N ? static_cast<float>(__ldg(a.CB + n * K + col)) : 0.0f;
+#pragma unroll
+        for (int t = 0; t < TP; ++t)
+          if (t < T)
+            part[t] = fmaf(__half2float(a.X[static_cast<int64_t>(t) * K + col]), cb, part[t]);
+      }
+    }
+    if (n < N) {
+#pragma unroll
+      for (int t = 0; t < TP; ++t)
+        if (t < T) a.C[static_cast<int64_t>(t) * N + n] = __float2half_rn(fmaf(part[t], ws, bn));
+    }
+  }
+}
+
+// ---------------------------------------------------------------------- the kernel
+// kRaw: the int8 product of given codes (a.Xq) written as int32 (a.acc); otherwise the
+// forward from a.X to a.C.  Launched with one CTA per SM, a multiple of S CTAs.
+template <int NT, bool kRaw>
+__global__ void __launch_bounds__(THREADS, 1)
+    decode_kernel(const __grid_constant__ CUtensorMap tmCB, const Args a) {
+  constexpr int TP = NT * 8;
   extern __shared__ uint8_t smraw[];
   const uint32_t raw_s = smem_u32(smraw);
   const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
   uint8_t* sm = smraw + pad;
-  const uint32_t ring = raw_s + pad;
+  const int T = a.T;
+  const int64_t N = a.N, K = a.K;
+  const Smem L = smem_layout(NT, K);
   const int64_t KS = slice_bytes(K);
   const int S = static_cast<int>(num_slices(K));
   const int64_t pitch = KS + 16;
-  uint8_t* xs = sm + static_cast<size_t>(STAGES) * STAGE_BYTES;
-  int32_t* red = reinterpret_cast<int32_t*>(xs + NT * 8 * pitch);
-  uint64_t* full = reinterpret_cast<uint64_t*>(red + CW * RP * NT * 8);
+  const uint32_t ring = raw_s + pad + L.ring;
+  const uint8_t* ring_p = sm + L.ring;
+  uint8_t* xs = sm + L.xs;
+  int32_t* red = reinterpret_cast<int32_t*>(sm + L.red);
+  uint8_t* cbo = sm + L.cbo;
+  uint32_t* maskall = reinterpret_cast<uint32_t*>(sm + L.mask);
+  int32_t* spre = reinterpret_cast<int32_t*>(sm + L.spre);
+  uint32_t* bm = reinterpret_cast<uint32_t*>(sm + L.bm);
+  int32_t* dl = reinterpret_cast<int32_t*>(sm + L.dl);
+  uint32_t* rmx = reinterpret_cast<uint32_t*>(sm + L.rmx);
+  int32_t* idx_s = reinterpret_cast<int32_t*>(sm + L.idx);
+  uint32_t* jinfo = reinterpret_cast<uint32_t*>(sm + L.jinfo);
+  __half* xo_s = reinterpret_cast<__half*>(sm + L.xo);
+  float* scx = reinterpret_cast<float*>(sm + L.scx);
+  float* scale = reinterpret_cast<float*>(sm + L.scale);
+  int32_t* jbase = reinterpret_cast<int32_t*>(sm + L.jbase);
+  int* misc = reinterpret_cast<int*>(sm + L.misc);  // [0] n_o, [1] abort flag, [2] scratch
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bars);
   uint64_t* empty = full + STAGES;
-  __shared__ int s_abort;
+  uint64_t* rfull = empty + STAGES;
+  uint64_t* rempty = rfull + EW;
+  uint64_t* xq_bar = rempty + EW;  // raw mode: the code rows have landed in xs
 
-  const int slice = blockIdx.x % S;
-  const int cta_in_slice = blockIdx.x / S;
+  const int slice = static_cast<int>(blockIdx.x % S);
+  const int cta_in_slice = static_cast<int>(blockIdx.x / S);
   const int ctas_in_slice = (static_cast<int>(gridDim.x) - slice + S - 1) / S;
   const int64_t k0 = static_cast<int64_t>(slice) * KS;
-  const int64_t klen = min(KS, K - k0);
-  const int spt = static_cast<int>((klen + CH - 1) / CH);   // stages per tile
+  const int64_t klen = KS < K - k0 ? KS : K - k0;
+  const int spt = static_cast<int>((klen + CH - 1) / CH);  // stages per tile
   const int64_t n_tiles = (N + ROWS - 1) / ROWS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -118,50 +749,88 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1)
       mbar_init(smem_u32(full + i), 1);
       mbar_init(smem_u32(empty + i), CW);
     }
-    s_abort = 0;
+    for (int i = 0; i < EW; ++i) {
+      mbar_init(smem_u32(rfull + i), CW);
+      mbar_init(smem_u32(rempty + i), 1);
+    }
+    mbar_init(smem_u32(xq_bar), 1);
+    misc[0] = 0;
+    misc[1] = 0;
     fence_mbar_init();
   }
-  if (warp == CW && lane == 0) tma_prefetch_desc(&tmCB);
-  grid_dep_wait();    // Xq comes from the previous kernel
-  grid_dep_launch();  // the finalize kernel may start launching
-  // stage Xq[:, k0 : k0+KS] (tokens >= T and columns >= K are zero)
-  const int64_t vec_per_row = KS / 16;
-  for (int64_t i = threadIdx.x; i < NT * 8 * vec_per_row; i += STREAM_THREADS) {
-    const int tok = static_cast<int>(i / vec_per_row);
-    const int64_t c16 = i - tok * vec_per_row;
-    const int64_t k = k0 + c16 * 16;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (tok < T && k < K) v = ldg_v4(Xq + static_cast<int64_t>(tok) * K + k);
-    *reinterpret_cast<uint4*>(xs + tok * pitch + c16 * 16) = v;
-  }
   __syncthreads();
-  volatile int* abort_flag = &s_abort;
+  volatile int* abort_flag = misc + 1;
 
-  if (warp == CW) {
+  if (warp == PRODUCER) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      tma_prefetch_desc(&tmCB);
       int s = 0;
       uint32_t ph = 0;
       uint32_t issued = 0;
       bool ok = true;
-      for (int64_t tile = cta_in_slice; tile < n_tiles && ok; tile += ctas_in_slice) {
-        const int y = static_cast<int>(tile * ROWS);
-        for (int st = 0; st < spt; ++st) {
-          if (!mbar_wait(smem_u32(empty + s), ph ^ 1u, abort_flag, lim)) {
+      // one ring stage per copy: wait until it is free, arm it, return its full barrier
+      auto acquire = [&](uint32_t bytes) -> uint32_t {
+        if (!mbar_wait(smem_u32(empty + s), ph ^ 1u, abort_flag, a.lim)) return 0u;
+        const uint32_t fb = smem_u32(full + s);
+        mbar_arrive_expect_tx(fb, bytes);
+        return fb;
+      };
+      auto advance = [&]() {
+        ++issued;
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      };
+      grid_dep_wait();  // X (or the codes) may come from the previous kernel
+      if constexpr (kRaw) {
+        // this slice of the code rows straight into xs
+        mbar_arrive_expect_tx(smem_u32(xq_bar), static_cast<uint32_t>(T * klen));
+        for (int t = 0; t < T; ++t)
+          bulk_load(smem_u32(xs + t * pitch), a.Xq + static_cast<int64_t>(t) * K + k0,
+                    static_cast<uint32_t>(klen), smem_u32(xq_bar));
+      } else {
+        const uint8_t* xb = reinterpret_cast<const uint8_t*>(a.X);
+        const int64_t xbytes = static_cast<int64_t>(T) * K * 2;
+        const int64_t pieces = a.coop ? 0 : (xbytes + STAGE_BYTES - 1) / STAGE_BYTES;
+        for (int64_t pc = 0; pc < pieces && ok; ++pc) {
+          const int64_t off = ((pc + blockIdx.x) % pieces) * STAGE_BYTES;
+          const uint32_t bytes =
+              static_cast<uint32_t>(min(static_cast<int64_t>(STAGE_BYTES), xbytes - off));
+          const uint32_t fb = acquire(bytes);
+          if (!fb) {
             ok = false;
             break;
           }
-          const uint32_t fb = smem_u32(full + s);
-          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          bulk_load(ring + s * STAGE_BYTES, xb + off, bytes, fb);
+          advance();
+        }
+        for (int tt = 0; tt < T && ok && !a.coop; ++tt) {
+          const int t = (tt + cta_in_slice) % T;
+          const uint32_t fb = acquire(static_cast<uint32_t>(klen * 2));
+          if (!fb) {
+            ok = false;
+            break;
+          }
+          bulk_load(ring + s * STAGE_BYTES, xb + (static_cast<int64_t>(t) * K + k0) * 2,
+                    static_cast<uint32_t>(klen * 2), fb);
+          advance();
+        }
+      }
+      for (int64_t tile = cta_in_slice; tile < n_tiles && ok; tile += ctas_in_slice) {
+        const int y = static_cast<int>(tile * ROWS);
+        for (int st = 0; st < spt; ++st) {
+          const uint32_t fb = acquire(STAGE_BYTES);
+          if (!fb) {
+            ok = false;
+            break;
+          }
           const int x = static_cast<int>(k0 + static_cast<int64_t>(st) * CH);
 #pragma unroll
           for (int c = 0; c < BOXES; ++c)
             tma_load_2d(ring + s * STAGE_BYTES + c * (ROWS * BOXW), &tmCB, fb, x + c * BOXW, y);
-          ++issued;
-          if (++s == STAGES) {
-            s = 0;
-            ph ^= 1u;
-          }
+          advance();
         }
       }
       if (!ok) {
@@ -170,136 +839,215 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1)
         const uint32_t inflight = issued < STAGES ? issued : STAGES;
         for (uint32_t i = 0; i < inflight; ++i) {
           const uint32_t u = issued - 1 - i;
-          mbar_wait(smem_u32(full + u % STAGES), (u / STAGES) & 1u, &no_abort, lim);
+          mbar_wait(smem_u32(full + u % STAGES), (u / STAGES) & 1u, &no_abort, a.lim);
         }
+      }
+      if constexpr (kRaw) {
+        int no_abort = 0;  // the code rows must land before the CTA may exit
+        mbar_wait(smem_u32(xq_bar), 0u, &no_abort, a.lim);
       }
     }
   } else {
-    // ------------------------------------------------------------ compute warps
-    const int g = lane >> 2, q = lane & 3;
-    int s = 0;
-    uint32_t ph = 0;
+    const int pt = warp < PRODUCER ? threadIdx.x : threadIdx.x - 32;
+    // zero the reduction buffers, (forward) the mask and block maxima, and every byte of
+    // xs that no code row writes: rows >= T, and columns >= klen of the others
+    for (int i = pt; i < EW * TP * RP; i += PRO_THREADS) red[i] = 0;
+    if constexpr (!kRaw) {
+      const int64_t MW = mask_words_smem(K), nbm = TP * ((K + XB - 1) / XB);
+      for (int64_t i = pt; i < MW; i += PRO_THREADS) maskall[i] = 0u;
+      for (int64_t i = pt; i < nbm; i += PRO_THREADS) bm[i] = 0u;
+      for (int i = pt; i < TP; i += PRO_THREADS) rmx[i] = 0u;
+    }
+    {
+      const int64_t tail = (pitch - klen) / 16, per_row = pitch / 16;
+      for (int64_t i = pt; i < T * tail; i += PRO_THREADS) {
+        const int64_t t = i / tail, c = i - t * tail;
+        *reinterpret_cast<uint4*>(xs + t * pitch + klen + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      for (int64_t i = pt; i < (TP - T) * per_row; i += PRO_THREADS)
+        reinterpret_cast<uint4*>(xs + T * pitch)[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    all_sync();
+    Ring rg;
+    rg.full = smem_u32(full);
+    rg.empty = smem_u32(empty);
     bool ok = true;
-    for (int64_t tile = cta_in_slice; tile < n_tiles; tile += ctas_in_slice) {
-      int c[NT][4];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) c[nt][0] = c[nt][1] = c[nt][2] = c[nt][3] = 0;
-      for (int st = 0; st < spt; ++st) {
-        if (ok) {
-          const bool got = mbar_wait(smem_u32(full + s), ph, abort_flag, lim);
+    if (warp < CW) {
+      if constexpr (kRaw) {
+        const bool got = mbar_wait(smem_u32(xq_bar), 0u, abort_flag, a.lim);
+        ok = __all_sync(0xffffffffu, got);
+      } else {
+        grid_dep_wait();  // the prologue re-reads a few blocks of X from global memory
+        ok = forward_prologue<NT>(a, threadIdx.x, slice, KS, S, rg, ring_p, xs, pitch, maskall,
+                                  spre, bm, dl, rmx, idx_s, jinfo, xo_s, scx, scale, jbase, misc,
+                                  xq_bar, abort_flag);
+        if (a.coop && ok) {
+          const bool got = mbar_wait(smem_u32(xq_bar), 0u, abort_flag, a.lim);
           ok = __all_sync(0xffffffffu, got);
         }
-        if (ok) {
-          // this warp's 64-byte step of the stage: box warp / 4, bytes 64 * (warp % 4) of
-          // each 256-byte row; k offset within the slice = stage * CH + 64 * warp
-          const uint32_t rowbase = ring + s * STAGE_BYTES + (warp >> 2) * (ROWS * BOXW) +
-                                   (warp & 3) * 64 + q * 16;
-          const int64_t kx = static_cast<int64_t>(st) * CH + 64 * warp + 16 * q;
-          const uint4 A0 = lds_v4(rowbase + g * BOXW);
-          const uint4 A1 = lds_v4(rowbase + (g + 8) * BOXW);
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const uint4 B = *reinterpret_cast<const uint4*>(xs + (nt * 8 + g) * pitch + kx);
-            mma_s8_16816(c[nt], A0.x, A1.x, A0.y, A1.y, B.x, B.y);
-            mma_s8_16816(c[nt], A0.z, A1.z, A0.w, A1.w, B.z, B.w);
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(empty + s));
-        }
-        if (++s == STAGES) {
-          s = 0;
-          ph ^= 1u;
-        }
       }
-      // ---- reduce the warps' partials of this tile (fixed order) and write P;
-      // the buffer is [warp][token][row] with row pitch RP
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int i0 = (warp * (NT * 8) + nt * 8 + 2 * q) * RP + g;
-        red[i0] = c[nt][0];
-        red[i0 + RP] = c[nt][1];
-        red[i0 + 8] = c[nt][2];
-        red[i0 + RP + 8] = c[nt][3];
-      }
-      asm volatile("bar.sync 1, %0;" ::"n"(CW * 32) : "memory");
-      const int64_t n0 = tile * ROWS;
-      for (int i = threadIdx.x; i < ROWS * NT * 8; i += CW * 32) {
-        const int tok = i / ROWS, rr = i - tok * ROWS;   // consecutive threads: consecutive n
-        int32_t sum = 0;
-#pragma unroll
-        for (int w = 0; w < CW; ++w) sum += red[(w * (NT * 8) + tok) * RP + rr];
-        const int64_t n = n0 + rr;
-        if (tok < T && n < N) P[(static_cast<int64_t>(slice) * T + tok) * N + n] = sum;
-      }
-      asm volatile("bar.sync 1, %0;" ::"n"(CW * 32) : "memory");
     }
-  }
-  __syncthreads();
-}
+    all_sync();
 
-// One thread per output channel n (consecutive threads on consecutive n) and group of TG
-// tokens (grid.y): the outlier bytes CB[n, idx[j]] are gathered once per group (8 loads in
-// flight; later groups find them in L2) and applied to the group's tokens in fp32, column
-// order j = 0 .. n_o-1; the slice partials are summed exactly (int32, slice order).
-// kRaw writes the int32 sums.
-template <bool kRaw>
-__global__ void __launch_bounds__(FIN_THREADS)
-    gemv_finalize_kernel(const int32_t* __restrict__ P, int S, int T, int64_t N, int64_t K,
-                         const float* __restrict__ SCx, const float* __restrict__ SCB,
-                         const __half* __restrict__ bias, const int8_t* __restrict__ CB,
-                         const int32_t* __restrict__ idx, const int32_t* __restrict__ n_o_ptr,
-                         const __half* __restrict__ X_o, __half* __restrict__ C,
-                         int32_t* __restrict__ acc_out) {
-  const int64_t n = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int t0 = blockIdx.y * TG;
-  const int tn = min(TG, T - t0);
-  grid_dep_wait();    // the partial sums come from the previous kernel
-  if (n >= N) return;
-  int32_t acc[TG];
+    if (warp < CW) {
+      // ---------------------------------------------------------- compute warps
+      const int g = lane >> 2, q = lane & 3;
+      const int64_t w0 = k0 / 32;
+      const int jb = kRaw ? 0 : jbase[slice];
+      int64_t it = 0;
+      for (int64_t tile = cta_in_slice; tile < n_tiles; tile += ctas_in_slice, ++it) {
+        const int b = static_cast<int>(it & (EW - 1));
+        const uint32_t use = static_cast<uint32_t>(it >> 2);
+        if (ok) {  // buffer b drained by its epilogue warp (tile it - EW)
+          const bool got = mbar_wait(smem_u32(rempty + b), (use & 1u) ^ 1u, abort_flag, a.lim);
+          ok = __all_sync(0xffffffffu, got);
+        }
+        uint8_t* cb_b = cbo + b * (MAXOS * ROWS);
+        int c[2][NT][4];
 #pragma unroll
-  for (int u = 0; u < TG; ++u) acc[u] = 0;
-  for (int sl = 0; sl < S; ++sl) {
-    const int32_t* p = P + (static_cast<int64_t>(sl) * T + t0) * N + n;
+        for (int h = 0; h < 2; ++h)
 #pragma unroll
-    for (int u = 0; u < TG; ++u)
-      if (u < tn) acc[u] += __ldcs(p + u * N);
-  }
-  if (kRaw) {
+          for (int nt = 0; nt < NT; ++nt) c[h][nt][0] = c[h][nt][1] = c[h][nt][2] = c[h][nt][3] = 0;
+        for (int st = 0; st < spt; ++st) {
+          if (ok) {
+            const bool got = mbar_wait(rg.full_bar(), rg.ph, abort_flag, a.lim);
+            ok = __all_sync(0xffffffffu, got);
+          }
+          if (ok) {
+            // this warp's 64-byte step of the stage: box warp / 4, bytes 64 * (warp % 4) of
+            // each 256-byte row; k offset within the slice = stage * CH + 64 * warp
+            const uint32_t rowbase = ring + rg.s * STAGE_BYTES + (warp >> 2) * (ROWS * BOXW) +
+                                     (warp & 3) * 64 + q * 16;
+            const int64_t kx = static_cast<int64_t>(st) * CH + 64 * warp + 16 * q;
+            const uint4 A0 = lds_v4(rowbase + g * BOXW);
+            const uint4 A1 = lds_v4(rowbase + (g + 8) * BOXW);
+            const uint4 A2 = lds_v4(rowbase + (g + 16) * BOXW);
+            const uint4 A3 = lds_v4(rowbase + (g + 24) * BOXW);
 #pragma unroll
-    for (int u = 0; u < TG; ++u)
-      if (u < tn) acc_out[static_cast<int64_t>(t0 + u) * N + n] = acc[u];
-    return;
-  }
-  float o[TG];
+            for (int nt = 0; nt < NT; ++nt) {
+              const uint4 B = *reinterpret_cast<const uint4*>(xs + (nt * 8 + g) * pitch + kx);
+              mma_s8_16816(c[0][nt], A0.x, A1.x, A0.y, A1.y, B.x, B.y);
+              mma_s8_16816(c[1][nt], A2.x, A3.x, A2.y, A3.y, B.x, B.y);
+              mma_s8_16816(c[0][nt], A0.z, A1.z, A0.w, A1.w, B.z, B.w);
+              mma_s8_16816(c[1][nt], A2.z, A3.z, A2.w, A3.w, B.z, B.w);
+            }
+            if constexpr (!kRaw) {
+              // copy out the bytes of outlier columns in this step (lane q holds columns
+              // 16q .. 16q+15 of rows g, g + 8, g + 16, g + 24)
+              const int wl = st * (CH / 32) + 2 * warp;  // slice-local mask word
+              if ((maskall[w0 + wl] | maskall[w0 + wl + 1]) != 0u) {
+                const int wq = wl + (q >> 1), sh = (q & 1) * 16;
+                const uint32_t mw = maskall[w0 + wq];
+                uint32_t bits = (mw >> sh) & 0xffffu;
+                while (bits) {
+                  const int bp = __ffs(bits) - 1;
+                  bits &= bits - 1u;
+                  const int jl = spre[wq] + __popc(mw & ((1u << (sh + bp)) - 1u)) - jb;
+                  if (jl < MAXOS && jl + jb < MAXO) {
+                    const int wi = bp >> 2, bs = 8 * (bp & 3);
+                    const uint32_t u0 = wi == 0 ? A0.x : wi == 1 ? A0.y : wi == 2 ? A0.z : A0.w;
+                    const uint32_t u1 = wi == 0 ? A1.x : wi == 1 ? A1.y : wi == 2 ? A1.z : A1.w;
+                    const uint32_t u2 = wi == 0 ? A2.x : wi == 1 ? A2.y : wi == 2 ? A2.z : A2.w;
+                    const uint32_t u3 = wi == 0 ? A3.x : wi == 1 ? A3.y : wi == 2 ? A3.z : A3.w;
+                    uint8_t* d = cb_b + jl * ROWS + g;
+                    d[0] = static_cast<uint8_t>(u0 >> bs);
+                    d[8] = static_cast<uint8_t>(u1 >> bs);
+                    d[16] = static_cast<uint8_t>(u2 >> bs);
+                    d[24] = static_cast<uint8_t>(u3 >> bs);
+                  }
+                }
+              }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(rg.empty_bar());
+          }
+          rg.advance();
+        }
+        if (ok) {
+          // this warp's 32 x TP partials into buffer b: c[h] covers rows 16h + (g, g + 8),
+          // elements 0/1 tokens 2q/2q+1 of row g, 2/3 of row g + 8 (integer adds: the order
+          // does not change the sums)
+          int32_t* rbuf = red + b * (TP * RP);
 #pragma unroll
-  for (int u = 0; u < TG; ++u) o[u] = 0.0f;
-  const int n_o = n_o_ptr == nullptr ? 0 : __ldg(n_o_ptr);
-  const int8_t* cbrow = CB + n * K;
-  for (int j0 = 0; j0 < n_o; j0 += 8) {
-    float cb[8];
+          for (int h = 0; h < 2; ++h)
 #pragma unroll
-    for (int v = 0; v < 8; ++v)
-      cb[v] = j0 + v < n_o ? static_cast<float>(cbrow[__ldg(idx + j0 + v)]) : 0.0f;
+            for (int nt = 0; nt < NT; ++nt) {
+              const int i0 = (nt * 8 + 2 * q) * RP + 16 * h + g;
+              atomicAdd(rbuf + i0, c[h][nt][0]);
+              atomicAdd(rbuf + i0 + RP, c[h][nt][1]);
+              atomicAdd(rbuf + i0 + 8, c[h][nt][2]);
+              atomicAdd(rbuf + i0 + RP + 8, c[h][nt][3]);
+            }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(rfull + b));
+        }
+      }
+    } else {
+      // ---------------------------------------------------------- epilogue warps
+      const int e = warp - EPI0;
+      const int rb = static_cast<int>(rec_bytes(T));
+      int nos = 0, jb = 0;  // this slice's copied outlier columns: ranks jb .. jb + nos - 1
+      if constexpr (!kRaw) {
+        jb = jbase[slice];
+        nos = jbase[slice + 1] - jb;
+        nos = min(nos, min(MAXOS, MAXO - jb));
+        if (nos < 0) nos = 0;
+      }
+      int32_t* rbuf = red + e * (TP * RP);
+      const uint8_t* cb_e = cbo + e * (MAXOS * ROWS);
+      int64_t it = e;
+      for (int64_t tile = cta_in_slice + static_cast<int64_t>(e) * ctas_in_slice; tile < n_tiles;
+           tile += static_cast<int64_t>(EW) * ctas_in_slice, it += EW) {
+        const uint32_t use = static_cast<uint32_t>(it >> 2);
+        const bool got = mbar_wait(smem_u32(rfull + e), use & 1u, abort_flag, a.lim);
+        if (!__all_sync(0xffffffffu, got)) break;
+        int32_t p[TP];
 #pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      const int j = j0 + v;
-      if (j >= n_o) break;
-      const __half* xo = X_o + (static_cast<int64_t>(j >> 6) * T + t0) * 64 + (j & 63);
+        for (int t = 0; t < TP; ++t) {
+          p[t] = rbuf[t * RP + lane];
+          rbuf[t * RP + lane] = 0;
+        }
+        // lane = row of the tile
+        uint8_t* rec = a.rec + (tile * S + slice) * rb + lane * 4;
+        if constexpr (kRaw) {
 #pragma unroll
-      for (int u = 0; u < TG; ++u)
-        if (u < tn) o[u] = fmaf(__half2float(xo[u * 64]), cb[v], o[u]);
+          for (int t = 0; t < TP; ++t)
+            if (t < T) reinterpret_cast<int32_t*>(rec)[t * ROWS] = p[t];
+        } else {
+          float o[TP];
+#pragma unroll
+          for (int t = 0; t < TP; ++t) o[t] = 0.0f;
+          for (int jl = 0; jl < nos; ++jl) {
+            const float cb = static_cast<float>(static_cast<int8_t>(cb_e[jl * ROWS + lane]));
+#pragma unroll
+            for (int t = 0; t < TP; ++t)
+              if (t < T) o[t] = fmaf(__half2float(xo_s[t * MAXO + jb + jl]), cb, o[t]);
+          }
+#pragma unroll
+          for (int t = 0; t < TP; ++t)
+            if (t < T)
+              reinterpret_cast<float*>(rec)[t * ROWS] =
+                  fmaf(static_cast<float>(p[t]), scx[t] * (1.0f / 127.0f), o[t]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(rempty + e));
+        fence_acq_rel_gpu();  // the record is visible before the arrival is counted
+        __syncwarp();
+        int arrivals = 0;
+        if (lane == 0) arrivals = tile_arrive(a.cnt + tile, static_cast<uint32_t>(a.epoch));
+        arrivals = __shfl_sync(0xffffffffu, arrivals, 0);
+        if (arrivals == S) {
+          fence_acq_rel_gpu();
+          finish_tile<NT, kRaw>(a, tile, S, rb, maskall, idx_s, jinfo, xo_s, misc);
+          __syncwarp();
+          if (lane == 0)
+            *reinterpret_cast<volatile unsigned long long*>(a.cnt + tile) = a.epoch << 32;
+        }
+      }
     }
   }
-  const float ws = __ldg(SCB + n) * (1.0f / 127.0f);
-  const float bn = bias ? __half2float(bias[n]) : 0.0f;
-#pragma unroll
-  for (int u = 0; u < TG; ++u) {
-    if (u < tn) {
-      const float part =
-          fmaf(static_cast<float>(acc[u]), __ldg(SCx + t0 + u) * (1.0f / 127.0f), o[u]);
-      C[static_cast<int64_t>(t0 + u) * N + n] = __float2half_rn(fmaf(part, ws, bn));
-    }
-  }
+  grid_dep_launch();
+  __syncthreads();
 }
 
 }  // namespace gemv

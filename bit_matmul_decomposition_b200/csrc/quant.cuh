@@ -237,6 +237,7 @@ constexpr int kPrepThreads = 512;
 constexpr int kPrepWarps = kPrepThreads / 32;
 constexpr int kPrepChunk = 32768;   // bytes per bulk copy of the row cache
 constexpr int kPrepMaxChunks = 8;
+constexpr int kPrepMaxIdx = 4096;    // outlier indices kept in shared memory
 
 struct PrepArgs {
   const __half* X;
@@ -348,18 +349,36 @@ __device__ __forceinline__ void row_codes(uint32_t base, const uint4* gbase, uin
   for (; v < gpr; v += step) q[v] = codes8(row_vec<kShared>(base, gbase, v), scan_bits(smask, v), s);
 }
 
+// Column of the j-th outlier (j < n_o) from the mask words and their exclusive popcount
+// prefix (spre[words] = n_o): the last word whose prefix is <= j holds it.
+__device__ __forceinline__ int32_t nth_outlier(const uint32_t* smask, const int32_t* spre,
+                                               int64_t words, int j) {
+  int64_t lo = 0, hi = words - 1;
+  while (lo < hi) {
+    const int64_t mid = (lo + hi + 1) >> 1;
+    if (spre[mid] <= j)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  uint32_t m = smask[lo];
+  for (int k = j - spre[lo]; k > 0; --k) m &= m - 1u;
+  return static_cast<int32_t>(lo * 32 + (__ffs(m) - 1));
+}
+
 __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs p) {
   extern __shared__ __align__(128) uint8_t psm[];
   const int64_t K = p.K;
   const int64_t words = (K + 31) / 32;
   const int64_t gpr = K / 8;  // 16-byte groups per row
-  // shared memory: [row cache][mask words][prefix words + 1][idx K][row scales]
+  // shared memory: [row cache][mask words][prefix words + 1][first kPrepMaxIdx indices]
+  // [row scales]; indices past kPrepMaxIdx are found from the mask and its prefix
   const size_t cache_bytes = static_cast<size_t>(p.cache_rows) * static_cast<size_t>(K) * 2;
   uint4* cache = reinterpret_cast<uint4*>(psm);
   uint32_t* smask = reinterpret_cast<uint32_t*>(psm + cache_bytes);
   int32_t* spre = reinterpret_cast<int32_t*>(smask + words);
   int32_t* sidx = spre + words + 1;
-  float* samax = reinterpret_cast<float*>(sidx + K);   // [rows_per_cta]
+  float* samax = reinterpret_cast<float*>(sidx + kPrepMaxIdx);   // [rows_per_cta]
   __shared__ __align__(8) uint64_t s_bar[kPrepMaxChunks];
   __shared__ int s_fail;
   __shared__ int s_wsum[kPrepWarps];
@@ -507,16 +526,19 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
     int pos = spre[w];
     while (m) {
       const int b = __ffs(m) - 1;
-      sidx[pos++] = static_cast<int32_t>(w * 32 + b);
+      const int32_t col = static_cast<int32_t>(w * 32 + b);
+      if (pos < kPrepMaxIdx) sidx[pos] = col;
+      if (blockIdx.x == 0) p.idx_out[pos] = col;
+      ++pos;
       m &= m - 1u;
     }
   }
   for (int64_t i = tid; i < nrows; i += kPrepThreads) samax[i] = 0.0f;
   __syncthreads();
-  if (blockIdx.x == 0) {
-    for (int j = tid; j < n_o; j += kPrepThreads) p.idx_out[j] = sidx[j];
-    if (tid == 0) *p.n_o_out = n_o;
-  }
+  if (blockIdx.x == 0 && tid == 0) *p.n_o_out = n_o;
+  auto idx_at = [&](int j) -> int64_t {
+    return j < kPrepMaxIdx ? sidx[j] : nth_outlier(smask, spre, words, j);
+  };
 
   // ------------------------------------------------ phase 3: quantise
   // Rows go in rounds of (16 / wpr) rows with wpr warps per row (wpr = 1 when the CTA owns
@@ -563,7 +585,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
       for (int j = start; j < padded; j += step) {
         __half v = __float2half_rn(0.0f);
         if (j < n_o) {
-          const int64_t k = sidx[j];
+          const int64_t k = idx_at(j);
           v = cached ? reinterpret_cast<const __half*>(cache + i * gpr)[k] : p.X[t * K + k];
         }
         p.X_o[(static_cast<int64_t>(j >> 6) * p.T + t) * 64 + (j & 63)] = v;
@@ -598,8 +620,9 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
           for (int64_t c = 0; c < chunks; ++c) {
             const int64_t j0 = c * 64 + 2 * lane;
             float v0 = 0.0f, v1 = 0.0f;
-            if (j0 < n_o) v0 = static_cast<float>(static_cast<int8_t>(rowbuf[sidx[j0]]));
-            if (j0 + 1 < n_o) v1 = static_cast<float>(static_cast<int8_t>(rowbuf[sidx[j0 + 1]]));
+            if (j0 < n_o) v0 = static_cast<float>(static_cast<int8_t>(rowbuf[idx_at(j0)]));
+            if (j0 + 1 < n_o)
+              v1 = static_cast<float>(static_cast<int8_t>(rowbuf[idx_at(j0 + 1)]));
             reinterpret_cast<__half2*>(p.CB_o + (c * p.N + n) * 64)[lane] =
                 __floats2half2_rn(v0, v1);
           }
@@ -623,8 +646,8 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
           if (it < items) {
             const int64_t c = it / p.N, n = it - c * p.N;
             const int64_t j0 = c * 64 + 2 * lane;
-            if (j0 < n_o) v0[u] = static_cast<float>(p.CB[n * K + sidx[j0]]);
-            if (j0 + 1 < n_o) v1[u] = static_cast<float>(p.CB[n * K + sidx[j0 + 1]]);
+            if (j0 < n_o) v0[u] = static_cast<float>(p.CB[n * K + idx_at(j0)]);
+            if (j0 + 1 < n_o) v1[u] = static_cast<float>(p.CB[n * K + idx_at(j0 + 1)]);
           }
         }
 #pragma unroll
@@ -642,11 +665,11 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
 }
 
 // Dynamic shared memory of prepare_kernel: a row cache of `cache_rows` rows, the mask,
-// its prefix, the index list and one scale per row of the CTA's block.
+// its prefix, the first kPrepMaxIdx indices and one scale per row of the CTA's block.
 __host__ inline size_t prepare_smem_bytes(int64_t K, int64_t cache_rows, int64_t rows_per_cta) {
   const int64_t words = (K + 31) / 32;
   return static_cast<size_t>(cache_rows) * static_cast<size_t>(K) * 2 +
-         static_cast<size_t>(2 * words + 1 + K + rows_per_cta) * 4;
+         static_cast<size_t>(2 * words + 1 + kPrepMaxIdx + rows_per_cta) * 4;
 }
 
 }  // namespace i8

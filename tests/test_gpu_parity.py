@@ -62,6 +62,7 @@ SCAN_CASES = [
     (4100, 1040, (7, 1039), 1e-4, 6.0),
     (3000, 16384, (0, 9000, 16383), 0.0, 6.0),    # rows beyond the per-CTA cache
     (16, 14336, (100, 14000), 0.0, 6.0),
+    (20, 6000, (), 0.0, 0.0),       # n_o = 6000: indices past the 4096 kept in shared memory
 ]
 
 
@@ -140,6 +141,14 @@ FORWARD_CASES = [
     (256, 4096, 512, (), 0.0, math.inf, True),      # GEMM, no outliers (2 TMEM buffers)
     (64, 208, 256, (9,), 0.0, 0.0, True),           # GEMM, thr 0: only the fp16 product
     (200, 128, 100, (1, 2, 3), 0.0, 6.0, False),
+    # decode kernel: more than 32 outlier columns in one K-slice (bytes read from CB
+    # instead of the copies), one token, a ragged 16-row tile
+    (1, 14336, 257, tuple(range(0, 3584, 89)) + (9000, 14335), 0.0, 6.0, True),
+    (9, 1024, 130, (), 0.0, 0.0, True),             # decode, n_o = K > 128 kept columns
+    (8, 65536, 40, (0, 30000, 65535), 0.0, 6.0, True),     # decode, largest K (19 slices)
+    (4, 65552, 33, (1, 65551), 0.0, 6.0, True),     # T <= 16 beyond 65536: GEMM path
+    (12, 3584, 48, (3583,), 0.0, 6.0, False),       # one slice, last column an outlier
+    (40, 8192, 96, (), 0.0, 0.0, True),             # GEMM, n_o = 8192 (> 4096 kept indices)
 ]
 
 
@@ -163,6 +172,55 @@ def test_forward_repeat_is_deterministic():
     C2 = host(gpu_forward(X_d, CB, SCB, b_d, 6.0))
     sync_ok()
     assert np.array_equal(C1.view(np.uint16), C2.view(np.uint16))
+
+
+@pytest.mark.parametrize("K", [2048, 4096], ids=["x_per_cta", "x_split"])
+def test_decode_row_max_next_to_an_outlier_column(K):
+    """SCx excludes outlier columns but keeps the other columns of their block: each row's
+    largest non-outlier value sits right beside an outlier column (K = 2048: every CTA
+    scans all of X; K = 4096: the CTAs split the scan)."""
+    T, N = 6, 96
+    w, X, W, b = _case(T, K, N, seed=21, cols=(300, 1500))
+    X = np.clip(X.astype(np.float32), -3.0, 3.0).astype(np.float16)
+    X[:, 300] = np.float16(9.0)
+    X[:, 1500] = np.float16(-7.5)
+    for t in range(T):
+        X[t, 301 if t % 2 else 1499] = np.float16(5.5 - 0.25 * t)
+    CB, SCB = gpu_quantize_weight(dev(W))
+    C = gpu_forward(dev(X), CB, SCB, dev(b), 6.0)
+    sync_ok()
+    CBr, SCBr = O.quantize_weight(W)
+    r = O.linear_forward(X, CBr, SCBr, b, 6.0)
+    assert np.array_equal(r["SCx"], np.array([5.5 - 0.25 * t for t in range(T)], np.float32))
+    check_output(host(C), r["C"])
+
+
+@pytest.mark.parametrize("T", [1, 16])
+def test_decode_workspace_garbage_and_reuse(T):
+    """The decode kernel's tile counters need no clearing: a workspace full of 0xff, then
+    reused by further calls (also of another shape), gives the same output every time."""
+    w, X, W, b = _case(T, 3600, 1000, seed=T + 40, cols=(10, 2000))
+    CB, SCB = gpu_quantize_weight(dev(W))
+    X_d, b_d = dev(X), dev(b)
+    nbytes = max(abi.i8_linear_workspace_size(T, 1000, 3600),
+                 abi.i8_linear_workspace_size(2, 500, 3600))
+    ws = torch.full((nbytes,), 255, dtype=torch.uint8, device="cuda")
+    CBr, SCBr = O.quantize_weight(W)
+    ref = O.linear_forward(X, CBr, SCBr, b, 6.0)["C"]
+    outs = []
+    for i in range(3):
+        C = torch.full((T, 1000), float("nan"), dtype=torch.float16, device="cuda")
+        abi.i8_linear_forward(X_d, CB, SCB, b_d, 6.0, C, ws)
+        outs.append(host(C))
+        if i == 1:  # another shape on the same workspace in between
+            X2 = dev(synth.random_fp16((2, 3600), seed=7, sigma=1.0))
+            C2 = torch.empty((2, 500), dtype=torch.float16, device="cuda")
+            abi.i8_linear_forward(X2, CB[:500].contiguous(), SCB[:500].contiguous(), None,
+                                  6.0, C2, ws)
+    sync_ok()
+    for C in outs:
+        check_output(C, ref)
+        assert np.array_equal(C.view(np.uint16), outs[0].view(np.uint16))
 
 
 def test_power_of_two_row_scaling_gpu():
