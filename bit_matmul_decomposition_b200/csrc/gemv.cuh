@@ -67,6 +67,8 @@ constexpr int CH = 64 * CW;                 // bytes of K per stage per row
 constexpr int BOXES = CH / BOXW;            // TMA boxes per stage
 constexpr int STAGES = 6;
 constexpr int STAGE_BYTES = ROWS * CH;      // 16 KB
+constexpr int XPAD = 64;                    // xs row pitch = KS + 64: a quarter-warp's B loads
+                                            // (tokens g, g+1 x 4 chunks) hit 8 bank groups
 constexpr int RP = ROWS + 4;                // token pitch of a reduction buffer (words):
                                             // the fragment adds fall on distinct banks
 constexpr int MAXO = 128;                   // outlier columns kept in shared memory
@@ -124,7 +126,7 @@ __host__ __device__ inline Smem smem_layout(int NT, int64_t K) {
   const int TP = NT * 8;                    // token rows held (padded)
   const int64_t KS = slice_bytes(K);
   s.ring = smem_take(off, static_cast<uint64_t>(STAGES) * STAGE_BYTES, 1024);
-  s.xs = smem_take(off, static_cast<uint64_t>(TP) * (KS + 16), 16);
+  s.xs = smem_take(off, static_cast<uint64_t>(TP) * (KS + XPAD), 16);
   s.red = smem_take(off, static_cast<uint64_t>(EW) * TP * RP * 4, 16);
   s.cbo = smem_take(off, static_cast<uint64_t>(EW) * MAXOS * ROWS, 16);
   s.mask = smem_take(off, static_cast<uint64_t>(mask_words_smem(K)) * 4, 16);
@@ -229,15 +231,20 @@ __device__ __forceinline__ int tile_arrive(unsigned long long* c, uint32_t e) {
   return static_cast<int>(static_cast<uint32_t>(atomicAdd(c, 1ull))) + 1;
 }
 
-// Grid barrier of the cooperative launch (one thread per CTA).  The counter only grows
-// within an epoch (a replay of the same launch starts the next generation of `target`
-// arrivals).  Bounded: false after `lim` ns (the error word records it).
-__device__ __forceinline__ bool grid_sync(unsigned long long* ctr, uint32_t e, uint32_t target,
-                                          uint64_t lim) {
+// Grid barrier of the cooperative launch (one thread per CTA), in two halves so that
+// independent work can go between them.  The counter only grows within an epoch (a replay
+// of the same launch starts the next generation of `target` arrivals).  The wait is
+// bounded: false after `lim` ns (the error word records it).
+__device__ __forceinline__ uint32_t grid_arrive(unsigned long long* ctr, uint32_t e,
+                                                uint32_t target) {
   fence_acq_rel_gpu();  // this CTA's writes before its arrival
   tag_claim(ctr, e);
   const uint32_t c = static_cast<uint32_t>(atomicAdd(ctr, 1ull));
-  const uint32_t goal = (c / target + 1) * target;
+  return (c / target + 1) * target;
+}
+
+__device__ __forceinline__ bool grid_wait(unsigned long long* ctr, uint32_t e, uint32_t goal,
+                                          uint64_t lim) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 0;; ++it) {
     const unsigned long long v = __ldcg(ctr);
@@ -249,6 +256,11 @@ __device__ __forceinline__ bool grid_sync(unsigned long long* ctr, uint32_t e, u
   }
   fence_acq_rel_gpu();
   return true;
+}
+
+__device__ __forceinline__ bool grid_sync(unsigned long long* ctr, uint32_t e, uint32_t target,
+                                          uint64_t lim) {
+  return grid_wait(ctr, e, grid_arrive(ctr, e, target), lim);
 }
 
 // Consumer side of the ring: wait for stage s (phase ph), then advance.
@@ -291,6 +303,8 @@ __device__ __forceinline__ bool forward_prologue(
   constexpr int GPB = XB / 8;  // groups per block
 
   bool ok = true;
+  const uint32_t e = static_cast<uint32_t>(a.epoch);
+  uint32_t goal3 = 0;  // cooperative path: third barrier, waited for after the tables below
   if (!a.coop) {
     // (a) step 1 and the block maxima, piece by piece
     const int64_t xbytes = static_cast<int64_t>(T) * K * 2;
@@ -355,7 +369,6 @@ __device__ __forceinline__ bool forward_prologue(
     // bits of its share into the global mask; grid barrier; each takes the masked maxima
     // of its share into the global row maxima; grid barrier; step 2 on its share into the
     // global codes; grid barrier; then this CTA's slice of the codes is copied into xs.
-    const uint32_t e = static_cast<uint32_t>(a.epoch);
     const int64_t TG = static_cast<int64_t>(T) * G;
     const int64_t f_lo = TG * blockIdx.x / gridDim.x, f_hi = TG * (blockIdx.x + 1) / gridDim.x;
     for (int64_t f = f_lo + ct; f < f_hi; f += CW * 32) {
@@ -407,23 +420,7 @@ __device__ __forceinline__ bool forward_prologue(
     // the codes are read back by TMA (the async proxy) in other CTAs
     asm volatile("fence.proxy.async.global;" ::: "memory");
     compute_sync();
-    if (ct == 0 && ok && !grid_sync(a.gbar + 2, e, gridDim.x, a.lim)) *abort_flag = 1;
-    if (ct == 0 && *abort_flag == 0) {
-      asm volatile("fence.proxy.async.global;" ::: "memory");
-      const int64_t k0 = static_cast<int64_t>(slice) * KS;
-      const int64_t klen = KS < K - k0 ? KS : K - k0;
-      mbar_arrive_expect_tx(smem_u32(xq_bar), static_cast<uint32_t>(T * klen));
-      for (int t = 0; t < T; ++t)
-        bulk_load(smem_u32(xs + t * pitch), a.xq + static_cast<int64_t>(t) * K + k0,
-                  static_cast<uint32_t>(klen), smem_u32(xq_bar));
-      // every CTA has read the mask and row maxima: CTA 0 puts them back to (epoch, 0)
-      if (blockIdx.x == 0) {
-        for (int64_t x = 0; x < KW; ++x) a.gmask[x] = static_cast<unsigned long long>(e) << 32;
-        for (int t = 0; t < T; ++t) a.gscx[t] = static_cast<unsigned long long>(e) << 32;
-      }
-    }
-    compute_sync();
-    ok = *abort_flag == 0;
+    if (ct == 0 && ok) goal3 = grid_arrive(a.gbar + 2, e, gridDim.x);
   }
 
   // (b) ranks (warp 0: lane l takes a contiguous run of mask words)
@@ -479,6 +476,26 @@ __device__ __forceinline__ bool forward_prologue(
   for (int i = ct; i < T * nf; i += CW * 32) {
     const int t = i / nf, j = i - t * nf;
     xo_s[t * MAXO + j] = X[static_cast<int64_t>(t) * K + idx_s[j]];
+  }
+  if (a.coop) {
+    // the third barrier: every CTA's codes are in global memory
+    if (ct == 0 && ok && !grid_wait(a.gbar + 2, e, goal3, a.lim)) *abort_flag = 1;
+    if (ct == 0 && *abort_flag == 0) {
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      const int64_t k0 = static_cast<int64_t>(slice) * KS;
+      const int64_t klen = KS < K - k0 ? KS : K - k0;
+      mbar_arrive_expect_tx(smem_u32(xq_bar), static_cast<uint32_t>(T * klen));
+      for (int t = 0; t < T; ++t)
+        bulk_load(smem_u32(xs + t * pitch), a.xq + static_cast<int64_t>(t) * K + k0,
+                  static_cast<uint32_t>(klen), smem_u32(xq_bar));
+      // every CTA has read the mask and row maxima: CTA 0 puts them back to (epoch, 0)
+      if (blockIdx.x == 0) {
+        for (int64_t x = 0; x < KW; ++x) a.gmask[x] = static_cast<unsigned long long>(e) << 32;
+        for (int t = 0; t < T; ++t) a.gscx[t] = static_cast<unsigned long long>(e) << 32;
+      }
+    }
+    compute_sync();
+    ok = *abort_flag == 0;
   }
   if (!a.coop) {
     // blocks holding outlier columns (warp 1 lists them); the other blocks give their
@@ -711,7 +728,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const Smem L = smem_layout(NT, K);
   const int64_t KS = slice_bytes(K);
   const int S = static_cast<int>(num_slices(K));
-  const int64_t pitch = KS + 16;
+  const int64_t pitch = KS + XPAD;
   const uint32_t ring = raw_s + pad + L.ring;
   const uint8_t* ring_p = sm + L.ring;
   uint8_t* xs = sm + L.xs;

@@ -237,7 +237,7 @@ constexpr int kPrepThreads = 512;
 constexpr int kPrepWarps = kPrepThreads / 32;
 constexpr int kPrepChunk = 32768;   // bytes per bulk copy of the row cache
 constexpr int kPrepMaxChunks = 8;
-constexpr int kPrepMaxIdx = 4096;    // outlier indices kept in shared memory
+constexpr int kPrepMaxIdx = 8192;    // outlier indices kept in shared memory
 
 struct PrepArgs {
   const __half* X;

@@ -62,7 +62,7 @@ SCAN_CASES = [
     (4100, 1040, (7, 1039), 1e-4, 6.0),
     (3000, 16384, (0, 9000, 16383), 0.0, 6.0),    # rows beyond the per-CTA cache
     (16, 14336, (100, 14000), 0.0, 6.0),
-    (20, 6000, (), 0.0, 0.0),       # n_o = 6000: indices past the 4096 kept in shared memory
+    (20, 10000, (), 0.0, 0.0),      # n_o = 10000: indices past the 8192 kept in shared memory
 ]
 
 
@@ -148,7 +148,7 @@ FORWARD_CASES = [
     (8, 65536, 40, (0, 30000, 65535), 0.0, 6.0, True),     # decode, largest K (19 slices)
     (4, 65552, 33, (1, 65551), 0.0, 6.0, True),     # T <= 16 beyond 65536: GEMM path
     (12, 3584, 48, (3583,), 0.0, 6.0, False),       # one slice, last column an outlier
-    (40, 8192, 96, (), 0.0, 0.0, True),             # GEMM, n_o = 8192 (> 4096 kept indices)
+    (40, 9216, 96, (), 0.0, 0.0, True),             # GEMM, n_o = 9216 (> 8192 kept indices)
 ]
 
 
