@@ -582,13 +582,21 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
       else
         row_codes<false>(sbase, gbase, qrow, g32, start, step, smask, sc);
       if (sub == 0 && lane == 0) p.SCx[t] = amax;
-      for (int j = start; j < padded; j += step) {
-        __half v = __float2half_rn(0.0f);
-        if (j < n_o) {
-          const int64_t k = idx_at(j);
-          v = cached ? reinterpret_cast<const __half*>(cache + i * gpr)[k] : p.X[t * K + k];
+      // the row's outlier values into X_o, eight loads in flight before their stores
+      const __half* xrow = cached ? reinterpret_cast<const __half*>(cache + i * gpr) : p.X + t * K;
+      for (int j0 = start; j0 < padded; j0 += 8 * step) {
+        __half v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int j = j0 + u * step;
+          v[u] = __float2half_rn(0.0f);
+          if (j < n_o) v[u] = xrow[idx_at(j)];
         }
-        p.X_o[(static_cast<int64_t>(j >> 6) * p.T + t) * 64 + (j & 63)] = v;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int j = j0 + u * step;
+          if (j < padded) p.X_o[(static_cast<int64_t>(j >> 6) * p.T + t) * 64 + (j & 63)] = v[u];
+        }
       }
     }
   }
