@@ -149,9 +149,9 @@ def work_counts(T, N, K, n_o):
     return i8_ops, f16_flops, eff_ops, bytes_
 
 
-def traffic_record(kernel):
+def traffic_record(kernel, workload):
     """DRAM bytes per launch from the committed ncu summary (profiles/dram_traffic.txt), if
-    it was taken on the current CUDA sources (else None)."""
+    it was taken on this workload and on the current CUDA sources (else None)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     try:
         with open(path) as f:
@@ -159,7 +159,8 @@ def traffic_record(kernel):
     except OSError:
         return None
     for parts in lines:
-        if len(parts) >= 3 and parts[0] == kernel and parts[2] == source_hash():
+        if (len(parts) >= 4 and parts[0] == kernel and parts[2] == source_hash()
+                and parts[3] == workload):
             return {"dram_bytes_per_launch": int(parts[1]),
                     "note": parts[4].strip() if len(parts) > 4 else ""}
     return None
@@ -391,7 +392,7 @@ def run_gpu(args, w0):
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
                 "frac": achieved / pk["hbm"], "kernel": "decode_kernel",
                 "algorithmic_bytes_per_launch": gemv_bytes}
-        tr = traffic_record("decode_kernel")
+        tr = traffic_record("decode_kernel", w0.name)
     else:
         # dominant kernel: the tcgen05 GEMM; int8 ops plus fp16 flops counted at the int8
         # rate x 2 (the nominal fp16 : int8 tensor rate is 1 : 2)
@@ -404,7 +405,7 @@ def run_gpu(args, w0):
                               % (pk["source"], pk["bf16_sus"]),
                 "frac_of_burst_peak": achieved / (2.0 * pk["bf16"]),
                 "algorithmic_ops_per_launch": equiv}
-        tr = traffic_record("i8_gemm_tcgen05_kernel")
+        tr = traffic_record("i8_gemm_tcgen05_kernel", w0.name)
     roof["kernel_ms"] = kern_per
     roof["traffic"] = None if tr is None else tr["dram_bytes_per_launch"]
     if tr is not None:
