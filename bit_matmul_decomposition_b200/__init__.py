@@ -4,4 +4,4 @@ The compute lives in the CUDA library ``libi8linear.so`` built from ``csrc/``; t
 side only marshals arguments (see ``abi.py``).  Importing the package does not load the
 library: the first call does, and fails loudly when it is missing.
 """
-__all__ = ["abi", "synth"]
+__all__ = ["abi", "linear", "synth"]

@@ -1,0 +1,97 @@
+"""The nn.Module front end on the GPU against the CPU oracle: quantisation bit for bit,
+outputs within the per-row tolerance on both the decode (T <= 16) and GEMM (T > 16)
+paths, exact restore of the quantised state, and a small layer stack converted with the
+replacement helper, checked layer by layer."""
+import io
+
+import numpy as np
+import pytest
+import torch
+
+from bit_matmul_decomposition_b200 import abi, synth
+from bit_matmul_decomposition_b200.linear import Linear8bitLt, replace_linear_with_int8
+from oracle import oracle as O
+from tests.gpu_util import check_output, host, sync_ok
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    abi.load()
+    yield
+    torch.cuda.synchronize()
+
+
+def _fp16_linear(K, N, seed, bias=True):
+    g = torch.Generator().manual_seed(seed)
+    lin = torch.nn.Linear(K, N, bias=bias).half()
+    with torch.no_grad():
+        lin.weight.copy_((torch.randn(N, K, generator=g) * 0.02).half())
+        if bias:
+            lin.bias.copy_((torch.randn(N, generator=g) * 0.02).half())
+    return lin.cuda()
+
+
+def _x(shape, K, cols, seed):
+    X = synth.random_fp16((int(np.prod(shape)), K), seed=seed)
+    X = synth.plant_columns(X, cols, seed=seed + 1)
+    return X.reshape(*shape, K)
+
+
+@pytest.mark.parametrize("lead", [(1, 5), (3, 7)], ids=["decode_T5", "gemm_T21"])
+def test_module_matches_oracle(lead):
+    K, N = 1024, 768
+    lin = _fp16_linear(K, N, seed=11)
+    m = Linear8bitLt.from_linear(lin, threshold=6.0)
+    W = host(lin.weight)
+    CBr, SCBr = O.quantize_weight(W)
+    assert np.array_equal(host(m.CB), CBr)
+    assert np.array_equal(host(m.SCB).view(np.uint32), SCBr.view(np.uint32))
+    X = _x(lead, K, (7, 500, 1000), seed=21)
+    y = m(torch.from_numpy(X.view(np.int16)).view(torch.float16).cuda())
+    sync_ok()
+    assert tuple(y.shape) == (*lead, N)
+    ref = O.linear_forward(X.reshape(-1, K), CBr, SCBr, host(lin.bias), 6.0)["C"]
+    check_output(host(y).reshape(-1, N), ref)
+
+
+def test_state_dict_restores_the_same_outputs():
+    K, N = 512, 256
+    m = Linear8bitLt.from_linear(_fp16_linear(K, N, seed=5))
+    buf = io.BytesIO()
+    torch.save(m.state_dict(), buf)
+    buf.seek(0)
+    m2 = Linear8bitLt(K, N, device="cuda")
+    m2.load_state_dict(torch.load(buf))
+    x = torch.from_numpy(_x((40,), K, (3,), seed=9).view(np.int16)).view(torch.float16).cuda()
+    y1, y2 = host(m(x)), host(m2(x))
+    sync_ok()
+    assert np.array_equal(y1.view(np.uint16), y2.view(np.uint16))
+
+
+def test_replaced_layer_stack_layer_by_layer():
+    """Linear -> GELU -> Linear (+ an fp16 head left alone): each int8 layer matches the
+    oracle on the activations it actually received."""
+    K, H = 512, 1024
+    model = torch.nn.Sequential(_fp16_linear(K, H, seed=1), torch.nn.GELU(),
+                                _fp16_linear(H, K, seed=2))
+    model.lm_head = _fp16_linear(K, 64, seed=3)
+    ws = [host(model[0].weight), host(model[2].weight)]
+    bs = [host(model[0].bias), host(model[2].bias)]
+    replace_linear_with_int8(model, threshold=6.0)
+    assert isinstance(model[0], Linear8bitLt) and isinstance(model[2], Linear8bitLt)
+    assert isinstance(model.lm_head, torch.nn.Linear)
+    X = _x((2, 24), K, (10, 300), seed=31)
+    x = torch.from_numpy(X.view(np.int16)).view(torch.float16).cuda()
+    h1 = model[0](x)
+    a1 = model[1](h1)
+    h2 = model[2](a1)
+    sync_ok()
+    for layer, (W, b, xin, y) in enumerate([(ws[0], bs[0], X, h1),
+                                            (ws[1], bs[1], host(a1), h2)]):
+        CBr, SCBr = O.quantize_weight(W)
+        ref = O.linear_forward(xin.reshape(-1, W.shape[1]), CBr, SCBr, b, 6.0)["C"]
+        check_output(host(y).reshape(-1, W.shape[0]), ref)

@@ -1,0 +1,66 @@
+"""Host-side checks of the nn.Module front end (no GPU): buffers, serialisation of the
+quantised state, argument checks, and the layer-replacement walk."""
+import io
+
+import pytest
+import torch
+
+from bit_matmul_decomposition_b200 import linear as L
+
+
+def test_buffers_and_shapes():
+    m = L.Linear8bitLt(64, 48, bias=True, threshold=6.0)
+    sd = m.state_dict()
+    assert set(sd) == {"CB", "SCB", "bias"}
+    assert sd["CB"].dtype == torch.int8 and tuple(sd["CB"].shape) == (48, 64)
+    assert sd["SCB"].dtype == torch.float32 and tuple(sd["SCB"].shape) == (48,)
+    assert sd["bias"].dtype == torch.float16 and tuple(sd["bias"].shape) == (48,)
+    assert set(L.Linear8bitLt(64, 48, bias=False).state_dict()) == {"CB", "SCB"}
+
+
+def test_in_features_must_be_a_multiple_of_16():
+    with pytest.raises(ValueError):
+        L.Linear8bitLt(40, 8)
+
+
+def test_state_dict_round_trip():
+    """CB / SCB serialisation: the quantised state saves and restores exactly."""
+    g = torch.Generator().manual_seed(3)
+    m = L.Linear8bitLt(32, 16)
+    m.CB.copy_(torch.randint(-127, 128, (16, 32), generator=g, dtype=torch.int8))
+    m.SCB.copy_(torch.rand(16, generator=g) + 0.25)
+    m.bias.copy_(torch.randn(16, generator=g).half())
+    buf = io.BytesIO()
+    torch.save(m.state_dict(), buf)
+    buf.seek(0)
+    m2 = L.Linear8bitLt(32, 16)
+    m2.load_state_dict(torch.load(buf))
+    assert torch.equal(m2.CB, m.CB) and torch.equal(m2.SCB, m.SCB) and torch.equal(m2.bias, m.bias)
+    # the dequantised weight is CB * SCB / 127 per output row
+    w = m.dequantized_weight()
+    assert torch.allclose(w[3], m.CB[3].float() * m.SCB[3] / 127.0)
+
+
+def test_forward_rejects_other_dtypes_before_any_call():
+    m = L.Linear8bitLt(32, 8)
+    with pytest.raises(TypeError):
+        m(torch.zeros(2, 32))
+    with pytest.raises(ValueError):
+        m(torch.zeros(2, 16, dtype=torch.float16))
+
+
+def test_replace_walk(monkeypatch):
+    made = []
+
+    def fake_from_linear(linear, threshold=6.0):
+        made.append((linear.in_features, linear.out_features, threshold))
+        return torch.nn.Identity()
+
+    monkeypatch.setattr(L.Linear8bitLt, "from_linear", staticmethod(fake_from_linear))
+    model = torch.nn.Sequential(torch.nn.Linear(32, 64), torch.nn.GELU(),
+                                torch.nn.Sequential(torch.nn.Linear(64, 32)))
+    model.lm_head = torch.nn.Linear(32, 10)
+    L.replace_linear_with_int8(model, threshold=5.0)
+    assert made == [(32, 64, 5.0), (64, 32, 5.0)]
+    assert isinstance(model[0], torch.nn.Identity) and isinstance(model[2][0], torch.nn.Identity)
+    assert isinstance(model.lm_head, torch.nn.Linear)
