@@ -236,9 +236,9 @@ __device__ __forceinline__ int tile_arrive(unsigned long long* c, uint32_t e) {
 // of the same launch starts the next generation of `target` arrivals).  The wait is
 // bounded: false after `lim` ns (the error word records it).
 __device__ __forceinline__ uint32_t grid_arrive(unsigned long long* ctr, uint32_t e,
-                                                uint32_t target) {
+                                                uint32_t target, bool claimed = false) {
   fence_acq_rel_gpu();  // this CTA's writes before its arrival
-  tag_claim(ctr, e);
+  if (!claimed) tag_claim(ctr, e);
   const uint32_t c = static_cast<uint32_t>(atomicAdd(ctr, 1ull));
   return (c / target + 1) * target;
 }
@@ -259,8 +259,8 @@ __device__ __forceinline__ bool grid_wait(unsigned long long* ctr, uint32_t e, u
 }
 
 __device__ __forceinline__ bool grid_sync(unsigned long long* ctr, uint32_t e, uint32_t target,
-                                          uint64_t lim) {
-  return grid_wait(ctr, e, grid_arrive(ctr, e, target), lim);
+                                          uint64_t lim, bool claimed = false) {
+  return grid_wait(ctr, e, grid_arrive(ctr, e, target, claimed), lim);
 }
 
 // Consumer side of the ring: wait for stage s (phase ph), then advance.
@@ -371,6 +371,12 @@ __device__ __forceinline__ bool forward_prologue(
     // global codes; grid barrier; then this CTA's slice of the codes is copied into xs.
     const int64_t TG = static_cast<int64_t>(T) * G;
     const int64_t f_lo = TG * blockIdx.x / gridDim.x, f_hi = TG * (blockIdx.x + 1) / gridDim.x;
+    // claim the barrier counters and the row-maximum words for this epoch now, while the
+    // scan's loads are in flight (every CTA does; all but the first claim of a word fail)
+    if (ct < 3)
+      tag_claim(a.gbar + ct, e);
+    else if (ct < 3 + T)
+      tag_claim(a.gscx + (ct - 3), e);
     for (int64_t f = f_lo + ct; f < f_hi; f += CW * 32) {
       const int64_t t = f / G, g = f - t * G;
       const uint4 v = ldg_v4(X + t * K + g * 8);
@@ -383,7 +389,7 @@ __device__ __forceinline__ bool forward_prologue(
       }
     }
     compute_sync();
-    if (ct == 0 && !grid_sync(a.gbar, e, gridDim.x, a.lim)) *abort_flag = 1;
+    if (ct == 0 && !grid_sync(a.gbar, e, gridDim.x, a.lim, true)) *abort_flag = 1;
     compute_sync();
     ok = *abort_flag == 0;
     for (int64_t x = ct; x < KW; x += CW * 32) maskall[x] = ok ? tagged_get(a.gmask + x, e) : 0u;
@@ -396,13 +402,10 @@ __device__ __forceinline__ bool forward_prologue(
     }
     compute_sync();
     for (int t = ct; t < T && ok; t += CW * 32) {
-      if (rmx[t] != 0u) {
-        tag_claim(a.gscx + t, e);
-        atomicMax(a.gscx + t, (static_cast<unsigned long long>(e) << 32) | rmx[t]);
-      }
+      if (rmx[t] != 0u) atomicMax(a.gscx + t, (static_cast<unsigned long long>(e) << 32) | rmx[t]);
     }
     compute_sync();
-    if (ct == 0 && ok && !grid_sync(a.gbar + 1, e, gridDim.x, a.lim)) *abort_flag = 1;
+    if (ct == 0 && ok && !grid_sync(a.gbar + 1, e, gridDim.x, a.lim, true)) *abort_flag = 1;
     compute_sync();
     ok = *abort_flag == 0;
     for (int t = ct; t < T; t += CW * 32) {
@@ -420,7 +423,7 @@ __device__ __forceinline__ bool forward_prologue(
     // the codes are read back by TMA (the async proxy) in other CTAs
     asm volatile("fence.proxy.async.global;" ::: "memory");
     compute_sync();
-    if (ct == 0 && ok) goal3 = grid_arrive(a.gbar + 2, e, gridDim.x);
+    if (ct == 0 && ok) goal3 = grid_arrive(a.gbar + 2, e, gridDim.x, true);
   }
 
   // (b) ranks (warp 0: lane l takes a contiguous run of mask words)

@@ -540,6 +540,47 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
     return j < kPrepMaxIdx ? sidx[j] : nth_outlier(smask, spre, words, j);
   };
 
+  // The CB_o gather of phase 4 for few outlier columns (one warp per (chunk, row) item,
+  // U4 items per batch) is bound by the latency of scattered byte reads of CB in HBM, so
+  // each warp issues its first batch here and stores it after the quantisation: those
+  // loads are in flight while the rows are quantised.
+  constexpr int U4 = 8;
+  const int64_t chunks4 = (n_o + 63) >> 6;
+  const int64_t nbuf4 = min(static_cast<int64_t>(kPrepWarps), p.cache_bytes_all / K);
+  const bool few4 = p.CB_o != nullptr && n_o > 0 &&
+                    !(static_cast<int64_t>(n_o) * 32 >= K && nbuf4 > 0);
+  const int64_t items4 = chunks4 * p.N;
+  const int64_t nw4 = static_cast<int64_t>(gridDim.x) * kPrepWarps;
+  const int64_t first4 = (static_cast<int64_t>(blockIdx.x) * kPrepWarps + warp) * U4;
+  // (the loaded bytes stay unconverted until the store, so nothing waits on them before)
+  auto gather_load = [&](int64_t it0, int (&v0)[U4], int (&v1)[U4]) {
+#pragma unroll
+    for (int u = 0; u < U4; ++u) {
+      const int64_t it = it0 + u;
+      v0[u] = 0;
+      v1[u] = 0;
+      if (it < items4) {
+        const int64_t c = it / p.N, n = it - c * p.N;
+        const int64_t j0 = c * 64 + 2 * lane;
+        if (j0 < n_o) v0[u] = p.CB[n * K + idx_at(j0)];
+        if (j0 + 1 < n_o) v1[u] = p.CB[n * K + idx_at(j0 + 1)];
+      }
+    }
+  };
+  auto gather_store = [&](int64_t it0, const int (&v0)[U4], const int (&v1)[U4]) {
+#pragma unroll
+    for (int u = 0; u < U4; ++u) {
+      const int64_t it = it0 + u;
+      if (it < items4) {
+        const int64_t c = it / p.N, n = it - c * p.N;
+        reinterpret_cast<__half2*>(p.CB_o + (c * p.N + n) * 64)[lane] =
+            __floats2half2_rn(static_cast<float>(v0[u]), static_cast<float>(v1[u]));
+      }
+    }
+  };
+  int pv0[U4], pv1[U4];
+  if (few4) gather_load(first4, pv0, pv1);
+
   // ------------------------------------------------ phase 3: quantise
   // Rows go in rounds of (16 / wpr) rows with wpr warps per row (wpr = 1 when the CTA owns
   // 16 rows or more; up to 16 when it owns one, as in decode batches).  Every warp walks
@@ -639,34 +680,13 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
       }
     } else {
       // Few outlier columns: one warp per (chunk, row) item, 8 items in flight per warp
-      // (the loads are scattered bytes of CB, so latency sets the pace).
-      constexpr int U = 8;
-      const int64_t items = chunks * p.N;
-      const int64_t nw = static_cast<int64_t>(gridDim.x) * kPrepWarps;
-      for (int64_t it0 = (static_cast<int64_t>(blockIdx.x) * kPrepWarps + warp) * U; it0 < items;
-           it0 += nw * U) {
-        float v0[U], v1[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int64_t it = it0 + u;
-          v0[u] = 0.0f;
-          v1[u] = 0.0f;
-          if (it < items) {
-            const int64_t c = it / p.N, n = it - c * p.N;
-            const int64_t j0 = c * 64 + 2 * lane;
-            if (j0 < n_o) v0[u] = static_cast<float>(p.CB[n * K + idx_at(j0)]);
-            if (j0 + 1 < n_o) v1[u] = static_cast<float>(p.CB[n * K + idx_at(j0 + 1)]);
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int64_t it = it0 + u;
-          if (it < items) {
-            const int64_t c = it / p.N, n = it - c * p.N;
-            reinterpret_cast<__half2*>(p.CB_o + (c * p.N + n) * 64)[lane] =
-                __floats2half2_rn(v0[u], v1[u]);
-          }
-        }
+      // (the loads are scattered bytes of CB, so latency sets the pace); the first batch
+      // was loaded before phase 3.
+      gather_store(first4, pv0, pv1);
+      for (int64_t it0 = first4 + nw4 * U4; it0 < items4; it0 += nw4 * U4) {
+        int v0[U4], v1[U4];
+        gather_load(it0, v0, v1);
+        gather_store(it0, v0, v1);
       }
     }
   }
