@@ -380,6 +380,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
   int32_t* sidx = spre + words + 1;
   float* samax = reinterpret_cast<float*>(sidx + kPrepMaxIdx);   // [rows_per_cta]
   __shared__ __align__(8) uint64_t s_bar[kPrepMaxChunks];
+  __shared__ __align__(8) uint64_t s_rbar[kPrepWarps];  // phase 4 row buffers
   __shared__ int s_fail;
   __shared__ int s_wsum[kPrepWarps];
   __shared__ float s_red[kPrepWarps];
@@ -396,6 +397,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
   if (tid == 0) {
     s_fail = 0;
     for (int c = 0; c < nchunks; ++c) mbar_init(smem_u32(&s_bar[c]), 1);
+    for (int c = 0; c < kPrepWarps; ++c) mbar_init(smem_u32(&s_rbar[c]), 1);
     fence_mbar_init();
   }
   for (int64_t w = tid; w < words; w += kPrepThreads) smask[w] = 0u;
@@ -648,32 +650,40 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
     const int64_t chunks = (n_o + 63) >> 6;
     const int64_t nbuf = min(static_cast<int64_t>(kPrepWarps), p.cache_bytes_all / K);
     if (static_cast<int64_t>(n_o) * 32 >= K && nbuf > 0) {
-      // Many outlier columns: stream whole CB rows (coalesced) into a per-warp buffer in
-      // the freed row cache and pick the outlier columns there.
+      // Many outlier columns: whole CB rows come by bulk copy into a per-warp buffer in the
+      // freed row cache (one round trip per row), and the warp picks the outlier columns
+      // there, four chunks' picks in flight at a time.
       if (warp < nbuf) {
         uint8_t* rowbuf = psm + static_cast<size_t>(warp) * static_cast<size_t>(K);
+        const uint32_t bar = smem_u32(&s_rbar[warp]);
         const int64_t nw = static_cast<int64_t>(gridDim.x) * nbuf;
+        uint32_t ph = 0;
+        int no_abort = 0;
         for (int64_t n = static_cast<int64_t>(blockIdx.x) * nbuf + warp; n < p.N; n += nw) {
-          const uint4* src = reinterpret_cast<const uint4*>(p.CB + n * K);
-          int v = lane;
-          for (; v + 96 < g32_of(K); v += 128) {
-            uint4 x0 = ldg_stream_v4(src + v), x1 = ldg_stream_v4(src + v + 32);
-            uint4 x2 = ldg_stream_v4(src + v + 64), x3 = ldg_stream_v4(src + v + 96);
-            reinterpret_cast<uint4*>(rowbuf)[v] = x0;
-            reinterpret_cast<uint4*>(rowbuf)[v + 32] = x1;
-            reinterpret_cast<uint4*>(rowbuf)[v + 64] = x2;
-            reinterpret_cast<uint4*>(rowbuf)[v + 96] = x3;
+          if (lane == 0) {
+            // the buffer's previous reads (generic proxy) come before the copy into it
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(K));
+            bulk_load(smem_u32(rowbuf), p.CB + n * K, static_cast<uint32_t>(K), bar);
           }
-          for (; v < g32_of(K); v += 32) reinterpret_cast<uint4*>(rowbuf)[v] = ldg_stream_v4(src + v);
-          __syncwarp();
-          for (int64_t c = 0; c < chunks; ++c) {
-            const int64_t j0 = c * 64 + 2 * lane;
-            float v0 = 0.0f, v1 = 0.0f;
-            if (j0 < n_o) v0 = static_cast<float>(static_cast<int8_t>(rowbuf[idx_at(j0)]));
-            if (j0 + 1 < n_o)
-              v1 = static_cast<float>(static_cast<int8_t>(rowbuf[idx_at(j0 + 1)]));
-            reinterpret_cast<__half2*>(p.CB_o + (c * p.N + n) * 64)[lane] =
-                __floats2half2_rn(v0, v1);
+          const bool got = mbar_wait(bar, ph, &no_abort, p.wait_limit_ns);
+          ph ^= 1u;
+          if (!__all_sync(0xffffffffu, got)) break;
+          for (int64_t c0 = 0; c0 < chunks; c0 += 4) {
+            float v0[4], v1[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int64_t j0 = (c0 + u) * 64 + 2 * lane;
+              v0[u] = j0 < n_o ? static_cast<float>(static_cast<int8_t>(rowbuf[idx_at(j0)])) : 0.0f;
+              v1[u] = j0 + 1 < n_o
+                          ? static_cast<float>(static_cast<int8_t>(rowbuf[idx_at(j0 + 1)]))
+                          : 0.0f;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              if (c0 + u < chunks)
+                reinterpret_cast<__half2*>(p.CB_o + ((c0 + u) * p.N + n) * 64)[lane] =
+                    __floats2half2_rn(v0[u], v1[u]);
           }
           __syncwarp();
         }
