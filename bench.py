@@ -449,6 +449,72 @@ def run_gpu(args, w0):
     return 0
 
 
+def run_train(args, w):
+    """--mode train (one GPU): a training step of the fp16-weight mode of the nn.Module
+    front end -- re-quantise the fp16 weight, the int8 decomposed forward (library kernels)
+    and the straight-through backward (dx = dy W, dW = dy^T x, db = sum dy; fp16 GEMMs) --
+    on the workload's shapes.  Reports 3 x 2TNK / step time (forward + two backward
+    products), separately from the forward benchmark."""
+    import torch
+
+    from bit_matmul_decomposition_b200.linear import Linear8bitLt
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    T, K, N = w.T, w.K, w.N
+    X = fp16_tensor(synth.make_x(w), dev).requires_grad_(True)
+    m = Linear8bitLt(K, N, bias=True, threshold=w.threshold, device=dev, has_fp16_weights=True)
+    with torch.no_grad():
+        m.weight.copy_(fp16_tensor(synth.make_w(w), dev))
+        b = synth.make_bias(w)
+        if b is not None:
+            m.bias.copy_(fp16_tensor(b, dev))
+    gy = torch.randn((T, N), device=dev, dtype=torch.float16) * 0.01
+    flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=dev)
+
+    def step():
+        X.grad = None
+        m.weight.grad = None
+        m.bias.grad = None
+        m(X).backward(gy)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    clocks = ClockSampler()
+    clocks.start()
+    time.sleep(0.3)
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record()
+        step()
+        e1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    flops = 3.0 * 2.0 * T * N * K
+    print(json.dumps({
+        "metric": "int8 decomposed linear, training step (fp16 weights re-quantised, "
+                  "int8 forward, straight-through fp16 backward)",
+        "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "mode": "train", "data": "synthetic",
+        "config": dict(w.describe(), l2="256 MiB buffer written between timed steps"),
+        "clocks": clk}), flush=True)
+    st = abi_status()
+    if st != 0:
+        raise RuntimeError("device error in the training loop: %s" % st)
+    return 0
+
+
+def abi_status():
+    from bit_matmul_decomposition_b200 import abi
+    return abi.i8_sync_status()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -458,11 +524,16 @@ def main():
     ap.add_argument("--workload", default="opt_ffn_up", choices=sorted(workloads()))
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", default="forward", choices=["forward", "train"],
+                    help="train: one GPU, the fp16-weight training step of the module "
+                         "front end (not the forward benchmark)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     w = workloads()[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.mode == "train":
+        return run_train(args, w)
     return run_gpu(args, w)
 
 

@@ -8,9 +8,14 @@ runs the mixed-precision decomposition with an outlier threshold (6.0 by default
 helper that swaps the nn.Linear layers of a model for such layers, leaving named ones
 (typically the output head) in fp16.
 
-Inference only: the forward has no backward (the blog's fp16-weight training mode is not
-built), so outputs never require grad.  Everything numerical runs in the library's CUDA
-kernels; this module allocates tensors and marshals arguments.
+The blog also names a mode that keeps the fp16 weights for mixed-precision training
+(``has_fp16_weights=True``): the weight stays an fp16 parameter, is re-quantised by every
+forward, and gradients pass straight through the quantisation -- the blog gives no
+gradient formulas, so the plainest reading is taken: the backward of y = x W^T + b, i.e.
+dx = dy W, dW = dy^T x, db = sum(dy), with fp16 operands.  Without fp16 weights the layer
+still passes dx = dy W' back (W' = CB * SCB / 127, the weight it computes with), so layers
+before it can train.  The forward runs in the library's CUDA kernels; the backward
+products are plain fp16 GEMMs (torch.matmul, cuBLAS) on the same device.
 """
 from __future__ import annotations
 
@@ -19,6 +24,34 @@ from typing import Dict, Iterable, Optional
 import torch
 
 from . import abi
+
+
+class _Int8LinearFn(torch.autograd.Function):
+    """Forward: the decomposed int8 layer (CUDA library).  Backward: straight through the
+    quantisation, fp16 GEMMs."""
+
+    @staticmethod
+    def forward(ctx, x2, weight, bias, layer):
+        out = layer._forward_kernel(x2)
+        ctx.layer = layer
+        ctx.save_for_backward(x2, weight)
+        ctx.has_bias = bias is not None
+        return out
+
+    @staticmethod
+    def backward(ctx, gy):
+        x2, weight = ctx.saved_tensors
+        layer = ctx.layer
+        gy = gy.to(torch.float16).contiguous()
+        gx = gw = gb = None
+        if ctx.needs_input_grad[0]:
+            w = weight if weight is not None else layer.dequantized_weight().to(torch.float16)
+            gx = gy @ w
+        if weight is not None and ctx.needs_input_grad[1]:
+            gw = gy.t() @ x2
+        if ctx.has_bias and ctx.needs_input_grad[2]:
+            gb = gy.float().sum(0).to(torch.float16)
+        return gx, gw, gb, None
 
 
 class Linear8bitLt(torch.nn.Module):
@@ -34,7 +67,7 @@ class Linear8bitLt(torch.nn.Module):
     """
 
     def __init__(self, in_features: int, out_features: int, bias: bool = True,
-                 threshold: float = 6.0, device=None):
+                 threshold: float = 6.0, device=None, has_fp16_weights: bool = False):
         super().__init__()
         if in_features <= 0 or out_features <= 0 or in_features % 16 != 0:
             raise ValueError("in_features must be a positive multiple of 16 (row pitch of the "
@@ -46,7 +79,14 @@ class Linear8bitLt(torch.nn.Module):
                                                device=device))
         self.register_buffer("SCB", torch.zeros((out_features,), dtype=torch.float32,
                                                 device=device))
-        if bias:
+        self.has_fp16_weights = bool(has_fp16_weights)
+        if self.has_fp16_weights:
+            # training mode: fp16 master weight (and bias) as parameters, CB / SCB derived
+            self.weight = torch.nn.Parameter(
+                torch.zeros((out_features, in_features), dtype=torch.float16, device=device))
+            self.bias = (torch.nn.Parameter(torch.zeros((out_features,), dtype=torch.float16,
+                                                        device=device)) if bias else None)
+        elif bias:
             self.register_buffer("bias", torch.zeros((out_features,), dtype=torch.float16,
                                                      device=device))
         else:
@@ -54,19 +94,27 @@ class Linear8bitLt(torch.nn.Module):
         self._ws: Dict[torch.device, torch.Tensor] = {}
 
     @classmethod
-    def from_linear(cls, linear: torch.nn.Linear, threshold: float = 6.0) -> "Linear8bitLt":
-        """Quantise an fp16 nn.Linear that lives on a CUDA device."""
+    def from_linear(cls, linear: torch.nn.Linear, threshold: float = 6.0,
+                    has_fp16_weights: bool = False) -> "Linear8bitLt":
+        """Quantise an nn.Linear that lives on a CUDA device (weights cast to fp16)."""
         w = linear.weight
         if not w.is_cuda:
             raise ValueError("the weight must be on a CUDA device (it is quantised there)")
         m = cls(linear.in_features, linear.out_features, bias=linear.bias is not None,
-                threshold=threshold, device=w.device)
-        m.quantize_(w.detach(), None if linear.bias is None else linear.bias.detach())
+                threshold=threshold, device=w.device, has_fp16_weights=has_fp16_weights)
+        if has_fp16_weights:
+            with torch.no_grad():
+                m.weight.copy_(w.detach().to(torch.float16))
+                if linear.bias is not None:
+                    m.bias.copy_(linear.bias.detach().to(torch.float16))
+        else:
+            m.quantize_(w.detach(), None if linear.bias is None else linear.bias.detach())
         return m
 
     @torch.no_grad()
     def quantize_(self, weight: torch.Tensor, bias: Optional[torch.Tensor] = None):
-        """Quantise an fp16 [out, in] weight (on this layer's CUDA device) into CB / SCB."""
+        """Quantise an fp16 [out, in] weight (on this layer's CUDA device) into CB / SCB
+        (inference mode; with fp16 weights every forward does this from ``weight``)."""
         if weight.shape != (self.out_features, self.in_features):
             raise ValueError("weight shape %s, expected %s"
                              % (tuple(weight.shape), (self.out_features, self.in_features)))
@@ -92,7 +140,16 @@ class Linear8bitLt(torch.nn.Module):
             self._ws[dev] = ws
         return ws
 
-    @torch.no_grad()
+    def _forward_kernel(self, x2: torch.Tensor) -> torch.Tensor:
+        """One i8_linear_forward call on a [T, in] fp16 input (no autograd)."""
+        T = x2.shape[0]
+        out = torch.empty((T, self.out_features), dtype=torch.float16, device=x2.device)
+        if T > 0:
+            bias = None if self.bias is None else self.bias.detach()
+            abi.i8_linear_forward(x2, self.CB, self.SCB, bias, self.threshold, out,
+                                  self._workspace(T))
+        return out
+
     def forward(self, x: torch.Tensor) -> torch.Tensor:
         if x.dtype != torch.float16:
             raise TypeError("input must be fp16 (got %s)" % x.dtype)
@@ -101,26 +158,33 @@ class Linear8bitLt(torch.nn.Module):
                              % (x.shape[-1], self.in_features))
         lead = x.shape[:-1]
         x2 = x.reshape(-1, self.in_features).contiguous()
-        T = x2.shape[0]
-        out = torch.empty((T, self.out_features), dtype=torch.float16, device=x2.device)
-        if T > 0:
-            abi.i8_linear_forward(x2, self.CB, self.SCB, self.bias, self.threshold, out,
-                                  self._workspace(T))
-        return out.reshape(*lead, self.out_features)
+        if self.has_fp16_weights:
+            with torch.no_grad():  # the weight may have changed since the last forward
+                abi.i8_quantize_weight(self.weight.detach().contiguous(), self.CB, self.SCB)
+        w = self.weight if self.has_fp16_weights else None
+        if torch.is_grad_enabled() and (x2.requires_grad or (w is not None and w.requires_grad)):
+            y = _Int8LinearFn.apply(x2, w, self.bias, self)
+        else:
+            y = self._forward_kernel(x2)
+        return y.reshape(*lead, self.out_features)
 
     def extra_repr(self) -> str:
-        return "in_features=%d, out_features=%d, bias=%s, threshold=%g" % (
-            self.in_features, self.out_features, self.bias is not None, self.threshold)
+        return "in_features=%d, out_features=%d, bias=%s, threshold=%g, has_fp16_weights=%s" % (
+            self.in_features, self.out_features, self.bias is not None, self.threshold,
+            self.has_fp16_weights)
 
 
 def replace_linear_with_int8(model: torch.nn.Module, threshold: float = 6.0,
-                             skip: Iterable[str] = ("lm_head",)) -> torch.nn.Module:
+                             skip: Iterable[str] = ("lm_head",),
+                             has_fp16_weights: bool = False) -> torch.nn.Module:
     """Swap every nn.Linear of `model` (weights on a CUDA device) for a Linear8bitLt, in
     place, except modules whose name (last path component) is in `skip`.  Returns `model`."""
     skip = set(skip)
     for name, child in list(model.named_children()):
         if isinstance(child, torch.nn.Linear) and name not in skip:
-            setattr(model, name, Linear8bitLt.from_linear(child, threshold=threshold))
+            setattr(model, name, Linear8bitLt.from_linear(child, threshold=threshold,
+                                                          has_fp16_weights=has_fp16_weights))
         elif name not in skip:
-            replace_linear_with_int8(child, threshold=threshold, skip=skip)
+            replace_linear_with_int8(child, threshold=threshold, skip=skip,
+                                     has_fp16_weights=has_fp16_weights)
     return model

@@ -95,3 +95,58 @@ def test_replaced_layer_stack_layer_by_layer():
         CBr, SCBr = O.quantize_weight(W)
         ref = O.linear_forward(xin.reshape(-1, W.shape[1]), CBr, SCBr, b, 6.0)["C"]
         check_output(host(y).reshape(-1, W.shape[0]), ref)
+
+
+def _ref_grads(X, W, gy):
+    """Backward of y = x W^T + b in fp64: dx = dy W, dW = dy^T x, db = sum(dy)."""
+    x64, w64, g64 = X.astype(np.float64), W.astype(np.float64), gy.astype(np.float64)
+    return g64 @ w64, g64.T @ x64, g64.sum(0)
+
+
+def _close(a, ref, rel=1e-2):
+    a = a.astype(np.float64)
+    assert np.isfinite(a).all()
+    err = np.abs(a - ref).max()
+    assert err <= rel * np.abs(ref).max() + 1e-3, (err, np.abs(ref).max())
+
+
+@pytest.mark.parametrize("T", [6, 40], ids=["decode", "gemm"])
+def test_training_mode_forward_backward_and_step(T):
+    K, N = 512, 384
+    lin = _fp16_linear(K, N, seed=7)
+    m = Linear8bitLt.from_linear(lin, threshold=6.0, has_fp16_weights=True)
+    X = _x((T,), K, (5, 77), seed=13)
+    x = torch.from_numpy(X.view(np.int16)).view(torch.float16).cuda().requires_grad_(True)
+    y = m(x)
+    W = host(m.weight)
+    CBr, SCBr = O.quantize_weight(W)
+    check_output(host(y), O.linear_forward(X, CBr, SCBr, host(m.bias), 6.0)["C"])
+    gy = synth.random_fp16((T, N), seed=17, sigma=0.5)
+    y.backward(torch.from_numpy(gy.view(np.int16)).view(torch.float16).cuda())
+    sync_ok()
+    gx_r, gw_r, gb_r = _ref_grads(X, W, gy)
+    _close(host(x.grad), gx_r)
+    _close(host(m.weight.grad), gw_r)
+    _close(host(m.bias.grad), gb_r)
+    # one SGD step on the fp16 weight; the next forward quantises the new weight
+    with torch.no_grad():
+        m.weight -= 1e-4 * m.weight.grad
+    y2 = m(x.detach())
+    sync_ok()
+    W2 = host(m.weight)
+    CB2, SCB2 = O.quantize_weight(W2)
+    assert np.array_equal(host(m.CB), CB2)
+    check_output(host(y2), O.linear_forward(X, CB2, SCB2, host(m.bias), 6.0)["C"])
+
+
+def test_inference_mode_passes_input_gradients():
+    K, N, T = 256, 128, 20
+    m = Linear8bitLt.from_linear(_fp16_linear(K, N, seed=19))
+    X = _x((T,), K, (9,), seed=23)
+    x = torch.from_numpy(X.view(np.int16)).view(torch.float16).cuda().requires_grad_(True)
+    gy = synth.random_fp16((T, N), seed=29, sigma=0.5)
+    m(x).backward(torch.from_numpy(gy.view(np.int16)).view(torch.float16).cuda())
+    sync_ok()
+    Wd = host(m.CB).astype(np.float64) * (host(m.SCB).astype(np.float64) / 127.0)[:, None]
+    _close(host(x.grad), gy.astype(np.float64) @ Wd)
+    assert all(p.grad is None for p in m.parameters())

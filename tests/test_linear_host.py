@@ -52,7 +52,7 @@ def test_forward_rejects_other_dtypes_before_any_call():
 def test_replace_walk(monkeypatch):
     made = []
 
-    def fake_from_linear(linear, threshold=6.0):
+    def fake_from_linear(linear, threshold=6.0, has_fp16_weights=False):
         made.append((linear.in_features, linear.out_features, threshold))
         return torch.nn.Identity()
 
@@ -64,3 +64,12 @@ def test_replace_walk(monkeypatch):
     assert made == [(32, 64, 5.0), (64, 32, 5.0)]
     assert isinstance(model[0], torch.nn.Identity) and isinstance(model[2][0], torch.nn.Identity)
     assert isinstance(model.lm_head, torch.nn.Linear)
+
+
+def test_training_mode_holds_fp16_parameters():
+    m = L.Linear8bitLt(64, 32, bias=True, has_fp16_weights=True)
+    assert {n for n, _ in m.named_parameters()} == {"weight", "bias"}
+    assert m.weight.dtype == torch.float16 and m.weight.requires_grad
+    assert {n for n, _ in m.named_buffers()} == {"CB", "SCB"}
+    assert set(m.state_dict()) == {"weight", "bias", "CB", "SCB"}
+    assert {n for n, _ in L.Linear8bitLt(64, 32).named_parameters()} == set()
