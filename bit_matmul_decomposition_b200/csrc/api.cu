@@ -367,10 +367,11 @@ i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t
 // decode: one launch of the decode kernel (forward from X, or the raw product of codes)
 std::atomic<unsigned long long> g_epoch{0};
 
-// The prologue of the forward reads all of X in every CTA when X fits two ring stages;
-// beyond that the CTAs split it (cooperative launch, three grid barriers).
+// The prologue of the forward reads all of X in every CTA when X fits eight ring stages
+// (128 KB: ~1 us per stage, against ~12 us for the cooperative prologue's three grid
+// barriers); beyond that the CTAs split it (cooperative launch).
 bool decode_coop(bool raw, int64_t T, int64_t K) {
-  return !raw && T * K * 2 > 2 * static_cast<int64_t>(gemv::STAGE_BYTES);
+  return !raw && T * K * 2 > 8 * static_cast<int64_t>(gemv::STAGE_BYTES);
 }
 
 i8_status run_decode(bool raw, const void* X, const int8_t* Xq, int64_t T, int64_t K,

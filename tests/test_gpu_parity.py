@@ -148,6 +148,7 @@ FORWARD_CASES = [
     (8, 65536, 40, (0, 30000, 65535), 0.0, 6.0, True),     # decode, largest K (19 slices)
     (4, 65552, 33, (1, 65551), 0.0, 6.0, True),     # T <= 16 beyond 65536: GEMM path
     (12, 3584, 48, (3583,), 0.0, 6.0, False),       # one slice, last column an outlier
+    (9, 8000, 333, (1, 4000, 7999), 0.0, 6.0, True),  # decode, X > 128 KB: split prologue
     (40, 9216, 96, (), 0.0, 0.0, True),             # GEMM, n_o = 9216 (> 8192 kept indices)
 ]
 
@@ -174,11 +175,11 @@ def test_forward_repeat_is_deterministic():
     assert np.array_equal(C1.view(np.uint16), C2.view(np.uint16))
 
 
-@pytest.mark.parametrize("K", [2048, 4096], ids=["x_per_cta", "x_split"])
+@pytest.mark.parametrize("K", [2048, 12288], ids=["x_per_cta", "x_split"])
 def test_decode_row_max_next_to_an_outlier_column(K):
     """SCx excludes outlier columns but keeps the other columns of their block: each row's
     largest non-outlier value sits right beside an outlier column (K = 2048: every CTA
-    scans all of X; K = 4096: the CTAs split the scan)."""
+    scans all of X; K = 12288, X > 128 KB: the CTAs split the scan)."""
     T, N = 6, 96
     w, X, W, b = _case(T, K, N, seed=21, cols=(300, 1500))
     X = np.clip(X.astype(np.float32), -3.0, 3.0).astype(np.float16)
@@ -197,13 +198,14 @@ def test_decode_row_max_next_to_an_outlier_column(K):
 
 @pytest.mark.parametrize("T", [1, 16])
 def test_decode_workspace_garbage_and_reuse(T):
-    """The decode kernel's tile counters need no clearing: a workspace full of 0xff, then
-    reused by further calls (also of another shape), gives the same output every time."""
-    w, X, W, b = _case(T, 3600, 1000, seed=T + 40, cols=(10, 2000))
+    """The decode kernel's counters and epoch-tagged words need no clearing: a workspace
+    full of 0xff, then reused by further calls (also of another shape), gives the same
+    output every time (T = 16: X > 128 KB, the cooperative prologue)."""
+    w, X, W, b = _case(T, 4608, 1000, seed=T + 40, cols=(10, 2000))
     CB, SCB = gpu_quantize_weight(dev(W))
     X_d, b_d = dev(X), dev(b)
-    nbytes = max(abi.i8_linear_workspace_size(T, 1000, 3600),
-                 abi.i8_linear_workspace_size(2, 500, 3600))
+    nbytes = max(abi.i8_linear_workspace_size(T, 1000, 4608),
+                 abi.i8_linear_workspace_size(2, 500, 4608))
     ws = torch.full((nbytes,), 255, dtype=torch.uint8, device="cuda")
     CBr, SCBr = O.quantize_weight(W)
     ref = O.linear_forward(X, CBr, SCBr, b, 6.0)["C"]
@@ -213,7 +215,7 @@ def test_decode_workspace_garbage_and_reuse(T):
         abi.i8_linear_forward(X_d, CB, SCB, b_d, 6.0, C, ws)
         outs.append(host(C))
         if i == 1:  # another shape on the same workspace in between
-            X2 = dev(synth.random_fp16((2, 3600), seed=7, sigma=1.0))
+            X2 = dev(synth.random_fp16((2, 4608), seed=7, sigma=1.0))
             C2 = torch.empty((2, 500), dtype=torch.float16, device="cuda")
             abi.i8_linear_forward(X2, CB[:500].contiguous(), SCB[:500].contiguous(), None,
                                   6.0, C2, ws)
