@@ -148,8 +148,11 @@ size_t i8_linear_workspace_size(int64_t T, int64_t N, int64_t K);
  *   workspace  device buffer of at least i8_linear_workspace_size(T, N, K) bytes, owned by
  *              the caller; its contents need no initialisation and are scratch after the
  *              call (calls sharing one workspace must be ordered on one stream).
- * T <= 16 runs the decode path (warp-level int8 tensor-core GEMV, split over K);
- * larger T runs the tcgen05 kind::i8 GEMM with the fused outlier/dequant epilogue.
+ * T <= 16 with K <= 65536 runs the decode path: one kernel (one CTA per SM, each on a
+ * K-slice; CB streamed once by TMA into warp-level int8 tensor-core MMAs; steps 1 and 2
+ * in its prologue, a cooperative launch when 2*T*K > 128 KB; the outlier sum per K-slice,
+ * then across slices, in fp32).  Otherwise: the fused prepare pass and the tcgen05
+ * kind::i8 GEMM with the outlier/dequant epilogue (a memset and two kernels).
  */
 i8_status i8_linear_forward(const void* X, int64_t T, int64_t K, const int8_t* CB,
                             const float* SCB, const void* bias, int64_t N, float threshold,
@@ -180,8 +183,8 @@ i8_status i8_linear_forward_noalloc(const void* X, int64_t T, int64_t K, const i
 
 /*
  * Step 4 alone -- acc[T, N] int32 = A[T, K] int8 * B[N, K]^T int8, on the same kernels
- * as i8_linear_forward (the tcgen05 GEMM for T > 16, the decode GEMV for T <= 16), with
- * the epilogue writing the raw accumulator.  Source: "内部的 MatMul" (the 8-bit matrix
+ * as i8_linear_forward (the tcgen05 GEMM, or the decode kernel for T <= 16 and
+ * K <= 65536), with the epilogue writing the raw accumulator.  Source: "内部的 MatMul" (the 8-bit matrix
  * multiplication).  Exact: |acc| <= K * 127^2 must fit in int32 (K <= 133144).
  *   workspace: at least i8_linear_workspace_size(T, N, K) bytes.
  */
@@ -198,7 +201,8 @@ i8_status i8_sync_status(void* stream);
 /*
  * Benchmark hook: when both are non-NULL cudaEvent_t handles, every following
  * i8_linear_forward records `start` just before and `stop` just after its dominant
- * kernel (the GEMM or the decode GEMV), on the call's stream.  NULL, NULL turns it off.
+ * kernel (the GEMM; on the decode path the decode kernel, i.e. the whole forward), on the
+ * call's stream.  NULL, NULL turns it off.
  * Process-wide; meant for single-threaded benchmarking.
  */
 i8_status i8_set_profile_events(void* start_event, void* stop_event);
