@@ -34,6 +34,10 @@ SIGNATURES = {
     "i8_linear_forward": (_ST, [_P, _I64, _I64, _P, _P, _P, _I64, _F, _P, _P, _SZ, _P]),
     "i8_igemm_s32": (_ST, [_P, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
     "i8_linear_forward_noalloc": (_ST, [_P, _I64, _I64, _P, _P, _P, _I64, _F, _P, _P]),
+    "i8_outlier_cache_size": (_SZ, [_I64, _I64, _I64]),
+    "i8_outlier_cache_reset": (_ST, [_P, _SZ, _P]),
+    "i8_linear_forward_cached": (_ST, [_P, _I64, _I64, _P, _P, _P, _I64, _F, _P, _P, _SZ, _P,
+                                       _SZ, _P]),
     "i8_sync_status": (_ST, [_P]),
     "i8_set_profile_events": (_ST, [_P, _P]),
     "i8_selftest_bounded_wait": (_ST, [_I64, _P]),
@@ -142,6 +146,28 @@ def i8_linear_forward_noalloc(X, CB, SCB, bias, threshold, C, stream=None):
     _check("i8_linear_forward_noalloc",
            load().i8_linear_forward_noalloc(_ptr(X), T, K, _ptr(CB), _ptr(SCB), _ptr(bias), N,
                                             float(threshold), _ptr(C), _stream(stream)))
+
+
+def i8_outlier_cache_size(N, K, max_cols) -> int:
+    return int(load().i8_outlier_cache_size(N, K, max_cols))
+
+
+def i8_outlier_cache_reset(cache, stream=None):
+    _check("i8_outlier_cache_reset",
+           load().i8_outlier_cache_reset(_ptr(cache), cache.numel() * cache.element_size(),
+                                         _stream(stream)))
+
+
+def i8_linear_forward_cached(X, CB, SCB, bias, threshold, C, workspace, cache, stream=None):
+    """i8_linear_forward keeping the weight's outlier-column codes in `cache` across calls."""
+    T, K = X.shape
+    N = CB.shape[0]
+    _check("i8_linear_forward_cached",
+           load().i8_linear_forward_cached(_ptr(X), T, K, _ptr(CB), _ptr(SCB), _ptr(bias), N,
+                                           float(threshold), _ptr(C), _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(),
+                                           _ptr(cache), cache.numel() * cache.element_size(),
+                                           _stream(stream)))
 
 
 def i8_igemm_s32(A, B, acc, workspace, stream=None):

@@ -134,12 +134,13 @@ size_t slice_elems(int64_t rows, int64_t K) {
 bool use_decode(int64_t T, int64_t K) { return T <= kDecodeMaxT && K <= gemv::MAX_K; }
 
 struct Workspace {
-  size_t mask, idx, n_o, scx, xq, xo, cbo, rec, cnt, gmask, gscx, gbar, total;
+  size_t mask, idx, n_o, sel, scx, xq, xo, cbo, rec, cnt, gmask, gscx, gbar, total;
   int64_t zero_words;  // words from `mask` on that must be zero when a forward starts
 };
 
-// GEMM path: the first region holds the packed outlier mask and the grid-barrier word of
-// the fused prepare pass; one memset clears both at the start of every forward.
+// GEMM path: the first region holds the packed outlier mask, the grid-barrier word of the
+// fused prepare pass and its outlier-cache update counter; one memset clears them at the
+// start of every forward.
 // Decode path: the slice records of every 32-row tile, the tiles' arrival counters and the
 // words of the cooperative prologue (none needs clearing: they carry the launch's epoch).
 Workspace layout(int64_t T, int64_t N, int64_t K) {
@@ -163,16 +164,33 @@ Workspace layout(int64_t T, int64_t N, int64_t K) {
     return w;
   }
   const int64_t words = (K + 31) / 32;
-  w.zero_words = words + 1;
+  w.zero_words = words + 2;
   w.mask = take(static_cast<size_t>(w.zero_words) * 4);
   w.idx = take(static_cast<size_t>(K) * 4);
   w.n_o = take(16);
+  w.sel = take(16);
   w.scx = take(static_cast<size_t>(T) * 4);
   w.xq = take(static_cast<size_t>(T) * static_cast<size_t>(K));
   w.xo = take(slice_elems(T, K) * 2);
   w.cbo = take(slice_elems(N, K) * 2);
   w.total = off;
   return w;
+}
+
+// ------------------------------------------------------------------ outlier cache
+// [header: kOcacheHdrWords words + ceil(K/32) mask words, padded to 256 B]
+// [CB_o slice: chunk-major [cols / 64][N][64] fp16]
+size_t ocache_header_bytes(int64_t K) {
+  return align_up(static_cast<size_t>(kOcacheHdrWords + (K + 31) / 32) * 4, 256);
+}
+
+// columns a cache of `bytes` holds for an [N, K] weight (0 when it holds none)
+int64_t ocache_cols(size_t bytes, int64_t N, int64_t K) {
+  const size_t head = ocache_header_bytes(K);
+  if (bytes < head) return 0;
+  int64_t cols = static_cast<int64_t>((bytes - head) / (static_cast<size_t>(N) * 128u)) * 64;
+  const int64_t kmax = (K + 63) / 64 * 64;
+  return cols < kmax ? cols : kmax;
 }
 
 // ------------------------------------------------------------------ TMA descriptors
@@ -274,10 +292,13 @@ i8_status run_quant_rows(const void* A, int64_t R, int64_t K, const uint32_t* ma
 // mask must hold ceil(K/32) + 1 words; the last one is the grid-barrier counter.
 // `zero_words` words from `mask` on are cleared first (at least the mask and the barrier
 // word, ceil(K/32) + 1).
+// With an outlier cache (`ocache` non-NULL, `ocache_cols` columns), CB_o is kept there
+// across calls and *cbo_sel tells the GEMM which slice holds this call's CB_o.
 i8_status run_prepare(const void* X, int64_t T, int64_t K, float thr, uint32_t* mask,
                       int64_t zero_words, int32_t* idx, int32_t* n_o, int8_t* Xq, float* SCx,
                       void* X_o, const int8_t* CB, int64_t N, void* CB_o, const DeviceInfo& d,
-                      cudaStream_t s) {
+                      cudaStream_t s, uint8_t* ocache = nullptr, int64_t ocols = 0,
+                      int32_t* cbo_sel = nullptr) {
   if (cudaMemsetAsync(mask, 0, static_cast<size_t>(zero_words) * 4, s) != cudaSuccess)
     return I8_ERR_CUDA;
   const int64_t G0 = d.sms;
@@ -310,6 +331,11 @@ i8_status run_prepare(const void* X, int64_t T, int64_t K, float thr, uint32_t* 
   a.CB = CB;
   a.N = N;
   a.CB_o = static_cast<__half*>(CB_o);
+  a.ocache = reinterpret_cast<uint32_t*>(ocache);
+  a.ocache_CB_o =
+      ocache ? reinterpret_cast<__half*>(ocache + ocache_header_bytes(K)) : nullptr;
+  a.ocache_cols = ocache ? ocols : 0;
+  a.cbo_sel = cbo_sel;
   a.rows_per_cta = rows_per_cta;
   a.cache_rows = cache_rows;
   a.cache_bytes_all = cache_rows * K * 2;
@@ -322,11 +348,14 @@ i8_status run_prepare(const void* X, int64_t T, int64_t K, float thr, uint32_t* 
 }
 
 // tcgen05 GEMM (pairs of CTAs, 256 x 256 tiles); raw=true writes the int32 accumulator.
+// B_c (ocols columns) is the outlier cache's CB_o slice, read instead of B_o when the
+// device word *cbo_sel is nonzero.
 i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t* B, int64_t N,
                    const void* A_o, const void* B_o, const int32_t* n_o, const float* SCx,
                    const float* SCB, const void* bias, void* C, int32_t* acc,
-                   const DeviceInfo& d, cudaStream_t s) {
-  CUtensorMap tA, tB, tAo, tBo;
+                   const DeviceInfo& d, cudaStream_t s, const void* B_c = nullptr,
+                   int64_t ocols = 0, const int32_t* cbo_sel = nullptr) {
+  CUtensorMap tA, tB, tAo, tBo, tBc;
   if (!map_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, T, K, gemm::BK, gemm::HM) ||
       !map_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, K, gemm::BK, gemm::HN))
     return I8_ERR_CUDA;
@@ -338,6 +367,10 @@ i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t
     if (!map_slice(&tAo, A_o, T, chunks, gemm::HM) || !map_slice(&tBo, B_o, N, chunks, gemm::HN))
       return I8_ERR_CUDA;
   }
+  tBc = tBo;
+  if (!raw && B_c != nullptr && cbo_sel != nullptr &&
+      !map_slice(&tBc, B_c, N, static_cast<uint64_t>(ocols / 64), gemm::HN))
+    return I8_ERR_CUDA;
   gemm::Args a;
   a.T = static_cast<int>(T);
   a.N = static_cast<int>(N);
@@ -346,6 +379,7 @@ i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t
   a.n_tiles = static_cast<int>((N + gemm::TN - 1) / gemm::TN);
   a.k_blocks = static_cast<int>((K + gemm::BK - 1) / gemm::BK);
   a.n_outliers = raw ? nullptr : n_o;
+  a.cbo_sel = (raw || B_c == nullptr) ? nullptr : cbo_sel;
   a.SCx = SCx;
   a.SCB = SCB;
   a.bias = static_cast<const __half*>(bias);
@@ -357,10 +391,10 @@ i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t
   cudaError_t e;
   if (raw)
     e = launch_overlapped(gemm::i8_gemm_tcgen05_kernel<true>, dim3(2 * clusters),
-                          dim3(gemm::THREADS), gemm::SMEM_BYTES, s, tA, tB, tAo, tBo, a);
+                          dim3(gemm::THREADS), gemm::SMEM_BYTES, s, tA, tB, tAo, tBo, tBc, a);
   else
     e = launch_overlapped(gemm::i8_gemm_tcgen05_kernel<false>, dim3(2 * clusters),
-                          dim3(gemm::THREADS), gemm::SMEM_BYTES, s, tA, tB, tAo, tBo, a);
+                          dim3(gemm::THREADS), gemm::SMEM_BYTES, s, tA, tB, tAo, tBo, tBc, a);
   return e == cudaSuccess ? launch_status() : I8_ERR_CUDA;
 }
 
@@ -477,6 +511,52 @@ i8_status static_scratch_address(void** out) {
   return I8_OK;
 }
 
+// The forward of both entry points; `cache` (ocols columns) is NULL for the uncached one.
+i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, const float* SCB,
+                       const void* bias, int64_t N, float threshold, void* C, void* workspace,
+                       size_t workspace_bytes, uint8_t* cache, int64_t ocols, void* stream) {
+  if (!X || !CB || !SCB || !C || !workspace) return I8_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(CB) || !aligned16(SCB) || !aligned16(C) ||
+      !aligned16(workspace) || (bias && !aligned16(bias)))
+    return I8_ERR_INVALID_ARG;
+  if (!shape_ok(T, K) || N <= 0 || N > 0x7fffffffLL || threshold != threshold)
+    return I8_ERR_INVALID_ARG;
+  const Workspace w = layout(T, N, K);
+  if (workspace_bytes < w.total) return I8_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  i8_status st = device_info(&d);
+  if (st != I8_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const bool prof = g_prof_start != nullptr && g_prof_stop != nullptr;
+  if (use_decode(T, K)) {
+    // (the decode kernel takes the outlier columns' codes out of its own CB stream)
+    if (prof && cudaEventRecord(g_prof_start, s) != cudaSuccess) return I8_ERR_CUDA;
+    st = run_decode(false, X, nullptr, T, K, CB, N, threshold, SCB, bias, C, nullptr, ws, w, *d,
+                    s);
+    if (st != I8_OK) return st;
+    if (prof && cudaEventRecord(g_prof_stop, s) != cudaSuccess) return I8_ERR_CUDA;
+    return I8_OK;
+  }
+  uint32_t* mask = reinterpret_cast<uint32_t*>(ws + w.mask);
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + w.idx);
+  int32_t* n_o = reinterpret_cast<int32_t*>(ws + w.n_o);
+  int32_t* sel = cache ? reinterpret_cast<int32_t*>(ws + w.sel) : nullptr;
+  float* SCx = reinterpret_cast<float*>(ws + w.scx);
+  int8_t* Xq = reinterpret_cast<int8_t*>(ws + w.xq);
+  void* X_o = ws + w.xo;
+  void* CB_o = ws + w.cbo;
+  st = run_prepare(X, T, K, threshold, mask, w.zero_words, idx, n_o, Xq, SCx, X_o, CB, N, CB_o,
+                   *d, s, cache, ocols, sel);
+  if (st != I8_OK) return st;
+  if (prof && cudaEventRecord(g_prof_start, s) != cudaSuccess) return I8_ERR_CUDA;
+  st = run_gemm(false, Xq, T, K, CB, N, X_o, CB_o, n_o, SCx, SCB, bias, C, nullptr, *d, s,
+                cache ? cache + ocache_header_bytes(K) : nullptr, ocols, sel);
+  if (st != I8_OK) return st;
+  if (prof && cudaEventRecord(g_prof_stop, s) != cudaSuccess) return I8_ERR_CUDA;
+  return I8_OK;
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -563,43 +643,36 @@ i8_status i8_prepare_act(const void* X, int64_t T, int64_t K, float threshold,
 i8_status i8_linear_forward(const void* X, int64_t T, int64_t K, const int8_t* CB,
                             const float* SCB, const void* bias, int64_t N, float threshold,
                             void* C, void* workspace, size_t workspace_bytes, void* stream) {
-  if (!X || !CB || !SCB || !C || !workspace) return I8_ERR_INVALID_ARG;
-  if (!aligned16(X) || !aligned16(CB) || !aligned16(SCB) || !aligned16(C) ||
-      !aligned16(workspace) || (bias && !aligned16(bias)))
-    return I8_ERR_INVALID_ARG;
-  if (!shape_ok(T, K) || N <= 0 || N > 0x7fffffffLL || threshold != threshold)
-    return I8_ERR_INVALID_ARG;
-  const Workspace w = layout(T, N, K);
-  if (workspace_bytes < w.total) return I8_ERR_INVALID_ARG;
-  DeviceInfo* d;
-  i8_status st = device_info(&d);
-  if (st != I8_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const bool prof = g_prof_start != nullptr && g_prof_stop != nullptr;
-  if (use_decode(T, K)) {
-    if (prof && cudaEventRecord(g_prof_start, s) != cudaSuccess) return I8_ERR_CUDA;
-    st = run_decode(false, X, nullptr, T, K, CB, N, threshold, SCB, bias, C, nullptr, ws, w, *d,
-                    s);
-    if (st != I8_OK) return st;
-    if (prof && cudaEventRecord(g_prof_stop, s) != cudaSuccess) return I8_ERR_CUDA;
-    return I8_OK;
-  }
-  uint32_t* mask = reinterpret_cast<uint32_t*>(ws + w.mask);
-  int32_t* idx = reinterpret_cast<int32_t*>(ws + w.idx);
-  int32_t* n_o = reinterpret_cast<int32_t*>(ws + w.n_o);
-  float* SCx = reinterpret_cast<float*>(ws + w.scx);
-  int8_t* Xq = reinterpret_cast<int8_t*>(ws + w.xq);
-  void* X_o = ws + w.xo;
-  void* CB_o = ws + w.cbo;
-  st = run_prepare(X, T, K, threshold, mask, w.zero_words, idx, n_o, Xq, SCx, X_o, CB, N, CB_o,
-                   *d, s);
-  if (st != I8_OK) return st;
-  if (prof && cudaEventRecord(g_prof_start, s) != cudaSuccess) return I8_ERR_CUDA;
-  st = run_gemm(false, Xq, T, K, CB, N, X_o, CB_o, n_o, SCx, SCB, bias, C, nullptr, *d, s);
-  if (st != I8_OK) return st;
-  if (prof && cudaEventRecord(g_prof_stop, s) != cudaSuccess) return I8_ERR_CUDA;
+  return forward_impl(X, T, K, CB, SCB, bias, N, threshold, C, workspace, workspace_bytes,
+                      nullptr, 0, stream);
+}
+
+size_t i8_outlier_cache_size(int64_t N, int64_t K, int64_t max_cols) {
+  if (N <= 0 || N > 0x7fffffffLL || !shape_ok(1, K) || max_cols <= 0) return 0;
+  const int64_t kmax = (K + 63) / 64 * 64;
+  const int64_t cols = max_cols < kmax ? (max_cols + 63) / 64 * 64 : kmax;
+  return ocache_header_bytes(K) + slice_elems(N, cols) * 2;
+}
+
+i8_status i8_outlier_cache_reset(void* cache, size_t cache_bytes, void* stream) {
+  if (!cache || !aligned16(cache) || cache_bytes < kOcacheHdrWords * 4) return I8_ERR_INVALID_ARG;
+  if (cudaMemsetAsync(cache, 0, kOcacheHdrWords * 4, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return I8_ERR_CUDA;
   return I8_OK;
+}
+
+i8_status i8_linear_forward_cached(const void* X, int64_t T, int64_t K, const int8_t* CB,
+                                   const float* SCB, const void* bias, int64_t N,
+                                   float threshold, void* C, void* workspace,
+                                   size_t workspace_bytes, void* cache, size_t cache_bytes,
+                                   void* stream) {
+  if (!cache || !aligned16(cache)) return I8_ERR_INVALID_ARG;
+  if (!shape_ok(T, K) || N <= 0 || N > 0x7fffffffLL) return I8_ERR_INVALID_ARG;
+  const int64_t ocols = ocache_cols(cache_bytes, N, K);
+  if (ocols < 64) return I8_ERR_INVALID_ARG;
+  return forward_impl(X, T, K, CB, SCB, bias, N, threshold, C, workspace, workspace_bytes,
+                      static_cast<uint8_t*>(cache), ocols, stream);
 }
 
 i8_status i8_igemm_s32(const int8_t* A, int64_t T, int64_t K, const int8_t* B, int64_t N,

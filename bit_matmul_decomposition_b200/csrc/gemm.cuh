@@ -59,6 +59,7 @@ struct Args {
   int T, N, K;
   int m_tiles, n_tiles, k_blocks;
   const int32_t* n_outliers;  // device scalar, NULL = no outlier phase
+  const int32_t* cbo_sel;     // device scalar or NULL: nonzero = B_o comes from tmBc
   const float* SCx;
   const float* SCB;
   const __half* bias;  // nullable
@@ -245,7 +246,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     i8_gemm_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmAo,
-                           const __grid_constant__ CUtensorMap tmBo, const Args a) {
+                           const __grid_constant__ CUtensorMap tmBo,
+                           const __grid_constant__ CUtensorMap tmBc, const Args a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
@@ -280,6 +282,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmAo);
     tma_prefetch_desc(&tmBo);
+    tma_prefetch_desc(&tmBc);
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(&bars->tmem_base), TMEM_COLS);
@@ -339,7 +342,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int coord[2] = {0, 0};
       const uint32_t full_leader0 = map_to_rank(smem_u32(&bars->full[0]), 0);
       const CUtensorMap* map_i = loads_a ? &tmA : &tmB;
-      const CUtensorMap* map_o = loads_a ? &tmAo : &tmBo;
+      // the prepare pass wrote the selector before this grid's dependency wait returned
+      const bool b_cached = !loads_a && a.cbo_sel != nullptr && __ldcg(a.cbo_sel) != 0;
+      const CUtensorMap* map_o = loads_a ? &tmAo : (b_cached ? &tmBc : &tmBo);
       const uint32_t half_off = loads_a ? 0u : static_cast<uint32_t>(A_BYTES);
       const bool ok = walk_schedule(L, KB, OC, [&](int kind, int it, int idx) -> bool {
         if (kind >= 2) return true;

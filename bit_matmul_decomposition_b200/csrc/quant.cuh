@@ -238,12 +238,15 @@ constexpr int kPrepWarps = kPrepThreads / 32;
 constexpr int kPrepChunk = 32768;   // bytes per bulk copy of the row cache
 constexpr int kPrepMaxChunks = 8;
 constexpr int kPrepMaxIdx = 8192;    // outlier indices kept in shared memory
+// Outlier cache header, 32-bit words: [0] valid, [1] n_o, [2] N, [3] K, [4..5] the CB
+// device pointer (low, high), [6..7] spare, then the ceil(K/32) mask words of the cached set.
+constexpr int kOcacheHdrWords = 8;
 
 struct PrepArgs {
   const __half* X;
   int64_t T, K;
   float thr;
-  uint32_t* mask;         // [words + 1]: mask, then the barrier counter
+  uint32_t* mask;         // [words + 2]: mask, the barrier counter, the cache-update counter
   int32_t* idx_out;       // [K]
   int32_t* n_o_out;       // [1]
   int8_t* Xq;
@@ -252,6 +255,13 @@ struct PrepArgs {
   const int8_t* CB;       // [N, K] (phase 4) or NULL
   int64_t N;
   __half* CB_o;           // chunk-major slice [ceil(K/64)][N][64] or NULL
+  // Outlier cache (NULL: none).  CB_o of a call whose outlier set (and weight) matches the
+  // cached one is the cache's slice as it stands; otherwise it is gathered, into the cache
+  // when n_o <= ocache_cols (which then keys it by this call's set), else into CB_o above.
+  uint32_t* ocache;       // header (kOcacheHdrWords words, then the mask words)
+  __half* ocache_CB_o;    // chunk-major slice [ocache_cols / 64][N][64]
+  int64_t ocache_cols;    // capacity in columns, a multiple of 64
+  int32_t* cbo_sel;       // out (may be NULL): 1 when this call's CB_o is the cache's slice
   int64_t rows_per_cta;
   int64_t cache_rows;     // rows of its block each CTA keeps in shared memory
   int64_t cache_bytes_all; // size of the row-cache region (reused by phase 4)
@@ -382,6 +392,8 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
   __shared__ __align__(8) uint64_t s_bar[kPrepMaxChunks];
   __shared__ __align__(8) uint64_t s_rbar[kPrepWarps];  // phase 4 row buffers
   __shared__ int s_fail;
+  __shared__ int s_gfail;  // phase 4 gave up on a wait: the cache is left invalid
+  __shared__ int s_last;
   __shared__ int s_wsum[kPrepWarps];
   __shared__ float s_red[kPrepWarps];
 
@@ -396,6 +408,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
   // ------------------------------------------------ phase 1: scan (and cache) the rows
   if (tid == 0) {
     s_fail = 0;
+    s_gfail = 0;
     for (int c = 0; c < nchunks; ++c) mbar_init(smem_u32(&s_bar[c]), 1);
     for (int c = 0; c < kPrepWarps; ++c) mbar_init(smem_u32(&s_rbar[c]), 1);
     fence_mbar_init();
@@ -542,6 +555,35 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
     return j < kPrepMaxIdx ? sidx[j] : nth_outlier(smask, spre, words, j);
   };
 
+  // Outlier cache: cmode 0 = not used, 1 = hit (CB_o is the cache's slice as it stands),
+  // 2 = miss (gather into the cache's slice, then key the cache by this call's set).  Every
+  // CTA reads the same header and the same final mask, so all take the same decision; a
+  // missing CTA clears the valid word before it writes the slice, which can only turn the
+  // decision of a CTA that reads the header later into the miss it takes anyway.
+  int cmode = 0;
+  if (p.ocache != nullptr && p.CB != nullptr && n_o > 0 && n_o <= p.ocache_cols) {
+    const uint32_t* h = p.ocache;
+    bool same = true;
+    if (tid == 0) {
+      const uint64_t cbp = reinterpret_cast<uint64_t>(p.CB);
+      same = __ldcg(h + 0) == 1u && __ldcg(h + 1) == static_cast<uint32_t>(n_o) &&
+             __ldcg(h + 2) == static_cast<uint32_t>(p.N) &&
+             __ldcg(h + 3) == static_cast<uint32_t>(K) &&
+             __ldcg(h + 4) == static_cast<uint32_t>(cbp) &&
+             __ldcg(h + 5) == static_cast<uint32_t>(cbp >> 32);
+    }
+    for (int64_t w = tid; w < words; w += kPrepThreads)
+      if (__ldcg(h + kOcacheHdrWords + w) != smask[w]) same = false;
+    cmode = __syncthreads_and(same) ? 1 : 2;
+    if (cmode == 2 && tid == 0) {
+      __stcg(p.ocache, 0u);
+      __threadfence();
+    }
+  }
+  __half* const cbo = cmode != 0 ? p.ocache_CB_o : p.CB_o;
+  const bool gather = cbo != nullptr && cmode != 1 && n_o > 0;
+  if (blockIdx.x == 0 && tid == 0 && p.cbo_sel != nullptr) *p.cbo_sel = cmode != 0 ? 1 : 0;
+
   // The CB_o gather of phase 4 for few outlier columns (one warp per (chunk, row) item,
   // U4 items per batch) is bound by the latency of scattered byte reads of CB in HBM, so
   // each warp issues its first batch here and stores it after the quantisation: those
@@ -549,8 +591,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
   constexpr int U4 = 8;
   const int64_t chunks4 = (n_o + 63) >> 6;
   const int64_t nbuf4 = min(static_cast<int64_t>(kPrepWarps), p.cache_bytes_all / K);
-  const bool few4 = p.CB_o != nullptr && n_o > 0 &&
-                    !(static_cast<int64_t>(n_o) * 32 >= K && nbuf4 > 0);
+  const bool few4 = gather && !(static_cast<int64_t>(n_o) * 32 >= K && nbuf4 > 0);
   const int64_t items4 = chunks4 * p.N;
   const int64_t nw4 = static_cast<int64_t>(gridDim.x) * kPrepWarps;
   const int64_t first4 = (static_cast<int64_t>(blockIdx.x) * kPrepWarps + warp) * U4;
@@ -575,7 +616,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
       const int64_t it = it0 + u;
       if (it < items4) {
         const int64_t c = it / p.N, n = it - c * p.N;
-        reinterpret_cast<__half2*>(p.CB_o + (c * p.N + n) * 64)[lane] =
+        reinterpret_cast<__half2*>(cbo + (c * p.N + n) * 64)[lane] =
             __floats2half2_rn(static_cast<float>(v0[u]), static_cast<float>(v1[u]));
       }
     }
@@ -646,7 +687,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
   __syncthreads();   // the row cache is free from here on (phase 4 may reuse it)
 
   // ------------------------------------------------ phase 4: fp16 outlier slice of CB
-  if (p.CB_o != nullptr && n_o > 0) {
+  if (gather) {
     const int64_t chunks = (n_o + 63) >> 6;
     const int64_t nbuf = min(static_cast<int64_t>(kPrepWarps), p.cache_bytes_all / K);
     if (static_cast<int64_t>(n_o) * 32 >= K && nbuf > 0) {
@@ -668,7 +709,10 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
           }
           const bool got = mbar_wait(bar, ph, &no_abort, p.wait_limit_ns);
           ph ^= 1u;
-          if (!__all_sync(0xffffffffu, got)) break;
+          if (!__all_sync(0xffffffffu, got)) {
+            if (lane == 0) s_gfail = 1;
+            break;
+          }
           for (int64_t c0 = 0; c0 < chunks; c0 += 4) {
             float v0[4], v1[4];
 #pragma unroll
@@ -682,7 +726,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
 #pragma unroll
             for (int u = 0; u < 4; ++u)
               if (c0 + u < chunks)
-                reinterpret_cast<__half2*>(p.CB_o + ((c0 + u) * p.N + n) * 64)[lane] =
+                reinterpret_cast<__half2*>(cbo + ((c0 + u) * p.N + n) * 64)[lane] =
                     __floats2half2_rn(v0[u], v1[u]);
           }
           __syncwarp();
@@ -697,6 +741,36 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
         int v0[U4], v1[U4];
         gather_load(it0, v0, v1);
         gather_store(it0, v0, v1);
+      }
+    }
+  }
+
+  // Cache miss: the last CTA to finish its part of the slice keys the cache by this call's
+  // outlier set (a CTA that gave up on a wait does not arrive, so the cache stays invalid).
+  if (cmode == 2) {
+    __syncthreads();
+    if (tid == 0) {
+      s_last = 0;
+      if (!s_gfail) {
+        __threadfence();
+        s_last = atomicAdd(p.mask + words + 1, 1u) == gridDim.x - 1u;
+      }
+    }
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      for (int64_t w = tid; w < words; w += kPrepThreads)
+        __stcg(p.ocache + kOcacheHdrWords + w, smask[w]);
+      __syncthreads();
+      if (tid == 0) {
+        const uint64_t cbp = reinterpret_cast<uint64_t>(p.CB);
+        __stcg(p.ocache + 1, static_cast<uint32_t>(n_o));
+        __stcg(p.ocache + 2, static_cast<uint32_t>(p.N));
+        __stcg(p.ocache + 3, static_cast<uint32_t>(K));
+        __stcg(p.ocache + 4, static_cast<uint32_t>(cbp));
+        __stcg(p.ocache + 5, static_cast<uint32_t>(cbp >> 32));
+        __threadfence();
+        __stcg(p.ocache, 1u);
       }
     }
   }

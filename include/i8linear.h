@@ -159,6 +159,54 @@ i8_status i8_linear_forward(const void* X, int64_t T, int64_t K, const int8_t* C
                             void* C, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Outlier cache: i8_linear_forward for a serving loop whose outlier columns repeat from
+ * call to call.  The blog ("LLM.int8() 的总结"; the emergent-feature discussion) notes that
+ * the outliers are systematic: the same few feature dimensions carry them in call after
+ * call.  The prefill path's prepare pass gathers the weight's codes in those columns,
+ * CB_o (fp16, chunk-major [ceil(n_o/64)][N][64]), on every call; this variant keeps CB_o
+ * in a caller-owned cache and skips the gather when a call's outlier set matches the
+ * cached one.  The output is bit-identical to i8_linear_forward's.
+ *
+ * i8_outlier_cache_size(N, K, max_cols): bytes of a cache that holds up to max_cols
+ * outlier columns (rounded up to a multiple of 64, at most K rounded up) of an [N, K]
+ * weight: a header (8 words and the ceil(K/32) mask words, padded to 256 B) plus
+ * N * 128 bytes per 64 columns.  Returns 0 for invalid arguments (N or K <= 0, K % 16 != 0,
+ * max_cols <= 0).  Host-only arithmetic.
+ *
+ * i8_outlier_cache_reset(cache, cache_bytes, stream): marks the cache empty (clears its
+ * header's first 8 words on `stream`).  Call it once on a new cache -- its memory starts
+ * undefined -- and again whenever the weight's codes CB change in place; the cache is keyed
+ * by the outlier set, N, K and the CB device pointer, not by CB's contents.  Returns
+ * I8_ERR_INVALID_ARG for a NULL or unaligned cache or cache_bytes < 32, I8_ERR_CUDA if the
+ * memset cannot be enqueued.
+ *
+ * i8_linear_forward_cached(X, T, K, CB, SCB, bias, N, threshold, C, workspace,
+ *                          workspace_bytes, cache, cache_bytes, stream):
+ *   every argument but the last three exactly as in i8_linear_forward (the workspace is
+ *   still needed, of the same size);
+ *   cache        device buffer, 16-byte aligned, owned by the caller, reset once before its
+ *                first use; cache_bytes its size, which sets its capacity in columns
+ *                (at least one 64-column chunk: i8_outlier_cache_size(N, K, 64)).
+ * The prepare pass decides on the device, with no host synchronisation: when the cache is
+ * valid and holds this call's exact outlier set for the same CB pointer, N and K, the GEMM
+ * reads CB_o from the cache and nothing is gathered; when the set differs (and n_o fits
+ * the capacity), CB_o is gathered into the cache, which is then keyed by this set; when
+ * n_o exceeds the capacity, CB_o is gathered into the workspace and the cache is left as
+ * it was.  Decode batches (T <= 16, K <= 65536) take the decode kernel, which needs no
+ * CB_o, and leave the cache untouched.  Calls sharing one cache must be ordered on one
+ * stream.  A call that fails on the device (I8_ERR_TIMEOUT from i8_sync_status) leaves the
+ * cache either as it was or empty, never keyed to a partly written slice.  Returns I8_ERR_INVALID_ARG, with nothing launched, for a NULL or unaligned
+ * cache, a capacity below 64 columns, or any argument i8_linear_forward rejects.
+ */
+size_t i8_outlier_cache_size(int64_t N, int64_t K, int64_t max_cols);
+i8_status i8_outlier_cache_reset(void* cache, size_t cache_bytes, void* stream);
+i8_status i8_linear_forward_cached(const void* X, int64_t T, int64_t K, const int8_t* CB,
+                                   const float* SCB, const void* bias, int64_t N,
+                                   float threshold, void* C, void* workspace,
+                                   size_t workspace_bytes, void* cache, size_t cache_bytes,
+                                   void* stream);
+
+/*
  * i8_linear_forward without a workspace argument: the same forward as i8_linear_forward,
  * with its scratch taken from a fixed 32 MiB array that the library itself holds in
  * device memory.  The pages have no counterpart to this call; it exists for callers that

@@ -108,3 +108,33 @@ def test_product_path_fails_loudly_without_library(tmp_path):
             abi.load(str(tmp_path / "missing.so"))
     finally:
         abi._lib = saved
+
+
+def test_outlier_cache_size_host_logic(lib):
+    cs = lib.i8_outlier_cache_size
+    assert cs(0, 64, 64) == 0 and cs(64, 0, 64) == 0 and cs(64, 72, 64) == 0
+    assert cs(64, 64, 0) == 0
+    head = 256                                        # 8 + 2 mask words, padded to 256 B
+    assert cs(64, 64, 1) == head + 64 * 64 * 2        # rounded up to one 64-column chunk
+    assert cs(64, 64, 1000) == head + 64 * 64 * 2     # at most K rounded up to 64
+    assert cs(300, 1040, 65) == head + 2 * 300 * 64 * 2
+    big = cs(16384, 4096, 256)                        # header: 8 + 128 words -> 768 B
+    assert big == 768 + 4 * 16384 * 64 * 2
+
+
+def test_cached_forward_rejects_bad_arguments_without_cuda(lib):
+    f = lib.i8_linear_forward_cached
+    ws_ok = lib.i8_linear_workspace_size(32, 64, 64)
+    c_ok = lib.i8_outlier_cache_size(64, 64, 64)
+
+    def call(cache=FAKE, cb=c_ok, X=FAKE, T=32, thr=6.0):
+        return f(X, T, 64, FAKE, FAKE, None, 64, thr, FAKE, FAKE, ws_ok, cache, cb, None)
+
+    assert call(cache=None) == INVALID
+    assert call(cache=FAKE + 8) == INVALID            # misaligned
+    assert call(cb=c_ok - 1) == INVALID               # less than one 64-column chunk
+    assert call(X=None) == INVALID
+    assert call(T=0) == INVALID
+    assert call(thr=math.nan) == INVALID
+    assert lib.i8_outlier_cache_reset(None, c_ok, None) == INVALID
+    assert lib.i8_outlier_cache_reset(FAKE, 16, None) == INVALID
