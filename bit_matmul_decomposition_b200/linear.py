@@ -16,6 +16,12 @@ dx = dy W, dW = dy^T x, db = sum(dy), with fp16 operands.  Without fp16 weights 
 still passes dx = dy W' back (W' = CB * SCB / 127, the weight it computes with), so layers
 before it can train.  The forward runs in the library's CUDA kernels; the backward
 products are plain fp16 GEMMs (torch.matmul, cuBLAS) on the same device.
+
+Serving with systematic outliers (the blog's observation that the same few feature
+dimensions carry the outliers call after call): ``outlier_cache_cols > 0`` keeps the
+weight's codes in the outlier columns (CB_o) in a device cache across forwards
+(``i8_linear_forward_cached``), so a call whose outlier set matches the cached one skips
+their gather; outputs are bit-identical to the uncached layer.
 """
 from __future__ import annotations
 
@@ -64,17 +70,29 @@ class Linear8bitLt(torch.nn.Module):
     ``forward(x)``: x fp16 [..., in] on the layer's CUDA device; the leading dimensions are
     flattened into T tokens of one call (T <= 16 takes the one-launch decode kernel, larger T
     the tensor-core GEMM).  The outlier columns are found per call from x.
+
+    ``outlier_cache_cols``: capacity (columns) of the outlier cache, 0 = no cache.  The cache
+    is not part of the state dict; ``quantize_`` and ``load_state_dict`` empty it, as they
+    rewrite CB in place (write CB through neither, and call ``invalidate_outlier_cache``).
     """
 
     def __init__(self, in_features: int, out_features: int, bias: bool = True,
-                 threshold: float = 6.0, device=None, has_fp16_weights: bool = False):
+                 threshold: float = 6.0, device=None, has_fp16_weights: bool = False,
+                 outlier_cache_cols: int = 0):
         super().__init__()
         if in_features <= 0 or out_features <= 0 or in_features % 16 != 0:
             raise ValueError("in_features must be a positive multiple of 16 (row pitch of the "
                              "int8 weight for TMA); out_features positive")
+        if outlier_cache_cols < 0:
+            raise ValueError("outlier_cache_cols must be >= 0")
+        if outlier_cache_cols and has_fp16_weights:
+            raise ValueError("the outlier cache needs fixed codes: not with has_fp16_weights "
+                             "(every forward re-quantises the weight)")
         self.in_features = in_features
         self.out_features = out_features
         self.threshold = float(threshold)
+        self.outlier_cache_cols = int(outlier_cache_cols)
+        self._ocache: Dict[torch.device, torch.Tensor] = {}
         self.register_buffer("CB", torch.zeros((out_features, in_features), dtype=torch.int8,
                                                device=device))
         self.register_buffer("SCB", torch.zeros((out_features,), dtype=torch.float32,
@@ -95,13 +113,15 @@ class Linear8bitLt(torch.nn.Module):
 
     @classmethod
     def from_linear(cls, linear: torch.nn.Linear, threshold: float = 6.0,
-                    has_fp16_weights: bool = False) -> "Linear8bitLt":
+                    has_fp16_weights: bool = False,
+                    outlier_cache_cols: int = 0) -> "Linear8bitLt":
         """Quantise an nn.Linear that lives on a CUDA device (weights cast to fp16)."""
         w = linear.weight
         if not w.is_cuda:
             raise ValueError("the weight must be on a CUDA device (it is quantised there)")
         m = cls(linear.in_features, linear.out_features, bias=linear.bias is not None,
-                threshold=threshold, device=w.device, has_fp16_weights=has_fp16_weights)
+                threshold=threshold, device=w.device, has_fp16_weights=has_fp16_weights,
+                outlier_cache_cols=outlier_cache_cols)
         if has_fp16_weights:
             with torch.no_grad():
                 m.weight.copy_(w.detach().to(torch.float16))
@@ -121,6 +141,7 @@ class Linear8bitLt(torch.nn.Module):
         if weight.device != self.CB.device:
             raise ValueError("weight on %s, layer on %s" % (weight.device, self.CB.device))
         abi.i8_quantize_weight(weight.to(torch.float16).contiguous(), self.CB, self.SCB)
+        self.invalidate_outlier_cache()
         if bias is not None:
             if self.bias is None:
                 raise ValueError("layer was built without bias")
@@ -140,14 +161,38 @@ class Linear8bitLt(torch.nn.Module):
             self._ws[dev] = ws
         return ws
 
+    def invalidate_outlier_cache(self):
+        """Empty the outlier cache (needed after CB changed in place)."""
+        for c in self._ocache.values():
+            abi.i8_outlier_cache_reset(c)
+
+    def _outlier_cache(self) -> torch.Tensor:
+        dev = self.CB.device
+        c = self._ocache.get(dev)
+        if c is None:
+            need = abi.i8_outlier_cache_size(self.out_features, self.in_features,
+                                             self.outlier_cache_cols)
+            c = torch.empty((need,), dtype=torch.uint8, device=dev)
+            abi.i8_outlier_cache_reset(c)
+            self._ocache[dev] = c
+        return c
+
+    def _load_from_state_dict(self, *args, **kwargs):
+        super()._load_from_state_dict(*args, **kwargs)
+        self.invalidate_outlier_cache()
+
     def _forward_kernel(self, x2: torch.Tensor) -> torch.Tensor:
-        """One i8_linear_forward call on a [T, in] fp16 input (no autograd)."""
+        """One i8_linear_forward(_cached) call on a [T, in] fp16 input (no autograd)."""
         T = x2.shape[0]
         out = torch.empty((T, self.out_features), dtype=torch.float16, device=x2.device)
         if T > 0:
             bias = None if self.bias is None else self.bias.detach()
-            abi.i8_linear_forward(x2, self.CB, self.SCB, bias, self.threshold, out,
-                                  self._workspace(T))
+            if self.outlier_cache_cols > 0:
+                abi.i8_linear_forward_cached(x2, self.CB, self.SCB, bias, self.threshold, out,
+                                             self._workspace(T), self._outlier_cache())
+            else:
+                abi.i8_linear_forward(x2, self.CB, self.SCB, bias, self.threshold, out,
+                                      self._workspace(T))
         return out
 
     def forward(self, x: torch.Tensor) -> torch.Tensor:
@@ -169,22 +214,26 @@ class Linear8bitLt(torch.nn.Module):
         return y.reshape(*lead, self.out_features)
 
     def extra_repr(self) -> str:
-        return "in_features=%d, out_features=%d, bias=%s, threshold=%g, has_fp16_weights=%s" % (
-            self.in_features, self.out_features, self.bias is not None, self.threshold,
-            self.has_fp16_weights)
+        return ("in_features=%d, out_features=%d, bias=%s, threshold=%g, has_fp16_weights=%s, "
+                "outlier_cache_cols=%d" % (self.in_features, self.out_features,
+                                           self.bias is not None, self.threshold,
+                                           self.has_fp16_weights, self.outlier_cache_cols))
 
 
 def replace_linear_with_int8(model: torch.nn.Module, threshold: float = 6.0,
                              skip: Iterable[str] = ("lm_head",),
-                             has_fp16_weights: bool = False) -> torch.nn.Module:
+                             has_fp16_weights: bool = False,
+                             outlier_cache_cols: int = 0) -> torch.nn.Module:
     """Swap every nn.Linear of `model` (weights on a CUDA device) for a Linear8bitLt, in
     place, except modules whose name (last path component) is in `skip`.  Returns `model`."""
     skip = set(skip)
     for name, child in list(model.named_children()):
         if isinstance(child, torch.nn.Linear) and name not in skip:
             setattr(model, name, Linear8bitLt.from_linear(child, threshold=threshold,
-                                                          has_fp16_weights=has_fp16_weights))
+                                                          has_fp16_weights=has_fp16_weights,
+                                                          outlier_cache_cols=outlier_cache_cols))
         elif name not in skip:
             replace_linear_with_int8(child, threshold=threshold, skip=skip,
-                                     has_fp16_weights=has_fp16_weights)
+                                     has_fp16_weights=has_fp16_weights,
+                                     outlier_cache_cols=outlier_cache_cols)
     return model

@@ -93,3 +93,11 @@ def test_reference_arm_other_ranks_exit_quietly():
     r = _run_ref({"RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_l2_policy_flushes_only_inputs_that_fit_twice_in_l2():
+    import bench
+    assert bench.l2_policy("auto", 2048, 16384, 4096)[0]            # 84 MB of inputs
+    no, desc = bench.l2_policy("auto", 16, 57344, 14336)             # CB 822 MB
+    assert not no and "no flush" in desc
+    assert bench.l2_policy("always", 16, 57344, 14336)[0]

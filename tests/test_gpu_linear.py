@@ -72,6 +72,27 @@ def test_state_dict_restores_the_same_outputs():
     assert np.array_equal(y1.view(np.uint16), y2.view(np.uint16))
 
 
+def test_outlier_cache_layer_matches_and_follows_new_weights():
+    K, N = 1024, 768
+    lin1, lin2 = _fp16_linear(K, N, seed=31), _fp16_linear(K, N, seed=32)
+    plain = Linear8bitLt.from_linear(lin1)
+    cached = Linear8bitLt.from_linear(lin1, outlier_cache_cols=64)
+    xs = [torch.from_numpy(_x((T,), K, cols, seed=40 + T).view(np.int16)).view(torch.float16).cuda()
+          for T, cols in ((300, (7, 900)), (300, (7, 900)), (48, (7, 900)), (5, (2,)),
+                          (300, (11,)))]
+    for x in xs:                       # miss, hit, hit at another T, decode, miss
+        assert torch.equal(plain(x).view(torch.int16), cached(x).view(torch.int16))
+    # new codes through load_state_dict (same CB buffer): the cache must not serve the old
+    cached.load_state_dict(Linear8bitLt.from_linear(lin2).state_dict())
+    plain2 = Linear8bitLt.from_linear(lin2)
+    for x in xs[:2]:
+        assert torch.equal(plain2(x).view(torch.int16), cached(x).view(torch.int16))
+    # and through quantize_
+    cached.quantize_(lin1.weight.detach(), lin1.bias.detach())
+    assert torch.equal(plain(xs[0]).view(torch.int16), cached(xs[0]).view(torch.int16))
+    sync_ok()
+
+
 def test_replaced_layer_stack_layer_by_layer():
     """Linear -> GELU -> Linear (+ an fp16 head left alone): each int8 layer matches the
     oracle on the activations it actually received."""

@@ -52,16 +52,16 @@ def test_forward_rejects_other_dtypes_before_any_call():
 def test_replace_walk(monkeypatch):
     made = []
 
-    def fake_from_linear(linear, threshold=6.0, has_fp16_weights=False):
-        made.append((linear.in_features, linear.out_features, threshold))
+    def fake_from_linear(linear, threshold=6.0, has_fp16_weights=False, outlier_cache_cols=0):
+        made.append((linear.in_features, linear.out_features, threshold, outlier_cache_cols))
         return torch.nn.Identity()
 
     monkeypatch.setattr(L.Linear8bitLt, "from_linear", staticmethod(fake_from_linear))
     model = torch.nn.Sequential(torch.nn.Linear(32, 64), torch.nn.GELU(),
                                 torch.nn.Sequential(torch.nn.Linear(64, 32)))
     model.lm_head = torch.nn.Linear(32, 10)
-    L.replace_linear_with_int8(model, threshold=5.0)
-    assert made == [(32, 64, 5.0), (64, 32, 5.0)]
+    L.replace_linear_with_int8(model, threshold=5.0, outlier_cache_cols=64)
+    assert made == [(32, 64, 5.0, 64), (64, 32, 5.0, 64)]
     assert isinstance(model[0], torch.nn.Identity) and isinstance(model[2][0], torch.nn.Identity)
     assert isinstance(model.lm_head, torch.nn.Linear)
 
@@ -73,3 +73,14 @@ def test_training_mode_holds_fp16_parameters():
     assert {n for n, _ in m.named_buffers()} == {"CB", "SCB"}
     assert set(m.state_dict()) == {"weight", "bias", "CB", "SCB"}
     assert {n for n, _ in L.Linear8bitLt(64, 32).named_parameters()} == set()
+
+
+def test_outlier_cache_option():
+    m = L.Linear8bitLt(64, 32, outlier_cache_cols=128)
+    assert "outlier_cache_cols=128" in repr(m)
+    assert set(m.state_dict()) == {"CB", "SCB", "bias"}    # the cache is not saved
+    m.load_state_dict(m.state_dict())                      # no cache allocated yet: no-op
+    with pytest.raises(ValueError):
+        L.Linear8bitLt(64, 32, outlier_cache_cols=-1)
+    with pytest.raises(ValueError):
+        L.Linear8bitLt(64, 32, outlier_cache_cols=64, has_fp16_weights=True)
