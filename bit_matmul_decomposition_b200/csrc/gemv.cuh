@@ -305,8 +305,12 @@ __device__ __forceinline__ bool forward_prologue(
   bool ok = true;
   const uint32_t e = static_cast<uint32_t>(a.epoch);
   uint32_t goal3 = 0;  // cooperative path: third barrier, waited for after the tables below
+  // One row: a column is an outlier column exactly when its one element reaches the
+  // threshold, so the row maximum over the other columns is the largest |x| below the
+  // threshold, taken in the same pass as the mask (no block maxima, no re-read).
+  const bool one_row = (T == 1);
   if (!a.coop) {
-    // (a) step 1 and the block maxima, piece by piece
+    // (a) step 1 and the block maxima (one row: the row maximum), piece by piece
     const int64_t xbytes = static_cast<int64_t>(T) * K * 2;
     const int64_t pieces = (xbytes + STAGE_BYTES - 1) / STAGE_BYTES;
     for (int64_t pc = 0; pc < pieces; ++pc) {
@@ -329,12 +333,19 @@ __device__ __forceinline__ bool forward_prologue(
             const int g = f0 - t * Gi + lane;
             const uint4 v = sp[i0 + lane];
             const uint32_t m = absmax8_bits(v);
+            uint32_t m1 = m;  // (one row) the largest |x| below the threshold
             if (half_bits_to_float(m) >= thr) {  // rare: an outlier in this group
               const uint32_t bits = outlier_bits8(v, thr);
               if (bits) atomicOr(&maskall[g >> 2], bits << (8 * (g & 3)));
+              m1 = __half_as_ushort(__float2half_rn(absmax8(v, bits)));
             }
-            const uint32_t mx = __reduce_max_sync(0xffffffffu, m);
-            if (lane == 0) atomicMax(&bm[t * NBK + g / GPB], mx);
+            if (one_row) {
+              const uint32_t mx = __reduce_max_sync(0xffffffffu, m1);
+              if (lane == 0) atomicMax(&rmx[0], __float_as_uint(half_bits_to_float(mx)));
+            } else {
+              const uint32_t mx = __reduce_max_sync(0xffffffffu, m);
+              if (lane == 0) atomicMax(&bm[t * NBK + g / GPB], mx);
+            }
           }
         } else {
           for (int i0 = w * 32; i0 < nvec; i0 += CW * 32) {
@@ -349,12 +360,18 @@ __device__ __forceinline__ bool forward_prologue(
               if (half_bits_to_float(m) >= thr) {
                 const uint32_t bits = outlier_bits8(v, thr);
                 if (bits) atomicOr(&maskall[g >> 2], bits << (8 * (g & 3)));
+                if (one_row) m = __half_as_ushort(__float2half_rn(absmax8(v, bits)));
               }
-              key = static_cast<uint32_t>(t * NBK + g / GPB);
+              key = one_row ? 0u : static_cast<uint32_t>(t * NBK + g / GPB);
             }
             const uint32_t peers = __match_any_sync(0xffffffffu, key);
             const uint32_t mx = __reduce_max_sync(peers, m);
-            if (valid && lane == __ffs(peers) - 1) atomicMax(&bm[key], mx);
+            if (valid && lane == __ffs(peers) - 1) {
+              if (one_row)
+                atomicMax(&rmx[0], __float_as_uint(half_bits_to_float(mx)));
+              else
+                atomicMax(&bm[key], mx);
+            }
           }
         }
         __syncwarp();
@@ -426,12 +443,13 @@ __device__ __forceinline__ bool forward_prologue(
     if (ct == 0 && ok) goal3 = grid_arrive(a.gbar + 2, e, gridDim.x, true);
   }
 
-  // (b) ranks (warp 0: lane l takes a contiguous run of mask words)
+  // (b) ranks: the compute threads take contiguous runs of mask words, and one block-wide
+  // exclusive scan of the runs' outlier counts gives each word its rank base
   const int WPS = static_cast<int>(KS / 32);  // mask words per slice
-  if (w == 0) {
+  {
     const int KWi = static_cast<int>(KW);
-    const int cw = (KWi + 31) / 32;
-    const int wb = lane * cw;
+    const int cw = (KWi + CW * 32 - 1) / (CW * 32);
+    const int wb = ct * cw < KWi ? ct * cw : KWi;
     const int we = wb + cw < KWi ? wb + cw : KWi;
     int cnt = 0;
     for (int x = wb; x < we; ++x) cnt += __popc(maskall[x]);
@@ -441,14 +459,20 @@ __device__ __forceinline__ bool forward_prologue(
       const int y = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += y;
     }
-    int run = incl - cnt;
-    int nb = (wb + WPS - 1) / WPS * WPS;  // next slice boundary at or after wb
+    int* wsum = reinterpret_cast<int*>(jinfo);  // scratch until (c) fills jinfo
+    if (lane == 31) wsum[w] = incl;
+    compute_sync();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int i = 0; i < CW; ++i) {
+      const int v = wsum[i];
+      before += i < w ? v : 0;
+      total += v;
+    }
+    int run = before + incl - cnt;
     const int sw0 = slice * WPS;
     for (int x = wb; x < we; ++x) {
-      if (x == nb) {
-        jbase[x / WPS] = run;
-        nb += WPS;
-      }
+      if (x % WPS == 0) jbase[x / WPS] = run;
       if (x >= sw0 && x < sw0 + WPS) spre[x - sw0] = run;
       uint32_t bits = maskall[x];
       while (bits) {
@@ -458,9 +482,9 @@ __device__ __forceinline__ bool forward_prologue(
         ++run;
       }
     }
-    if (lane == 31) {
-      misc[0] = run;  // n_o
-      jbase[S] = run;
+    if (ct == 0) {
+      misc[0] = total;  // n_o
+      jbase[S] = total;
     }
   }
   compute_sync();
@@ -500,7 +524,7 @@ __device__ __forceinline__ bool forward_prologue(
     compute_sync();
     ok = *abort_flag == 0;
   }
-  if (!a.coop) {
+  if (!a.coop && !one_row) {
     // blocks holding outlier columns (warp 1 lists them); the other blocks give their
     // maxima from (a)
     if (w == 1) {
