@@ -199,6 +199,157 @@ int64_t oracle_linear_forward_rows(const uint16_t *X, int64_t T, int64_t K,
     return overflow;
 }
 
+/* ---------------------------------------------------------------------------------
+ * FP8 (e4m3) variant of the decomposition.  The pages name 8-bit floating point only as
+ * the next step ("LLM.int8() 的总结" / the closing outlook); the plainest reading keeps
+ * every step above and swaps the int8 absmax code for an e4m3 code of the same scaled
+ * value: scale = fl32(448 / absmax) (448 is the largest finite e4m3 magnitude, as 127 is
+ * the largest int8 code used), code = e4m3 rounding of fl32(x * scale), and 448 in place
+ * of 127 in every dequantisation (acc * SCx * SCB / 448^2, weights CB * SCB / 448).
+ *
+ * e4m3 is the "fn" format of the OCP 8-bit floating-point specification: 1 sign bit,
+ * 4 exponent bits (bias 7), 3 fraction bits; exponent field 0 holds zero and the
+ * subnormals (fraction * 2^-9); S.1111.111 is NaN; there are no infinities, and the
+ * largest finite magnitude is 1.75 * 2^8 = 448. */
+
+/* Decode one e4m3 code to its exact value. */
+double oracle_e4m3_to_double(uint8_t c)
+{
+    int e = (c >> 3) & 0xF, m = c & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);
+    else
+        v = ldexp(1.0 + m / 8.0, e - 7);
+    return (c & 0x80) ? -v : v;
+}
+
+/* Encode: round to the nearest e4m3 value, ties to the even fraction; magnitudes of 448
+ * and above give 448 (round-to-nearest already does below 464, the midpoint to the next
+ * power-of-two step; the scaled values of this layer never exceed 448 * (1 + 2^-23)). */
+uint8_t oracle_e4m3_from_float(float v)
+{
+    if (isnan(v))
+        return 0x7F;
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs((double)v);
+    if (a >= 448.0)
+        return sign | 0x7E;
+    if (a == 0.0)
+        return sign;
+    int e;
+    frexp(a, &e);                    /* a in [2^(e-1), 2^e) */
+    int E = e - 1;
+    if (E < -6)
+        E = -6;                      /* subnormals share the 2^-6 binade's step */
+    double step = ldexp(1.0, E - 3); /* three fraction bits */
+    double r = nearbyint(a / step) * step;   /* default rounding: nearest, ties to even */
+    if (r == 0.0)
+        return sign;
+    int e2;
+    frexp(r, &e2);
+    int E2 = e2 - 1;
+    if (E2 < -6)
+        return sign | (uint8_t)(r / ldexp(1.0, -9));
+    int m = (int)((ldexp(r, -E2) - 1.0) * 8.0);
+    return sign | (uint8_t)(((E2 + 7) << 3) | m);
+}
+
+/* Row-wise absmax e4m3 quantisation of an fp16 matrix A [R,K] (activations with `skip`,
+ * weights with skip NULL): scale[r] = max |A[r,k]| over the kept columns (fp32);
+ * q[r,k] = e4m3(fl32(A[r,k] * fl32(448 / scale[r]))); skipped columns and zero rows give
+ * code 0. */
+void oracle_absmax_quantize_rows_e4m3(const uint16_t *A, int64_t R, int64_t K,
+                                      const uint8_t *skip, uint8_t *q, float *scale)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r) {
+        const uint16_t *row = A + r * K;
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            if (skip && skip[k])
+                continue;
+            float a = fabsf(oracle_half_to_float(row[k]));
+            if (a > amax)
+                amax = a;
+        }
+        scale[r] = amax;
+        uint8_t *qr = q + r * K;
+        if (amax == 0.0f) {
+            for (int64_t k = 0; k < K; ++k)
+                qr[k] = 0;
+            continue;
+        }
+        float s = 448.0f / amax;
+        for (int64_t k = 0; k < K; ++k) {
+            if (skip && skip[k]) {
+                qr[k] = 0;
+                continue;
+            }
+            float v = oracle_half_to_float(row[k]) * s;
+            qr[k] = oracle_e4m3_from_float(v);
+        }
+    }
+}
+
+/* The e4m3 product acc[i,n] = sum_k dec(A[rows[i],k]) * dec(B[n,k]) in fp64.  Every
+ * product of two e4m3 values has at most 8 significant bits between 2^-18 and 2^17, so
+ * sums of up to 2^16 of them are exact in fp64: acc is the exact product. */
+void oracle_e4m3_matmul(const uint8_t *A, const uint8_t *B, int64_t nrows,
+                        const int64_t *rows, int64_t N, int64_t K, double *acc)
+{
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t i = 0; i < nrows; ++i) {
+        for (int64_t n = 0; n < N; ++n) {
+            const uint8_t *a = A + (rows ? rows[i] : i) * K;
+            const uint8_t *b = B + n * K;
+            double s = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                s += oracle_e4m3_to_double(a[k]) * oracle_e4m3_to_double(b[k]);
+            acc[i * N + n] = s;
+        }
+    }
+}
+
+/* The whole e4m3 forward for a subset of rows, in fp64:
+ *   C[i,n] = acc[i,n] * SCx[t] * SCB[n] / 448^2
+ *          + sum_{j < n_o} X[t, idx[j]] * dec(CB[n, idx[j]]) * SCB[n] / 448 + bias[n]
+ * with the mask and SCx over ALL rows of X, as in the int8 forward. */
+int64_t oracle_linear_forward_rows_e4m3(const uint16_t *X, int64_t T, int64_t K,
+                                        const uint8_t *CB, const float *SCB,
+                                        const uint16_t *bias, int64_t N, float threshold,
+                                        const int64_t *rows, int64_t nrows,
+                                        uint32_t *mask_words, int32_t *idx, int32_t *n_o,
+                                        uint8_t *Xq, float *SCx, double *acc, double *C)
+{
+    uint8_t *is_outlier = (uint8_t *)malloc((size_t)(K > 0 ? K : 1));
+    if (!is_outlier)
+        return -1;
+    oracle_outlier_scan(X, T, K, threshold, is_outlier, mask_words, idx, n_o);
+    oracle_absmax_quantize_rows_e4m3(X, T, K, is_outlier, Xq, SCx);
+    oracle_e4m3_matmul(Xq, CB, nrows, rows, N, K, acc);
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t i = 0; i < nrows; ++i) {
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t t = rows ? rows[i] : i;
+            double main_part = acc[i * N + n] * (double)SCx[t] * (double)SCB[n]
+                               / (448.0 * 448.0);
+            double out_part = 0.0;
+            for (int32_t j = 0; j < *n_o; ++j) {
+                int64_t k = idx[j];
+                double w = oracle_e4m3_to_double(CB[n * K + k]) * (double)SCB[n] / 448.0;
+                out_part += (double)oracle_half_to_float(X[t * K + k]) * w;
+            }
+            double b = bias ? (double)oracle_half_to_float(bias[n]) : 0.0;
+            C[i * N + n] = main_part + out_part + b;
+        }
+    }
+    free(is_outlier);
+    return 0;
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

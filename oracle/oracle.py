@@ -58,6 +58,17 @@ def _load(path):
     L.oracle_linear_forward_rows.argtypes = [P, i64, i64, P, P, P, i64, ctypes.c_float,
                                              P, i64, P, P, P, P, P, P, P]
     L.oracle_linear_forward_rows.restype = i64
+    L.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+    L.oracle_e4m3_to_double.restype = ctypes.c_double
+    L.oracle_e4m3_from_float.argtypes = [ctypes.c_float]
+    L.oracle_e4m3_from_float.restype = ctypes.c_uint8
+    L.oracle_absmax_quantize_rows_e4m3.argtypes = [P, i64, i64, P, P, P]
+    L.oracle_absmax_quantize_rows_e4m3.restype = None
+    L.oracle_e4m3_matmul.argtypes = [P, P, i64, P, i64, i64, P]
+    L.oracle_e4m3_matmul.restype = None
+    L.oracle_linear_forward_rows_e4m3.argtypes = [P, i64, i64, P, P, P, i64, ctypes.c_float,
+                                                  P, i64, P, P, P, P, P, P, P]
+    L.oracle_linear_forward_rows_e4m3.restype = i64
     L.oracle_num_threads.argtypes = []
     L.oracle_num_threads.restype = ctypes.c_int
     return L
@@ -156,5 +167,80 @@ def linear_forward(X, CB, SCB, bias, threshold, rows=None):
         raise MemoryError("oracle allocation failed")
     if ov:
         raise OverflowError("int32 accumulator overflow in %d results" % ov)
+    n = int(n_o[0])
+    return dict(mask_words=words, idx=idx[:n].copy(), n_o=n, Xq=Xq, SCx=SCx, acc=acc, C=C)
+
+
+# ------------------------------------------------------------------- e4m3 variant
+def e4m3_to_float(code: int) -> float:
+    return lib().oracle_e4m3_to_double(int(code) & 0xFF)
+
+
+def e4m3_from_float(v: float) -> int:
+    return int(lib().oracle_e4m3_from_float(float(v)))
+
+
+def e4m3_decode(codes):
+    """Exact values (float64) of an array of e4m3 codes."""
+    table = np.array([e4m3_to_float(c) for c in range(256)], np.float64)
+    return table[np.asarray(codes, np.uint8)]
+
+
+def absmax_quantize_rows_e4m3(A, skip=None):
+    """Row-wise absmax e4m3 codes: returns (codes uint8 [R,K], scale float32 [R])."""
+    Ab = _bits(A)
+    R, K = Ab.shape
+    q = np.zeros((R, K), np.uint8)
+    s = np.zeros(R, np.float32)
+    sk = None if skip is None else np.ascontiguousarray(skip, dtype=np.uint8)
+    lib().oracle_absmax_quantize_rows_e4m3(_ptr(Ab), R, K, _ptr(sk), _ptr(q), _ptr(s))
+    return q, s
+
+
+def quantize_weight_e4m3(W):
+    """Per-output-channel e4m3 quantisation of W [N,K] -> (CB uint8 [N,K], SCB float32 [N])."""
+    return absmax_quantize_rows_e4m3(W, None)
+
+
+def e4m3_matmul(A, B, rows=None):
+    """Exact product of e4m3 code matrices: float64 [len(rows) or A.shape[0], N]."""
+    A = np.ascontiguousarray(A, np.uint8)
+    B = np.ascontiguousarray(B, np.uint8)
+    K = A.shape[1]
+    assert B.shape[1] == K
+    r = None if rows is None else np.ascontiguousarray(rows, np.int64)
+    nrows = A.shape[0] if r is None else r.shape[0]
+    N = B.shape[0]
+    acc = np.zeros((nrows, N), np.float64)
+    lib().oracle_e4m3_matmul(_ptr(A), _ptr(B), nrows, _ptr(r), N, K, _ptr(acc))
+    return acc
+
+
+def linear_forward_e4m3(X, CB, SCB, bias, threshold, rows=None):
+    """The e4m3 forward (mask and SCx over all rows; product and output for `rows`).
+
+    Returns a dict with mask_words, idx, n_o, Xq (uint8 codes), SCx, acc (fp64) and C.
+    """
+    Xb = _bits(X)
+    T, K = Xb.shape
+    CB = np.ascontiguousarray(CB, np.uint8)
+    SCB = np.ascontiguousarray(SCB, np.float32)
+    N = CB.shape[0]
+    bb = None if bias is None else _bits(bias)
+    r = None if rows is None else np.ascontiguousarray(rows, np.int64)
+    nrows = T if r is None else r.shape[0]
+    words = np.zeros((K + 31) // 32, np.uint32)
+    idx = np.zeros(max(K, 1), np.int32)
+    n_o = np.zeros(1, np.int32)
+    Xq = np.zeros((T, K), np.uint8)
+    SCx = np.zeros(T, np.float32)
+    acc = np.zeros((nrows, N), np.float64)
+    C = np.zeros((nrows, N), np.float64)
+    st = lib().oracle_linear_forward_rows_e4m3(_ptr(Xb), T, K, _ptr(CB), _ptr(SCB), _ptr(bb),
+                                               N, float(threshold), _ptr(r), nrows,
+                                               _ptr(words), _ptr(idx), _ptr(n_o), _ptr(Xq),
+                                               _ptr(SCx), _ptr(acc), _ptr(C))
+    if st < 0:
+        raise MemoryError("oracle allocation failed")
     n = int(n_o[0])
     return dict(mask_words=words, idx=idx[:n].copy(), n_o=n, Xq=Xq, SCx=SCx, acc=acc, C=C)

@@ -335,4 +335,175 @@ def pin_row_subset_matches_full():
     assert np.array_equal(rs["C"], r["C"][rows])
 
 
+# ---------------------------------------------------------------- e4m3 variant
+# The pages name 8-bit floating point only as the next step; the variant keeps every step
+# of the decomposition with e4m3 codes (scale 448 / absmax) in place of int8 ones.  The
+# pins below tie the e4m3 arithmetic to the format's definition (OCP 8-bit floating point,
+# e4m3 "fn": bias 7, 3 fraction bits, max 448, no infinities) through an independent
+# library cast and brute force, and the forward to the same closed forms as the int8 one.
+
+def _e4m3_values():
+    """The 127 finite non-negative e4m3 values, by code 0x00..0x7E, from torch's cast."""
+    import torch
+    codes = torch.arange(0, 0x7F, dtype=torch.uint8)
+    return codes.view(torch.float8_e4m3fn).float().double().numpy()
+
+
+def pin_e4m3_decode_against_torch():
+    """All 256 codes decode as torch's float8_e4m3fn (NaN exactly at S.1111.111)."""
+    import torch
+    ref = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn)
+    ref = ref.float().double().numpy()
+    got = np.array([O.e4m3_to_float(c) for c in range(256)])
+    nan = np.isnan(ref)
+    assert nan.tolist() == np.isnan(got).tolist() and nan.sum() == 2
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def pin_e4m3_encode_against_torch():
+    """Encoding (nearest, ties to even) agrees with torch's float8_e4m3fn cast on every
+    finite fp16 value below 464 in magnitude, on the exact midpoints between neighbouring
+    e4m3 values (the ties), and on random fp32 values."""
+    import torch
+    h = np.arange(0, 0x10000, dtype=np.uint32).astype(np.uint16).view(np.float16)
+    h = h[np.isfinite(h)].astype(np.float32)
+    h = h[np.abs(h) < 464.0]
+    v = _e4m3_values()
+    mids = ((v[1:] + v[:-1]) / 2).astype(np.float32)
+    rng = np.random.default_rng(7)
+    rnd = (rng.standard_normal(20000) * np.exp2(rng.uniform(-12, 8, 20000))).astype(np.float32)
+    rnd = rnd[np.abs(rnd) < 464.0]
+    x = np.concatenate([h, mids, -mids, rnd])
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([O.e4m3_from_float(float(t)) for t in x], np.uint8)
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, (x[bad[:5]], got[bad[:5]], ref[bad[:5]])
+
+
+def pin_e4m3_encode_brute_force():
+    """Independent of any library: the code is the nearest of the 127 finite magnitudes
+    (ties to the even code), the sign is kept, and 448 and beyond saturate to 448."""
+    v = _e4m3_values()
+    rng = np.random.default_rng(8)
+    xs = np.concatenate([rng.uniform(0, 460, 3000), np.exp2(rng.uniform(-12, 9, 3000)),
+                         (v[1:] + v[:-1]) / 2]).astype(np.float32)
+    for x in xs[:4000]:
+        a = float(abs(x))
+        d = np.abs(v - a)
+        best = np.nonzero(d == d.min())[0]
+        want = best[0] if best.size == 1 else [c for c in best if c % 2 == 0][0]
+        if a >= 448.0:
+            want = 0x7E
+        assert O.e4m3_from_float(float(x)) == want, (x, want)
+        assert O.e4m3_from_float(-float(x)) == (want | 0x80 if want else 0x80), x
+    assert O.e4m3_from_float(1e6) == 0x7E and O.e4m3_from_float(-1e6) == 0xFE
+
+
+def pin_e4m3_rows_absmax_and_scaling():
+    """Row quantisation: the absmax element codes to +-448 (0x7E / 0xFE), skipped columns
+    and zero rows give code 0 and scale 0, and scaling a row by 2^j (exact in fp16) keeps
+    its codes and scales its absmax by 2^j."""
+    rng = np.random.default_rng(9)
+    A = (rng.standard_normal((5, 40)) * 0.7).astype(np.float16)
+    A[2] = 0
+    A[3, 7] = -2.5          # the largest magnitude of row 3
+    skip = np.zeros(40, np.uint8)
+    skip[[4, 11]] = 1
+    q, s = O.absmax_quantize_rows_e4m3(A, skip)
+    assert not q[2].any() and s[2] == 0
+    assert not q[:, [4, 11]].any()
+    assert q[3, 7] == 0xFE and s[3] == 2.5
+    for r in (0, 1, 3, 4):
+        kept = np.abs(A[r].astype(np.float32)) * (1 - skip)
+        assert s[r] == kept.max()
+        k = int(np.argmax(kept))
+        assert q[r, k] & 0x7F == 0x7E
+    q2, s2 = O.absmax_quantize_rows_e4m3((A.astype(np.float32) * 4).astype(np.float16), skip)
+    assert np.array_equal(q2, q) and np.array_equal(s2, s * 4)
+
+
+def pin_e4m3_hand_worked_example():
+    """A 1x4 by 4x2 case worked by hand with exact fractions (threshold 6):
+      X = [1, 0.15185546875, 8, -0.5]: column 2 is the outlier; SCx = 1, scale 448;
+          0.15185546875 * 448 = 68.03125 lies just past the midpoint 68 of the e4m3 step
+          [64, 72], so it codes to 72 (0x69); codes [448, 72, 0, -224] = [7E, 69, 00, F6].
+      W row 0 = [1, .5, .25, -1]: SCB 1, codes [448, 224, 112, -448] = [7E, 76, 6E, FE];
+      W row 1 = [.5, .5, .5, .5]: SCB .5, scale 896, codes all 448.
+      acc = [448*448 + 72*224 + 224*448, 448*448 + 72*448 - 224*448] = [317184, 132608].
+      C0 = 317184 * 1 * 1 / 448^2 + 8 * 112 * 1 / 448 + 0
+      C1 = 132608 * 1 * .5 / 448^2 + 8 * 448 * .5 / 448 + 1"""
+    X = _f16([[1.0, 0.15185546875, 8.0, -0.5]])
+    assert float(X[0, 1]) == 0.15185546875
+    W = _f16([[1.0, 0.5, 0.25, -1.0], [0.5, 0.5, 0.5, 0.5]])
+    b = _f16([0.0, 1.0])
+    CB, SCB = O.quantize_weight_e4m3(W)
+    assert CB.tolist() == [[0x7E, 0x76, 0x6E, 0xFE], [0x7E] * 4]
+    assert SCB.tolist() == [1.0, 0.5]
+    r = O.linear_forward_e4m3(X, CB, SCB, b, 6.0)
+    assert r["idx"].tolist() == [2] and r["SCx"].tolist() == [1.0]
+    assert r["Xq"].tolist() == [[0x7E, 0x69, 0x00, 0xF6]]
+    assert r["acc"].tolist() == [[317184.0, 132608.0]]
+    exp = [Fraction(317184, 448 ** 2) + Fraction(8 * 112, 448),
+           Fraction(132608, 2 * 448 ** 2) + Fraction(8 * 448, 2 * 448) + 1]
+    for got, e in zip(r["C"][0], exp):
+        assert abs(Fraction(got) - e) < Fraction(1, 10 ** 12)
+
+
+def _linear_case_e4m3(T, K, N, seed, cols, thr, bias_sigma=0.02):
+    w = synth.Workload("pin8", T, K, N, seed=seed, fixed_cols=cols, b_sigma=bias_sigma)
+    X, W, b = synth.make_x(w), synth.make_w(w), synth.make_bias(w)
+    CB, SCB = O.quantize_weight_e4m3(W)
+    return X, W, b, CB, SCB, O.linear_forward_e4m3(X, CB, SCB, b, thr)
+
+
+def pin_e4m3_threshold_zero_is_fp16_gemm():
+    """thr = 0: every column is an outlier column, so the e4m3 layer is the plain product
+    X @ (dec(CB) * SCB / 448)^T + bias, against numpy's fp64 matmul."""
+    X, W, b, CB, SCB, r = _linear_case_e4m3(9, 48, 11, 26, (2, 30), 0.0)
+    assert r["n_o"] == 48 and not r["Xq"].any() and not r["SCx"].any()
+    Wr = O.e4m3_decode(CB) * SCB.astype(np.float64)[:, None] / 448.0
+    ref = X.astype(np.float64) @ Wr.T + b.astype(np.float64)
+    assert np.allclose(r["C"], ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_e4m3_threshold_inf_is_vectorwise():
+    """thr = +inf: the e4m3 part alone.  The exact product equals numpy's fp64 matmul of
+    the decoded codes (every partial sum is exact), and the output is its outer-product
+    dequantisation by SCx * SCB / 448^2 plus the bias."""
+    X, W, b, CB, SCB, r = _linear_case_e4m3(6, 64, 10, 27, (4,), math.inf)
+    assert r["n_o"] == 0
+    acc = O.e4m3_decode(r["Xq"]) @ O.e4m3_decode(CB).T
+    assert np.array_equal(r["acc"], acc)
+    ref = acc * np.outer(r["SCx"].astype(np.float64), SCB.astype(np.float64)) / 448.0 ** 2
+    ref += b.astype(np.float64)
+    assert np.allclose(r["C"], ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_e4m3_error_bound_against_unquantised_product():
+    """Closed-form bound versus the unquantised X W^T + b (numpy fp64).  An e4m3 code is
+    within half a step of the scaled value: relative 2^-4 for normal values, 2^-10 absolute
+    below 2^-6 (plus fp32 slack), so with e(x) = 2^-4 |x| + 2^-10 SCx / 448:
+      non-outlier k: |x w - x^ w^| <= |x| e(w) + (|w| + e(w)) e(x)
+      outlier k:     |x w - x w^|  <= |x| e(w)"""
+    X, W, b, CB, SCB, r = _linear_case_e4m3(13, 80, 9, 28, (1, 33, 70), 6.0, bias_sigma=3.0)
+    assert set(r["idx"].tolist()) >= {1, 33, 70}
+    x, w = X.astype(np.float64), W.astype(np.float64)
+    ref = x @ w.T + b.astype(np.float64)
+    out = np.zeros(80, bool)
+    out[r["idx"]] = True
+    slack = 1 + 2.0 ** -20
+    ex = (2.0 ** -4 * np.abs(x) + 2.0 ** -10 * r["SCx"].astype(np.float64)[:, None] / 448) * slack
+    ew = (2.0 ** -4 * np.abs(w) + 2.0 ** -10 * SCB.astype(np.float64)[:, None] / 448) * slack
+    ax, aw = np.abs(x), np.abs(w)
+    bound = ax @ ew.T                                    # every column: |x| e(w)
+    keep = ~out
+    bound += ex[:, keep] @ (aw[:, keep] + ew[:, keep]).T  # non-outlier columns: e(x) terms
+    bound += 1e-9
+    err = np.abs(r["C"] - ref)
+    assert (err <= bound).all(), float((err - bound).max())
+    # and the bound is not vacuous: dropping the outlier columns breaks it
+    contrib = np.abs(x[:, out] @ w[:, out].T)
+    assert (contrib > 3 * bound).mean() > 0.5
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -32,6 +32,22 @@ MUTATIONS = [
     ("mask_bit_order", "mask_words[k / 32] |= (uint32_t)1 << (k % 32);",
      "mask_words[k / 32] |= (uint32_t)1 << (31 - k % 32);"),
     ("subnormal_decode", "v = ldexpf((float)f, -24);", "v = ldexpf((float)f, -25);"),
+    # e4m3 variant
+    ("e4m3_scale_447", "float s = 448.0f / amax;", "float s = 447.0f / amax;"),
+    ("e4m3_ties_away", "double r = nearbyint(a / step) * step;",
+     "double r = round(a / step) * step;"),
+    ("e4m3_exponent_bias_8", "v = ldexp(1.0 + m / 8.0, e - 7);",
+     "v = ldexp(1.0 + m / 8.0, e - 8);"),
+    ("e4m3_two_fraction_bits", "double step = ldexp(1.0, E - 3);",
+     "double step = ldexp(1.0, E - 2);"),
+    ("e4m3_dequant_127", "/ (448.0 * 448.0);", "/ (448.0 * 127.0);"),
+    ("e4m3_recovery_127", "(double)SCB[n] / 448.0;", "(double)SCB[n] / 127.0;"),
+    ("e4m3_outlier_dropped", "out_part += (double)oracle_half_to_float(X[t * K + k]) * w;\n"
+     "            }\n            double b = bias ? (double)oracle_half_to_float(bias[n]) : 0.0;\n"
+     "            C[i * N + n] = main_part",
+     "out_part += 0.0;\n"
+     "            }\n            double b = bias ? (double)oracle_half_to_float(bias[n]) : 0.0;\n"
+     "            C[i * N + n] = main_part"),
 ]
 
 
