@@ -34,6 +34,10 @@ SIGNATURES = {
     "i8_linear_forward": (_ST, [_P, _I64, _I64, _P, _P, _P, _I64, _F, _P, _P, _SZ, _P]),
     "i8_igemm_s32": (_ST, [_P, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
     "i8_linear_forward_noalloc": (_ST, [_P, _I64, _I64, _P, _P, _P, _I64, _F, _P, _P]),
+    "i8_quantize_weight_e4m3": (_ST, [_P, _I64, _I64, _P, _P, _P]),
+    "i8_prepare_act_e4m3": (_ST, [_P, _I64, _I64, _F, _P, _P, _P, _P, _P, _P, _P]),
+    "i8_linear_workspace_size_e4m3": (_SZ, [_I64, _I64, _I64]),
+    "i8_linear_forward_e4m3": (_ST, [_P, _I64, _I64, _P, _P, _P, _I64, _F, _P, _P, _SZ, _P]),
     "i8_outlier_cache_size": (_SZ, [_I64, _I64, _I64]),
     "i8_outlier_cache_reset": (_ST, [_P, _SZ, _P]),
     "i8_linear_forward_cached": (_ST, [_P, _I64, _I64, _P, _P, _P, _I64, _F, _P, _P, _SZ, _P,
@@ -146,6 +150,36 @@ def i8_linear_forward_noalloc(X, CB, SCB, bias, threshold, C, stream=None):
     _check("i8_linear_forward_noalloc",
            load().i8_linear_forward_noalloc(_ptr(X), T, K, _ptr(CB), _ptr(SCB), _ptr(bias), N,
                                             float(threshold), _ptr(C), _stream(stream)))
+
+
+def i8_quantize_weight_e4m3(W, CB, SCB, stream=None):
+    """e4m3 variant of i8_quantize_weight: CB is a uint8 [N, K] tensor of e4m3 codes."""
+    N, K = W.shape
+    _check("i8_quantize_weight_e4m3",
+           load().i8_quantize_weight_e4m3(_ptr(W), N, K, _ptr(CB), _ptr(SCB), _stream(stream)))
+
+
+def i8_prepare_act_e4m3(X, threshold, col_mask, outlier_idx, n_outliers, Xq, SCx, X_o,
+                        stream=None):
+    T, K = X.shape
+    _check("i8_prepare_act_e4m3",
+           load().i8_prepare_act_e4m3(_ptr(X), T, K, float(threshold), _ptr(col_mask),
+                                      _ptr(outlier_idx), _ptr(n_outliers), _ptr(Xq), _ptr(SCx),
+                                      _ptr(X_o), _stream(stream)))
+
+
+def i8_linear_workspace_size_e4m3(T, N, K) -> int:
+    return int(load().i8_linear_workspace_size_e4m3(T, N, K))
+
+
+def i8_linear_forward_e4m3(X, CB, SCB, bias, threshold, C, workspace, stream=None):
+    T, K = X.shape
+    N = CB.shape[0]
+    _check("i8_linear_forward_e4m3",
+           load().i8_linear_forward_e4m3(_ptr(X), T, K, _ptr(CB), _ptr(SCB), _ptr(bias), N,
+                                         float(threshold), _ptr(C), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(),
+                                         _stream(stream)))
 
 
 def i8_outlier_cache_size(N, K, max_cols) -> int:

@@ -64,6 +64,8 @@ i8_status device_info(DeviceInfo** out) {
     if (cudaFuncSetAttribute(gemm::i8_gemm_tcgen05_kernel<false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
         cudaFuncSetAttribute(gemm::i8_gemm_tcgen05_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(gemm::i8_gemm_tcgen05_kernel<false, true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
       return I8_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
@@ -143,7 +145,7 @@ struct Workspace {
 // start of every forward.
 // Decode path: the slice records of every 32-row tile, the tiles' arrival counters and the
 // words of the cooperative prologue (none needs clearing: they carry the launch's epoch).
-Workspace layout(int64_t T, int64_t N, int64_t K) {
+Workspace layout(int64_t T, int64_t N, int64_t K, bool gemm_path = false) {
   Workspace w{};
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -151,7 +153,7 @@ Workspace layout(int64_t T, int64_t N, int64_t K) {
     off = align_up(off + bytes, 256);
     return o;
   };
-  if (use_decode(T, K)) {
+  if (!gemm_path && use_decode(T, K)) {
     const size_t n_tiles = static_cast<size_t>((N + gemv::ROWS - 1) / gemv::ROWS);
     w.rec = take(n_tiles * static_cast<size_t>(gemv::num_slices(K)) *
                  static_cast<size_t>(gemv::rec_bytes(T)));
@@ -282,9 +284,10 @@ i8_status run_scan(const void* X, int64_t T, int64_t K, float thr, uint32_t* mas
 
 i8_status run_quant_rows(const void* A, int64_t R, int64_t K, const uint32_t* mask, int8_t* Q,
                          float* scale, const int32_t* idx, const int32_t* n_o, void* A_o,
-                         cudaStream_t s) {
+                         cudaStream_t s, bool e4m3 = false) {
   quantize_rows_kernel<<<static_cast<unsigned>(R), kQuantThreads, 0, s>>>(
-      static_cast<const __half*>(A), R, K, mask, Q, scale, idx, n_o, static_cast<__half*>(A_o));
+      static_cast<const __half*>(A), R, K, mask, Q, scale, idx, n_o, static_cast<__half*>(A_o),
+      e4m3);
   return launch_status();
 }
 
@@ -298,7 +301,7 @@ i8_status run_prepare(const void* X, int64_t T, int64_t K, float thr, uint32_t* 
                       int64_t zero_words, int32_t* idx, int32_t* n_o, int8_t* Xq, float* SCx,
                       void* X_o, const int8_t* CB, int64_t N, void* CB_o, const DeviceInfo& d,
                       cudaStream_t s, uint8_t* ocache = nullptr, int64_t ocols = 0,
-                      int32_t* cbo_sel = nullptr) {
+                      int32_t* cbo_sel = nullptr, bool e4m3 = false) {
   if (cudaMemsetAsync(mask, 0, static_cast<size_t>(zero_words) * 4, s) != cudaSuccess)
     return I8_ERR_CUDA;
   const int64_t G0 = d.sms;
@@ -336,6 +339,7 @@ i8_status run_prepare(const void* X, int64_t T, int64_t K, float thr, uint32_t* 
       ocache ? reinterpret_cast<__half*>(ocache + ocache_header_bytes(K)) : nullptr;
   a.ocache_cols = ocache ? ocols : 0;
   a.cbo_sel = cbo_sel;
+  a.e4m3 = e4m3;
   a.rows_per_cta = rows_per_cta;
   a.cache_rows = cache_rows;
   a.cache_bytes_all = cache_rows * K * 2;
@@ -354,7 +358,7 @@ i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t
                    const void* A_o, const void* B_o, const int32_t* n_o, const float* SCx,
                    const float* SCB, const void* bias, void* C, int32_t* acc,
                    const DeviceInfo& d, cudaStream_t s, const void* B_c = nullptr,
-                   int64_t ocols = 0, const int32_t* cbo_sel = nullptr) {
+                   int64_t ocols = 0, const int32_t* cbo_sel = nullptr, bool e4m3 = false) {
   CUtensorMap tA, tB, tAo, tBo, tBc;
   if (!map_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, T, K, gemm::BK, gemm::HM) ||
       !map_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, K, gemm::BK, gemm::HN))
@@ -389,7 +393,10 @@ i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t
   const int64_t tiles = static_cast<int64_t>(a.m_tiles) * a.n_tiles;
   const int clusters = static_cast<int>(tiles < d.gemm_clusters ? tiles : d.gemm_clusters);
   cudaError_t e;
-  if (raw)
+  if (e4m3 && !raw)
+    e = launch_overlapped(gemm::i8_gemm_tcgen05_kernel<false, true>, dim3(2 * clusters),
+                          dim3(gemm::THREADS), gemm::SMEM_BYTES, s, tA, tB, tAo, tBo, tBc, a);
+  else if (raw)
     e = launch_overlapped(gemm::i8_gemm_tcgen05_kernel<true>, dim3(2 * clusters),
                           dim3(gemm::THREADS), gemm::SMEM_BYTES, s, tA, tB, tAo, tBo, tBc, a);
   else
@@ -659,6 +666,75 @@ i8_status i8_outlier_cache_reset(void* cache, size_t cache_bytes, void* stream) 
   if (cudaMemsetAsync(cache, 0, kOcacheHdrWords * 4, static_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
     return I8_ERR_CUDA;
+  return I8_OK;
+}
+
+size_t i8_linear_workspace_size_e4m3(int64_t T, int64_t N, int64_t K) {
+  if (!shape_ok(T, K) || N <= 0 || N > 0x7fffffffLL) return 0;
+  return layout(T, N, K, true).total;
+}
+
+i8_status i8_quantize_weight_e4m3(const void* W, int64_t N, int64_t K, uint8_t* CB, float* SCB,
+                                  void* stream) {
+  if (!W || !CB || !SCB || !aligned16(W) || !aligned16(CB) || !aligned16(SCB)) return I8_ERR_INVALID_ARG;
+  if (!shape_ok(N, K)) return I8_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  i8_status st = device_info(&d);
+  if (st != I8_OK) return st;
+  return run_quant_rows(W, N, K, nullptr, reinterpret_cast<int8_t*>(CB), SCB, nullptr, nullptr,
+                        nullptr, static_cast<cudaStream_t>(stream), true);
+}
+
+i8_status i8_prepare_act_e4m3(const void* X, int64_t T, int64_t K, float threshold,
+                              uint32_t* col_mask, int32_t* outlier_idx, int32_t* n_outliers,
+                              uint8_t* Xq, float* SCx, void* X_o, void* stream) {
+  if (!X || !col_mask || !outlier_idx || !n_outliers || !Xq || !SCx || !X_o)
+    return I8_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(col_mask) || !aligned16(outlier_idx) || !aligned16(Xq) ||
+      !aligned16(SCx) || !aligned16(X_o) || !aligned16(n_outliers))
+    return I8_ERR_INVALID_ARG;
+  if (!shape_ok(T, K) || threshold != threshold) return I8_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  i8_status st = device_info(&d);
+  if (st != I8_OK) return st;
+  return run_prepare(X, T, K, threshold, col_mask, (K + 31) / 32 + 1, outlier_idx, n_outliers,
+                     reinterpret_cast<int8_t*>(Xq), SCx, X_o, nullptr, 0, nullptr, *d,
+                     static_cast<cudaStream_t>(stream), nullptr, 0, nullptr, true);
+}
+
+i8_status i8_linear_forward_e4m3(const void* X, int64_t T, int64_t K, const uint8_t* CB,
+                                 const float* SCB, const void* bias, int64_t N, float threshold,
+                                 void* C, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!X || !CB || !SCB || !C || !workspace) return I8_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(CB) || !aligned16(SCB) || !aligned16(C) ||
+      !aligned16(workspace) || (bias && !aligned16(bias)))
+    return I8_ERR_INVALID_ARG;
+  if (!shape_ok(T, K) || N <= 0 || N > 0x7fffffffLL || threshold != threshold)
+    return I8_ERR_INVALID_ARG;
+  const Workspace w = layout(T, N, K, true);
+  if (workspace_bytes < w.total) return I8_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  i8_status st = device_info(&d);
+  if (st != I8_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const bool prof = g_prof_start != nullptr && g_prof_stop != nullptr;
+  uint32_t* mask = reinterpret_cast<uint32_t*>(ws + w.mask);
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + w.idx);
+  int32_t* n_o = reinterpret_cast<int32_t*>(ws + w.n_o);
+  float* SCx = reinterpret_cast<float*>(ws + w.scx);
+  int8_t* Xq = reinterpret_cast<int8_t*>(ws + w.xq);
+  void* X_o = ws + w.xo;
+  void* CB_o = ws + w.cbo;
+  const int8_t* CBb = reinterpret_cast<const int8_t*>(CB);
+  st = run_prepare(X, T, K, threshold, mask, w.zero_words, idx, n_o, Xq, SCx, X_o, CBb, N, CB_o,
+                   *d, s, nullptr, 0, nullptr, true);
+  if (st != I8_OK) return st;
+  if (prof && cudaEventRecord(g_prof_start, s) != cudaSuccess) return I8_ERR_CUDA;
+  st = run_gemm(false, Xq, T, K, CBb, N, X_o, CB_o, n_o, SCx, SCB, bias, C, nullptr, *d, s,
+                nullptr, 0, nullptr, true);
+  if (st != I8_OK) return st;
+  if (prof && cudaEventRecord(g_prof_stop, s) != cudaSuccess) return I8_ERR_CUDA;
   return I8_OK;
 }
 

@@ -205,11 +205,17 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t smem_addr) {
   return d;
 }
 
-// Instruction descriptors (kind::i8 and kind::f16), both operands K-major, dense.
+// Instruction descriptors (kind::i8, kind::f8f6f4 and kind::f16), both operands K-major, dense.
 //   bits 4-5 accumulator format (1 = f32, 2 = s32)   bits 7-9 / 10-12 A / B format
 //   bits 17-22 N >> 3                                 bits 24-28 M >> 4
 __host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N) {
   return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// kind::f8f6f4 with e4m3 A and B (format code 0) and an fp32 accumulator
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 

@@ -44,6 +44,7 @@ constexpr int THREADS = 224;     // warps 0,6 TMA (A, B); 1 MMA; 2..5 epilogue
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC_I8 = idesc_s8_s32(TM, TN);
 constexpr uint32_t IDESC_F16 = idesc_f16_f32(TM, TN);
+constexpr uint32_t IDESC_E4M3 = idesc_e4m3_f32(TM, TN);
 constexpr int INSERT_AT = 8;    // K-blocks of tile i+1 issued before the outlier MMAs of tile i
 constexpr int GROUP_M = 16;     // m-tiles per raster group (L2 reuse of Xq)
 constexpr int COL_BYTES = 2 * 2 * TN * 4;        // SCB/127 and bias as fp32, two buffers
@@ -147,6 +148,16 @@ __device__ __forceinline__ void umma_i8_pair(uint32_t d_tmem, uint64_t adesc, ui
       : "memory");
 }
 
+__device__ __forceinline__ void umma_e4m3_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                               uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -186,6 +197,12 @@ __device__ __forceinline__ void tmem_st_wait() {
 
 __device__ __forceinline__ void epilogue_bar() {
   asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// An accumulator word as fp32: an int32 sum of int8 products, or already fp32 (e4m3).
+template <bool kE4M3>
+__device__ __forceinline__ float acc_value(uint32_t r) {
+  return kE4M3 ? __uint_as_float(r) : static_cast<float>(static_cast<int32_t>(r));
 }
 
 // Stores 32 consecutive fp16 outputs of one row (c0 = first column of the chunk).
@@ -241,7 +258,10 @@ __device__ __forceinline__ bool walk_schedule(int L, int KB, int OC, F&& visit) 
   return true;
 }
 
-template <bool kRaw>
+// kRaw: write the int32 accumulators (int8 codes only).  kE4M3: the codes are e4m3
+// (kind::f8f6f4, fp32 accumulators, scales over 448) instead of int8 (kind::i8, int32
+// accumulators, scales over 127).
+template <bool kRaw, bool kE4M3 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     i8_gemm_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmB,
@@ -293,6 +313,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = bars->tmem_base;
+  constexpr float kInvQ = kE4M3 ? 1.0f / 448.0f : 1.0f / 127.0f;
   // everything above overlaps the previous kernel; its outputs are read from here on
   grid_dep_wait();
 
@@ -409,7 +430,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const uint32_t sa = ring + s * STAGE_BYTES;
         const uint32_t sb = sa + A_BYTES;
         const uint32_t d = tmem_base + static_cast<uint32_t>(b * TN);
-        if (kind == 0) {
+        if (kind == 0 && kE4M3) {
+#pragma unroll
+          for (int kk = 0; kk < BK / 32; ++kk)
+            umma_e4m3_pair(d, sdesc_k_sw128(sa + kk * 32), sdesc_k_sw128(sb + kk * 32),
+                           IDESC_E4M3, (idx | kk) != 0);
+        } else if (kind == 0) {
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk)
             umma_i8_pair(d, sdesc_k_sw128(sa + kk * 32), sdesc_k_sw128(sb + kk * 32), IDESC_I8,
@@ -455,17 +481,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       if (!kRaw) {
         for (int j = et; j < TN; j += 128) {
           const int n = n0 + j;
-          ws[j] = n < a.N ? __ldg(a.SCB + n) * (1.0f / 127.0f) : 0.0f;
+          ws[j] = n < a.N ? __ldg(a.SCB + n) * kInvQ : 0.0f;
           bs[j] = (n < a.N && a.bias) ? __half2float(a.bias[n]) : 0.0f;
         }
       }
       epilogue_bar();
       if (dead) continue;
-      const float sx = (!kRaw && row_ok) ? __ldg(a.SCx + t) * (1.0f / 127.0f) : 0.0f;
+      const float sx = (!kRaw && row_ok) ? __ldg(a.SCx + t) * kInvQ : 0.0f;
       const uint32_t tb = lane_base + static_cast<uint32_t>(b * TN);
 
       if (!kRaw && OC > 0) {
-        // int32 -> fp32 * SCx/127 in place; the outlier MMAs then add on top
+        // accumulator (int32, or fp32 for e4m3) -> fp32 * SCx/127 (/448) in place; the
+        // outlier MMAs then add on top
         bool got = mbar_wait(smem_u32(&bars->int_full[b]), use & 1u, abort_flag, lim);
         if (!__all_sync(0xffffffffu, got)) {
           dead = true;
@@ -479,7 +506,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            r[j] = __float_as_uint(static_cast<float>(static_cast<int32_t>(r[j])) * sx);
+            r[j] = __float_as_uint(acc_value<kE4M3>(r[j]) * sx);
           tmem_st_32x32b_x32(tb + static_cast<uint32_t>(c * 32), r);
         }
         tmem_st_wait();
@@ -524,7 +551,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             } else {
 #pragma unroll
               for (int j = 0; j < 32; ++j)
-                v[j] = fmaf(static_cast<float>(static_cast<int32_t>(r[j])) * sx, wsc[j], bsc[j]);
+                v[j] = fmaf(acc_value<kE4M3>(r[j]) * sx, wsc[j], bsc[j]);
             }
             store_row32_f16(a.C + static_cast<int64_t>(t) * a.N, c0, a.N, v, vec_ok);
           }

@@ -156,6 +156,46 @@ __device__ __forceinline__ uint2 codes8(const uint4 v, uint32_t skip, float s) {
   return make_uint2(out[0], out[1]);
 }
 
+// e4m3 variant: the codes of 8 fp16 values are the e4m3 roundings (nearest, ties to even;
+// magnitudes beyond 448 saturate) of fl32(x * s); excluded columns, and every column of
+// a row whose scale is 0, give code 0.  Two values per conversion instruction: the
+// second source goes to the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ uint2 codes8_e4m3(const uint4 v, uint32_t skip, float s) {
+  if (s == 0.0f) return make_uint2(0u, 0u);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t out[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = h2f2(w[i]);
+    const float p0 = ((skip >> (2 * i)) & 1u) ? 0.0f : __fmul_rn(f.x, s);
+    const float p1 = ((skip >> (2 * i + 1)) & 1u) ? 0.0f : __fmul_rn(f.y, s);
+    out[i >> 1] |= e4m3x2(p0, p1) << (16 * (i & 1));
+  }
+  return make_uint2(out[0], out[1]);
+}
+
+// codes of 8 values in the layer's code format (int8, or e4m3 when e4m3 is set)
+__device__ __forceinline__ uint2 codes8_fmt(const uint4 v, uint32_t skip, float s, bool e4m3) {
+  return e4m3 ? codes8_e4m3(v, skip, s) : codes8(v, skip, s);
+}
+
+// largest code magnitude of the format: the absmax maps onto it
+__device__ __forceinline__ float code_max(bool e4m3) { return e4m3 ? 448.0f : 127.0f; }
+
+// fp16 value of one weight code (an int8 code, or an e4m3 code in the low byte of c)
+__device__ __forceinline__ __half code_to_half(int c, bool e4m3) {
+  if (!e4m3) return __int2half_rn(c);
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(c & 0xff)));
+  return __ushort_as_half(static_cast<unsigned short>(h & 0xffffu));
+}
+
 __device__ __forceinline__ uint32_t skip_bits8(const uint32_t* mask, int64_t v) {
   return mask ? ((__ldg(mask + (v >> 2)) >> (8 * (v & 3))) & 0xffu) : 0u;
 }
@@ -166,7 +206,8 @@ __global__ void __launch_bounds__(kQuantThreads)
     quantize_rows_kernel(const __half* __restrict__ A, int64_t R, int64_t K,
                          const uint32_t* __restrict__ mask, int8_t* __restrict__ Q,
                          float* __restrict__ scale, const int32_t* __restrict__ idx,
-                         const int32_t* __restrict__ n_o_ptr, __half* __restrict__ A_o) {
+                         const int32_t* __restrict__ n_o_ptr, __half* __restrict__ A_o,
+                         bool e4m3 = false) {
   __shared__ float red[kQuantThreads / 32];
   const int64_t r = blockIdx.x;
   const int64_t nv = K >> 3;
@@ -196,16 +237,16 @@ __global__ void __launch_bounds__(kQuantThreads)
 #pragma unroll
   for (int w = 1; w < kQuantThreads / 32; ++w) amax = fmaxf(amax, red[w]);
 
-  const float s = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+  const float s = amax > 0.0f ? __fdiv_rn(code_max(e4m3), amax) : 0.0f;
   uint2* qrow = reinterpret_cast<uint2*>(Q + r * K);
 #pragma unroll
   for (int i = 0; i < kQuantCacheVec; ++i) {
     const int64_t v = threadIdx.x + static_cast<int64_t>(i) * kQuantThreads;
-    if (v < nv) qrow[v] = codes8(cache[i], skip[i], s);
+    if (v < nv) qrow[v] = codes8_fmt(cache[i], skip[i], s, e4m3);
   }
   for (int64_t v = threadIdx.x + static_cast<int64_t>(kQuantCacheVec) * kQuantThreads; v < nv;
        v += kQuantThreads)
-    qrow[v] = codes8(ldg_v4(row + v), skip_bits8(mask, v), s);
+    qrow[v] = codes8_fmt(ldg_v4(row + v), skip_bits8(mask, v), s, e4m3);
   if (threadIdx.x == 0) scale[r] = amax;
 
   if (A_o != nullptr) {
@@ -262,6 +303,7 @@ struct PrepArgs {
   __half* ocache_CB_o;    // chunk-major slice [ocache_cols / 64][N][64]
   int64_t ocache_cols;    // capacity in columns, a multiple of 64
   int32_t* cbo_sel;       // out (may be NULL): 1 when this call's CB_o is the cache's slice
+  bool e4m3;              // codes in e4m3 (scale 448 / absmax) instead of int8
   int64_t rows_per_cta;
   int64_t cache_rows;     // rows of its block each CTA keeps in shared memory
   int64_t cache_bytes_all; // size of the row-cache region (reused by phase 4)
@@ -341,22 +383,24 @@ __device__ __forceinline__ float row_absmax(uint32_t base, const uint4* gbase, i
   return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 }
 
-// int8 codes of groups start, start+step, ... of one row.
+// codes (int8, or e4m3) of groups start, start+step, ... of one row.
 template <bool kShared>
 __device__ __forceinline__ void row_codes(uint32_t base, const uint4* gbase, uint2* q, int gpr,
-                                          int start, int step, const uint32_t* smask, float s) {
+                                          int start, int step, const uint32_t* smask, float s,
+                                          bool e4m3) {
   int v = start;
   for (; v + 3 * step < gpr; v += 4 * step) {
     const uint4 x0 = row_vec<kShared>(base, gbase, v);
     const uint4 x1 = row_vec<kShared>(base, gbase, v + step);
     const uint4 x2 = row_vec<kShared>(base, gbase, v + 2 * step);
     const uint4 x3 = row_vec<kShared>(base, gbase, v + 3 * step);
-    q[v] = codes8(x0, scan_bits(smask, v), s);
-    q[v + step] = codes8(x1, scan_bits(smask, v + step), s);
-    q[v + 2 * step] = codes8(x2, scan_bits(smask, v + 2 * step), s);
-    q[v + 3 * step] = codes8(x3, scan_bits(smask, v + 3 * step), s);
+    q[v] = codes8_fmt(x0, scan_bits(smask, v), s, e4m3);
+    q[v + step] = codes8_fmt(x1, scan_bits(smask, v + step), s, e4m3);
+    q[v + 2 * step] = codes8_fmt(x2, scan_bits(smask, v + 2 * step), s, e4m3);
+    q[v + 3 * step] = codes8_fmt(x3, scan_bits(smask, v + 3 * step), s, e4m3);
   }
-  for (; v < gpr; v += step) q[v] = codes8(row_vec<kShared>(base, gbase, v), scan_bits(smask, v), s);
+  for (; v < gpr; v += step)
+    q[v] = codes8_fmt(row_vec<kShared>(base, gbase, v), scan_bits(smask, v), s, e4m3);
 }
 
 // Column of the j-th outlier (j < n_o) from the mask words and their exclusive popcount
@@ -617,7 +661,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
       if (it < items4) {
         const int64_t c = it / p.N, n = it - c * p.N;
         reinterpret_cast<__half2*>(cbo + (c * p.N + n) * 64)[lane] =
-            __floats2half2_rn(static_cast<float>(v0[u]), static_cast<float>(v1[u]));
+            __halves2half2(code_to_half(v0[u], p.e4m3), code_to_half(v1[u], p.e4m3));
       }
     }
   };
@@ -659,12 +703,12 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
         for (int w2 = 0; w2 < wpr; ++w2) amax = fmaxf(amax, s_red[rr * wpr + w2]);
       }
       if (!have) continue;
-      const float sc = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+      const float sc = amax > 0.0f ? __fdiv_rn(code_max(p.e4m3), amax) : 0.0f;
       uint2* qrow = reinterpret_cast<uint2*>(p.Xq + t * K);
       if (cached)
-        row_codes<true>(sbase, gbase, qrow, g32, start, step, smask, sc);
+        row_codes<true>(sbase, gbase, qrow, g32, start, step, smask, sc, p.e4m3);
       else
-        row_codes<false>(sbase, gbase, qrow, g32, start, step, smask, sc);
+        row_codes<false>(sbase, gbase, qrow, g32, start, step, smask, sc, p.e4m3);
       if (sub == 0 && lane == 0) p.SCx[t] = amax;
       // the row's outlier values into X_o, eight loads in flight before their stores
       const __half* xrow = cached ? reinterpret_cast<const __half*>(cache + i * gpr) : p.X + t * K;
@@ -714,20 +758,18 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
             break;
           }
           for (int64_t c0 = 0; c0 < chunks; c0 += 4) {
-            float v0[4], v1[4];
+            int v0[4], v1[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const int64_t j0 = (c0 + u) * 64 + 2 * lane;
-              v0[u] = j0 < n_o ? static_cast<float>(static_cast<int8_t>(rowbuf[idx_at(j0)])) : 0.0f;
-              v1[u] = j0 + 1 < n_o
-                          ? static_cast<float>(static_cast<int8_t>(rowbuf[idx_at(j0 + 1)]))
-                          : 0.0f;
+              v0[u] = j0 < n_o ? static_cast<int8_t>(rowbuf[idx_at(j0)]) : 0;
+              v1[u] = j0 + 1 < n_o ? static_cast<int8_t>(rowbuf[idx_at(j0 + 1)]) : 0;
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u)
               if (c0 + u < chunks)
                 reinterpret_cast<__half2*>(cbo + ((c0 + u) * p.N + n) * 64)[lane] =
-                    __floats2half2_rn(v0[u], v1[u]);
+                    __halves2half2(code_to_half(v0[u], p.e4m3), code_to_half(v1[u], p.e4m3));
           }
           __syncwarp();
         }

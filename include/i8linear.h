@@ -207,6 +207,44 @@ i8_status i8_linear_forward_cached(const void* X, int64_t T, int64_t K, const in
                                    void* stream);
 
 /*
+ * FP8 (e4m3) variant of the layer.  The blog names 8-bit floating point only as the next
+ * step after int8 (its closing outlook); these calls take the plainest reading of it:
+ * every step above is kept, and the int8 absmax code is replaced by an e4m3 code of the
+ * same scaled value --
+ *   scale s = fl32(448 / absmax)   (448 = the largest finite e4m3 magnitude),
+ *   code    = e4m3 rounding of fl32(x * s): nearest, ties to even, beyond 448 saturating,
+ * with 448 in place of 127 in both dequantisations:
+ *   C[t,n] = fp16_rn( (acc[t,n] * SCx[t] / 448 + sum_j X[t,idx_j] * dec(CB[n,idx_j]))
+ *                     * SCB[n] / 448 + bias[n] ),
+ * acc being the e4m3 x e4m3 product accumulated in fp32 by the tensor cores
+ * (tcgen05 kind::f8f6f4).  e4m3 is the "fn" format of the OCP 8-bit floating-point
+ * specification (1 sign, 4 exponent bits with bias 7, 3 fraction bits, no infinities).
+ * Codes are stored one byte each (uint8_t), row-major, like the int8 codes.
+ *
+ * i8_quantize_weight_e4m3(W, N, K, CB, SCB, stream): as i8_quantize_weight, with CB [N, K]
+ *   e4m3 codes.
+ * i8_prepare_act_e4m3(...): as i8_prepare_act, with Xq [T, K] e4m3 codes (outlier columns
+ *   code 0).
+ * i8_linear_workspace_size_e4m3(T, N, K): workspace bytes of i8_linear_forward_e4m3 (0 for
+ *   invalid shapes).
+ * i8_linear_forward_e4m3(X, T, K, CB, SCB, bias, N, threshold, C, workspace,
+ *   workspace_bytes, stream): the e4m3 forward; arguments as in i8_linear_forward, with CB
+ *   from i8_quantize_weight_e4m3 and a workspace of i8_linear_workspace_size_e4m3 bytes.
+ *   Every T takes the fused prepare pass and the tensor-core GEMM (there is no separate
+ *   decode kernel for this variant).
+ * Errors as for the int8 calls.
+ */
+i8_status i8_quantize_weight_e4m3(const void* W, int64_t N, int64_t K, uint8_t* CB, float* SCB,
+                                  void* stream);
+i8_status i8_prepare_act_e4m3(const void* X, int64_t T, int64_t K, float threshold,
+                              uint32_t* col_mask, int32_t* outlier_idx, int32_t* n_outliers,
+                              uint8_t* Xq, float* SCx, void* X_o, void* stream);
+size_t i8_linear_workspace_size_e4m3(int64_t T, int64_t N, int64_t K);
+i8_status i8_linear_forward_e4m3(const void* X, int64_t T, int64_t K, const uint8_t* CB,
+                                 const float* SCB, const void* bias, int64_t N, float threshold,
+                                 void* C, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * i8_linear_forward without a workspace argument: the same forward as i8_linear_forward,
  * with its scratch taken from a fixed 32 MiB array that the library itself holds in
  * device memory.  The pages have no counterpart to this call; it exists for callers that
