@@ -297,23 +297,28 @@ def run_gpu(args, w0):
 
     X_d, W_d = fp16_tensor(X, dev), fp16_tensor(W, dev)
     b_d = None if b is None else fp16_tensor(b, dev)
-    CB = torch.empty((N, K), dtype=torch.int8, device=dev)
+    e4m3 = args.format == "e4m3"
+    if e4m3 and args.outlier_cache:
+        raise SystemExit("--outlier-cache applies to the int8 forward only")
+    CB = torch.empty((N, K), dtype=torch.uint8 if e4m3 else torch.int8, device=dev)
+    quantize_weight = abi.i8_quantize_weight_e4m3 if e4m3 else abi.i8_quantize_weight
     SCB = torch.empty((N,), dtype=torch.float32, device=dev)
 
     # weight quantisation (once per weight): timed on its own
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    abi.i8_quantize_weight(W_d, CB, SCB)
+    quantize_weight(W_d, CB, SCB)
     torch.cuda.synchronize()
     reps = 5
     ev[0].record(stream)
     for _ in range(reps):
-        abi.i8_quantize_weight(W_d, CB, SCB)
+        quantize_weight(W_d, CB, SCB)
     ev[1].record(stream)
     torch.cuda.synchronize()
     wq_ms = ev[0].elapsed_time(ev[1]) / reps
     del W_d
 
-    ws = torch.empty((abi.i8_linear_workspace_size(T, N, K),), dtype=torch.uint8, device=dev)
+    ws_size = abi.i8_linear_workspace_size_e4m3 if e4m3 else abi.i8_linear_workspace_size
+    ws = torch.empty((ws_size(T, N, K),), dtype=torch.uint8, device=dev)
     C = torch.empty((T, N), dtype=torch.float16, device=dev)
     use_flush, l2_desc = l2_policy(args.l2_flush, T, N, K)
     flush = torch.empty((L2_FLUSH_BYTES if use_flush else 16,), dtype=torch.uint8, device=dev)
@@ -330,7 +335,9 @@ def run_gpu(args, w0):
         abi.i8_outlier_cache_reset(cache)
 
     def forward(X_in):
-        if cache is None:
+        if e4m3:
+            abi.i8_linear_forward_e4m3(X_in, CB, SCB, b_d, w.threshold, C, ws)
+        elif cache is None:
             abi.i8_linear_forward(X_in, CB, SCB, b_d, w.threshold, C, ws)
         else:
             abi.i8_linear_forward_cached(X_in, CB, SCB, b_d, w.threshold, C, ws, cache)
@@ -431,7 +438,7 @@ def run_gpu(args, w0):
     if st != 0:
         raise RuntimeError("device error in the e2e loop: %s" % abi.STATUS.get(st, st))
 
-    decode = T <= 16
+    decode = T <= 16 and not e4m3   # (the e4m3 forward runs the GEMM for every T)
     pk = peaks()
     kern_per = kern_ms / K_steps
     if decode:
@@ -444,18 +451,18 @@ def run_gpu(args, w0):
                 "algorithmic_bytes_per_launch": gemv_bytes}
         tr = traffic_record("decode_kernel", w0.name)
     else:
-        # dominant kernel: the tcgen05 GEMM; int8 ops plus fp16 flops counted at the int8
-        # rate x 2 (the nominal fp16 : int8 tensor rate is 1 : 2)
+        # dominant kernel: the tcgen05 GEMM; int8 (or e4m3) ops plus fp16 flops counted at
+        # the 8-bit rate x 2 (the nominal fp16 : int8 : fp8 dense rates are 1 : 2 : 2)
         equiv = i8_ops + 2.0 * f16_flops
         achieved = equiv / (kern_per * 1e-3) / 1e12
         peak_i8 = 2.0 * pk["bf16_sus"]
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak_i8, "unit": "TOPS",
                 "frac": achieved / peak_i8, "kernel": "i8_gemm_tcgen05_kernel",
-                "peak_basis": "%s sustained bf16 %.1f TF/s x 2 (nominal int8:bf16 ratio)"
-                              % (pk["source"], pk["bf16_sus"]),
+                "peak_basis": "%s sustained bf16 %.1f TF/s x 2 (nominal %s:bf16 ratio)"
+                              % (pk["source"], pk["bf16_sus"], "fp8" if e4m3 else "int8"),
                 "frac_of_burst_peak": achieved / (2.0 * pk["bf16"]),
                 "algorithmic_ops_per_launch": equiv}
-        tr = traffic_record("i8_gemm_tcgen05_kernel", w0.name)
+        tr = None if e4m3 else traffic_record("i8_gemm_tcgen05_kernel", w0.name)
     roof["kernel_ms"] = kern_per
     roof["traffic"] = None if tr is None else tr["dram_bytes_per_launch"]
     if tr is not None:
@@ -464,11 +471,13 @@ def run_gpu(args, w0):
     line = {"metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
             "steps": K_steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "int8", "data": "synthetic",
+            "dtype": "e4m3" if e4m3 else "int8", "data": "synthetic",
             "config": dict(w0.describe(), n_outliers=n_o,
                            parallelism="column-parallel x%d (own output-channel block per GPU)"
                                        % world,
                            l2=l2_desc,
+                           **({"code_format": "e4m3 (the FP8 variant of the decomposition)"}
+                              if e4m3 else {}),
                            **({"outlier_cache": "on: the fixed input's outlier set is cached "
                                                 "during warm-up, every timed step hits"}
                               if cache is not None else {})),
@@ -484,7 +493,7 @@ def run_gpu(args, w0):
             "clocks": clk}
 
     # CPU baseline: the oracle on this host, rank 0 at N = 1 only
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not e4m3:
         from oracle import oracle as O
         CB_h = CB.cpu().numpy()
         SCB_h = SCB.cpu().numpy()
@@ -580,6 +589,9 @@ def main():
     ap.add_argument("--l2-flush", default="auto", choices=["auto", "always"],
                     help="auto: flush the L2 between timed steps only when the inputs are "
                          "smaller than twice the L2")
+    ap.add_argument("--format", default="int8", choices=["int8", "e4m3"],
+                    help="code format of the decomposition's 8-bit part (e4m3: the FP8 "
+                         "variant, not the benchmark's headline configuration)")
     ap.add_argument("--outlier-cache", action="store_true",
                     help="forward through i8_linear_forward_cached (the weight's outlier "
                          "columns kept across calls)")
