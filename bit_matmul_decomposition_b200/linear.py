@@ -22,6 +22,9 @@ dimensions carry the outliers call after call): ``outlier_cache_cols > 0`` keeps
 weight's codes in the outlier columns (CB_o) in a device cache across forwards
 (``i8_linear_forward_cached``), so a call whose outlier set matches the cached one skips
 their gather; outputs are bit-identical to the uncached layer.
+
+``code_format="e4m3"`` selects the FP8 variant of the decomposition (e4m3 codes scaled by
+448 / absmax, the library's ``i8_*_e4m3`` calls); CB then holds e4m3 codes as uint8.
 """
 from __future__ import annotations
 
@@ -78,8 +81,13 @@ class Linear8bitLt(torch.nn.Module):
 
     def __init__(self, in_features: int, out_features: int, bias: bool = True,
                  threshold: float = 6.0, device=None, has_fp16_weights: bool = False,
-                 outlier_cache_cols: int = 0):
+                 outlier_cache_cols: int = 0, code_format: str = "int8"):
         super().__init__()
+        if code_format not in ("int8", "e4m3"):
+            raise ValueError("code_format must be 'int8' or 'e4m3'")
+        if code_format == "e4m3" and outlier_cache_cols:
+            raise ValueError("the outlier cache serves the int8 forward only")
+        self.code_format = code_format
         if in_features <= 0 or out_features <= 0 or in_features % 16 != 0:
             raise ValueError("in_features must be a positive multiple of 16 (row pitch of the "
                              "int8 weight for TMA); out_features positive")
@@ -93,7 +101,8 @@ class Linear8bitLt(torch.nn.Module):
         self.threshold = float(threshold)
         self.outlier_cache_cols = int(outlier_cache_cols)
         self._ocache: Dict[torch.device, torch.Tensor] = {}
-        self.register_buffer("CB", torch.zeros((out_features, in_features), dtype=torch.int8,
+        cb_dtype = torch.uint8 if code_format == "e4m3" else torch.int8
+        self.register_buffer("CB", torch.zeros((out_features, in_features), dtype=cb_dtype,
                                                device=device))
         self.register_buffer("SCB", torch.zeros((out_features,), dtype=torch.float32,
                                                 device=device))
@@ -114,14 +123,14 @@ class Linear8bitLt(torch.nn.Module):
     @classmethod
     def from_linear(cls, linear: torch.nn.Linear, threshold: float = 6.0,
                     has_fp16_weights: bool = False,
-                    outlier_cache_cols: int = 0) -> "Linear8bitLt":
+                    outlier_cache_cols: int = 0, code_format: str = "int8") -> "Linear8bitLt":
         """Quantise an nn.Linear that lives on a CUDA device (weights cast to fp16)."""
         w = linear.weight
         if not w.is_cuda:
             raise ValueError("the weight must be on a CUDA device (it is quantised there)")
         m = cls(linear.in_features, linear.out_features, bias=linear.bias is not None,
                 threshold=threshold, device=w.device, has_fp16_weights=has_fp16_weights,
-                outlier_cache_cols=outlier_cache_cols)
+                outlier_cache_cols=outlier_cache_cols, code_format=code_format)
         if has_fp16_weights:
             with torch.no_grad():
                 m.weight.copy_(w.detach().to(torch.float16))
@@ -140,7 +149,7 @@ class Linear8bitLt(torch.nn.Module):
                              % (tuple(weight.shape), (self.out_features, self.in_features)))
         if weight.device != self.CB.device:
             raise ValueError("weight on %s, layer on %s" % (weight.device, self.CB.device))
-        abi.i8_quantize_weight(weight.to(torch.float16).contiguous(), self.CB, self.SCB)
+        self._quantize(weight.to(torch.float16).contiguous())
         self.invalidate_outlier_cache()
         if bias is not None:
             if self.bias is None:
@@ -148,12 +157,24 @@ class Linear8bitLt(torch.nn.Module):
             self.bias.copy_(bias.to(torch.float16))
         return self
 
+    def _quantize(self, weight16: torch.Tensor):
+        if self.code_format == "e4m3":
+            abi.i8_quantize_weight_e4m3(weight16, self.CB, self.SCB)
+        else:
+            abi.i8_quantize_weight(weight16, self.CB, self.SCB)
+
     def dequantized_weight(self) -> torch.Tensor:
-        """The weight the layer computes with, CB * SCB / 127 (fp32), for inspection."""
+        """The weight the layer computes with (fp32): CB * SCB / 127, or for e4m3 codes
+        their values * SCB / 448."""
+        if self.code_format == "e4m3":
+            vals = self.CB.view(torch.float8_e4m3fn).float()
+            return vals * (self.SCB.float() / 448.0)[:, None]
         return self.CB.float() * (self.SCB.float() / 127.0)[:, None]
 
     def _workspace(self, T: int) -> torch.Tensor:
-        need = abi.i8_linear_workspace_size(T, self.out_features, self.in_features)
+        size = (abi.i8_linear_workspace_size_e4m3 if self.code_format == "e4m3"
+                else abi.i8_linear_workspace_size)
+        need = size(T, self.out_features, self.in_features)
         dev = self.CB.device
         ws = self._ws.get(dev)
         if ws is None or ws.numel() < need:
@@ -187,7 +208,10 @@ class Linear8bitLt(torch.nn.Module):
         out = torch.empty((T, self.out_features), dtype=torch.float16, device=x2.device)
         if T > 0:
             bias = None if self.bias is None else self.bias.detach()
-            if self.outlier_cache_cols > 0:
+            if self.code_format == "e4m3":
+                abi.i8_linear_forward_e4m3(x2, self.CB, self.SCB, bias, self.threshold, out,
+                                           self._workspace(T))
+            elif self.outlier_cache_cols > 0:
                 abi.i8_linear_forward_cached(x2, self.CB, self.SCB, bias, self.threshold, out,
                                              self._workspace(T), self._outlier_cache())
             else:
@@ -205,7 +229,7 @@ class Linear8bitLt(torch.nn.Module):
         x2 = x.reshape(-1, self.in_features).contiguous()
         if self.has_fp16_weights:
             with torch.no_grad():  # the weight may have changed since the last forward
-                abi.i8_quantize_weight(self.weight.detach().contiguous(), self.CB, self.SCB)
+                self._quantize(self.weight.detach().contiguous())
         w = self.weight if self.has_fp16_weights else None
         if torch.is_grad_enabled() and (x2.requires_grad or (w is not None and w.requires_grad)):
             y = _Int8LinearFn.apply(x2, w, self.bias, self)
@@ -215,15 +239,16 @@ class Linear8bitLt(torch.nn.Module):
 
     def extra_repr(self) -> str:
         return ("in_features=%d, out_features=%d, bias=%s, threshold=%g, has_fp16_weights=%s, "
-                "outlier_cache_cols=%d" % (self.in_features, self.out_features,
-                                           self.bias is not None, self.threshold,
-                                           self.has_fp16_weights, self.outlier_cache_cols))
+                "outlier_cache_cols=%d, code_format=%s"
+                % (self.in_features, self.out_features, self.bias is not None, self.threshold,
+                   self.has_fp16_weights, self.outlier_cache_cols, self.code_format))
 
 
 def replace_linear_with_int8(model: torch.nn.Module, threshold: float = 6.0,
                              skip: Iterable[str] = ("lm_head",),
                              has_fp16_weights: bool = False,
-                             outlier_cache_cols: int = 0) -> torch.nn.Module:
+                             outlier_cache_cols: int = 0,
+                             code_format: str = "int8") -> torch.nn.Module:
     """Swap every nn.Linear of `model` (weights on a CUDA device) for a Linear8bitLt, in
     place, except modules whose name (last path component) is in `skip`.  Returns `model`."""
     skip = set(skip)
@@ -231,9 +256,11 @@ def replace_linear_with_int8(model: torch.nn.Module, threshold: float = 6.0,
         if isinstance(child, torch.nn.Linear) and name not in skip:
             setattr(model, name, Linear8bitLt.from_linear(child, threshold=threshold,
                                                           has_fp16_weights=has_fp16_weights,
-                                                          outlier_cache_cols=outlier_cache_cols))
+                                                          outlier_cache_cols=outlier_cache_cols,
+                                                          code_format=code_format))
         elif name not in skip:
             replace_linear_with_int8(child, threshold=threshold, skip=skip,
                                      has_fp16_weights=has_fp16_weights,
-                                     outlier_cache_cols=outlier_cache_cols)
+                                     outlier_cache_cols=outlier_cache_cols,
+                                     code_format=code_format)
     return model

@@ -93,6 +93,25 @@ def test_outlier_cache_layer_matches_and_follows_new_weights():
     sync_ok()
 
 
+@pytest.mark.parametrize("lead", [(1, 5), (3, 7)], ids=["T5", "T21"])
+def test_e4m3_module_matches_oracle(lead):
+    K, N = 1024, 768
+    lin = _fp16_linear(K, N, seed=13)
+    m = Linear8bitLt.from_linear(lin, code_format="e4m3")
+    W = host(lin.weight)
+    CBr, SCBr = O.quantize_weight_e4m3(W)
+    assert np.array_equal(host(m.CB), CBr)
+    X = _x(lead, K, (7, 500, 1000), seed=23)
+    y = m(torch.from_numpy(X.view(np.int16)).view(torch.float16).cuda())
+    sync_ok()
+    ref = O.linear_forward_e4m3(X.reshape(-1, K), CBr, SCBr, host(lin.bias), 6.0)["C"]
+    check_output(host(y).reshape(-1, N), ref)
+    # the weight the layer computes with is the decoded codes times SCB / 448
+    wd = host(m.dequantized_weight()).astype(np.float64)
+    want = O.e4m3_decode(CBr) * SCBr.astype(np.float64)[:, None] / 448.0
+    assert np.allclose(wd, want, rtol=2.0 ** -22, atol=0)
+
+
 def test_replaced_layer_stack_layer_by_layer():
     """Linear -> GELU -> Linear (+ an fp16 head left alone): each int8 layer matches the
     oracle on the activations it actually received."""

@@ -52,7 +52,8 @@ def test_forward_rejects_other_dtypes_before_any_call():
 def test_replace_walk(monkeypatch):
     made = []
 
-    def fake_from_linear(linear, threshold=6.0, has_fp16_weights=False, outlier_cache_cols=0):
+    def fake_from_linear(linear, threshold=6.0, has_fp16_weights=False, outlier_cache_cols=0,
+                         code_format="int8"):
         made.append((linear.in_features, linear.out_features, threshold, outlier_cache_cols))
         return torch.nn.Identity()
 
@@ -84,3 +85,18 @@ def test_outlier_cache_option():
         L.Linear8bitLt(64, 32, outlier_cache_cols=-1)
     with pytest.raises(ValueError):
         L.Linear8bitLt(64, 32, outlier_cache_cols=64, has_fp16_weights=True)
+
+
+def test_e4m3_code_format_option():
+    m = L.Linear8bitLt(64, 32, code_format="e4m3")
+    assert m.CB.dtype == torch.uint8 and "code_format=e4m3" in repr(m)
+    # dequantised weight: e4m3 values * SCB / 448 (0x38 = 1.0, 0x7E = 448, 0xFE = -448)
+    m.CB.zero_()
+    m.CB[0, :3] = torch.tensor([0x38, 0x7E, 0xFE], dtype=torch.uint8)
+    m.SCB.fill_(2.0)
+    w = m.dequantized_weight()
+    assert w[0, :3].tolist() == pytest.approx([2.0 / 448, 2.0, -2.0], rel=1e-6)
+    with pytest.raises(ValueError):
+        L.Linear8bitLt(64, 32, code_format="int4")
+    with pytest.raises(ValueError):
+        L.Linear8bitLt(64, 32, code_format="e4m3", outlier_cache_cols=64)
