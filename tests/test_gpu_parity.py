@@ -150,6 +150,11 @@ FORWARD_CASES = [
     (12, 3584, 48, (3583,), 0.0, 6.0, False),       # one slice, last column an outlier
     (9, 8000, 333, (1, 4000, 7999), 0.0, 6.0, True),  # decode, X > 128 KB: split prologue
     (40, 9216, 96, (), 0.0, 0.0, True),             # GEMM, n_o = 9216 (> 8192 kept indices)
+    # GEMM, one outlier chunk with adjacent and far-apart columns, and a single outlier
+    # column on ragged tiles without bias
+    (300, 1040, 700, (0, 1, 2, 3, 4, 5, 6, 1039), 0.0, 6.0, True),      # n_o = 8
+    (300, 1040, 700, (0, 1, 2, 3, 4, 5, 6, 7, 1039), 0.0, 6.0, True),   # n_o = 9
+    (513, 4096, 1000, (77,), 0.0, 6.0, False),      # n_o = 1
 ]
 
 
