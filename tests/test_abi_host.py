@@ -138,3 +138,24 @@ def test_cached_forward_rejects_bad_arguments_without_cuda(lib):
     assert call(thr=math.nan) == INVALID
     assert lib.i8_outlier_cache_reset(None, c_ok, None) == INVALID
     assert lib.i8_outlier_cache_reset(FAKE, 16, None) == INVALID
+
+
+def test_e4m3_calls_reject_bad_arguments_without_cuda(lib):
+    # the e4m3 forward always takes the GEMM path, so its workspace for a decode-size batch
+    # is the GEMM layout (outlier slices sized for n_o = K), larger than the decode one
+    assert lib.i8_linear_workspace_size_e4m3(8, 4096, 4096) > \
+        lib.i8_linear_workspace_size(8, 4096, 4096)
+    assert lib.i8_linear_workspace_size_e4m3(2048, 16384, 4096) == \
+        lib.i8_linear_workspace_size(2048, 16384, 4096)
+    assert lib.i8_linear_workspace_size_e4m3(0, 64, 64) == 0
+    assert lib.i8_linear_workspace_size_e4m3(8, 64, 72) == 0
+    ws_ok = lib.i8_linear_workspace_size_e4m3(32, 64, 64)
+    f = lib.i8_linear_forward_e4m3
+    assert f(None, 32, 64, FAKE, FAKE, None, 64, 6.0, FAKE, FAKE, ws_ok, None) == INVALID
+    assert f(FAKE, 32, 64, FAKE, FAKE, None, 64, math.nan, FAKE, FAKE, ws_ok, None) == INVALID
+    assert f(FAKE, 32, 64, FAKE, FAKE, None, 64, 6.0, FAKE, FAKE, ws_ok - 1, None) == INVALID
+    assert f(FAKE, 32, 72, FAKE, FAKE, None, 64, 6.0, FAKE, FAKE, ws_ok, None) == INVALID
+    assert lib.i8_quantize_weight_e4m3(FAKE, 64, 40, FAKE, FAKE, None) == INVALID
+    assert lib.i8_quantize_weight_e4m3(None, 64, 64, FAKE, FAKE, None) == INVALID
+    assert lib.i8_prepare_act_e4m3(FAKE, 4, 64, 6.0, FAKE, FAKE, FAKE, None, FAKE, FAKE,
+                                   None) == INVALID
