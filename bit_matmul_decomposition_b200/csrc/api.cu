@@ -518,17 +518,19 @@ i8_status static_scratch_address(void** out) {
   return I8_OK;
 }
 
-// The forward of both entry points; `cache` (ocols columns) is NULL for the uncached one.
+// The forward of every entry point: int8 codes (with `cache`, ocols columns, or without:
+// NULL), or e4m3 codes (no cache; the prepare pass and the GEMM for every T).
 i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, const float* SCB,
                        const void* bias, int64_t N, float threshold, void* C, void* workspace,
-                       size_t workspace_bytes, uint8_t* cache, int64_t ocols, void* stream) {
+                       size_t workspace_bytes, uint8_t* cache, int64_t ocols, void* stream,
+                       bool e4m3 = false) {
   if (!X || !CB || !SCB || !C || !workspace) return I8_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(CB) || !aligned16(SCB) || !aligned16(C) ||
       !aligned16(workspace) || (bias && !aligned16(bias)))
     return I8_ERR_INVALID_ARG;
   if (!shape_ok(T, K) || N <= 0 || N > 0x7fffffffLL || threshold != threshold)
     return I8_ERR_INVALID_ARG;
-  const Workspace w = layout(T, N, K);
+  const Workspace w = layout(T, N, K, e4m3);
   if (workspace_bytes < w.total) return I8_ERR_INVALID_ARG;
   DeviceInfo* d;
   i8_status st = device_info(&d);
@@ -536,7 +538,7 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const bool prof = g_prof_start != nullptr && g_prof_stop != nullptr;
-  if (use_decode(T, K)) {
+  if (!e4m3 && use_decode(T, K)) {
     // (the decode kernel takes the outlier columns' codes out of its own CB stream)
     if (prof && cudaEventRecord(g_prof_start, s) != cudaSuccess) return I8_ERR_CUDA;
     st = run_decode(false, X, nullptr, T, K, CB, N, threshold, SCB, bias, C, nullptr, ws, w, *d,
@@ -554,11 +556,11 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   void* X_o = ws + w.xo;
   void* CB_o = ws + w.cbo;
   st = run_prepare(X, T, K, threshold, mask, w.zero_words, idx, n_o, Xq, SCx, X_o, CB, N, CB_o,
-                   *d, s, cache, ocols, sel);
+                   *d, s, cache, ocols, sel, e4m3);
   if (st != I8_OK) return st;
   if (prof && cudaEventRecord(g_prof_start, s) != cudaSuccess) return I8_ERR_CUDA;
   st = run_gemm(false, Xq, T, K, CB, N, X_o, CB_o, n_o, SCx, SCB, bias, C, nullptr, *d, s,
-                cache ? cache + ocache_header_bytes(K) : nullptr, ocols, sel);
+                cache ? cache + ocache_header_bytes(K) : nullptr, ocols, sel, e4m3);
   if (st != I8_OK) return st;
   if (prof && cudaEventRecord(g_prof_stop, s) != cudaSuccess) return I8_ERR_CUDA;
   return I8_OK;
@@ -705,37 +707,8 @@ i8_status i8_prepare_act_e4m3(const void* X, int64_t T, int64_t K, float thresho
 i8_status i8_linear_forward_e4m3(const void* X, int64_t T, int64_t K, const uint8_t* CB,
                                  const float* SCB, const void* bias, int64_t N, float threshold,
                                  void* C, void* workspace, size_t workspace_bytes, void* stream) {
-  if (!X || !CB || !SCB || !C || !workspace) return I8_ERR_INVALID_ARG;
-  if (!aligned16(X) || !aligned16(CB) || !aligned16(SCB) || !aligned16(C) ||
-      !aligned16(workspace) || (bias && !aligned16(bias)))
-    return I8_ERR_INVALID_ARG;
-  if (!shape_ok(T, K) || N <= 0 || N > 0x7fffffffLL || threshold != threshold)
-    return I8_ERR_INVALID_ARG;
-  const Workspace w = layout(T, N, K, true);
-  if (workspace_bytes < w.total) return I8_ERR_INVALID_ARG;
-  DeviceInfo* d;
-  i8_status st = device_info(&d);
-  if (st != I8_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const bool prof = g_prof_start != nullptr && g_prof_stop != nullptr;
-  uint32_t* mask = reinterpret_cast<uint32_t*>(ws + w.mask);
-  int32_t* idx = reinterpret_cast<int32_t*>(ws + w.idx);
-  int32_t* n_o = reinterpret_cast<int32_t*>(ws + w.n_o);
-  float* SCx = reinterpret_cast<float*>(ws + w.scx);
-  int8_t* Xq = reinterpret_cast<int8_t*>(ws + w.xq);
-  void* X_o = ws + w.xo;
-  void* CB_o = ws + w.cbo;
-  const int8_t* CBb = reinterpret_cast<const int8_t*>(CB);
-  st = run_prepare(X, T, K, threshold, mask, w.zero_words, idx, n_o, Xq, SCx, X_o, CBb, N, CB_o,
-                   *d, s, nullptr, 0, nullptr, true);
-  if (st != I8_OK) return st;
-  if (prof && cudaEventRecord(g_prof_start, s) != cudaSuccess) return I8_ERR_CUDA;
-  st = run_gemm(false, Xq, T, K, CBb, N, X_o, CB_o, n_o, SCx, SCB, bias, C, nullptr, *d, s,
-                nullptr, 0, nullptr, true);
-  if (st != I8_OK) return st;
-  if (prof && cudaEventRecord(g_prof_stop, s) != cudaSuccess) return I8_ERR_CUDA;
-  return I8_OK;
+  return forward_impl(X, T, K, reinterpret_cast<const int8_t*>(CB), SCB, bias, N, threshold, C,
+                      workspace, workspace_bytes, nullptr, 0, stream, true);
 }
 
 i8_status i8_linear_forward_cached(const void* X, int64_t T, int64_t K, const int8_t* CB,

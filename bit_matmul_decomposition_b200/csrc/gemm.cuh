@@ -14,8 +14,10 @@
 // Design (sm_100a): persistent clusters of two CTAs on an SM pair, 256 x 256 output tiles,
 // tcgen05.mma.cta_group::2 (M = 256: each CTA holds 128 rows of A and 128 rows of B in its
 // own shared memory, and 128 rows x 256 columns of the accumulator in its own TMEM).
-//   warp 0      TMA producer (both CTAs): 128 B of K per stage, 128-byte swizzle, no
-//               multicast; both CTAs' loads complete on the leader CTA's barrier.
+//   warps 0, 6  TMA producers (both CTAs; warp 0 loads A, warp 6 loads B): 128 B of K per
+//               stage, 128-byte swizzle, no multicast; both CTAs' loads complete on the
+//               leader CTA's barrier.  B_o comes from one of two tensor maps (the
+//               workspace's CB_o slice, or an outlier cache's), chosen by a device word.
 //   warp 1      TMEM allocation (both CTAs); the leader's lane 0 issues every MMA and
 //               commits with multicast to both CTAs' barriers.
 //   warps 2..5  epilogue (both CTAs): tcgen05.ld / tcgen05.st, per-column scales staged in
@@ -24,6 +26,8 @@
 // MMAs of the next.  With outlier columns, the int32 accumulator of tile i is converted in
 // place to fp32 (times SCx/127) by the epilogue, and the fp16 outlier MMAs of tile i,
 // issued after the first few K-blocks of tile i+1, accumulate on top of it.
+// FP8 variant (kE4M3): e4m3 codes, tcgen05.mma kind::f8f6f4 with an fp32 accumulator that
+// the epilogue reads as it is, and 448 in place of 127 in both scales.
 #pragma once
 
 #include "common.cuh"

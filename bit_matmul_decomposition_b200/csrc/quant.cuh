@@ -4,7 +4,10 @@
 //   quantize_rows_kernel   steps 2/3: row absmax (over the non-outlier columns) and int8
 //                          codes; for the hidden states also the fp16 outlier slice X_o
 //   prepare_kernel         steps 1 and 2 fused (one read of X), plus the fp16 outlier
-//                          slices of X and of CB for step 6
+//                          slices of X and of CB for step 6 (CB's kept across calls in an
+//                          outlier cache when the caller provides one)
+// Both quantisers also produce the e4m3 codes of the FP8 variant (scale 448 / absmax,
+// nearest-even e4m3 rounding) when asked.
 // Source: "A Gentle Introduction to 8-bit Matrix Multiplication for transformers at
 // scale" (Hugging Face blog), sections "absmax 量化", "LLM.int8() 的总结", "内部的 MatMul".
 #pragma once
