@@ -245,6 +245,19 @@ bool map_2d_plain(CUtensorMap* m, const void* base, uint64_t inner, uint64_t out
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp16 output C [rows, cols] for TMA stores of 32 x 32 boxes (cols % 8 == 0).
+bool map_c(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Chunk-major outlier slice [chunks][rows][64] fp16; box [1][box_rows][64].
 bool map_slice(CUtensorMap* m, const void* base, uint64_t rows, uint64_t chunks,
                uint32_t box_rows) {
@@ -359,7 +372,7 @@ i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t
                    const float* SCB, const void* bias, void* C, int32_t* acc,
                    const DeviceInfo& d, cudaStream_t s, const void* B_c = nullptr,
                    int64_t ocols = 0, const int32_t* cbo_sel = nullptr, bool e4m3 = false) {
-  CUtensorMap tA, tB, tAo, tBo, tBc;
+  CUtensorMap tA, tB, tAo, tBo, tBc, tC;
   if (!map_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A, K, T, K, gemm::BK, gemm::HM) ||
       !map_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B, K, N, K, gemm::BK, gemm::HN))
     return I8_ERR_CUDA;
@@ -372,6 +385,11 @@ i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t
       return I8_ERR_CUDA;
   }
   tBc = tBo;
+  // C goes out by TMA stores when its row pitch allows a tensor map (N % 8 == 0)
+  tC = tA;
+  const bool c_tma = !raw && C != nullptr && (N % 8) == 0;
+  if (c_tma && !map_c(&tC, C, static_cast<uint64_t>(N), static_cast<uint64_t>(T)))
+    return I8_ERR_CUDA;
   if (!raw && B_c != nullptr && cbo_sel != nullptr &&
       !map_slice(&tBc, B_c, N, static_cast<uint64_t>(ocols / 64), gemm::HN))
     return I8_ERR_CUDA;
@@ -389,19 +407,20 @@ i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t
   a.bias = static_cast<const __half*>(bias);
   a.C = static_cast<__half*>(C);
   a.acc_out = acc;
+  a.c_tma = c_tma;
   a.wait_limit_ns = kWaitLimitNs;
   const int64_t tiles = static_cast<int64_t>(a.m_tiles) * a.n_tiles;
   const int clusters = static_cast<int>(tiles < d.gemm_clusters ? tiles : d.gemm_clusters);
   cudaError_t e;
   if (e4m3 && !raw)
     e = launch_overlapped(gemm::i8_gemm_tcgen05_kernel<false, true>, dim3(2 * clusters),
-                          dim3(gemm::THREADS), gemm::SMEM_BYTES, s, tA, tB, tAo, tBo, tBc, a);
+                          dim3(gemm::THREADS), gemm::SMEM_BYTES, s, tA, tB, tAo, tBo, tBc, tC, a);
   else if (raw)
     e = launch_overlapped(gemm::i8_gemm_tcgen05_kernel<true>, dim3(2 * clusters),
-                          dim3(gemm::THREADS), gemm::SMEM_BYTES, s, tA, tB, tAo, tBo, tBc, a);
+                          dim3(gemm::THREADS), gemm::SMEM_BYTES, s, tA, tB, tAo, tBo, tBc, tC, a);
   else
     e = launch_overlapped(gemm::i8_gemm_tcgen05_kernel<false>, dim3(2 * clusters),
-                          dim3(gemm::THREADS), gemm::SMEM_BYTES, s, tA, tB, tAo, tBo, tBc, a);
+                          dim3(gemm::THREADS), gemm::SMEM_BYTES, s, tA, tB, tAo, tBo, tBc, tC, a);
   return e == cudaSuccess ? launch_status() : I8_ERR_CUDA;
 }
 

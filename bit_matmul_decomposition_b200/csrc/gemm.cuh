@@ -52,9 +52,11 @@ constexpr uint32_t IDESC_E4M3 = idesc_e4m3_f32(TM, TN);
 constexpr int INSERT_AT = 8;    // K-blocks of tile i+1 issued before the outlier MMAs of tile i
 constexpr int GROUP_M = 16;     // m-tiles per raster group (L2 reuse of Xq)
 constexpr int COL_BYTES = 2 * 2 * TN * 4;        // SCB/127 and bias as fp32, two buffers
+// fp16 output staging for the TMA stores of C: per epilogue warp two 32 x 32 blocks
+constexpr int CST_BYTES = 4 * 2 * 32 * 64;
 constexpr int BAR_BYTES = 256;
 constexpr size_t SMEM_BYTES =
-    static_cast<size_t>(STAGES) * STAGE_BYTES + COL_BYTES + BAR_BYTES + 1024;
+    static_cast<size_t>(STAGES) * STAGE_BYTES + COL_BYTES + CST_BYTES + BAR_BYTES + 1024;
 constexpr uint16_t PAIR_MASK = 0x3;
 
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
@@ -70,6 +72,7 @@ struct Args {
   const __half* bias;  // nullable
   __half* C;
   int32_t* acc_out;  // raw-accumulator mode
+  bool c_tma;        // C is written by TMA stores through tmC (N % 8 == 0), else by threads
   uint64_t wait_limit_ns;
 };
 
@@ -209,6 +212,55 @@ __device__ __forceinline__ float acc_value(uint32_t r) {
   return kE4M3 ? __uint_as_float(r) : static_cast<float>(static_cast<int32_t>(r));
 }
 
+// fp32 outputs of one 32-column chunk of a row from its accumulator words: with outlier
+// MMAs the words already hold acc*SCx/127 + the outlier product (fp32); without, the raw
+// accumulator (int32, or fp32 for e4m3) is scaled here.  Then * SCB/127 (/448) + bias.
+template <bool kE4M3>
+__device__ __forceinline__ void epilogue_values(const uint32_t (&r)[32], int OC, float sx,
+                                                const float* wsc, const float* bsc,
+                                                float (&v)[32]) {
+  if (OC > 0) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = fmaf(__uint_as_float(r[j]), wsc[j], bsc[j]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = fmaf(acc_value<kE4M3>(r[j]) * sx, wsc[j], bsc[j]);
+  }
+}
+
+__device__ __forceinline__ void sts_v4(uint32_t addr, uint32_t x, uint32_t y, uint32_t z,
+                                       uint32_t w) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z),
+               "r"(w)
+               : "memory");
+}
+
+// TMA store of a shared-memory box to global memory (bulk-group completion).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// wait until at most the most recent bulk group still reads its shared-memory source
+__device__ __forceinline__ void bulk_wait_read_1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// this thread's generic-proxy shared-memory writes become visible to the async proxy
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Stores 32 consecutive fp16 outputs of one row (c0 = first column of the chunk).
 __device__ __forceinline__ void store_row32_f16(__half* crow, int c0, int N, const float (&v)[32],
                                                 bool vec_ok) {
@@ -271,15 +323,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                            const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmAo,
                            const __grid_constant__ CUtensorMap tmBo,
-                           const __grid_constant__ CUtensorMap tmBc, const Args a) {
+                           const __grid_constant__ CUtensorMap tmBc,
+                           const __grid_constant__ CUtensorMap tmC, const Args a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
   const uint32_t ring = raw_s + pad;  // 1024-aligned shared address of stage 0
   float* colbuf = reinterpret_cast<float*>(smem + static_cast<size_t>(STAGES) * STAGE_BYTES);
+  const uint32_t cstage = ring + static_cast<uint32_t>(STAGES * STAGE_BYTES + COL_BYTES);
   SmemBars* bars = reinterpret_cast<SmemBars*>(smem + static_cast<size_t>(STAGES) * STAGE_BYTES +
-                                               COL_BYTES);
+                                               COL_BYTES + CST_BYTES);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -307,6 +361,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tma_prefetch_desc(&tmAo);
     tma_prefetch_desc(&tmBo);
     tma_prefetch_desc(&tmBc);
+    if (a.c_tma) tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(&bars->tmem_base), TMEM_COLS);
@@ -466,19 +521,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   } else if (warp >= 2 && warp <= 5) {
     // -------------------------------------------------------------- epilogue warps
     const int q = warp & 3;
-    const int row = q * 32 + lane;
     const int et = threadIdx.x - 64;  // 0..127 among the epilogue threads
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     const bool vec_ok = (a.N % 8) == 0;
     // A warp that gives up on a wait keeps walking the tiles (it must still meet the
     // other epilogue warps at every named barrier) but touches TMEM no more.
     bool dead = false;
+    int cbuf = 0;  // this warp's C staging buffer for the next TMA store
     for (int it = 0; it < L; ++it) {
       const int b = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
       const int m0 = tile_m0(it);
       const int n0 = tile_n0(it);
-      const int t = m0 + static_cast<int>(rank) * HM + row;
+      const int trow0 = m0 + static_cast<int>(rank) * HM + q * 32;  // the warp's first row
+      const int t = trow0 + lane;
       const bool row_ok = t < a.T;
       float* ws = colbuf + b * (2 * TN);
       float* bs = ws + TN;
@@ -545,26 +601,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               for (int j = 0; j < 32; ++j)
                 if (c0 + j < a.N) arow[c0 + j] = static_cast<int32_t>(r[j]);
             }
-          } else {
+          } else if (!a.c_tma) {
             float v[32];
-            const float* wsc = ws + c * 32;
-            const float* bsc = bs + c * 32;
-            if (OC > 0) {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = fmaf(__uint_as_float(r[j]), wsc[j], bsc[j]);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                v[j] = fmaf(acc_value<kE4M3>(r[j]) * sx, wsc[j], bsc[j]);
-            }
+            epilogue_values<kE4M3>(r, OC, sx, ws + c * 32, ws + TN + c * 32, v);
             store_row32_f16(a.C + static_cast<int64_t>(t) * a.N, c0, a.N, v, vec_ok);
           }
+        }
+        if (!kRaw && a.c_tma && c0 < a.N && trow0 < a.T) {
+          // the warp's 32 rows x 32 columns in fp16 through shared memory, one TMA store
+          // (rows past T and columns past N are clipped by the tensor map)
+          float v[32];
+          epilogue_values<kE4M3>(r, OC, sx, ws + c * 32, ws + TN + c * 32, v);
+          const uint32_t sb = cstage + static_cast<uint32_t>((q * 2 + cbuf) * 2048);
+          if (lane == 0) bulk_wait_read_1();  // the store that last read this buffer is done
+          __syncwarp();
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            __half2 h0 = __floats2half2_rn(v[8 * q4 + 0], v[8 * q4 + 1]);
+            __half2 h1 = __floats2half2_rn(v[8 * q4 + 2], v[8 * q4 + 3]);
+            __half2 h2 = __floats2half2_rn(v[8 * q4 + 4], v[8 * q4 + 5]);
+            __half2 h3 = __floats2half2_rn(v[8 * q4 + 6], v[8 * q4 + 7]);
+            sts_v4(sb + static_cast<uint32_t>(lane * 64 + q4 * 16),
+                   *reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
+                   *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmC, sb, c0, trow0);
+            bulk_commit();
+          }
+          cbuf ^= 1;
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(map_to_rank(smem_u32(&bars->tmem_empty[b]), 0));
     }
+    // the shared-memory reads and global writes of this warp's TMA stores are complete
+    // before the CTA can exit
+    if (lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
