@@ -506,4 +506,16 @@ def pin_e4m3_error_bound_against_unquantised_product():
     assert (contrib > 3 * bound).mean() > 0.5
 
 
+
+def pin_e4m3_row_subset_matches_full():
+    """The e4m3 forward on a row subset gives exactly the same rows as on all rows (the
+    mask and row scales still come from every row, and each selected row keeps its own
+    scale)."""
+    X, W, b, CB, SCB, r = _linear_case_e4m3(12, 64, 6, 29, (3,), 6.0)
+    rows = np.array([11, 0, 5])
+    rs = O.linear_forward_e4m3(X, CB, SCB, b, 6.0, rows=rows)
+    assert np.array_equal(rs["SCx"], r["SCx"])
+    assert np.array_equal(rs["acc"], r["acc"][rows])
+    assert np.array_equal(rs["C"], r["C"][rows])
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

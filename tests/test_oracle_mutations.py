@@ -48,6 +48,64 @@ MUTATIONS = [
      "out_part += 0.0;\n"
      "            }\n            double b = bias ? (double)oracle_half_to_float(bias[n]) : 0.0;\n"
      "            C[i * N + n] = main_part"),
+    ("e4m3_subnormal_binade", "    if (E < -6)\n        E = -6;", "    if (E < -7)\n        E = -7;"),
+    ("e4m3_decode_subnormal", "v = ldexp((double)m, -9);", "v = ldexp((double)m, -10);"),
+    ("e4m3_saturate_below_448", "    if (a >= 448.0)\n        return sign | 0x7E;",
+     "    if (a >= 416.0)\n        return sign | 0x7E;"),
+    ("e4m3_outlier_codes_kept",
+     "            if (skip && skip[k]) {\n                qr[k] = 0;\n                continue;\n"
+     "            }\n            float v = oracle_half_to_float(row[k]) * s;\n            qr[k]",
+     "            float v = oracle_half_to_float(row[k]) * s;\n            qr[k]"),
+    ("e4m3_act_scale_row_index", "main_part = acc[i * N + n] * (double)SCx[t]",
+     "main_part = acc[i * N + n] * (double)SCx[i]"),
+    # scan, index list and half decode
+    ("idx_descending",
+     "    for (int64_t k = 0; k < K; ++k)\n        if (is_outlier[k])\n            idx[count++]",
+     "    for (int64_t k = K - 1; k >= 0; --k)\n        if (is_outlier[k])\n            idx[count++]"),
+    ("scan_first_row_only",
+     "    for (int64_t t = 0; t < T; ++t)\n        for (int64_t k = 0; k < K; ++k)\n"
+     "            if (fabsf",
+     "    for (int64_t t = 0; t < 1; ++t)\n        for (int64_t k = 0; k < K; ++k)\n"
+     "            if (fabsf"),
+    ("scan_signed", "if (fabsf(oracle_half_to_float(X[t * K + k])) >= threshold)",
+     "if (oracle_half_to_float(X[t * K + k]) >= threshold)"),
+    ("half_exponent_bias_14", "v = ldexpf((float)(f + 1024), e - 25);",
+     "v = ldexpf((float)(f + 1024), e - 24);"),
+    # int8 quantiser
+    ("outlier_codes_kept",
+     "            if (skip && skip[k]) {\n                qr[k] = 0;\n                continue;\n"
+     "            }\n            float v = oracle_half_to_float(row[k]) * s;\n            float c",
+     "            float v = oracle_half_to_float(row[k]) * s;\n            float c"),
+    ("weight_absmax_half_row",
+     "        for (int64_t k = 0; k < K; ++k) {\n            if (skip && skip[k])\n"
+     "                continue;\n            float a = fabsf(oracle_half_to_float(row[k]));\n"
+     "            if (a > amax)\n                amax = a;\n        }\n"
+     "        scale[r] = amax;\n        int8_t",
+     "        for (int64_t k = 0; k < (skip ? K : K / 2); ++k) {\n            if (skip && skip[k])\n"
+     "                continue;\n            float a = fabsf(oracle_half_to_float(row[k]));\n"
+     "            if (a > amax)\n                amax = a;\n        }\n"
+     "        scale[r] = amax;\n        int8_t"),
+    ("clamp_126", "if (c > 127.0f) c = 127.0f;", "if (c > 126.0f) c = 126.0f;"),
+    # product and output
+    ("matmul_drops_last_k",
+     "            for (int64_t k = 0; k < K; ++k)\n                s += (int64_t)a[k] * (int64_t)b[k];",
+     "            for (int64_t k = 0; k + 1 < K; ++k)\n                s += (int64_t)a[k] * (int64_t)b[k];"),
+    ("act_scale_row_index", "(double)acc[i * N + n] * (double)SCx[t] * (double)SCB[n]",
+     "(double)acc[i * N + n] * (double)SCx[i] * (double)SCB[n]"),
+    ("outlier_part_wrong_column",
+     "out_part += (double)oracle_half_to_float(X[t * K + k]) * w;\n            }\n"
+     "            double b = bias ? (double)oracle_half_to_float(bias[n]) : 0.0;\n"
+     "            C[i * N + n] = int_part",
+     "out_part += (double)oracle_half_to_float(X[t * K + j]) * w;\n            }\n"
+     "            double b = bias ? (double)oracle_half_to_float(bias[n]) : 0.0;\n"
+     "            C[i * N + n] = int_part"),
+    ("dequant_single_127", "                              / (127.0 * 127.0);",
+     "                              / (127.0);"),
+    ("bias_index_row",
+     "double b = bias ? (double)oracle_half_to_float(bias[n]) : 0.0;\n"
+     "            C[i * N + n] = int_part",
+     "double b = bias ? (double)oracle_half_to_float(bias[i % N]) : 0.0;\n"
+     "            C[i * N + n] = int_part"),
 ]
 
 
