@@ -84,7 +84,73 @@ def _ptr(t) -> Optional[int]:
         raise ValueError("expected a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError("expected a contiguous tensor")
+    import torch
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError("tensor on %s, but the current device is cuda:%d: the call would "
+                         "launch there (use torch.cuda.device)"
+                         % (t.device, torch.cuda.current_device()))
     return t.data_ptr()
+
+
+# The C calls take bare pointers, and most buffers have no size argument: the library
+# trusts that X is [T, K], C is [T, N], and so on.  These checks hold every tensor to the
+# dtype and the element count that its header comment states, so that a wrong or short
+# buffer raises here instead of being read or written out of bounds on the device.
+def _dt(*names):
+    import torch
+    return tuple(getattr(torch, n) for n in names)
+
+
+def _arg(t, name, dtypes, elems):
+    if t is None:
+        raise ValueError("%s: a tensor is required" % name)
+    if t.dtype not in dtypes:
+        raise TypeError("%s: dtype %s, expected %s"
+                        % (name, t.dtype, " or ".join(str(d) for d in dtypes)))
+    if t.numel() < elems:
+        raise ValueError("%s: %d elements, the call needs at least %d"
+                         % (name, t.numel(), elems))
+
+
+def _mat(t, name, dtypes):
+    """A 2-D operand: checks its dtype and returns its shape."""
+    if t is None or t.dim() != 2:
+        raise ValueError("%s: a 2-D tensor is required" % name)
+    _arg(t, name, dtypes, 0)
+    return t.shape
+
+
+def _slice_elems(rows, K):
+    # host copy of i8_outlier_slice_elems: ceil(K/64) chunks of rows x 64 fp16
+    return (K + 63) // 64 * rows * 64
+
+
+def _check_weight(CB, SCB, K, codes):
+    N, Kc = _mat(CB, "CB", codes)
+    if Kc != K:
+        raise ValueError("CB has %d columns, X has %d" % (Kc, K))
+    _arg(SCB, "SCB", _dt("float32"), N)
+    return N
+
+
+def _check_forward(X, CB, SCB, bias, C, codes):
+    T, K = _mat(X, "X", _dt("float16"))
+    N = _check_weight(CB, SCB, K, codes)
+    if bias is not None:
+        _arg(bias, "bias", _dt("float16"), N)
+    _arg(C, "C", _dt("float16"), T * N)
+    return T, K, N
+
+
+def _check_act_outputs(T, K, col_mask, mask_words, outlier_idx, n_outliers, Xq, SCx, X_o,
+                       codes):
+    w32 = _dt("int32", "uint32")
+    _arg(col_mask, "col_mask", w32, mask_words)
+    _arg(outlier_idx, "outlier_idx", w32, K)
+    _arg(n_outliers, "n_outliers", w32, 1)
+    _arg(Xq, "Xq", codes, T * K)
+    _arg(SCx, "SCx", _dt("float32"), T)
+    _arg(X_o, "X_o", _dt("float16"), _slice_elems(T, K))
 
 
 def _stream(stream):
@@ -96,13 +162,19 @@ def _stream(stream):
 
 # ----------------------------------------------------------------- the C calls
 def i8_quantize_weight(W, CB, SCB, stream=None):
-    N, K = W.shape
+    N, K = _mat(W, "W", _dt("float16"))
+    _arg(CB, "CB", _dt("int8"), N * K)
+    _arg(SCB, "SCB", _dt("float32"), N)
     _check("i8_quantize_weight",
            load().i8_quantize_weight(_ptr(W), N, K, _ptr(CB), _ptr(SCB), _stream(stream)))
 
 
 def i8_outlier_scan(X, threshold, col_mask, outlier_idx, n_outliers, stream=None):
-    T, K = X.shape
+    T, K = _mat(X, "X", _dt("float16"))
+    w32 = _dt("int32", "uint32")
+    _arg(col_mask, "col_mask", w32, (K + 31) // 32)
+    _arg(outlier_idx, "outlier_idx", w32, K)
+    _arg(n_outliers, "n_outliers", w32, 1)
     _check("i8_outlier_scan",
            load().i8_outlier_scan(_ptr(X), T, K, float(threshold), _ptr(col_mask),
                                   _ptr(outlier_idx), _ptr(n_outliers), _stream(stream)))
@@ -113,7 +185,9 @@ def i8_outlier_slice_elems(rows, K) -> int:
 
 
 def i8_quantize_act(X, col_mask, outlier_idx, n_outliers, Xq, SCx, X_o, stream=None):
-    T, K = X.shape
+    T, K = _mat(X, "X", _dt("float16"))
+    _check_act_outputs(T, K, col_mask, (K + 31) // 32, outlier_idx, n_outliers, Xq, SCx, X_o,
+                       _dt("int8"))
     _check("i8_quantize_act",
            load().i8_quantize_act(_ptr(X), T, K, _ptr(col_mask), _ptr(outlier_idx),
                                   _ptr(n_outliers), _ptr(Xq), _ptr(SCx), _ptr(X_o),
@@ -122,7 +196,9 @@ def i8_quantize_act(X, col_mask, outlier_idx, n_outliers, Xq, SCx, X_o, stream=N
 
 def i8_prepare_act(X, threshold, col_mask, outlier_idx, n_outliers, Xq, SCx, X_o, stream=None):
     """col_mask needs ceil(K/32) + 1 words (the last is scratch)."""
-    T, K = X.shape
+    T, K = _mat(X, "X", _dt("float16"))
+    _check_act_outputs(T, K, col_mask, (K + 31) // 32 + 1, outlier_idx, n_outliers, Xq, SCx,
+                       X_o, _dt("int8"))
     _check("i8_prepare_act",
            load().i8_prepare_act(_ptr(X), T, K, float(threshold), _ptr(col_mask),
                                  _ptr(outlier_idx), _ptr(n_outliers), _ptr(Xq), _ptr(SCx),
@@ -134,8 +210,7 @@ def i8_linear_workspace_size(T, N, K) -> int:
 
 
 def i8_linear_forward(X, CB, SCB, bias, threshold, C, workspace, stream=None):
-    T, K = X.shape
-    N = CB.shape[0]
+    T, K, N = _check_forward(X, CB, SCB, bias, C, _dt("int8"))
     _check("i8_linear_forward",
            load().i8_linear_forward(_ptr(X), T, K, _ptr(CB), _ptr(SCB), _ptr(bias), N,
                                     float(threshold), _ptr(C), _ptr(workspace),
@@ -145,8 +220,7 @@ def i8_linear_forward(X, CB, SCB, bias, threshold, C, workspace, stream=None):
 
 def i8_linear_forward_noalloc(X, CB, SCB, bias, threshold, C, stream=None):
     """i8_linear_forward with the library's fixed 32 MiB device scratch (no workspace)."""
-    T, K = X.shape
-    N = CB.shape[0]
+    T, K, N = _check_forward(X, CB, SCB, bias, C, _dt("int8"))
     _check("i8_linear_forward_noalloc",
            load().i8_linear_forward_noalloc(_ptr(X), T, K, _ptr(CB), _ptr(SCB), _ptr(bias), N,
                                             float(threshold), _ptr(C), _stream(stream)))
@@ -154,14 +228,18 @@ def i8_linear_forward_noalloc(X, CB, SCB, bias, threshold, C, stream=None):
 
 def i8_quantize_weight_e4m3(W, CB, SCB, stream=None):
     """e4m3 variant of i8_quantize_weight: CB is a uint8 [N, K] tensor of e4m3 codes."""
-    N, K = W.shape
+    N, K = _mat(W, "W", _dt("float16"))
+    _arg(CB, "CB", _dt("uint8", "float8_e4m3fn"), N * K)
+    _arg(SCB, "SCB", _dt("float32"), N)
     _check("i8_quantize_weight_e4m3",
            load().i8_quantize_weight_e4m3(_ptr(W), N, K, _ptr(CB), _ptr(SCB), _stream(stream)))
 
 
 def i8_prepare_act_e4m3(X, threshold, col_mask, outlier_idx, n_outliers, Xq, SCx, X_o,
                         stream=None):
-    T, K = X.shape
+    T, K = _mat(X, "X", _dt("float16"))
+    _check_act_outputs(T, K, col_mask, (K + 31) // 32 + 1, outlier_idx, n_outliers, Xq, SCx,
+                       X_o, _dt("uint8", "float8_e4m3fn"))
     _check("i8_prepare_act_e4m3",
            load().i8_prepare_act_e4m3(_ptr(X), T, K, float(threshold), _ptr(col_mask),
                                       _ptr(outlier_idx), _ptr(n_outliers), _ptr(Xq), _ptr(SCx),
@@ -173,8 +251,7 @@ def i8_linear_workspace_size_e4m3(T, N, K) -> int:
 
 
 def i8_linear_forward_e4m3(X, CB, SCB, bias, threshold, C, workspace, stream=None):
-    T, K = X.shape
-    N = CB.shape[0]
+    T, K, N = _check_forward(X, CB, SCB, bias, C, _dt("uint8", "float8_e4m3fn"))
     _check("i8_linear_forward_e4m3",
            load().i8_linear_forward_e4m3(_ptr(X), T, K, _ptr(CB), _ptr(SCB), _ptr(bias), N,
                                          float(threshold), _ptr(C), _ptr(workspace),
@@ -194,8 +271,7 @@ def i8_outlier_cache_reset(cache, stream=None):
 
 def i8_linear_forward_cached(X, CB, SCB, bias, threshold, C, workspace, cache, stream=None):
     """i8_linear_forward keeping the weight's outlier-column codes in `cache` across calls."""
-    T, K = X.shape
-    N = CB.shape[0]
+    T, K, N = _check_forward(X, CB, SCB, bias, C, _dt("int8"))
     _check("i8_linear_forward_cached",
            load().i8_linear_forward_cached(_ptr(X), T, K, _ptr(CB), _ptr(SCB), _ptr(bias), N,
                                            float(threshold), _ptr(C), _ptr(workspace),
@@ -205,8 +281,11 @@ def i8_linear_forward_cached(X, CB, SCB, bias, threshold, C, workspace, cache, s
 
 
 def i8_igemm_s32(A, B, acc, workspace, stream=None):
-    T, K = A.shape
-    N = B.shape[0]
+    T, K = _mat(A, "A", _dt("int8"))
+    N, Kb = _mat(B, "B", _dt("int8"))
+    if Kb != K:
+        raise ValueError("B has %d columns, A has %d" % (Kb, K))
+    _arg(acc, "acc", _dt("int32"), T * N)
     _check("i8_igemm_s32",
            load().i8_igemm_s32(_ptr(A), T, K, _ptr(B), N, _ptr(acc), _ptr(workspace),
                                workspace.numel() * workspace.element_size(), _stream(stream)))

@@ -158,10 +158,11 @@ class Linear8bitLt(torch.nn.Module):
         return self
 
     def _quantize(self, weight16: torch.Tensor):
-        if self.code_format == "e4m3":
-            abi.i8_quantize_weight_e4m3(weight16, self.CB, self.SCB)
-        else:
-            abi.i8_quantize_weight(weight16, self.CB, self.SCB)
+        with torch.cuda.device(self.CB.device):   # the library launches on the current device
+            if self.code_format == "e4m3":
+                abi.i8_quantize_weight_e4m3(weight16, self.CB, self.SCB)
+            else:
+                abi.i8_quantize_weight(weight16, self.CB, self.SCB)
 
     def dequantized_weight(self) -> torch.Tensor:
         """The weight the layer computes with (fp32): CB * SCB / 127, or for e4m3 codes
@@ -185,7 +186,8 @@ class Linear8bitLt(torch.nn.Module):
     def invalidate_outlier_cache(self):
         """Empty the outlier cache (needed after CB changed in place)."""
         for c in self._ocache.values():
-            abi.i8_outlier_cache_reset(c)
+            with torch.cuda.device(c.device):
+                abi.i8_outlier_cache_reset(c)
 
     def _outlier_cache(self) -> torch.Tensor:
         dev = self.CB.device
@@ -194,7 +196,8 @@ class Linear8bitLt(torch.nn.Module):
             need = abi.i8_outlier_cache_size(self.out_features, self.in_features,
                                              self.outlier_cache_cols)
             c = torch.empty((need,), dtype=torch.uint8, device=dev)
-            abi.i8_outlier_cache_reset(c)
+            with torch.cuda.device(dev):
+                abi.i8_outlier_cache_reset(c)
             self._ocache[dev] = c
         return c
 
@@ -207,17 +210,22 @@ class Linear8bitLt(torch.nn.Module):
         T = x2.shape[0]
         out = torch.empty((T, self.out_features), dtype=torch.float16, device=x2.device)
         if T > 0:
-            bias = None if self.bias is None else self.bias.detach()
-            if self.code_format == "e4m3":
-                abi.i8_linear_forward_e4m3(x2, self.CB, self.SCB, bias, self.threshold, out,
-                                           self._workspace(T))
-            elif self.outlier_cache_cols > 0:
-                abi.i8_linear_forward_cached(x2, self.CB, self.SCB, bias, self.threshold, out,
-                                             self._workspace(T), self._outlier_cache())
-            else:
-                abi.i8_linear_forward(x2, self.CB, self.SCB, bias, self.threshold, out,
-                                      self._workspace(T))
+            with torch.cuda.device(self.CB.device):
+                self._launch_forward(x2, out)
         return out
+
+    def _launch_forward(self, x2: torch.Tensor, out: torch.Tensor):
+        T = x2.shape[0]
+        bias = None if self.bias is None else self.bias.detach()
+        if self.code_format == "e4m3":
+            abi.i8_linear_forward_e4m3(x2, self.CB, self.SCB, bias, self.threshold, out,
+                                       self._workspace(T))
+        elif self.outlier_cache_cols > 0:
+            abi.i8_linear_forward_cached(x2, self.CB, self.SCB, bias, self.threshold, out,
+                                         self._workspace(T), self._outlier_cache())
+        else:
+            abi.i8_linear_forward(x2, self.CB, self.SCB, bias, self.threshold, out,
+                                  self._workspace(T))
 
     def forward(self, x: torch.Tensor) -> torch.Tensor:
         if x.dtype != torch.float16:
@@ -225,6 +233,8 @@ class Linear8bitLt(torch.nn.Module):
         if x.shape[-1] != self.in_features:
             raise ValueError("last input dimension %d, expected %d"
                              % (x.shape[-1], self.in_features))
+        if x.device != self.CB.device:
+            raise ValueError("input on %s, layer on %s" % (x.device, self.CB.device))
         lead = x.shape[:-1]
         x2 = x.reshape(-1, self.in_features).contiguous()
         if self.has_fp16_weights:
