@@ -101,3 +101,23 @@ def test_l2_policy_flushes_only_inputs_that_fit_twice_in_l2():
     no, desc = bench.l2_policy("auto", 16, 57344, 14336)             # CB 822 MB
     assert not no and "no flush" in desc
     assert bench.l2_policy("always", 16, 57344, 14336)[0]
+
+
+def test_work_counts_split_the_product_at_the_outlier_columns():
+    T, N, K = 2048, 16384, 4096
+    i8, f16, eff, nbytes = bench.work_counts(T, N, K, 0)
+    assert i8 == eff == 2.0 * T * N * K and f16 == 0.0
+    i8, f16, eff, _ = bench.work_counts(T, N, K, 6)
+    assert i8 + f16 == eff and f16 == 2.0 * T * N * 6
+    # the bytes include at least CB once, X once and C once
+    assert nbytes >= N * K + 2 * T * K + 2 * T * N
+
+
+def test_traffic_is_reported_only_for_the_sources_it_was_measured_on(monkeypatch):
+    rec = bench.traffic_record("i8_gemm_tcgen05_kernel", "opt6.7b_ffn_up_prefill_2048x4096x16384")
+    if rec is not None:   # the committed capture matches the current CUDA sources
+        assert rec["dram_bytes_per_launch"] > 0
+    monkeypatch.setattr(bench, "source_hash", lambda: "0" * 64)
+    assert bench.traffic_record("i8_gemm_tcgen05_kernel",
+                                "opt6.7b_ffn_up_prefill_2048x4096x16384") is None
+    assert bench.traffic_record("decode_kernel", "no_such_workload") is None
