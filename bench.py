@@ -14,7 +14,10 @@ launching stream, with a 256 MiB buffer written between steps (outside the event
 flush the 126 MB L2 when the step's inputs (X and CB) are smaller than twice the L2 --
 larger inputs stream from HBM every step anyway, and the config line says which was
 done; barrier + synchronize around the loop; value = total effective
-ops of all ranks / the slowest rank's summed step time.  Multi-GPU: one process per GPU
+ops of all ranks / the slowest rank's summed step time.  "e2e" is the same metric through
+the public call with host buffers: each step uploads X from pinned host memory and reads
+the whole C back, with the copies on two streams of their own overlapping the forward
+(two buffer slots); the read-backs are checked bit for bit.  Multi-GPU: one process per GPU
 (torchrun), each rank owns a disjoint block of output channels of a layer N*world wide
 (column-parallel, no collective on the data path): weak scaling.
 
