@@ -159,3 +159,32 @@ def test_e4m3_calls_reject_bad_arguments_without_cuda(lib):
     assert lib.i8_quantize_weight_e4m3(None, 64, 64, FAKE, FAKE, None) == INVALID
     assert lib.i8_prepare_act_e4m3(FAKE, 4, 64, 6.0, FAKE, FAKE, FAKE, None, FAKE, FAKE,
                                    None) == INVALID
+
+
+def test_header_serves_a_plain_c_caller(lib, tmp_path):
+    """The boundary is a C ABI: a C99 program (no C++, no CUDA headers) includes
+    i8linear.h with every warning on, links against the library and calls it; the call
+    with NULL pointers is refused before any CUDA work, so this runs without a GPU."""
+    src = tmp_path / "caller.c"
+    src.write_text(
+        '#include "i8linear.h"\n'
+        "#include <stdio.h>\n"
+        "int main(void) {\n"
+        "    size_t ws = i8_linear_workspace_size(2048, 16384, 4096);\n"
+        "    i8_status s = i8_linear_forward(NULL, 4, 64, NULL, NULL, NULL, 8, 6.0f, NULL,\n"
+        "                                    NULL, 0, NULL);\n"
+        '    printf("%zu %s\\n", ws, i8_status_string(s));\n'
+        "    return (s == I8_ERR_INVALID_ARG && ws > 0) ? 0 : 1;\n"
+        "}\n", encoding="utf-8")
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(abi.LIB_PATH)
+    import subprocess
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                           "-I", os.path.join(ROOT, "include"), str(src),
+                           "-L", libdir, "-l:libi8linear.so", "-Wl,-rpath," + libdir,
+                           "-o", str(exe)])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stdout + out.stderr
+    ws, name = out.stdout.split()
+    assert int(ws) == lib.i8_linear_workspace_size(2048, 16384, 4096)
+    assert name == "I8_ERR_INVALID_ARG"
