@@ -325,7 +325,6 @@ class Linear8bit:
         self.bias = bias
         i8_quantize_weight(W, self.CB, self.SCB, stream)
         self._ws = None
-        self._ws_T = -1
 
     def workspace(self, T):
         import torch
