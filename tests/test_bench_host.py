@@ -121,3 +121,13 @@ def test_traffic_is_reported_only_for_the_sources_it_was_measured_on(monkeypatch
     assert bench.traffic_record("i8_gemm_tcgen05_kernel",
                                 "opt6.7b_ffn_up_prefill_2048x4096x16384") is None
     assert bench.traffic_record("decode_kernel", "no_such_workload") is None
+
+
+def test_tensor_peak_follows_the_power_cap_seen_while_timing():
+    pk = dict(hbm=6459.3, bf16=1679.9, bf16_sus=1418.9, source="measured")
+    burst, why = bench.tensor_peak(pk, {"sm_mhz": 1965.0, "reasons": []})
+    assert burst == 2 * 1679.9 and "burst" in why
+    capped, why = bench.tensor_peak(pk, {"sm_mhz": 1380.0, "reasons": ["sw_power_cap"]})
+    assert capped == 2 * 1418.9 and "sustained" in why
+    unknown, why = bench.tensor_peak(pk, None, e4m3=True)
+    assert unknown == 2 * 1679.9 and "fp8" in why and "no clock record" in why
