@@ -6,20 +6,32 @@ A step is one i8_linear_forward over one batch (outlier scan, activation quantis
 int8 tcgen05 GEMM with the fused fp16 outlier product, dequantisation and bias).  The
 weight is quantised once before timing (i8_quantize_weight; timed separately and reported
 under "weight_quant").  Inputs are synthetic (numpy PCG64, see synth.py) with the shape of
-the named workload; the default is the OPT-6.7B FFN up-projection prefill,
-X [2048, 4096] x W [16384, 4096] with 6 fixed outlier columns.
+the named workload; the default, and the line's headline, is the OPT-175B-shaped layer,
+X [8192, 12288] x W [49152, 12288] with 8 planted outlier columns at threshold 6 (the
+largest of the layer shapes, and the one the outlier-density sweep is quoted on).
 
 Timing: W untimed warm-up steps; then K timed steps, each bracketed by CUDA events on the
 launching stream, with a 256 MiB buffer written between steps (outside the events) to
 flush the 126 MB L2 when the step's inputs (X and CB) are smaller than twice the L2 --
 larger inputs stream from HBM every step anyway, and the config line says which was
-done; barrier + synchronize around the loop; value = total effective
-ops of all ranks / the slowest rank's summed step time.  "e2e" is the same metric through
-the public call with host buffers: each step uploads X from pinned host memory and reads
-the whole C back, with the copies on two streams of their own overlapping the forward
-(two buffer slots); the read-backs are checked bit for bit.  Multi-GPU: one process per GPU
-(torchrun), each rank owns a disjoint block of output channels of a layer N*world wide
-(column-parallel, no collective on the data path): weak scaling.
+done; barrier + synchronize around the loop; value = total effective ops of all ranks /
+the slowest rank's summed step time.  A second loop of the same steps records events
+around the dominant kernel alone (the "roofline" record).  "e2e" is the same metric
+through the public call with host buffers: each step uploads X from pinned host memory
+and reads the whole C back, with the copies on two streams of their own overlapping the
+forward (two buffer slots); the read-backs are checked bit for bit.
+
+At one GPU, with the default workload, the same run also measures the rest of the layer
+shapes (unless --no-extras): "sweep" holds the OPT-175B outlier-density sweep (planted
+columns {0, 8, 64, 256} x threshold {6, +inf}) and "per_config" the BLOOM-176B FFN decode
+batches (T = 1, 8, 16; bound by HBM), the BLOOM-176B QKV prefill and the OPT-6.7B FFN-up
+prefill, each with its step time, effective TOPS and dominant-kernel roofline fraction.
+
+Multi-GPU: one process per GPU (torchrun).  At N GPUs the layer is N times as wide (N x
+49152 output channels by default) and rank r holds output channels [r*N0, (r+1)*N0) of
+that one layer -- its own rows of the one weight, scales and bias -- with the hidden
+states replicated: every rank computes the same outlier mask and row scales and writes its
+own columns of C, with no collective on the data path (weak scaling).
 
 --impl reference times the CPU oracle (oracle/, plain C) on this host's cores on the
 same workload, each step a bounded row sample, and prints the same line with
@@ -43,8 +55,15 @@ sys.path.insert(0, ROOT)
 from bit_matmul_decomposition_b200 import synth  # noqa: E402
 
 METRIC = "int8 decomposed linear: effective TOPS & HBM GB/s, % of sm_100a roofline"
+DEFAULT_WORKLOAD = "opt175b_cols8_thr6"
 L2_FLUSH_BYTES = 256 << 20
 L2_BYTES = 126 * 1000 * 1000      # B200 L2 capacity (nominal)
+# int8 (and e4m3) dense tensor ops per SM per clock of tcgen05 (8192 multiply-adds), the
+# instruction rate ncu reports for the int8 pipe; x SMs x SM clock = the pipe's peak
+PIPE_OPS_PER_SM_CLK = 16384
+# NVIDIA's dense B200 figures, for context: int8 4.5 POPS, HBM3e 8 TB/s class
+DATASHEET_I8_TOPS = 4500.0
+DATASHEET_HBM_GBS = 8000.0
 
 
 def l2_policy(mode, T, N, K):
@@ -98,6 +117,18 @@ def tensor_peak(pk, clk, e4m3=False):
     return 2.0 * bf16, basis
 
 
+def json_threshold(t):
+    """A threshold for the JSON line: +inf as the string "inf" (JSON has no infinity)."""
+    return "inf" if math.isinf(t) else t
+
+
+def pipe_peak_tops(sms, sm_mhz):
+    """The tensor pipe's int8 instruction rate at the given SM clock (TOPS)."""
+    if not sms or not sm_mhz:
+        return None
+    return PIPE_OPS_PER_SM_CLK * sms * sm_mhz * 1e6 / 1e12
+
+
 def max_over_ranks(values, device=None):
     """Element-wise max of a list of floats over all ranks of the default process group
     (identity without one).  Used for every device time the line reports."""
@@ -109,13 +140,15 @@ def max_over_ranks(values, device=None):
     return [float(v) for v in t.cpu()]
 
 
-def rank_workload(w, rank):
-    """Weak scaling: rank r owns the r-th block of output channels (its own weight shard);
-    the hidden states are replicated."""
-    if rank == 0:
-        return w, w
+def rank_workload(w, rank, world):
+    """Weak scaling over one layer: with `world` GPUs the layer has world * N output
+    channels, and rank r holds rows synth.shard_rows(world * N, r, world) of its weight,
+    scales and bias (N of them).  Returns (layer, rows): the layer's workload and the rank's
+    [r0, r1).  The hidden states are the same on every rank."""
     import dataclasses
-    return w, dataclasses.replace(w, seed=w.seed * 1000 + rank)
+    layer = w if world == 1 else dataclasses.replace(
+        w, N=w.N * world, name="%s_x%d_wide" % (w.name, world))
+    return layer, synth.shard_rows(layer.N, rank, world)
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -203,7 +236,7 @@ def traffic_record(kernel, workload):
 
 def source_hash():
     h = hashlib.sha256()
-    for f in ("api.cu", "common.cuh", "quant.cuh", "gemm.cuh", "gemv.cuh"):
+    for f in ("api.cu", "common.cuh", "quant.cuh", "gemm.cuh", "gemv.cuh", "bwd.cuh"):
         with open(os.path.join(ROOT, "bit_matmul_decomposition_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
@@ -286,6 +319,214 @@ def run_reference(args, w):
 
 
 # ----------------------------------------------------------------------------- GPU arm
+class Layer:
+    """One workload's device tensors: X, CB/SCB (quantised here, timed), bias, C and the
+    forward's workspace."""
+
+    def __init__(self, abi, w, dev, rows=None, e4m3=False, X=None, CB=None, SCB=None):
+        import torch
+        self.w, self.dev, self.e4m3 = w, dev, e4m3
+        r0, r1 = (0, w.N) if rows is None else rows
+        self.T, self.K, self.N = w.T, w.K, r1 - r0
+        self.X_h = synth.make_x(w) if X is None else X
+        self.X = fp16_tensor(self.X_h, dev)
+        b = synth.make_bias(w, (r0, r1))
+        self.b = None if b is None else fp16_tensor(b, dev)
+        self.wq_ms = None
+        if CB is None:
+            W = fp16_tensor(synth.make_w(w, (r0, r1)), dev)
+            self.CB = torch.empty((self.N, self.K), dtype=torch.uint8 if e4m3 else torch.int8,
+                                  device=dev)
+            self.SCB = torch.empty((self.N,), dtype=torch.float32, device=dev)
+            quantize = abi.i8_quantize_weight_e4m3 if e4m3 else abi.i8_quantize_weight
+            quantize(W, self.CB, self.SCB)
+            torch.cuda.synchronize()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            reps = 5
+            ev[0].record()
+            for _ in range(reps):
+                quantize(W, self.CB, self.SCB)
+            ev[1].record()
+            torch.cuda.synchronize()
+            self.wq_ms = ev[0].elapsed_time(ev[1]) / reps
+            del W
+        else:
+            self.CB, self.SCB = CB, SCB
+        size = abi.i8_linear_workspace_size_e4m3 if e4m3 else abi.i8_linear_workspace_size
+        self.ws = torch.empty((size(self.T, self.N, self.K),), dtype=torch.uint8, device=dev)
+        self.C = torch.empty((self.T, self.N), dtype=torch.float16, device=dev)
+        # outlier count of this input (the scan's device scalar), for the work accounting
+        mask = torch.empty(((self.K + 31) // 32,), dtype=torch.int32, device=dev)
+        idx = torch.empty((self.K,), dtype=torch.int32, device=dev)
+        n_o = torch.empty((4,), dtype=torch.int32, device=dev)
+        abi.i8_outlier_scan(self.X, w.threshold, mask, idx, n_o)
+        self.n_o = int(n_o[0].item())
+
+    def weight_quant(self, pk):
+        if self.wq_ms is None:
+            return None
+        gbs = 3.0 * self.N * self.K / (self.wq_ms * 1e-3) / 1e9
+        return {"ms": self.wq_ms, "gbs": gbs, "frac_hbm": gbs / pk["hbm"],
+                "frac_of_datasheet_hbm": gbs / DATASHEET_HBM_GBS,
+                "bytes": 3 * self.N * self.K + 4 * self.N}
+
+
+def time_forward(abi, forward, steps, warmup, flush_l2, stream, uuid, barrier=lambda: None):
+    """Region 1: `steps` whole steps, each bracketed by events (clocks sampled meanwhile).
+    Region 2: the same steps with events around the dominant kernel alone.  Returns
+    (summed step ms, summed kernel ms, clock record)."""
+    import torch
+    for _ in range(warmup):
+        flush_l2()
+        forward()
+    st = abi.i8_sync_status()
+    if st != 0:
+        raise RuntimeError("device error during warm-up: %s" % abi.STATUS.get(st, st))
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    kv_s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    kv_e = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for e in kv_s + kv_e:          # torch creates the CUDA event on its first record
+        e.record(stream)
+    clocks = ClockSampler(uuid)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(steps):
+        flush_l2()
+        ev_s[i].record(stream)
+        forward()
+        ev_e[i].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    st = abi.i8_sync_status()
+    if st != 0:
+        raise RuntimeError("device error in the timed loop: %s" % abi.STATUS.get(st, st))
+    # (recording events between kernels costs the launch overlap, so region 1 runs without)
+    for i in range(steps):
+        flush_l2()
+        abi.i8_set_profile_events(kv_s[i], kv_e[i])
+        forward()
+    abi.i8_set_profile_events(None, None)
+    torch.cuda.synchronize()
+    barrier()
+    st = abi.i8_sync_status()
+    if st != 0:
+        raise RuntimeError("device error in the kernel-timing loop: %s" % abi.STATUS.get(st, st))
+    step_ms = sum(ev_s[i].elapsed_time(ev_e[i]) for i in range(steps))
+    kern_ms = sum(kv_s[i].elapsed_time(kv_e[i]) for i in range(steps))
+    return step_ms, kern_ms, clk
+
+
+def roofline(L, kern_per, clk, pk, sms):
+    """The dominant kernel against its roofline: the decode kernel (the whole forward of a
+    decode batch, one stream of CB) against HBM bandwidth, else the tcgen05 GEMM against
+    the 8-bit tensor peak.  `peak` is the measured figure; the pipe instruction rate at the
+    sampled SM clock and the datasheet figure are given beside it."""
+    T, N, K, n_o = L.T, L.N, L.K, L.n_o
+    i8_ops, f16_flops, _, _ = work_counts(T, N, K, n_o)
+    if T <= 16 and not L.e4m3:
+        nbytes = N * K + 2 * T * K + 4 * N + (2 * N if L.b is not None else 0) + 2 * T * N
+        achieved = nbytes / (kern_per * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                "frac": achieved / pk["hbm"], "kernel": "decode_kernel",
+                "peak_basis": "%s HBM copy bandwidth" % pk["source"],
+                "frac_of_datasheet_peak": achieved / DATASHEET_HBM_GBS,
+                "algorithmic_bytes_per_launch": nbytes, "kernel_ms": kern_per}
+    # int8 (or e4m3) ops plus the fp16 flops counted at the 8-bit rate x 2 (the nominal
+    # fp16 : int8 : fp8 dense rates are 1 : 2 : 2)
+    equiv = i8_ops + 2.0 * f16_flops
+    achieved = equiv / (kern_per * 1e-3) / 1e12
+    peak_i8, basis = tensor_peak(pk, clk, L.e4m3)
+    mhz = clk.get("sm_mhz") if clk else None
+    pipe = pipe_peak_tops(sms, mhz)
+    return {"bound": "tensor", "achieved": achieved, "peak": peak_i8, "unit": "TOPS",
+            "frac": achieved / peak_i8, "kernel": "i8_gemm_tcgen05_kernel",
+            "peak_basis": basis,
+            "frac_of_burst_peak": achieved / (2.0 * pk["bf16"]),
+            "frac_of_sustained_peak": achieved / (2.0 * pk["bf16_sus"]),
+            "frac_of_pipe_peak": None if pipe is None else achieved / pipe,
+            "pipe_peak_basis": None if pipe is None else (
+                "%d ops/clk/SM x %d SMs x median %.0f MHz sampled in the timed loop = %.0f TOPS"
+                % (PIPE_OPS_PER_SM_CLK, sms, mhz, pipe)),
+            "frac_of_datasheet_peak": achieved / DATASHEET_I8_TOPS,
+            "algorithmic_ops_per_launch": equiv, "kernel_ms": kern_per}
+
+
+def measure_layer(abi, L, steps, warmup, l2_mode, stream, uuid, pk, sms, forward=None):
+    """Step time, effective TOPS and the dominant kernel's roofline of one layer."""
+    import torch
+    use_flush, l2_desc = l2_policy(l2_mode, L.T, L.N, L.K)
+    flush = torch.empty((L2_FLUSH_BYTES if use_flush else 16,), dtype=torch.uint8,
+                        device=L.dev)
+
+    def flush_l2():
+        if use_flush:
+            flush.zero_()
+
+    if forward is None:
+        def forward():
+            abi.i8_linear_forward(L.X, L.CB, L.SCB, L.b, L.w.threshold, L.C, L.ws)
+    step_ms, kern_ms, clk = time_forward(abi, forward, steps, warmup, flush_l2, stream, uuid)
+    ms = step_ms / steps
+    _, _, eff, nbytes = work_counts(L.T, L.N, L.K, L.n_o)
+    roof = roofline(L, kern_ms / steps, clk, pk, sms)
+    return {"workload": L.w.name, "T": L.T, "N": L.N, "K": L.K,
+            "threshold": json_threshold(L.w.threshold),
+            "n_outliers": L.n_o, "steps": steps, "ms_per_step": ms,
+            "effective_tops": eff / (ms * 1e-3) / 1e12,
+            "hbm_gbs": nbytes / (ms * 1e-3) / 1e9, "l2": l2_desc,
+            "roofline": {k: v for k, v in roof.items()
+                         if k not in ("pipe_peak_basis", "peak_basis")},
+            "clocks": None if clk is None else {"sm_mhz": clk["sm_mhz"],
+                                                "reasons": clk["reasons"]}}
+
+
+def run_extras(abi, head, dev, stream, uuid, pk, sms, steps):
+    """The other layer shapes, measured in the same run: the OPT-175B density sweep (same
+    weight as the headline) and the BLOOM decode / QKV and OPT-6.7B FFN-up layers."""
+    import torch
+    sweep = []
+    xs = {}
+    for c in (0, 8, 64, 256):
+        for thr in (6.0, math.inf):
+            w = synth.opt175b_sweep(c, thr)
+            if w.name == head.w.name:
+                continue
+            if c not in xs:      # the two thresholds share their hidden states
+                xs = {c: synth.make_x(w)}
+            L = Layer(abi, w, dev, X=xs[c], CB=head.CB, SCB=head.SCB)
+            sweep.append(measure_layer(abi, L, max(5, steps // 2), 3, "auto", stream, uuid,
+                                       pk, sms))
+            del L
+            torch.cuda.empty_cache()
+    per = {}
+    jobs = [("bloom_ffn_decode_T%d" % T, synth.bloom_ffn_decode(T), 100) for T in (1, 8, 16)]
+    jobs += [("bloom_qkv_prefill", synth.bloom_qkv_prefill(), max(5, steps // 2)),
+             ("opt6.7b_ffn_up_prefill", synth.opt_ffn_up_prefill(), 200)]
+    shared = None      # the three decode batches share one weight
+    for key, w, n in jobs:
+        if shared is not None and w.seed == shared.w.seed:
+            L = Layer(abi, w, dev, CB=shared.CB, SCB=shared.SCB)
+        else:
+            shared = None
+            torch.cuda.empty_cache()
+            L = Layer(abi, w, dev)
+        rec = measure_layer(abi, L, n, 5, "auto", stream, uuid, pk, sms)
+        wq = L.weight_quant(pk)
+        if wq is not None:
+            rec["weight_quant"] = wq
+        per[key] = rec
+        if w.T <= 16:
+            shared = L
+        del L
+    del shared
+    torch.cuda.empty_cache()
+    return sweep, per
+
+
 def run_gpu(args, w0):
     import torch
     import torch.distributed as dist
@@ -306,39 +547,15 @@ def run_gpu(args, w0):
         if world > 1:
             dist.barrier()
 
-    _, w = rank_workload(w0, rank)
-    X = synth.make_x(w0)                      # replicated hidden states
-    W = synth.make_w(w)
-    b = synth.make_bias(w)
-    T, K, N = w.T, w.K, w.N
+    layer, rows = rank_workload(w0, rank, world)
     abi.load()
     stream = torch.cuda.current_stream()
-
-    X_d, W_d = fp16_tensor(X, dev), fp16_tensor(W, dev)
-    b_d = None if b is None else fp16_tensor(b, dev)
+    sms = torch.cuda.get_device_properties(local).multi_processor_count
     e4m3 = args.format == "e4m3"
     if e4m3 and args.outlier_cache:
         raise SystemExit("--outlier-cache applies to the int8 forward only")
-    CB = torch.empty((N, K), dtype=torch.uint8 if e4m3 else torch.int8, device=dev)
-    quantize_weight = abi.i8_quantize_weight_e4m3 if e4m3 else abi.i8_quantize_weight
-    SCB = torch.empty((N,), dtype=torch.float32, device=dev)
-
-    # weight quantisation (once per weight): timed on its own
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    quantize_weight(W_d, CB, SCB)
-    torch.cuda.synchronize()
-    reps = 5
-    ev[0].record(stream)
-    for _ in range(reps):
-        quantize_weight(W_d, CB, SCB)
-    ev[1].record(stream)
-    torch.cuda.synchronize()
-    wq_ms = ev[0].elapsed_time(ev[1]) / reps
-    del W_d
-
-    ws_size = abi.i8_linear_workspace_size_e4m3 if e4m3 else abi.i8_linear_workspace_size
-    ws = torch.empty((ws_size(T, N, K),), dtype=torch.uint8, device=dev)
-    C = torch.empty((T, N), dtype=torch.float16, device=dev)
+    L = Layer(abi, layer, dev, rows=rows, e4m3=e4m3)
+    T, K, N = L.T, L.K, L.N
     use_flush, l2_desc = l2_policy(args.l2_flush, T, N, K)
     flush = torch.empty((L2_FLUSH_BYTES if use_flush else 16,), dtype=torch.uint8, device=dev)
 
@@ -353,78 +570,26 @@ def run_gpu(args, w0):
                             device=dev)
         abi.i8_outlier_cache_reset(cache)
 
-    def forward(X_in, C_out=C):
+    def forward(X_in, C_out):
         if e4m3:
-            abi.i8_linear_forward_e4m3(X_in, CB, SCB, b_d, w.threshold, C_out, ws)
+            abi.i8_linear_forward_e4m3(X_in, L.CB, L.SCB, L.b, layer.threshold, C_out, L.ws)
         elif cache is None:
-            abi.i8_linear_forward(X_in, CB, SCB, b_d, w.threshold, C_out, ws)
+            abi.i8_linear_forward(X_in, L.CB, L.SCB, L.b, layer.threshold, C_out, L.ws)
         else:
-            abi.i8_linear_forward_cached(X_in, CB, SCB, b_d, w.threshold, C_out, ws, cache)
+            abi.i8_linear_forward_cached(X_in, L.CB, L.SCB, L.b, layer.threshold, C_out, L.ws,
+                                         cache)
 
-    def step():
-        forward(X_d)
-
-    for _ in range(args.warmup):
-        flush_l2()
-        step()
-    st = abi.i8_sync_status()
-    if st != 0:
-        raise RuntimeError("device error during warm-up: %s" % abi.STATUS.get(st, st))
-    # outlier count of this input (the scan's device scalar), for the work accounting
-    mask = torch.empty(((K + 31) // 32,), dtype=torch.int32, device=dev)
-    idx = torch.empty((K,), dtype=torch.int32, device=dev)
-    n_o_d = torch.empty((4,), dtype=torch.int32, device=dev)
-    abi.i8_outlier_scan(X_d, w.threshold, mask, idx, n_o_d)
-    n_o = int(n_o_d[0].item())
-
-    K_steps = args.steps
-    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K_steps)]
-    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K_steps)]
-    kv_s = [torch.cuda.Event(enable_timing=True) for _ in range(K_steps)]
-    kv_e = [torch.cuda.Event(enable_timing=True) for _ in range(K_steps)]
     uuid = None
     try:
         uuid = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
     except Exception:
         pass
-    for e in kv_s + kv_e:          # torch creates the CUDA event on its first record
-        e.record(stream)
-    clocks = ClockSampler(uuid)
-    # timed region 1: K whole steps (each step bracketed by events; the L2 is flushed
-    # between steps, outside the events)
-    barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)
-    for i in range(K_steps):
-        flush_l2()
-        ev_s[i].record(stream)
-        step()
-        ev_e[i].record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    clk = clocks.stop()
-    st = abi.i8_sync_status()
-    if st != 0:
-        raise RuntimeError("device error in the timed loop: %s" % abi.STATUS.get(st, st))
-    # timed region 2: the same steps with events around the dominant kernel (recording
-    # them between kernels costs the launch overlap, so region 1 runs without them)
-    for i in range(K_steps):
-        flush_l2()
-        abi.i8_set_profile_events(kv_s[i], kv_e[i])
-        step()
-    abi.i8_set_profile_events(None, None)
-    torch.cuda.synchronize()
-    barrier()
-    st = abi.i8_sync_status()
-    if st != 0:
-        raise RuntimeError("device error in the kernel-timing loop: %s" % abi.STATUS.get(st, st))
-
-    step_ms = sum(ev_s[i].elapsed_time(ev_e[i]) for i in range(K_steps))
-    kern_ms = sum(kv_s[i].elapsed_time(kv_e[i]) for i in range(K_steps))
+    K_steps = args.steps
+    step_ms, kern_ms, clk = time_forward(abi, lambda: forward(L.X, L.C), K_steps, args.warmup,
+                                         flush_l2, stream, uuid, barrier)
     step_ms, kern_ms = max_over_ranks([step_ms, kern_ms], dev)
 
-    i8_ops, f16_flops, eff_ops, bytes_ = work_counts(T, N, K, n_o)
+    i8_ops, f16_flops, eff_ops, bytes_ = work_counts(T, N, K, L.n_o)
     ms_per_step = step_ms / K_steps
     value = world * eff_ops / (ms_per_step * 1e-3) / 1e12
     hbm_gbs = bytes_ / (ms_per_step * 1e-3) / 1e9
@@ -438,10 +603,11 @@ def run_gpu(args, w0):
     # asks for one, runs on the forward stream inside the timed region.
     e2e_steps = max(3, min(K_steps, 50))
     depth = 2
-    X_h = torch.from_numpy(np.ascontiguousarray(X).view(np.int16)).view(torch.float16).pin_memory()
+    X_h = torch.from_numpy(np.ascontiguousarray(L.X_h).view(np.int16)).view(
+        torch.float16).pin_memory()
     C_h = [torch.empty((T, N), dtype=torch.float16).pin_memory() for _ in range(depth)]
-    X_in = [torch.empty_like(X_d) for _ in range(depth)]
-    C_out = [torch.empty_like(C) for _ in range(depth)]
+    X_in = [torch.empty_like(L.X) for _ in range(depth)]
+    C_out = [torch.empty_like(L.C) for _ in range(depth)]
     up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     ev_up = [torch.cuda.Event() for _ in range(depth)]
     ev_fw = [torch.cuda.Event() for _ in range(depth)]
@@ -492,39 +658,18 @@ def run_gpu(args, w0):
     if st != 0:
         raise RuntimeError("device error in the e2e loop: %s" % abi.STATUS.get(st, st))
     # every read-back holds the forward's output (the forward is deterministic)
-    C_ref_bits = C.cpu().view(torch.int16)
+    C_ref_bits = L.C.cpu().view(torch.int16)
     for j in range(depth):
         if not torch.equal(C_h[j].view(torch.int16), C_ref_bits):
             raise RuntimeError("e2e read-back %d differs from the device-timed output" % j)
+    del C_h, X_in, C_out, X_h, C_ref_bits
     e2e_per = max_over_ranks([e2e_ms], dev)[0] / e2e_steps
     e2e_value = world * eff_ops / (e2e_per * 1e-3) / 1e12
 
     decode = T <= 16 and not e4m3   # (the e4m3 forward runs the GEMM for every T)
     pk = peaks()
-    kern_per = kern_ms / K_steps
-    if decode:
-        # the whole decode forward is one kernel streaming CB once: algorithmic bytes are
-        # CB, X, the scales, the bias and C
-        gemv_bytes = N * K + 2 * T * K + 4 * N + (2 * N if b is not None else 0) + 2 * T * N
-        achieved = gemv_bytes / (kern_per * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
-                "frac": achieved / pk["hbm"], "kernel": "decode_kernel",
-                "algorithmic_bytes_per_launch": gemv_bytes}
-        tr = traffic_record("decode_kernel", w0.name)
-    else:
-        # dominant kernel: the tcgen05 GEMM; int8 (or e4m3) ops plus fp16 flops counted at
-        # the 8-bit rate x 2 (the nominal fp16 : int8 : fp8 dense rates are 1 : 2 : 2)
-        equiv = i8_ops + 2.0 * f16_flops
-        achieved = equiv / (kern_per * 1e-3) / 1e12
-        peak_i8, basis = tensor_peak(pk, clk, e4m3)
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak_i8, "unit": "TOPS",
-                "frac": achieved / peak_i8, "kernel": "i8_gemm_tcgen05_kernel",
-                "peak_basis": basis,
-                "frac_of_burst_peak": achieved / (2.0 * pk["bf16"]),
-                "frac_of_sustained_peak": achieved / (2.0 * pk["bf16_sus"]),
-                "algorithmic_ops_per_launch": equiv}
-        tr = None if e4m3 else traffic_record("i8_gemm_tcgen05_kernel", w0.name)
-    roof["kernel_ms"] = kern_per
+    roof = roofline(L, kern_ms / K_steps, clk, pk, sms)
+    tr = traffic_record(roof["kernel"], w0.name) if not e4m3 else None
     roof["traffic"] = None if tr is None else tr["dram_bytes_per_launch"]
     if tr is not None:
         roof["traffic_note"] = tr.get("note", "")
@@ -533,9 +678,11 @@ def run_gpu(args, w0):
             "steps": K_steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3" if e4m3 else "int8", "data": "synthetic",
-            "config": dict(w0.describe(), n_outliers=n_o,
-                           parallelism="column-parallel x%d (own output-channel block per GPU)"
-                                       % world,
+            "config": dict(w0.describe(), n_outliers=L.n_o,
+                           parallelism=("one layer of %d x %d output channels split by output "
+                                        "channel over %d GPUs; this rank holds [%d, %d)"
+                                        % (world, w0.N, world, rows[0], rows[1])
+                                        if world > 1 else "one GPU, the whole layer"),
                            l2=l2_desc,
                            **({"code_format": "e4m3 (the FP8 variant of the decomposition)"}
                               if e4m3 else {}),
@@ -544,31 +691,46 @@ def run_gpu(args, w0):
                               if cache is not None else {})),
             "hbm_gbs": hbm_gbs * world, "hbm_frac": hbm_gbs / pk["hbm"],
             "roofline": roof,
-            "weight_quant": {"ms": wq_ms, "gbs": 3.0 * N * K / (wq_ms * 1e-3) / 1e9,
-                             "frac_hbm": 3.0 * N * K / (wq_ms * 1e-3) / 1e9 / pk["hbm"]},
+            "weight_quant": L.weight_quant(pk),
             "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": 2 * T * K,
                     "d2h_bytes_per_step": 2 * T * N, "ms_per_step": e2e_per,
                     "steps": e2e_steps,
                     "pipeline": "forward on one stream; X uploads and C read-backs on two "
                                 "copy streams, %d buffer slots; read-backs checked "
                                 "bit-exact against the device-timed output" % depth},
-            # launches of this library's kernels per step: fused prepare + GEMM (the mask
-            # clear before them is a memset, not a kernel), or the one decode kernel
+            # launches of this library's kernels per step: fused prepare + GEMM, or the one
+            # decode kernel (the memsets before them are not kernels of this library)
             "gpu_launches": K_steps * (1 if decode else 2),
             "clocks": clk}
 
     # CPU baseline: the oracle on this host, rank 0 at N = 1 only
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not e4m3:
         from oracle import oracle as O
-        CB_h = CB.cpu().numpy()
-        SCB_h = SCB.cpu().numpy()
-        dt, rows, ops = oracle_sample(w, X, CB_h, SCB_h, b, args.cpu_budget)
+        CB_h = L.CB.cpu().numpy()
+        SCB_h = L.SCB.cpu().numpy()
+        b_h = None if L.b is None else L.b.cpu().view(torch.int16).numpy().view(np.float16)
+        dt, nrows, ops = oracle_sample(layer, L.X_h, CB_h, SCB_h, b_h, args.cpu_budget)
+        del CB_h
         line["cpu_baseline"] = {
             "value": ops / dt / 1e12, "unit": "TOPS", "cores": O.num_threads(),
             "kind": "oracle",
             "sample": "scan + row quantisation of all %d rows, then int8 product, dequant, "
                       "fp64 outlier part and bias for %d evenly spaced rows (repeated calls "
-                      "count again) x all %d outputs (%.1f s)" % (T, rows, N, dt)}
+                      "count again) x all %d outputs (%.1f s)" % (T, nrows, N, dt)}
+
+    if (world == 1 and not args.no_extras and not e4m3 and cache is None
+            and w0.name == workloads()[DEFAULT_WORKLOAD].name):
+        keep = L
+        del L
+        sweep, per = run_extras(abi, keep, dev, stream, uuid, pk, sms, K_steps)
+        head = {"workload": keep.w.name, "threshold": json_threshold(keep.w.threshold),
+                "n_outliers": keep.n_o, "ms_per_step": ms_per_step,
+                "effective_tops": value, "roofline": {k: roof[k] for k in (
+                    "achieved", "peak", "frac", "frac_of_pipe_peak",
+                    "frac_of_datasheet_peak", "kernel_ms")}}
+        line["sweep"] = sorted([head] + sweep,
+                               key=lambda r: (r["threshold"] == "inf", r["n_outliers"]))
+        line["per_config"] = per
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -648,9 +810,12 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--workload", default="opt_ffn_up", choices=sorted(workloads()))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads()))
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other layer shapes (sweep and per_config records) that the "
+                         "default workload's run also measures")
     ap.add_argument("--l2-flush", default="auto", choices=["auto", "always"],
                     help="auto: flush the L2 between timed steps only when the inputs are "
                          "smaller than twice the L2")

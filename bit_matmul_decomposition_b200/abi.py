@@ -42,6 +42,11 @@ SIGNATURES = {
     "i8_outlier_cache_reset": (_ST, [_P, _SZ, _P]),
     "i8_linear_forward_cached": (_ST, [_P, _I64, _I64, _P, _P, _P, _I64, _F, _P, _P, _SZ, _P,
                                        _SZ, _P]),
+    "i8_linear_backward_input": (_ST, [_P, _I64, _I64, _P, _I64, _P, _P]),
+    "i8_linear_backward_weight": (_ST, [_P, _P, _I64, _I64, _I64, _P, _P]),
+    "i8_bias_grad": (_ST, [_P, _I64, _I64, _P, _P]),
+    "i8_dequantize_weight": (_ST, [_P, _P, _I64, _I64, _P, _P]),
+    "i8_dequantize_weight_e4m3": (_ST, [_P, _P, _I64, _I64, _P, _P]),
     "i8_sync_status": (_ST, [_P]),
     "i8_set_profile_events": (_ST, [_P, _P]),
     "i8_selftest_bounded_wait": (_ST, [_I64, _P]),
@@ -289,6 +294,48 @@ def i8_igemm_s32(A, B, acc, workspace, stream=None):
     _check("i8_igemm_s32",
            load().i8_igemm_s32(_ptr(A), T, K, _ptr(B), N, _ptr(acc), _ptr(workspace),
                                workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def i8_linear_backward_input(dY, W, dX, stream=None):
+    """dX[T, K] = dY[T, N] W[N, K] (fp16, tensor cores, fp32 sums)."""
+    T, N = _mat(dY, "dY", _dt("float16"))
+    Nw, K = _mat(W, "W", _dt("float16"))
+    if Nw != N:
+        raise ValueError("W has %d rows, dY has %d columns" % (Nw, N))
+    _arg(dX, "dX", _dt("float16"), T * K)
+    _check("i8_linear_backward_input",
+           load().i8_linear_backward_input(_ptr(dY), T, N, _ptr(W), K, _ptr(dX),
+                                           _stream(stream)))
+
+
+def i8_linear_backward_weight(dY, X, dW, stream=None):
+    """dW[N, K] = dY[T, N]^T X[T, K] (fp16, tensor cores, fp32 sums)."""
+    T, N = _mat(dY, "dY", _dt("float16"))
+    Tx, K = _mat(X, "X", _dt("float16"))
+    if Tx != T:
+        raise ValueError("X has %d rows, dY has %d" % (Tx, T))
+    _arg(dW, "dW", _dt("float16"), N * K)
+    _check("i8_linear_backward_weight",
+           load().i8_linear_backward_weight(_ptr(dY), _ptr(X), T, N, K, _ptr(dW),
+                                            _stream(stream)))
+
+
+def i8_bias_grad(dY, db, stream=None):
+    """db[N] = sum over rows of dY[T, N] (fp32 sums, fp16 result)."""
+    T, N = _mat(dY, "dY", _dt("float16"))
+    _arg(db, "db", _dt("float16"), N)
+    _check("i8_bias_grad", load().i8_bias_grad(_ptr(dY), T, N, _ptr(db), _stream(stream)))
+
+
+def i8_dequantize_weight(CB, SCB, W, stream=None):
+    """W[N, K] fp16 = CB * SCB / 127 (int8 codes) or the e4m3 codes' values * SCB / 448
+    (uint8 / float8_e4m3fn codes)."""
+    N, K = _mat(CB, "CB", _dt("int8", "uint8", "float8_e4m3fn"))
+    _arg(SCB, "SCB", _dt("float32"), N)
+    _arg(W, "W", _dt("float16"), N * K)
+    import torch
+    fn = "i8_dequantize_weight" if CB.dtype == torch.int8 else "i8_dequantize_weight_e4m3"
+    _check(fn, getattr(load(), fn)(_ptr(CB), _ptr(SCB), N, K, _ptr(W), _stream(stream)))
 
 
 def i8_sync_status(stream=None) -> int:

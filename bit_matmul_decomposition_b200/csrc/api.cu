@@ -9,6 +9,7 @@
 #include <utility>
 
 #include "../../include/i8linear.h"
+#include "bwd.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
 #include "gemv.cuh"
@@ -29,6 +30,7 @@ struct DeviceInfo {
   int sms = 0;
   bool gemm_attr = false;
   int gemm_clusters = 0;  // co-resident CTA pairs of the GEMM kernel
+  int bwd_clusters = 0;   // co-resident CTA pairs of the backward fp16 GEMM
   int prep_smem_max = 0;  // dynamic shared memory granted to prepare_kernel
   int smem_optin = 0;     // largest dynamic shared memory a kernel may opt in to
 };
@@ -66,7 +68,13 @@ i8_status device_info(DeviceInfo** out) {
         cudaFuncSetAttribute(gemm::i8_gemm_tcgen05_kernel<true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
         cudaFuncSetAttribute(gemm::i8_gemm_tcgen05_kernel<false, true>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(bwd::f16_gemm_kernel<false, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(bwd::SMEM_BYTES)) != cudaSuccess ||
+        cudaFuncSetAttribute(bwd::f16_gemm_kernel<true, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(bwd::SMEM_BYTES)) != cudaSuccess)
       return I8_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * d.sms, 1, 1);
@@ -78,6 +86,14 @@ i8_status device_info(DeviceInfo** out) {
         clusters < 1)
       return I8_ERR_CUDA;
     d.gemm_clusters = clusters;
+    cfg.dynamicSmemBytes = bwd::SMEM_BYTES;
+    cfg.blockDim = dim3(bwd::THREADS, 1, 1);
+    clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, bwd::f16_gemm_kernel<true, true>, &cfg) !=
+            cudaSuccess ||
+        clusters < 1)
+      return I8_ERR_CUDA;
+    d.bwd_clusters = clusters;
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, prepare_kernel) != cudaSuccess) return I8_ERR_CUDA;
     const int prep_max =
@@ -88,6 +104,9 @@ i8_status device_info(DeviceInfo** out) {
       return I8_ERR_CUDA;
     d.prep_smem_max = prep_max;
     d.smem_optin = static_cast<int>(p_smem_optin(dev));
+    if (cudaFuncSetAttribute(quantize_weight_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kWqRingBytes)) != cudaSuccess)
+      return I8_ERR_CUDA;
     d.gemm_attr = true;
   }
   *out = &d;
@@ -308,6 +327,29 @@ i8_status run_quant_rows(const void* A, int64_t R, int64_t K, const uint32_t* ma
   return launch_status();
 }
 
+// Step 3 for a whole weight: the streaming quantiser (rows of up to 64 KB), else one CTA
+// per row.
+i8_status run_quant_weight(const void* W, int64_t N, int64_t K, int8_t* CB, float* SCB,
+                           const DeviceInfo& d, cudaStream_t s, bool e4m3 = false) {
+  if (K * 2 > kWqMaxRowBytes)
+    return run_quant_rows(W, N, K, nullptr, CB, SCB, nullptr, nullptr, nullptr, s, e4m3);
+  WqArgs a;
+  a.W = static_cast<const __half*>(W);
+  a.N = N;
+  a.K = K;
+  a.CB = CB;
+  a.SCB = SCB;
+  a.e4m3 = e4m3;
+  a.R = wq_rows_per_stage(K);
+  a.stages = (N + a.R - 1) / a.R;
+  a.slots = wq_slots(K);
+  a.wait_limit_ns = kWaitLimitNs;
+  const int64_t grid = a.stages < d.sms ? a.stages : d.sms;
+  const size_t smem = static_cast<size_t>(a.slots) * static_cast<size_t>(a.R * K * 2);
+  quantize_weight_kernel<<<static_cast<unsigned>(grid), kWqThreads, smem, s>>>(a);
+  return launch_status();
+}
+
 // Fused steps 1 + 2 (+ the fp16 outlier slices): one cooperative launch.
 // mask must hold ceil(K/32) + 1 words; the last one is the grid-barrier counter.
 // `zero_words` words from `mask` on are cleared first (at least the mask and the barrier
@@ -425,6 +467,48 @@ i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t
   else
     e = launch_overlapped(gemm::i8_gemm_tcgen05_kernel<false>, dim3(2 * clusters),
                           dim3(gemm::THREADS), gemm::SMEM_BYTES, s, tA, tB, tAo, tBo, tBc, tC, a);
+  return e == cudaSuccess ? launch_status() : I8_ERR_CUDA;
+}
+
+// Backward fp16 GEMM: C[M, Nc] = sum_r A(m, r) B(n, r); a_mn / b_mn: the operand's rows run
+// along m / n (MN-major) instead of the reduction.  lda / ldb: elements per row in memory.
+i8_status run_f16_gemm(bool a_mn, const void* A, int64_t lda, bool b_mn, const void* B,
+                       int64_t ldb, int64_t M, int64_t Nc, int64_t R, void* C,
+                       const DeviceInfo& d, cudaStream_t s) {
+  CUtensorMap tA, tB, tC;
+  const auto F16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  // K-major: [M rows][R] with 128 x 64 boxes; MN-major: [R rows][M] with 64 x 64 boxes
+  const bool okA = a_mn ? map_2d(&tA, F16, A, M, R, lda * 2, 64, 64)
+                        : map_2d(&tA, F16, A, R, M, lda * 2, 64, 128);
+  const bool okB = b_mn ? map_2d(&tB, F16, B, Nc, R, ldb * 2, 64, 64)
+                        : map_2d(&tB, F16, B, R, Nc, ldb * 2, 64, 128);
+  if (!okA || !okB) return I8_ERR_CUDA;
+  tC = tA;
+  const bool c_tma = (Nc % 8) == 0;
+  if (c_tma && !map_c(&tC, C, static_cast<uint64_t>(Nc), static_cast<uint64_t>(M)))
+    return I8_ERR_CUDA;
+  bwd::Args a;
+  a.M = static_cast<int>(M);
+  a.Nc = static_cast<int>(Nc);
+  a.R = static_cast<int>(R);
+  a.m_tiles = static_cast<int>((M + bwd::TM - 1) / bwd::TM);
+  a.n_tiles = static_cast<int>((Nc + bwd::TN - 1) / bwd::TN);
+  a.k_blocks = static_cast<int>((R + bwd::BK - 1) / bwd::BK);
+  a.C = static_cast<__half*>(C);
+  a.ldc = static_cast<int>(Nc);
+  a.c_tma = c_tma;
+  a.wait_limit_ns = kWaitLimitNs;
+  const int64_t tiles = static_cast<int64_t>(a.m_tiles) * a.n_tiles;
+  const int clusters = static_cast<int>(tiles < d.bwd_clusters ? tiles : d.bwd_clusters);
+  cudaError_t e;
+  if (a_mn && b_mn)
+    e = launch_overlapped(bwd::f16_gemm_kernel<true, true>, dim3(2 * clusters),
+                          dim3(bwd::THREADS), bwd::SMEM_BYTES, s, tA, tB, tC, a);
+  else if (!a_mn && b_mn)
+    e = launch_overlapped(bwd::f16_gemm_kernel<false, true>, dim3(2 * clusters),
+                          dim3(bwd::THREADS), bwd::SMEM_BYTES, s, tA, tB, tC, a);
+  else
+    return I8_ERR_INVALID_ARG;
   return e == cudaSuccess ? launch_status() : I8_ERR_CUDA;
 }
 
@@ -625,8 +709,7 @@ i8_status i8_quantize_weight(const void* W, int64_t N, int64_t K, int8_t* CB, fl
   DeviceInfo* d;
   i8_status st = device_info(&d);
   if (st != I8_OK) return st;
-  return run_quant_rows(W, N, K, nullptr, CB, SCB, nullptr, nullptr, nullptr,
-                        static_cast<cudaStream_t>(stream));
+  return run_quant_weight(W, N, K, CB, SCB, *d, static_cast<cudaStream_t>(stream));
 }
 
 i8_status i8_outlier_scan(const void* X, int64_t T, int64_t K, float threshold, uint32_t* col_mask,
@@ -708,8 +791,8 @@ i8_status i8_quantize_weight_e4m3(const void* W, int64_t N, int64_t K, uint8_t* 
   DeviceInfo* d;
   i8_status st = device_info(&d);
   if (st != I8_OK) return st;
-  return run_quant_rows(W, N, K, nullptr, reinterpret_cast<int8_t*>(CB), SCB, nullptr, nullptr,
-                        nullptr, static_cast<cudaStream_t>(stream), true);
+  return run_quant_weight(W, N, K, reinterpret_cast<int8_t*>(CB), SCB, *d,
+                          static_cast<cudaStream_t>(stream), true);
 }
 
 i8_status i8_prepare_act_e4m3(const void* X, int64_t T, int64_t K, float threshold,
@@ -766,6 +849,70 @@ i8_status i8_igemm_s32(const int8_t* A, int64_t T, int64_t K, const int8_t* B, i
                     nullptr, acc, *d, s);
   return run_decode(true, nullptr, A, T, K, B, N, 0.0f, nullptr, nullptr, nullptr, acc,
                     static_cast<uint8_t*>(workspace), w, *d, s);
+}
+
+i8_status i8_linear_backward_input(const void* dY, int64_t T, int64_t N, const void* W,
+                                   int64_t K, void* dX, void* stream) {
+  if (!dY || !W || !dX || !aligned16(dY) || !aligned16(W) || !aligned16(dX))
+    return I8_ERR_INVALID_ARG;
+  if (!shape_ok(T, K) || N <= 0 || N > 0x7fffffffLL || (N % 8) != 0) return I8_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  i8_status st = device_info(&d);
+  if (st != I8_OK) return st;
+  return run_f16_gemm(false, dY, N, true, W, K, T, K, N, dX, *d,
+                      static_cast<cudaStream_t>(stream));
+}
+
+i8_status i8_linear_backward_weight(const void* dY, const void* X, int64_t T, int64_t N,
+                                    int64_t K, void* dW, void* stream) {
+  if (!dY || !X || !dW || !aligned16(dY) || !aligned16(X) || !aligned16(dW))
+    return I8_ERR_INVALID_ARG;
+  if (!shape_ok(T, K) || N <= 0 || N > 0x7fffffffLL || (N % 8) != 0) return I8_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  i8_status st = device_info(&d);
+  if (st != I8_OK) return st;
+  return run_f16_gemm(true, dY, N, true, X, K, N, K, T, dW, *d,
+                      static_cast<cudaStream_t>(stream));
+}
+
+i8_status i8_bias_grad(const void* dY, int64_t T, int64_t N, void* db, void* stream) {
+  if (!dY || !db || !aligned16(dY) || !aligned16(db)) return I8_ERR_INVALID_ARG;
+  if (T <= 0 || T > 0x7fffffffLL || N <= 0 || N > 0x7fffffffLL || (N % 8) != 0)
+    return I8_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  i8_status st = device_info(&d);
+  if (st != I8_OK) return st;
+  bwd::bias_grad_kernel<<<static_cast<unsigned>((N + 63) / 64), bwd::kBiasThreads, 0,
+                          static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __half*>(dY), T, N, static_cast<__half*>(db));
+  return launch_status();
+}
+
+static i8_status dequantize(const void* CB, const float* SCB, int64_t N, int64_t K, void* W,
+                            void* stream, bool e4m3) {
+  if (!CB || !SCB || !W || !aligned16(CB) || !aligned16(SCB) || !aligned16(W))
+    return I8_ERR_INVALID_ARG;
+  if (!shape_ok(N, K)) return I8_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  i8_status st = device_info(&d);
+  if (st != I8_OK) return st;
+  const int64_t groups = N * K / 16;
+  int64_t grid = (groups + bwd::kDequantThreads - 1) / bwd::kDequantThreads;
+  if (grid > static_cast<int64_t>(d->sms) * 16) grid = static_cast<int64_t>(d->sms) * 16;
+  bwd::dequantize_kernel<<<static_cast<unsigned>(grid), bwd::kDequantThreads, 0,
+                           static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const int8_t*>(CB), SCB, N, K, static_cast<__half*>(W), e4m3);
+  return launch_status();
+}
+
+i8_status i8_dequantize_weight(const int8_t* CB, const float* SCB, int64_t N, int64_t K, void* W,
+                               void* stream) {
+  return dequantize(CB, SCB, N, K, W, stream, false);
+}
+
+i8_status i8_dequantize_weight_e4m3(const uint8_t* CB, const float* SCB, int64_t N, int64_t K,
+                                    void* W, void* stream) {
+  return dequantize(CB, SCB, N, K, W, stream, true);
 }
 
 i8_status i8_sync_status(void* stream) {

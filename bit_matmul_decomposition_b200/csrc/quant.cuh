@@ -3,6 +3,7 @@
 //   compact_kernel         step 1: mask -> ascending outlier index list + count
 //   quantize_rows_kernel   steps 2/3: row absmax (over the non-outlier columns) and int8
 //                          codes; for the hidden states also the fp16 outlier slice X_o
+//   quantize_weight_kernel step 3 for a whole weight: rows streamed through shared memory
 //   prepare_kernel         steps 1 and 2 fused (one read of X), plus the fp16 outlier
 //                          slices of X and of CB for step 6 (CB's kept across calls in an
 //                          outlier cache when the caller provides one)
@@ -818,6 +819,172 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
         __stcg(p.ocache, 1u);
       }
     }
+  }
+}
+
+// ====================================================================== weight quantiser
+// quantize_weight_kernel: step 3 over a whole weight at the speed of HBM.  The weight is cut
+// into stages of R consecutive rows (R a power of two, R * K * 2 bytes up to 32 KB); CTA b
+// takes stages b, b + G, ...  Its producer thread copies each stage into a ring of
+// shared-memory slots with one bulk (TMA) copy, so that several stages per SM are always
+// in flight; 8 consumer warps take each row's absmax and write its codes and scale from
+// shared memory: a warp per row when R >= 8, else 8 / R warps per row, combining their
+// maxima through shared memory.  Codes and scales are those of quantize_rows_kernel with no
+// excluded column.
+constexpr int kWqWarps = 8;                            // consumer warps
+constexpr int kWqThreads = (kWqWarps + 1) * 32;        // + the producer warp
+constexpr int64_t kWqStageTarget = 32768;              // bytes per stage (at most)
+constexpr int64_t kWqRingBytes = 196608;               // shared-memory ring (at most)
+constexpr int kWqMaxSlots = 8;
+constexpr int64_t kWqMaxRowBytes = 65536;              // longer rows: quantize_rows_kernel
+
+struct WqArgs {
+  const __half* W;
+  int64_t N, K;
+  int8_t* CB;
+  float* SCB;
+  bool e4m3;
+  int64_t R;            // rows per stage
+  int64_t stages;       // ceil(N / R)
+  int slots;            // ring slots
+  uint64_t wait_limit_ns;
+};
+
+__host__ __device__ inline int64_t wq_rows_per_stage(int64_t K) {
+  int64_t r = 1;
+  while (r < 256 && 2 * r * K * 2 <= kWqStageTarget) r *= 2;
+  return r;
+}
+
+__host__ __device__ inline int wq_slots(int64_t K) {
+  const int64_t stage = wq_rows_per_stage(K) * K * 2;
+  const int64_t n = kWqRingBytes / stage;
+  return static_cast<int>(n < kWqMaxSlots ? n : kWqMaxSlots);
+}
+
+__device__ __forceinline__ void wq_consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kWqWarps * 32) : "memory");
+}
+
+// true when `v` holds in every consumer thread (a barrier of the consumer warps)
+__device__ __forceinline__ bool wq_consumers_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "n"(kWqWarps * 32)
+      : "memory");
+  return r != 0;
+}
+
+__global__ void __launch_bounds__(kWqThreads, 1) quantize_weight_kernel(const WqArgs a) {
+  extern __shared__ __align__(128) uint8_t wsm[];
+  __shared__ __align__(8) uint64_t full[kWqMaxSlots];
+  __shared__ __align__(8) uint64_t empty[kWqMaxSlots];
+  __shared__ float red[2][kWqWarps];
+  __shared__ int abort_flag_s;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t K = a.K, R = a.R;
+  const int64_t stage_bytes = R * K * 2;
+  const int NS = a.slots;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&empty[i]), kWqWarps);
+    }
+    abort_flag_s = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  volatile int* abort_flag = &abort_flag_s;
+  const uint32_t ring = smem_u32(wsm);
+
+  if (warp == kWqWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t issued = 0;
+      bool ok = true;
+      for (int64_t j = blockIdx.x; j < a.stages; j += gridDim.x, ++issued) {
+        const int slot = static_cast<int>(issued % NS);
+        const uint32_t ph = (issued / NS) & 1u;
+        if (!mbar_wait(smem_u32(&empty[slot]), ph ^ 1u, abort_flag, a.wait_limit_ns)) {
+          ok = false;
+          break;
+        }
+        // the slot's previous reads (generic proxy) come before the copy into it
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        const int64_t r0 = j * R;
+        const int64_t rows = min(R, a.N - r0);
+        const uint32_t bytes = static_cast<uint32_t>(rows * K * 2);
+        mbar_arrive_expect_tx(smem_u32(&full[slot]), bytes);
+        bulk_load(ring + static_cast<uint32_t>(slot * stage_bytes), a.W + r0 * K, bytes,
+                  smem_u32(&full[slot]));
+      }
+      if (!ok) {
+        // wind down: the copies in flight land (bounded) before the CTA exits
+        int no_abort = 0;
+        const uint32_t inflight = issued < static_cast<uint32_t>(NS) ? issued : NS;
+        for (uint32_t i = 0; i < inflight; ++i) {
+          const uint32_t u = issued - 1 - i;
+          mbar_wait(smem_u32(&full[u % NS]), (u / NS) & 1u, &no_abort, a.wait_limit_ns);
+        }
+      }
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int wpr = R >= kWqWarps ? 1 : static_cast<int>(kWqWarps / R);   // warps per row
+  const int gpr = static_cast<int>(K / 8);                             // 16-byte groups
+  const int sub = warp % wpr;
+  const int start = sub * 32 + lane, step = 32 * wpr;
+  const float cmax = code_max(a.e4m3);
+  uint32_t it = 0;
+  for (int64_t j = blockIdx.x; j < a.stages; j += gridDim.x, ++it) {
+    const int slot = static_cast<int>(it % NS);
+    const bool got = mbar_wait(smem_u32(&full[slot]), (it / NS) & 1u, abort_flag,
+                               a.wait_limit_ns);
+    // warps that share rows meet at barriers below: they must all take the same branch
+    if (wpr > 1 ? !wq_consumers_all(got) : !__all_sync(0xffffffffu, got)) break;
+    const int64_t r0 = j * R;
+    const int64_t rows = min(R, a.N - r0);
+    const uint32_t sbase = ring + static_cast<uint32_t>(slot * stage_bytes);
+    // row i of the stage goes to warps i * wpr .. i * wpr + wpr - 1 (wpr > 1), or to warp
+    // i % 8 (wpr == 1)
+    for (int64_t i = (wpr > 1 ? warp / wpr : warp); i < (wpr > 1 ? R : rows);
+         i += (wpr > 1 ? R : kWqWarps)) {
+      const bool have = i < rows;
+      const uint32_t rbase = sbase + static_cast<uint32_t>(i * K * 2);
+      float amax = 0.0f;
+      if (have) {
+        float m0 = 0.0f, m1 = 0.0f;
+        int v = start;
+        for (; v + step < gpr; v += 2 * step) {
+          m0 = fmaxf(m0, absmax8_all(lds_v4(rbase + static_cast<uint32_t>(v) * 16u)));
+          m1 = fmaxf(m1, absmax8_all(lds_v4(rbase + static_cast<uint32_t>(v + step) * 16u)));
+        }
+        if (v < gpr) m0 = fmaxf(m0, absmax8_all(lds_v4(rbase + static_cast<uint32_t>(v) * 16u)));
+        amax = warp_max(fmaxf(m0, m1));
+      }
+      if (wpr > 1) {
+        if (lane == 0) red[it & 1u][warp] = amax;
+        wq_consumer_sync();
+        const int base = (warp / wpr) * wpr;
+        for (int w2 = 0; w2 < wpr; ++w2) amax = fmaxf(amax, red[it & 1u][base + w2]);
+      }
+      if (have) {
+        const float sc = amax > 0.0f ? __fdiv_rn(cmax, amax) : 0.0f;
+        uint2* q = reinterpret_cast<uint2*>(a.CB + (r0 + i) * K);
+        for (int v = start; v < gpr; v += step)
+          q[v] = codes8_fmt(lds_v4(rbase + static_cast<uint32_t>(v) * 16u), 0u, sc, a.e4m3);
+        if (sub == 0 && lane == 0) a.SCB[r0 + i] = amax;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&empty[slot]));
   }
 }
 

@@ -14,8 +14,10 @@ forward, and gradients pass straight through the quantisation -- the blog gives 
 gradient formulas, so the plainest reading is taken: the backward of y = x W^T + b, i.e.
 dx = dy W, dW = dy^T x, db = sum(dy), with fp16 operands.  Without fp16 weights the layer
 still passes dx = dy W' back (W' = CB * SCB / 127, the weight it computes with), so layers
-before it can train.  The forward runs in the library's CUDA kernels; the backward
-products are plain fp16 GEMMs (torch.matmul, cuBLAS) on the same device.
+before it can train.  Forward and backward run in the library's CUDA kernels: the two
+backward products on the tcgen05 tensor cores (i8_linear_backward_input / _weight), the
+bias gradient and W' in HBM-bound passes (i8_bias_grad, i8_dequantize_weight).  The
+backward needs out_features % 8 == 0 (the row pitch of dy must suit TMA).
 
 Serving with systematic outliers (the blog's observation that the same few feature
 dimensions carry the outliers call after call): ``outlier_cache_cols > 0`` keeps the
@@ -37,7 +39,7 @@ from . import abi
 
 class _Int8LinearFn(torch.autograd.Function):
     """Forward: the decomposed int8 layer (CUDA library).  Backward: straight through the
-    quantisation, fp16 GEMMs."""
+    quantisation, the library's fp16 tensor-core products."""
 
     @staticmethod
     def forward(ctx, x2, weight, bias, layer):
@@ -52,14 +54,32 @@ class _Int8LinearFn(torch.autograd.Function):
         x2, weight = ctx.saved_tensors
         layer = ctx.layer
         gy = gy.to(torch.float16).contiguous()
+        T, N = gy.shape
+        K = layer.in_features
+        dev = gy.device
         gx = gw = gb = None
-        if ctx.needs_input_grad[0]:
-            w = weight if weight is not None else layer.dequantized_weight().to(torch.float16)
-            gx = gy @ w
-        if weight is not None and ctx.needs_input_grad[1]:
-            gw = gy.t() @ x2
-        if ctx.has_bias and ctx.needs_input_grad[2]:
-            gb = gy.float().sum(0).to(torch.float16)
+        want_x = ctx.needs_input_grad[0]
+        want_w = weight is not None and ctx.needs_input_grad[1]
+        want_b = ctx.has_bias and ctx.needs_input_grad[2]
+        if T == 0:
+            z = lambda *shape: torch.zeros(shape, dtype=torch.float16, device=dev)  # noqa: E731
+            return (z(0, K) if want_x else None, z(N, K) if want_w else None,
+                    z(N) if want_b else None, None)
+        if N % 8:
+            raise NotImplementedError("the backward needs out_features % 8 == 0 (got %d): "
+                                      "the row pitch of dy must be a multiple of 16 bytes" % N)
+        with torch.cuda.device(dev):
+            if want_x:
+                w = (weight.detach().contiguous() if weight is not None
+                     else layer.dequantized_weight())
+                gx = torch.empty((T, K), dtype=torch.float16, device=dev)
+                abi.i8_linear_backward_input(gy, w, gx)
+            if want_w:
+                gw = torch.empty((N, K), dtype=torch.float16, device=dev)
+                abi.i8_linear_backward_weight(gy, x2.detach(), gw)
+            if want_b:
+                gb = torch.empty((N,), dtype=torch.float16, device=dev)
+                abi.i8_bias_grad(gy, gb)
         return gx, gw, gb, None
 
 
@@ -165,12 +185,16 @@ class Linear8bitLt(torch.nn.Module):
                 abi.i8_quantize_weight(weight16, self.CB, self.SCB)
 
     def dequantized_weight(self) -> torch.Tensor:
-        """The weight the layer computes with (fp32): CB * SCB / 127, or for e4m3 codes
-        their values * SCB / 448."""
-        if self.code_format == "e4m3":
-            vals = self.CB.view(torch.float8_e4m3fn).float()
-            return vals * (self.SCB.float() / 448.0)[:, None]
-        return self.CB.float() * (self.SCB.float() / 127.0)[:, None]
+        """The weight the layer computes with, fp16 [out, in], from the library's kernel:
+        CB * SCB / 127, or for e4m3 codes their values * SCB / 448 (the layer must be on a
+        CUDA device)."""
+        if not self.CB.is_cuda:
+            raise ValueError("dequantized_weight() runs on the layer's CUDA device")
+        W = torch.empty((self.out_features, self.in_features), dtype=torch.float16,
+                        device=self.CB.device)
+        with torch.cuda.device(self.CB.device):
+            abi.i8_dequantize_weight(self.CB, self.SCB, W)
+        return W
 
     def _workspace(self, T: int) -> torch.Tensor:
         size = (abi.i8_linear_workspace_size_e4m3 if self.code_format == "e4m3"

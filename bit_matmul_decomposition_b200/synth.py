@@ -6,6 +6,9 @@ so that the CUDA path and the CPU oracle can be fed identical bytes.
 Recipe (shared by every workload):
   * numpy ``Generator(PCG64)``; one child seed per tensor from ``SeedSequence(seed)``
     (child 0: hidden states X, child 1: weight W, child 2: bias, child 3: outlier layout);
+    the weight is drawn in blocks of W_BLOCK rows, block i from the seed sequence with
+    spawn key (1, i), so that any range of output channels (one GPU's shard of the layer)
+    can be drawn on its own and equals the same rows of the whole weight;
   * N(mu, sigma) is drawn in fp32 and cast to fp16 with round-to-nearest-even;
   * "+-U[a,b]" means magnitude U[a,b] with an independent random sign per entry;
   * fixed outlier columns are drawn without replacement from [0, K) and overwritten in
@@ -19,8 +22,10 @@ shapes, whose real weights are not available, stand in for the evaluated models.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
 import math
+import os
 from typing import Optional, Sequence
 
 import numpy as np
@@ -46,7 +51,7 @@ class Workload:
 
     def describe(self) -> dict:
         d = dict(workload=self.name, T=self.T, K=self.K, N=self.N, seed=self.seed,
-                 threshold=self.threshold)
+                 threshold="inf" if math.isinf(self.threshold) else self.threshold)
         if self.fixed_cols is not None:
             d["outlier_cols"] = list(self.fixed_cols)
         else:
@@ -141,15 +146,57 @@ def make_x(w: Workload, T: Optional[int] = None) -> np.ndarray:
     return X
 
 
-def make_w(w: Workload) -> np.ndarray:
-    """Weight W [N, K] fp16 in the nn.Linear [out, in] layout."""
-    return _normal_fp16(_children(w.seed)[1], (w.N, w.K), w.w_sigma)
+W_BLOCK = 2048   # rows of the weight drawn from one generator
 
 
-def make_bias(w: Workload) -> Optional[np.ndarray]:
+def _w_block_rng(seed: int, blk: int):
+    return np.random.Generator(np.random.PCG64(
+        np.random.SeedSequence(entropy=seed, spawn_key=(1, blk))))
+
+
+def make_w(w: Workload, rows: Optional[tuple] = None) -> np.ndarray:
+    """Weight W [N, K] fp16 in the nn.Linear [out, in] layout, or only its rows
+    [rows[0], rows[1]) (bit for bit the same rows of the whole weight)."""
+    r0, r1 = (0, w.N) if rows is None else (int(rows[0]), int(rows[1]))
+    if not 0 <= r0 <= r1 <= w.N:
+        raise ValueError("rows %r outside [0, %d]" % (rows, w.N))
+    out = np.empty((r1 - r0, w.K), np.float16)
+
+    def draw(blk):
+        b0, b1 = blk * W_BLOCK, min(w.N, (blk + 1) * W_BLOCK)
+        lo, hi = max(b0, r0), min(b1, r1)
+        if lo == b0 and hi == b1:   # a whole block: straight into the output
+            out[lo - r0:hi - r0] = _normal_fp16(_w_block_rng(w.seed, blk), (b1 - b0, w.K),
+                                                w.w_sigma, chunk_rows=W_BLOCK)
+        else:
+            full = _normal_fp16(_w_block_rng(w.seed, blk), (b1 - b0, w.K), w.w_sigma,
+                                chunk_rows=W_BLOCK)
+            out[lo - r0:hi - r0] = full[lo - b0:hi - b0]
+
+    blocks = range(r0 // W_BLOCK, (r1 + W_BLOCK - 1) // W_BLOCK)
+    if len(blocks) <= 1:
+        for blk in blocks:
+            draw(blk)
+    else:   # blocks are independent streams: draw them on several threads
+        with concurrent.futures.ThreadPoolExecutor(min(len(blocks), os.cpu_count() or 1)) as ex:
+            list(ex.map(draw, blocks))
+    return out
+
+
+def make_bias(w: Workload, rows: Optional[tuple] = None) -> Optional[np.ndarray]:
+    """Bias [N] fp16 (or its entries [rows[0], rows[1])), None for a layer without."""
     if not w.bias:
         return None
-    return _normal_fp16(_children(w.seed)[2], (w.N,), w.b_sigma)
+    b = _normal_fp16(_children(w.seed)[2], (w.N,), w.b_sigma)
+    return b if rows is None else b[int(rows[0]):int(rows[1])].copy()
+
+
+def shard_rows(N: int, rank: int, world: int) -> tuple:
+    """Output channels [r0, r1) of rank `rank` when an N-wide layer is split over `world`
+    GPUs by output channel: contiguous blocks, sizes differing by at most one."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("rank %d of %d" % (rank, world))
+    return (N * rank) // world, (N * (rank + 1)) // world
 
 
 def random_fp16(shape, seed: int, sigma: float = 1.0) -> np.ndarray:

@@ -268,6 +268,43 @@ i8_status i8_linear_forward_noalloc(const void* X, int64_t T, int64_t K, const i
                                     float threshold, void* C, void* stream);
 
 /*
+ * Backward of the fp16-weight training mode.  Source: "用法" (usage) -- a layer built with
+ * has_fp16_weights=True keeps its fp16 weights for int8/fp16 mixed-precision training and
+ * re-quantises them for every forward; CB * SCB / 127 recovers the weight.  The blog gives
+ * no gradient formulas; these calls take the plainest reading, the backward of
+ * y = x W^T + b passed straight through the quantisation:
+ *
+ * i8_linear_backward_input(dY, T, N, W, K, dX, stream):
+ *   dX[T, K] = dY[T, N] * W[N, K]             (dY, W, dX fp16; W may be the fp16 weight
+ *                                             or the dequantised weight below)
+ * i8_linear_backward_weight(dY, X, T, N, K, dW, stream):
+ *   dW[N, K] = dY[T, N]^T * X[T, K]           (dY, X, dW fp16)
+ *   Both on the tcgen05 tensor cores (kind::f16): fp16 products summed in fp32, one
+ *   round-to-nearest-even to fp16 at the end.  W and X are read in their stored layout
+ *   (row-major [N, K] and [T, K]); the tensor cores take them as MN-major operands.
+ * i8_bias_grad(dY, T, N, db, stream):
+ *   db[N] = fp16(sum_t dY[t, n]), summed in fp32 in a fixed order (deterministic).
+ * i8_dequantize_weight(CB, SCB, N, K, W, stream):
+ *   W[n, k] = fp16_rn(fl32(CB[n, k] * fl32(SCB[n] / 127)))   (W fp16 [N, K], written)
+ * i8_dequantize_weight_e4m3(CB, SCB, N, K, W, stream):
+ *   the same with e4m3 codes: their values times fl32(SCB[n] / 448).
+ *
+ * Shapes: T, N, K > 0, K % 16 == 0, and N % 8 == 0 for the three calls that read dY (its
+ * row pitch must be a multiple of 16 bytes for TMA).  Every pointer is a 16-byte aligned
+ * device pointer owned by the caller; outputs are written in full.  Violations return
+ * I8_ERR_INVALID_ARG with nothing launched; errors otherwise as for the forward.
+ */
+i8_status i8_linear_backward_input(const void* dY, int64_t T, int64_t N, const void* W,
+                                   int64_t K, void* dX, void* stream);
+i8_status i8_linear_backward_weight(const void* dY, const void* X, int64_t T, int64_t N,
+                                    int64_t K, void* dW, void* stream);
+i8_status i8_bias_grad(const void* dY, int64_t T, int64_t N, void* db, void* stream);
+i8_status i8_dequantize_weight(const int8_t* CB, const float* SCB, int64_t N, int64_t K, void* W,
+                               void* stream);
+i8_status i8_dequantize_weight_e4m3(const uint8_t* CB, const float* SCB, int64_t N, int64_t K,
+                                    void* W, void* stream);
+
+/*
  * Step 4 alone -- acc[T, N] int32 = A[T, K] int8 * B[N, K]^T int8, on the same kernels
  * as i8_linear_forward (the tcgen05 GEMM, or the decode kernel for T <= 16 and
  * K <= 65536), with the epilogue writing the raw accumulator.  Source: "内部的 MatMul" (the 8-bit matrix

@@ -1,6 +1,7 @@
 """Host logic of bench.py on the CPU: the max-over-ranks reduction across two gloo ranks,
-the per-rank output-channel sharding (weak scaling), and the JSON contract of the
-reference arm (the CPU oracle timed on this host)."""
+the output-channel sharding of one layer (each rank its own rows of one weight; two gloo
+ranks running the oracle on their shards reproduce the unsharded layer bit for bit), and
+the JSON contract of the reference arm (the CPU oracle timed on this host)."""
 import json
 import os
 import socket
@@ -50,15 +51,88 @@ def test_max_over_ranks_without_process_group_is_identity():
     assert bench.max_over_ranks([1.5, 2.5]) == [1.5, 2.5]
 
 
-def test_each_rank_owns_its_own_output_channels():
-    w = synth.Workload("t", 8, 64, 32, seed=7)
-    w0, r0 = bench.rank_workload(w, 0)
-    _, r1 = bench.rank_workload(w, 1)
-    # the hidden states are replicated (same seed for X on every rank) ...
-    assert np.array_equal(synth.make_x(w0), synth.make_x(w))
-    # ... while every rank draws a different weight block
-    assert r0.seed == w.seed and r1.seed != w.seed
-    assert not np.array_equal(synth.make_w(r0), synth.make_w(r1))
+def test_shard_rows_partition_the_output_channels():
+    for N in (1, 7, 101, 49152):
+        for world in (1, 2, 3, 8):
+            if world > N:
+                continue
+            blocks = [synth.shard_rows(N, r, world) for r in range(world)]
+            assert blocks[0][0] == 0 and blocks[-1][1] == N
+            assert all(blocks[i][1] == blocks[i + 1][0] for i in range(world - 1))
+            sizes = [b - a for a, b in blocks]
+            assert max(sizes) - min(sizes) <= 1
+
+
+def test_each_rank_holds_rows_of_one_weight():
+    w = synth.Workload("t", 8, 64, 2500, seed=7)
+    for world in (1, 2, 3):
+        layer, _ = bench.rank_workload(w, 0, world)
+        assert layer.N == world * w.N and layer.seed == w.seed
+        W = synth.make_w(layer)
+        b = synth.make_bias(layer)
+        parts = []
+        for r in range(world):
+            lay_r, rows = bench.rank_workload(w, r, world)
+            assert lay_r == layer and rows[1] - rows[0] == w.N   # weak scaling: N per rank
+            parts.append(synth.make_w(layer, rows))
+            assert np.array_equal(synth.make_bias(layer, rows), b[rows[0]:rows[1]])
+        # the ranks' blocks are the rows of the one weight, in order
+        assert np.array_equal(np.concatenate(parts), W)
+        # the hidden states are the same on every rank
+        assert np.array_equal(synth.make_x(layer), synth.make_x(w))
+    layer1, rows1 = bench.rank_workload(w, 0, 1)
+    assert layer1 == w and rows1 == (0, w.N)     # one GPU: the workload itself
+
+
+def _shard_worker(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=120))
+    try:
+        from oracle import oracle as O
+        w = synth.Workload("shard", 24, 128, 101, seed=5, fixed_cols=(3, 77))
+        rows = synth.shard_rows(w.N, rank, world)
+        X = synth.make_x(w)                      # replicated
+        W_r = synth.make_w(w, rows)
+        b_r = synth.make_bias(w, rows)
+        CB_r, SCB_r = O.quantize_weight(W_r)
+        r = O.linear_forward(X, CB_r, SCB_r, b_r, w.threshold)
+        mine = dict(rows=rows, mask=r["mask_words"], SCx=r["SCx"], Xq=r["Xq"], CB=CB_r,
+                    SCB=SCB_r, C=r["C"])
+        got = [None] * world
+        dist.all_gather_object(got, mine)
+        if rank == 0:
+            full_W, full_b = synth.make_w(w), synth.make_bias(w)
+            CB, SCB = O.quantize_weight(full_W)
+            ref = O.linear_forward(X, CB, SCB, full_b, w.threshold)
+            ok = [got[i]["rows"] == synth.shard_rows(w.N, i, world) for i in range(world)]
+            for g in got:   # every rank found the same outlier columns and row scales
+                ok.append(np.array_equal(g["mask"], ref["mask_words"]))
+                ok.append(np.array_equal(g["SCx"].view(np.uint32), ref["SCx"].view(np.uint32)))
+                ok.append(np.array_equal(g["Xq"], ref["Xq"]))
+            ok.append(np.array_equal(np.concatenate([g["CB"] for g in got]), CB))
+            ok.append(np.array_equal(np.concatenate([g["SCB"] for g in got]).view(np.uint32),
+                                     SCB.view(np.uint32)))
+            C = np.concatenate([g["C"] for g in got], axis=1)
+            ok.append(C.shape == ref["C"].shape
+                      and np.array_equal(C.view(np.uint64), ref["C"].view(np.uint64)))
+            out["ok"] = ok
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_shard_one_layer_like_one_gpu():
+    """N = 101 over two ranks (blocks of 50 and 51 channels): each rank runs the oracle on
+    its rows of the one weight; the gathered blocks equal the unsharded layer bit for bit
+    (mask, row scales, codes, CB/SCB and the fp64 output)."""
+    world = 2
+    port = _free_port()
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_shard_worker, args=(world, port, out), nprocs=world, join=True)
+    assert out["ok"] and all(out["ok"]), out["ok"]
 
 
 REQUIRED = ["metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",

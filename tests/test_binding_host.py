@@ -166,3 +166,35 @@ def test_slice_size_matches_the_library():
     real.i8_outlier_slice_elems.argtypes = [ctypes.c_int64, ctypes.c_int64]
     for rows, k in [(1, 16), (5, 96), (300, 464), (2048, 4096), (7, 65552)]:
         assert abi._slice_elems(rows, k) == real.i8_outlier_slice_elems(rows, k)
+
+
+def test_backward_bindings_marshal_and_check(rec):
+    dY, W, X = _t((T, N), torch.float16), _t((N, K), torch.float16), _t((T, K), torch.float16)
+    dX, dW, db = _t((T, K), torch.float16), _t((N, K), torch.float16), _t((N,), torch.float16)
+    abi.i8_linear_backward_input(dY, W, dX)
+    assert rec.calls[-1][0] == "i8_linear_backward_input"
+    assert rec.calls[-1][1][1:3] == (T, N) and rec.calls[-1][1][4] == K
+    abi.i8_linear_backward_weight(dY, X, dW)
+    assert rec.calls[-1][0] == "i8_linear_backward_weight" and rec.calls[-1][1][2:5] == (T, N, K)
+    abi.i8_bias_grad(dY, db)
+    assert rec.calls[-1][0] == "i8_bias_grad" and rec.calls[-1][1][1:3] == (T, N)
+    with pytest.raises(ValueError):
+        abi.i8_linear_backward_input(dY, _t((N + 1, K), torch.float16), dX)   # rows != N
+    with pytest.raises(ValueError):
+        abi.i8_linear_backward_input(dY, W, _t((T, K - 1), torch.float16))   # short dX
+    with pytest.raises(ValueError):
+        abi.i8_linear_backward_weight(dY, _t((T + 1, K), torch.float16), dW)  # rows != T
+    with pytest.raises(TypeError):
+        abi.i8_bias_grad(_t((T, N), torch.float32), db)
+    with pytest.raises(ValueError):
+        abi.i8_bias_grad(dY, _t((N - 1,), torch.float16))
+
+
+def test_dequantize_binding_picks_the_code_format(rec):
+    SCB, Wd = _t((N,), torch.float32), _t((N, K), torch.float16)
+    abi.i8_dequantize_weight(_t((N, K), torch.int8), SCB, Wd)
+    assert rec.calls[-1][0] == "i8_dequantize_weight" and rec.calls[-1][1][2:4] == (N, K)
+    abi.i8_dequantize_weight(_t((N, K), torch.uint8), SCB, Wd)
+    assert rec.calls[-1][0] == "i8_dequantize_weight_e4m3"
+    with pytest.raises(ValueError):
+        abi.i8_dequantize_weight(_t((N, K), torch.int8), SCB, _t((N, K - 1), torch.float16))

