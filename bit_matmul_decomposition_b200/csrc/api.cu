@@ -143,8 +143,12 @@ struct Workspace {
 // GEMM path: the first region holds the packed outlier mask, the grid-barrier word of the
 // fused prepare pass and its outlier-cache update counter; one memset clears them at the
 // start of every forward.
-// Decode path: the slice records of every 32-row tile, the tiles' arrival counters and the
-// words of the cooperative prologue (none needs clearing: they carry the launch's epoch).
+// Decode path: the slice records of every 32-row tile, then the control words -- the
+// tiles' arrival counters and the words of the cooperative prologue, contiguous from `cnt`
+// to `xq` -- which one memset clears at the start of every decode call.  The words carry
+// the launch's epoch in their upper half; a zero upper half never matches an epoch, so no
+// bytes left in the workspace by an earlier call of another shape or path, or by another
+// user of the memory, can pose as a counter of this launch.
 Workspace layout(int64_t T, int64_t N, int64_t K, bool gemm_path = false) {
   Workspace w{};
   size_t off = 0;
@@ -443,6 +447,8 @@ i8_status run_decode(bool raw, const void* X, const int8_t* Xq, int64_t T, int64
   if (smem > static_cast<size_t>(d.smem_optin)) return I8_ERR_INVALID_ARG;
   CUtensorMap tCB;
   if (!map_2d_plain(&tCB, CB, K, N, K, gemv::BOXW, gemv::ROWS)) return I8_ERR_CUDA;
+  // the tile counters and the prologue's words (contiguous, cnt .. xq) start at zero
+  if (cudaMemsetAsync(ws + w.cnt, 0, w.xq - w.cnt, s) != cudaSuccess) return I8_ERR_CUDA;
   const int S = static_cast<int>(gemv::num_slices(K));
   int grid = (d.sms / S) * S;  // one CTA per SM, the same number of CTAs on every slice
   if (grid > 255) grid = (255 / S) * S;  // arrival counts are 8-bit

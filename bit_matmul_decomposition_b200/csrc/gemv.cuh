@@ -42,10 +42,11 @@
 //                        the S records in slice order and writes
 //                          C[t,n] = fp16((sum_s P_s[t,n]) * SCB[n]/127 + bias[n]).
 //
-// The tile counters and the words of the cooperative prologue carry the launch's epoch in
-// their upper 32 bits: a word of an earlier launch (or uninitialised memory) is claimed
-// afresh by the first update, and every word is put back to (epoch, 0) before the launch
-// ends, so the workspace needs no clearing between calls, graph replays included.
+// The tile counters and the words of the cooperative prologue carry the launch's epoch
+// (1 .. 2^32 - 1) in their upper 32 bits.  The host clears them (one memset) before every
+// launch, so no leftover bytes can carry this launch's epoch; the first update in the
+// launch claims a word, plain atomics follow, and every word is put back to (epoch, 0)
+// before the launch ends.
 #pragma once
 
 #include "common.cuh"
