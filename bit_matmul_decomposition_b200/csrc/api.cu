@@ -368,7 +368,7 @@ i8_status run_prepare(const void* X, int64_t T, int64_t K, float thr, uint32_t* 
   const size_t head = prepare_smem_bytes(K, 0, rows_per_cta);
   const size_t budget = static_cast<size_t>(d.prep_smem_max);
   if (head + 16 > budget) return I8_ERR_INVALID_ARG;
-  int64_t cache_rows = static_cast<int64_t>((budget - head) / (static_cast<size_t>(K) * 2));
+  int64_t cache_rows = static_cast<int64_t>((budget - head) / prepare_row_bytes(K));
   if (cache_rows > rows_per_cta) cache_rows = rows_per_cta;
   if (cache_rows * K * 2 > static_cast<int64_t>(kPrepChunk) * kPrepMaxChunks)
     cache_rows = static_cast<int64_t>(kPrepChunk) * kPrepMaxChunks / (K * 2);

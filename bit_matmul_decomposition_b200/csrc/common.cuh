@@ -245,14 +245,18 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-// Absmax code: round half away from zero of v = fl32(x * s), as truncation of
-// fl32(v + copysign(0.5, v)).  For |v| < 2^22 the sum is exact or its rounding cannot cross
-// an integer, except at |v| = 0.5 - 2^-25; an exhaustive search over every fp16 absmax and
-// every fp16 x near absmax/254 shows no input reaches that value.  |v| <= 127.0000077
+// Absmax code: round half away from zero of v = fl32(x * s), with no float-to-int
+// conversion.  For a = |v|, floor(fl_rz(a + 0.5)) = floor(a + 0.5): when a + 0.5 is an
+// integer it is representable, and otherwise rounding toward zero cannot cross the integer
+// below it.  For 0 <= b < 2^22, fl_rz(b + 1.5 * 2^23) = 1.5 * 2^23 + floor(b), so floor(b)
+// is that sum's bit pattern minus the pattern of 1.5 * 2^23.  |v| <= 127.0000077
 // (x = absmax gives the largest product), so the code never leaves [-127, 127].
 __device__ __forceinline__ int quant_code(float x, float s) {
   const float v = __fmul_rn(x, s);
-  return __float2int_rz(__fadd_rn(v, copysignf(0.5f, v)));
+  const float r = __fadd_rz(__fadd_rz(fabsf(v), 0.5f), 12582912.0f);
+  const int m = __float_as_int(r) - 0x4B400000;
+  const int sgn = __float_as_int(v) >> 31;  // 0, or -1 when v is negative
+  return (m ^ sgn) - sgn;
 }
 
 }  // namespace i8

@@ -283,6 +283,7 @@ constexpr int kPrepWarps = kPrepThreads / 32;
 constexpr int kPrepChunk = 32768;   // bytes per bulk copy of the row cache
 constexpr int kPrepMaxChunks = 8;
 constexpr int kPrepMaxIdx = 8192;    // outlier indices kept in shared memory
+constexpr int kSpecMinRows = 8;      // cached rows from which a CTA quantises early
 // Outlier cache header, 32-bit words: [0] valid, [1] n_o, [2] N, [3] K, [4..5] the CB
 // device pointer (low, high), [6..7] spare, then the ceil(K/32) mask words of the cached set.
 constexpr int kOcacheHdrWords = 8;
@@ -430,13 +431,15 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
   const int64_t words = (K + 31) / 32;
   const int64_t gpr = K / 8;  // 16-byte groups per row
   // shared memory: [row cache][mask words][prefix words + 1][first kPrepMaxIdx indices]
-  // [row scales]; indices past kPrepMaxIdx are found from the mask and its prefix
+  // [speculative row scales][speculative block maxima, 128 columns per block, cached rows];
+  // indices past kPrepMaxIdx are found from the mask and its prefix
   const size_t cache_bytes = static_cast<size_t>(p.cache_rows) * static_cast<size_t>(K) * 2;
   uint4* cache = reinterpret_cast<uint4*>(psm);
   uint32_t* smask = reinterpret_cast<uint32_t*>(psm + cache_bytes);
   int32_t* spre = reinterpret_cast<int32_t*>(smask + words);
   int32_t* sidx = spre + words + 1;
   float* samax = reinterpret_cast<float*>(sidx + kPrepMaxIdx);   // [rows_per_cta]
+  float* sbm = samax + p.rows_per_cta;                           // [cache_rows][nblk]
   __shared__ __align__(8) uint64_t s_bar[kPrepMaxChunks];
   __shared__ __align__(8) uint64_t s_rbar[kPrepWarps];  // phase 4 row buffers
   __shared__ int s_fail;
@@ -498,8 +501,59 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
       }
     }
   }
-  // cached rows: scan each chunk as it lands
-  {
+  // Cached rows.  A CTA that keeps at least kSpecMinRows rows in shared memory quantises
+  // them speculatively before the grid barrier: one warp per row, as soon as the chunks
+  // holding it have landed, scans the row (its outlier bits go into the CTA's mask), takes
+  // the largest |x| below the threshold per 128-column block and over the row, and writes
+  // the row's codes at that scale.  The final mask can only add columns in which this
+  // row's elements are below the threshold; phase 3 takes the true scale from the block
+  // maxima (re-reading only the blocks that hold outlier columns) and, when it is the
+  // speculative one, only clears the codes of the outlier columns.  Other CTAs scan each
+  // chunk as it lands and quantise in phase 3.
+  const bool spec = ncached >= kSpecMinRows;
+  const int nblk = static_cast<int>((gpr + 15) / 16);
+  if (spec) {
+    int no_abort = 0;
+    const int g32 = static_cast<int>(gpr);
+    const uint32_t cache_s = smem_u32(cache);
+    for (int64_t i = warp; i < ncached; i += kPrepWarps) {
+      const int c_first = static_cast<int>(i * K * 2 / kPrepChunk);
+      const int c_last = static_cast<int>(((i + 1) * K * 2 - 1) / kPrepChunk);
+      bool got = true;
+      for (int c = c_first; c <= c_last; ++c)
+        got = mbar_wait(smem_u32(&s_bar[c]), 0u, &no_abort, p.wait_limit_ns) && got;
+      if (!__all_sync(0xffffffffu, got)) {
+        if (lane == 0) s_fail = 1;
+        continue;
+      }
+      const uint32_t rbase = cache_s + static_cast<uint32_t>(i * gpr * 16);
+      float mrow = 0.0f;
+      for (int g0 = 0; g0 < g32; g0 += 32) {  // 32 groups: two blocks, one per half-warp
+        const int g = g0 + lane;
+        float m = 0.0f;
+        if (g < g32) {
+          const uint4 x = lds_v4(rbase + static_cast<uint32_t>(g) * 16u);
+          const uint32_t f = outlier_bits8(x, p.thr);
+          if (f) atomicOr(smask + (g >> 2), f << (8 * (g & 3)));
+          m = f ? absmax8(x, f) : absmax8_all(x);
+        }
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        if ((lane & 15) == 0 && g < g32) sbm[i * nblk + (g >> 4)] = m;
+        mrow = fmaxf(mrow, m);
+      }
+      mrow = fmaxf(mrow, __shfl_xor_sync(0xffffffffu, mrow, 16));
+      __syncwarp();  // every lane sees the row's own outlier bits in the mask
+      // codes at the speculative scale; columns already in the CTA's mask (the row's own
+      // outliers among them) get code 0, as every column of the final mask must
+      const float sc = mrow > 0.0f ? __fdiv_rn(code_max(p.e4m3), mrow) : 0.0f;
+      row_codes<true>(rbase, nullptr, reinterpret_cast<uint2*>(p.Xq + (r0 + i) * K), g32, lane,
+                      32, smask, sc, p.e4m3);
+      if (lane == 0) samax[i] = mrow;
+    }
+  } else {
     int no_abort = 0;
     for (int c = 0; c < nchunks; ++c) {
       const bool got = mbar_wait(smem_u32(&s_bar[c]), 0u, &no_abort, p.wait_limit_ns);
@@ -596,7 +650,6 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
       m &= m - 1u;
     }
   }
-  for (int64_t i = tid; i < nrows; i += kPrepThreads) samax[i] = 0.0f;
   __syncthreads();
   if (blockIdx.x == 0 && tid == 0) *p.n_o_out = n_o;
   auto idx_at = [&](int j) -> int64_t {
@@ -694,11 +747,30 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
       const int64_t t = r0 + i;
       const uint32_t sbase = cache_s + static_cast<uint32_t>(i * gpr * 16);
       const uint4* gbase = reinterpret_cast<const uint4*>(p.X + t * K);
+      const bool specrow = spec && cached;
       float amax = 0.0f;
-      if (cached)
+      if (specrow) {
+        // blocks free of outlier columns: their speculative maxima are exact; the others
+        // are read again without the outlier columns
+        for (int b = start; b < nblk; b += step) {
+          const int ga = b * 16, gb = min(ga + 16, g32);
+          bool dirty = false;
+          for (int g = ga; g < gb; g += 4) dirty = dirty || smask[g >> 2] != 0u;
+          if (!dirty) {
+            amax = fmaxf(amax, sbm[i * nblk + b]);
+          } else {
+            for (int g = ga; g < gb; ++g) {
+              const uint32_t k = scan_bits(smask, g);
+              const uint4 x = lds_v4(sbase + static_cast<uint32_t>(g) * 16u);
+              amax = fmaxf(amax, k ? absmax8(x, k) : absmax8_all(x));
+            }
+          }
+        }
+      } else if (cached) {
         amax = row_absmax<true>(sbase, gbase, g32, start, step, smask);
-      else if (have)
+      } else if (have) {
         amax = row_absmax<false>(sbase, gbase, g32, start, step, smask);
+      }
       amax = warp_max(amax);
       if (wpr > 1) {
         __syncthreads();
@@ -709,10 +781,15 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
       if (!have) continue;
       const float sc = amax > 0.0f ? __fdiv_rn(code_max(p.e4m3), amax) : 0.0f;
       uint2* qrow = reinterpret_cast<uint2*>(p.Xq + t * K);
-      if (cached)
+      if (specrow && amax == samax[i] && static_cast<int64_t>(n_o) * 8 <= K) {
+        // the speculative codes stand: clear those of the outlier columns
+        int8_t* qb = p.Xq + t * K;
+        for (int j = start; j < n_o; j += step) qb[idx_at(j)] = 0;
+      } else if (cached) {
         row_codes<true>(sbase, gbase, qrow, g32, start, step, smask, sc, p.e4m3);
-      else
+      } else {
         row_codes<false>(sbase, gbase, qrow, g32, start, step, smask, sc, p.e4m3);
+      }
       if (sub == 0 && lane == 0) p.SCx[t] = amax;
       // the row's outlier values into X_o, eight loads in flight before their stores
       const __half* xrow = cached ? reinterpret_cast<const __half*>(cache + i * gpr) : p.X + t * K;
@@ -988,11 +1065,17 @@ __global__ void __launch_bounds__(kWqThreads, 1) quantize_weight_kernel(const Wq
   }
 }
 
+// Shared-memory bytes per cached row of prepare_kernel: the row and its block maxima.
+__host__ inline size_t prepare_row_bytes(int64_t K) {
+  return static_cast<size_t>(K) * 2 + static_cast<size_t>((K + 127) / 128) * 4;
+}
+
 // Dynamic shared memory of prepare_kernel: a row cache of `cache_rows` rows, the mask,
-// its prefix, the first kPrepMaxIdx indices and one scale per row of the CTA's block.
+// its prefix, the first kPrepMaxIdx indices, one scale per row of the CTA's block and the
+// block maxima of the cached rows.
 __host__ inline size_t prepare_smem_bytes(int64_t K, int64_t cache_rows, int64_t rows_per_cta) {
   const int64_t words = (K + 31) / 32;
-  return static_cast<size_t>(cache_rows) * static_cast<size_t>(K) * 2 +
+  return static_cast<size_t>(cache_rows) * prepare_row_bytes(K) +
          static_cast<size_t>(2 * words + 1 + kPrepMaxIdx + rows_per_cta) * 4;
 }
 

@@ -70,6 +70,13 @@ SCAN_CASES = [
     (3000, 16384, (0, 9000, 16383), 0.0, 6.0),    # rows beyond the per-CTA cache
     (16, 14336, (100, 14000), 0.0, 6.0),
     (20, 10000, (), 0.0, 0.0),      # n_o = 10000: indices past the 8192 kept in shared memory
+    # >= 8 cached rows per CTA: rows quantised before the grid barrier.  Random outliers
+    # flag columns in which the other rows hold ordinary values, so some rows keep their
+    # early codes (outlier columns cleared) and others, whose largest value sits in such a
+    # column, are coded again; K = 2064 ends in a partial 128-column block
+    (2000, 2064, (5, 100, 2063), 5e-5, 6.0),
+    (1500, 1040, (), 0.0, math.inf),
+    (1400, 256, (3,), 0.0, 0.0),
 ]
 
 
@@ -162,6 +169,7 @@ FORWARD_CASES = [
     (300, 1040, 700, (0, 1, 2, 3, 4, 5, 6, 1039), 0.0, 6.0, True),      # n_o = 8
     (300, 1040, 700, (0, 1, 2, 3, 4, 5, 6, 7, 1039), 0.0, 6.0, True),   # n_o = 9
     (513, 4096, 1000, (77,), 0.0, 6.0, False),      # n_o = 1
+    (1500, 1040, 300, (7, 1039), 5e-5, 6.0, True),  # rows quantised before the grid barrier
 ]
 
 
