@@ -825,12 +825,20 @@ def main():
     ap.add_argument("--outlier-cache", action="store_true",
                     help="forward through i8_linear_forward_cached (the weight's outlier "
                          "columns kept across calls)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the workload's token count T (a smaller case of the same "
+                         "layer, e.g. for profiler captures); the line then names T")
     ap.add_argument("--mode", default="forward", choices=["forward", "train"],
                     help="train: one GPU, the fp16-weight training step of the module "
                          "front end (not the forward benchmark)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     w = workloads()[args.workload]
+    if args.tokens is not None:
+        import dataclasses
+        if args.tokens < 1:
+            raise SystemExit("--tokens must be positive")
+        w = dataclasses.replace(w, T=args.tokens, name="%s_T%d" % (w.name, args.tokens))
     if args.impl == "reference":
         return run_reference(args, w)
     if args.mode == "train":

@@ -25,6 +25,7 @@ _SZ = ctypes.c_size_t
 _ST = ctypes.c_int
 SIGNATURES = {
     "i8_status_string": (ctypes.c_char_p, [_ST]),
+    "i8_last_error": (ctypes.c_char_p, []),
     "i8_quantize_weight": (_ST, [_P, _I64, _I64, _P, _P, _P]),
     "i8_outlier_scan": (_ST, [_P, _I64, _I64, _F, _P, _P, _P, _P]),
     "i8_outlier_slice_elems": (_SZ, [_I64, _I64]),
@@ -54,9 +55,11 @@ SIGNATURES = {
 
 
 class I8Error(RuntimeError):
-    def __init__(self, fn, code):
-        super().__init__("%s returned %s" % (fn, STATUS.get(code, code)))
+    def __init__(self, fn, code, detail=""):
+        msg = "%s returned %s" % (fn, STATUS.get(code, code))
+        super().__init__(msg + (" (%s)" % detail if detail else ""))
         self.code = code
+        self.detail = detail
 
 
 _lib = None
@@ -79,7 +82,10 @@ def load(path: str = LIB_PATH):
 
 def _check(fn, code):
     if code != 0:
-        raise I8Error(fn, code)
+        detail = ""
+        if code == 3 and _lib is not None:   # I8_ERR_CUDA: which CUDA call failed
+            detail = (_lib.i8_last_error() or b"").decode("utf-8", "replace")
+        raise I8Error(fn, code, detail)
 
 
 def _ptr(t) -> Optional[int]:

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cstdio>
 #include <mutex>
 #include <utility>
 
@@ -22,6 +23,21 @@ using namespace i8;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s for every device-side wait
 constexpr int64_t kDecodeMaxT = 16;               // T <= 16 takes the decode kernel
 constexpr int kMaxDevices = 64;
+
+// ------------------------------------------------------------------ errors
+// The CUDA call behind the last I8_ERR_CUDA returned to this thread (i8_last_error()).
+thread_local char g_last_err[192] = "";
+
+void note_cuda(const char* what, int code, const char* name) {
+  snprintf(g_last_err, sizeof(g_last_err), "%s failed: %s (%d)", what, name, code);
+}
+
+// true when e is cudaSuccess; else records `what` and the error for i8_last_error()
+bool cuda_ok(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return true;
+  note_cuda(what, static_cast<int>(e), cudaGetErrorName(e));
+  return false;
+}
 
 // ------------------------------------------------------------------ device info
 struct DeviceInfo {
@@ -49,13 +65,22 @@ size_t p_smem_optin(int dev) {
 
 i8_status device_info(DeviceInfo** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return I8_ERR_CUDA;
+  if (!cuda_ok(cudaGetDevice(&dev), "cudaGetDevice")) return I8_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return I8_ERR_UNSUPPORTED;
+  // The driver calls of this library (the tensor-map encoder) need the device's context to
+  // be current in the calling thread; a thread in which no CUDA runtime has made it current
+  // yet (e.g. PyTorch's autograd worker thread) has none: make it current once per thread
+  // and device.
+  thread_local int ctx_dev = -1;
+  if (ctx_dev != dev) {
+    if (!cuda_ok(cudaSetDevice(dev), "cudaSetDevice")) return I8_ERR_CUDA;
+    ctx_dev = dev;
+  }
   std::lock_guard<std::mutex> lk(g_mu);
   DeviceInfo& d = g_dev[dev];
   if (!d.init) {
     cudaDeviceProp p;
-    if (cudaGetDeviceProperties(&p, dev) != cudaSuccess) return I8_ERR_CUDA;
+    if (!cuda_ok(cudaGetDeviceProperties(&p, dev), "cudaGetDeviceProperties")) return I8_ERR_CUDA;
     d.sm100 = (p.major == 10 && p.minor == 0);
     d.sms = p.multiProcessorCount;
     d.init = true;
@@ -63,49 +88,54 @@ i8_status device_info(DeviceInfo** out) {
   if (!d.sm100) return I8_ERR_UNSUPPORTED;
   if (!d.gemm_attr) {
     const int bytes = static_cast<int>(gemm::SMEM_BYTES);
-    if (cudaFuncSetAttribute(gemm::i8_gemm_tcgen05_kernel<false>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
-        cudaFuncSetAttribute(gemm::i8_gemm_tcgen05_kernel<true>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
-        cudaFuncSetAttribute(gemm::i8_gemm_tcgen05_kernel<false, true>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
-        cudaFuncSetAttribute(bwd::f16_gemm_kernel<false, true>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(bwd::SMEM_BYTES)) != cudaSuccess ||
-        cudaFuncSetAttribute(bwd::f16_gemm_kernel<true, true>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(bwd::SMEM_BYTES)) != cudaSuccess)
+    const int bwd_bytes = static_cast<int>(bwd::SMEM_BYTES);
+    const auto smem_attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
+    if (!cuda_ok(cudaFuncSetAttribute(gemm::i8_gemm_tcgen05_kernel<false>, smem_attr, bytes),
+                 "cudaFuncSetAttribute(gemm)") ||
+        !cuda_ok(cudaFuncSetAttribute(gemm::i8_gemm_tcgen05_kernel<true>, smem_attr, bytes),
+                 "cudaFuncSetAttribute(gemm raw)") ||
+        !cuda_ok(cudaFuncSetAttribute(gemm::i8_gemm_tcgen05_kernel<false, true>, smem_attr, bytes),
+                 "cudaFuncSetAttribute(gemm e4m3)") ||
+        !cuda_ok(cudaFuncSetAttribute(bwd::f16_gemm_kernel<false, true>, smem_attr, bwd_bytes),
+                 "cudaFuncSetAttribute(f16 gemm)") ||
+        !cuda_ok(cudaFuncSetAttribute(bwd::f16_gemm_kernel<true, true>, smem_attr, bwd_bytes),
+                 "cudaFuncSetAttribute(f16 gemm)"))
       return I8_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * d.sms, 1, 1);
     cfg.blockDim = dim3(gemm::THREADS, 1, 1);
     cfg.dynamicSmemBytes = gemm::SMEM_BYTES;
     int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, gemm::i8_gemm_tcgen05_kernel<false>, &cfg) !=
-            cudaSuccess ||
-        clusters < 1)
+    if (!cuda_ok(cudaOccupancyMaxActiveClusters(&clusters, gemm::i8_gemm_tcgen05_kernel<false>,
+                                                &cfg),
+                 "cudaOccupancyMaxActiveClusters(gemm)"))
       return I8_ERR_CUDA;
+    if (clusters < 1) return I8_ERR_UNSUPPORTED;
     d.gemm_clusters = clusters;
     cfg.dynamicSmemBytes = bwd::SMEM_BYTES;
     cfg.blockDim = dim3(bwd::THREADS, 1, 1);
     clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, bwd::f16_gemm_kernel<true, true>, &cfg) !=
-            cudaSuccess ||
-        clusters < 1)
+    if (!cuda_ok(cudaOccupancyMaxActiveClusters(&clusters, bwd::f16_gemm_kernel<true, true>, &cfg),
+                 "cudaOccupancyMaxActiveClusters(f16 gemm)"))
       return I8_ERR_CUDA;
+    if (clusters < 1) return I8_ERR_UNSUPPORTED;
     d.bwd_clusters = clusters;
     cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, prepare_kernel) != cudaSuccess) return I8_ERR_CUDA;
+    if (!cuda_ok(cudaFuncGetAttributes(&fa, prepare_kernel<false>), "cudaFuncGetAttributes"))
+      return I8_ERR_CUDA;
     const int prep_max =
         static_cast<int>(p_smem_optin(dev)) - static_cast<int>(fa.sharedSizeBytes) - 1024;
-    if (prep_max < 32 * 1024 ||
-        cudaFuncSetAttribute(prepare_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             prep_max) != cudaSuccess)
+    if (prep_max < 32 * 1024) return I8_ERR_UNSUPPORTED;
+    if (!cuda_ok(cudaFuncSetAttribute(prepare_kernel<false>, smem_attr, prep_max),
+                 "cudaFuncSetAttribute(prepare)") ||
+        !cuda_ok(cudaFuncSetAttribute(prepare_kernel<true>, smem_attr, prep_max),
+                 "cudaFuncSetAttribute(prepare e4m3)"))
       return I8_ERR_CUDA;
     d.prep_smem_max = prep_max;
     d.smem_optin = static_cast<int>(p_smem_optin(dev));
-    if (cudaFuncSetAttribute(quantize_weight_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kWqRingBytes)) != cudaSuccess)
+    if (!cuda_ok(cudaFuncSetAttribute(quantize_weight_kernel, smem_attr,
+                                      static_cast<int>(kWqRingBytes)),
+                 "cudaFuncSetAttribute(quantize_weight)"))
       return I8_ERR_CUDA;
     d.gemm_attr = true;
   }
@@ -142,7 +172,7 @@ bool shape_ok(int64_t T, int64_t K) {
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 i8_status launch_status() {
-  return cudaGetLastError() == cudaSuccess ? I8_OK : I8_ERR_CUDA;
+  return cuda_ok(cudaGetLastError(), "kernel launch") ? I8_OK : I8_ERR_CUDA;
 }
 
 size_t slice_elems(int64_t rows, int64_t K) {
@@ -155,7 +185,7 @@ size_t slice_elems(int64_t rows, int64_t K) {
 bool use_decode(int64_t T, int64_t K) { return T <= kDecodeMaxT && K <= gemv::MAX_K; }
 
 struct Workspace {
-  size_t mask, idx, n_o, sel, scx, xq, xo, cbo, rec, cnt, gmask, gscx, gbar, total;
+  size_t mask, idx, n_o, sel, scx, xq, xo, cbo, rec, cnt, gmask, gbm, gbar, total;
   int64_t zero_words;  // words from `mask` on that must be zero when a forward starts
 };
 
@@ -164,7 +194,7 @@ struct Workspace {
 // start of every forward.
 // Decode path: the slice records of every 32-row tile, then the control words -- the
 // tiles' arrival counters and the words of the cooperative prologue, contiguous from `cnt`
-// to `xq` -- which one memset clears at the start of every decode call.  The words carry
+// to the end -- which one memset clears at the start of every decode call.  The words carry
 // the launch's epoch in their upper half; a zero upper half never matches an epoch, so no
 // bytes left in the workspace by an earlier call of another shape or path, or by another
 // user of the memory, can pose as a counter of this launch.
@@ -182,9 +212,8 @@ Workspace layout(int64_t T, int64_t N, int64_t K, bool gemm_path = false) {
                  static_cast<size_t>(gemv::rec_bytes(T)));
     w.cnt = take(n_tiles * 8);
     w.gmask = take(static_cast<size_t>((K + 31) / 32) * 8);
-    w.gscx = take(static_cast<size_t>(T) * 8);
-    w.gbar = take(24);
-    w.xq = take(static_cast<size_t>(T) * static_cast<size_t>(K));
+    w.gbm = take(static_cast<size_t>(T) * static_cast<size_t>((K + gemv::XB - 1) / gemv::XB) * 8);
+    w.gbar = take(8);
     w.total = off;
     return w;
   }
@@ -224,6 +253,13 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// records a failed tensor-map encoding for i8_last_error()
+bool encoded(CUresult r) {
+  if (r == CUDA_SUCCESS) return true;
+  note_cuda("cuTensorMapEncodeTiled", static_cast<int>(r), "CUresult");
+  return false;
+}
+
 EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
   static std::once_flag once;
@@ -242,65 +278,77 @@ EncodeTiledFn encode_fn() {
 bool map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
             uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
   EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
+  if (!enc) {
+    note_cuda("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", 0, "not found");
+    return false;
+  }
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
-  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
+  return encoded(enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE));
 }
 
 // 2-D row-major uint8 tensor without swizzle (box inner extent up to 256 bytes).
 bool map_2d_plain(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
   EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
+  if (!enc) {
+    note_cuda("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", 0, "not found");
+    return false;
+  }
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+  return encoded(enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE));
 }
 
 // fp16 output C [rows, cols] for TMA stores of 32 x 32 boxes (cols % 8 == 0).
 bool map_c(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows) {
   EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
+  if (!enc) {
+    note_cuda("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", 0, "not found");
+    return false;
+  }
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
   cuuint32_t box[2] = {32, 32};
   cuuint32_t es[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, es,
+  return encoded(enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE));
 }
 
 // Chunk-major outlier slice [chunks][rows][64] fp16; box [1][box_rows][64].
 bool map_slice(CUtensorMap* m, const void* base, uint64_t rows, uint64_t chunks,
                uint32_t box_rows) {
   EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
+  if (!enc) {
+    note_cuda("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", 0, "not found");
+    return false;
+  }
   cuuint64_t dims[3] = {64, rows, chunks};
   cuuint64_t strides[2] = {128, rows * 128};
   cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+  return encoded(enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box,
              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE));
 }
 
 // ------------------------------------------------------------------ stage launchers
 i8_status run_scan(const void* X, int64_t T, int64_t K, float thr, uint32_t* mask, int32_t* idx,
                    int32_t* n_o, const DeviceInfo& d, cudaStream_t s) {
   const int64_t words = (K + 31) / 32;
-  if (cudaMemsetAsync(mask, 0, static_cast<size_t>(words) * 4, s) != cudaSuccess)
+  if (!cuda_ok(cudaMemsetAsync(mask, 0, static_cast<size_t>(words) * 4, s), "cudaMemsetAsync"))
     return I8_ERR_CUDA;
   const int64_t groups = K / 8;
   const int64_t gx = (groups + kScanThreads - 1) / kScanThreads;
@@ -344,7 +392,7 @@ i8_status run_quant_weight(const void* W, int64_t N, int64_t K, int8_t* CB, floa
   a.stages = (N + a.R - 1) / a.R;
   a.slots = wq_slots(K);
   a.wait_limit_ns = kWaitLimitNs;
-  const int64_t grid = a.stages < d.sms ? a.stages : d.sms;
+  const int64_t grid = a.stages < 2 * d.sms ? a.stages : 2 * d.sms;   // two CTAs per SM
   const size_t smem = static_cast<size_t>(a.slots) * static_cast<size_t>(a.R * K * 2);
   quantize_weight_kernel<<<static_cast<unsigned>(grid), kWqThreads, smem, s>>>(a);
   return launch_status();
@@ -361,7 +409,7 @@ i8_status run_prepare(const void* X, int64_t T, int64_t K, float thr, uint32_t* 
                       void* X_o, const int8_t* CB, int64_t N, void* CB_o, const DeviceInfo& d,
                       cudaStream_t s, uint8_t* ocache = nullptr, int64_t ocols = 0,
                       int32_t* cbo_sel = nullptr, bool e4m3 = false) {
-  if (cudaMemsetAsync(mask, 0, static_cast<size_t>(zero_words) * 4, s) != cudaSuccess)
+  if (!cuda_ok(cudaMemsetAsync(mask, 0, static_cast<size_t>(zero_words) * 4, s), "cudaMemsetAsync"))
     return I8_ERR_CUDA;
   const int64_t G0 = d.sms;
   const int64_t rows_per_cta = (T + G0 - 1) / G0;
@@ -374,10 +422,13 @@ i8_status run_prepare(const void* X, int64_t T, int64_t K, float thr, uint32_t* 
     cache_rows = static_cast<int64_t>(kPrepChunk) * kPrepMaxChunks / (K * 2);
   const size_t smem = prepare_smem_bytes(K, cache_rows, rows_per_cta);
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prepare_kernel, kPrepThreads,
-                                                    smem) != cudaSuccess ||
-      per_sm < 1)
+  const void* kernel = e4m3 ? reinterpret_cast<const void*>(prepare_kernel<true>)
+                            : reinterpret_cast<const void*>(prepare_kernel<false>);
+  if (!cuda_ok(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kPrepThreads,
+                                                             smem),
+               "cudaOccupancyMaxActiveBlocksPerMultiprocessor(prepare)"))
     return I8_ERR_CUDA;
+  if (per_sm < 1) return I8_ERR_INVALID_ARG;
   const int grid = d.sms;  // one CTA per SM: every CTA is resident for the grid barrier
   PrepArgs a;
   a.X = static_cast<const __half*>(X);
@@ -398,14 +449,13 @@ i8_status run_prepare(const void* X, int64_t T, int64_t K, float thr, uint32_t* 
       ocache ? reinterpret_cast<__half*>(ocache + ocache_header_bytes(K)) : nullptr;
   a.ocache_cols = ocache ? ocols : 0;
   a.cbo_sel = cbo_sel;
-  a.e4m3 = e4m3;
   a.rows_per_cta = rows_per_cta;
   a.cache_rows = cache_rows;
   a.cache_bytes_all = cache_rows * K * 2;
   a.wait_limit_ns = kWaitLimitNs;
   void* params[] = {&a};
-  if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(prepare_kernel), dim3(grid),
-                                  dim3(kPrepThreads), params, smem, s) != cudaSuccess)
+  if (!cuda_ok(cudaLaunchCooperativeKernel(kernel, dim3(grid),
+                                  dim3(kPrepThreads), params, smem, s), "cudaLaunchCooperativeKernel"))
     return I8_ERR_CUDA;
   return launch_status();
 }
@@ -467,7 +517,7 @@ i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t
   else
     e = launch_overlapped(gemm::i8_gemm_tcgen05_kernel<false>, dim3(2 * clusters),
                           dim3(gemm::THREADS), gemm::SMEM_BYTES, s, tA, tB, tAo, tBo, tBc, tC, a);
-  return e == cudaSuccess ? launch_status() : I8_ERR_CUDA;
+  return cuda_ok(e, "kernel launch") ? launch_status() : I8_ERR_CUDA;
 }
 
 // Backward fp16 GEMM: C[M, Nc] = sum_r A(m, r) B(n, r); a_mn / b_mn: the operand's rows run
@@ -509,15 +559,15 @@ i8_status run_f16_gemm(bool a_mn, const void* A, int64_t lda, bool b_mn, const v
                           dim3(bwd::THREADS), bwd::SMEM_BYTES, s, tA, tB, tC, a);
   else
     return I8_ERR_INVALID_ARG;
-  return e == cudaSuccess ? launch_status() : I8_ERR_CUDA;
+  return cuda_ok(e, "kernel launch") ? launch_status() : I8_ERR_CUDA;
 }
 
 // decode: one launch of the decode kernel (forward from X, or the raw product of codes)
 std::atomic<unsigned long long> g_epoch{0};
 
 // The prologue of the forward reads all of X in every CTA when X fits eight ring stages
-// (128 KB: ~1 us per stage, against ~12 us for the cooperative prologue's three grid
-// barriers); beyond that the CTAs split it (cooperative launch).
+// (128 KB, ~1 us per stage); beyond that the CTAs split the scan and meet at one grid
+// barrier (cooperative launch).
 bool decode_coop(bool raw, int64_t T, int64_t K) {
   return !raw && T * K * 2 > 8 * static_cast<int64_t>(gemv::STAGE_BYTES);
 }
@@ -531,8 +581,8 @@ i8_status run_decode(bool raw, const void* X, const int8_t* Xq, int64_t T, int64
   if (smem > static_cast<size_t>(d.smem_optin)) return I8_ERR_INVALID_ARG;
   CUtensorMap tCB;
   if (!map_2d_plain(&tCB, CB, K, N, K, gemv::BOXW, gemv::ROWS)) return I8_ERR_CUDA;
-  // the tile counters and the prologue's words (contiguous, cnt .. xq) start at zero
-  if (cudaMemsetAsync(ws + w.cnt, 0, w.xq - w.cnt, s) != cudaSuccess) return I8_ERR_CUDA;
+  // the tile counters and the prologue's words (contiguous from cnt) start at zero
+  if (!cuda_ok(cudaMemsetAsync(ws + w.cnt, 0, w.total - w.cnt, s), "cudaMemsetAsync")) return I8_ERR_CUDA;
   const int S = static_cast<int>(gemv::num_slices(K));
   int grid = (d.sms / S) * S;  // one CTA per SM, the same number of CTAs on every slice
   if (grid > 255) grid = (255 / S) * S;  // arrival counts are 8-bit
@@ -555,9 +605,8 @@ i8_status run_decode(bool raw, const void* X, const int8_t* Xq, int64_t T, int64
   a.lim = kWaitLimitNs;
   a.coop = decode_coop(raw, T, K);
   a.gmask = reinterpret_cast<unsigned long long*>(ws + w.gmask);
-  a.gscx = reinterpret_cast<unsigned long long*>(ws + w.gscx);
+  a.gbm = reinterpret_cast<unsigned long long*>(ws + w.gbm);
   a.gbar = reinterpret_cast<unsigned long long*>(ws + w.gbar);
-  a.xq = reinterpret_cast<int8_t*>(ws + w.xq);
   auto go = [&](auto kernel) -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -585,7 +634,7 @@ i8_status run_decode(bool raw, const void* X, const int8_t* Xq, int64_t T, int64
     e = raw ? go(gemv::decode_kernel<1, true>) : go(gemv::decode_kernel<1, false>);
   else
     e = raw ? go(gemv::decode_kernel<2, true>) : go(gemv::decode_kernel<2, false>);
-  return e == cudaSuccess ? launch_status() : I8_ERR_CUDA;
+  return cuda_ok(e, "kernel launch") ? launch_status() : I8_ERR_CUDA;
 }
 
 __global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
@@ -614,12 +663,13 @@ void* g_static_scratch_addr[kMaxDevices] = {};
 // Device address of g_static_scratch on the current device (looked up on first use).
 i8_status static_scratch_address(void** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return I8_ERR_CUDA;
+  if (!cuda_ok(cudaGetDevice(&dev), "cudaGetDevice")) return I8_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return I8_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_static_scratch_addr[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr)
+    if (!cuda_ok(cudaGetSymbolAddress(&p, g_static_scratch), "cudaGetSymbolAddress") ||
+        p == nullptr)
       return I8_ERR_CUDA;
     g_static_scratch_addr[dev] = p;
   }
@@ -649,11 +699,11 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   const bool prof = g_prof_start != nullptr && g_prof_stop != nullptr;
   if (!e4m3 && use_decode(T, K)) {
     // (the decode kernel takes the outlier columns' codes out of its own CB stream)
-    if (prof && cudaEventRecord(g_prof_start, s) != cudaSuccess) return I8_ERR_CUDA;
+    if (prof && !cuda_ok(cudaEventRecord(g_prof_start, s), "cudaEventRecord")) return I8_ERR_CUDA;
     st = run_decode(false, X, nullptr, T, K, CB, N, threshold, SCB, bias, C, nullptr, ws, w, *d,
                     s);
     if (st != I8_OK) return st;
-    if (prof && cudaEventRecord(g_prof_stop, s) != cudaSuccess) return I8_ERR_CUDA;
+    if (prof && !cuda_ok(cudaEventRecord(g_prof_stop, s), "cudaEventRecord")) return I8_ERR_CUDA;
     return I8_OK;
   }
   uint32_t* mask = reinterpret_cast<uint32_t*>(ws + w.mask);
@@ -667,11 +717,11 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
   st = run_prepare(X, T, K, threshold, mask, w.zero_words, idx, n_o, Xq, SCx, X_o, CB, N, CB_o,
                    *d, s, cache, ocols, sel, e4m3);
   if (st != I8_OK) return st;
-  if (prof && cudaEventRecord(g_prof_start, s) != cudaSuccess) return I8_ERR_CUDA;
+  if (prof && !cuda_ok(cudaEventRecord(g_prof_start, s), "cudaEventRecord")) return I8_ERR_CUDA;
   st = run_gemm(false, Xq, T, K, CB, N, X_o, CB_o, n_o, SCx, SCB, bias, C, nullptr, *d, s,
                 cache ? cache + ocache_header_bytes(K) : nullptr, ocols, sel, e4m3);
   if (st != I8_OK) return st;
-  if (prof && cudaEventRecord(g_prof_stop, s) != cudaSuccess) return I8_ERR_CUDA;
+  if (prof && !cuda_ok(cudaEventRecord(g_prof_stop, s), "cudaEventRecord")) return I8_ERR_CUDA;
   return I8_OK;
 }
 
@@ -679,6 +729,8 @@ i8_status forward_impl(const void* X, int64_t T, int64_t K, const int8_t* CB, co
 
 // ====================================================================== C ABI
 extern "C" {
+
+const char* i8_last_error(void) { return g_last_err; }
 
 const char* i8_status_string(i8_status s) {
   switch (s) {
@@ -916,13 +968,13 @@ i8_status i8_dequantize_weight_e4m3(const uint8_t* CB, const float* SCB, int64_t
 }
 
 i8_status i8_sync_status(void* stream) {
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return I8_ERR_CUDA;
+  if (!cuda_ok(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)), "cudaStreamSynchronize")) return I8_ERR_CUDA;
   unsigned int word = 0;
-  if (cudaMemcpyFromSymbol(&word, i8::g_error_word, sizeof(word)) != cudaSuccess)
+  if (!cuda_ok(cudaMemcpyFromSymbol(&word, i8::g_error_word, sizeof(word)), "cudaMemcpyFromSymbol"))
     return I8_ERR_CUDA;
   if (word == 0) return I8_OK;
   const unsigned int zero = 0;
-  if (cudaMemcpyToSymbol(i8::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return I8_ERR_CUDA;
+  if (!cuda_ok(cudaMemcpyToSymbol(i8::g_error_word, &zero, sizeof(zero)), "cudaMemcpyToSymbol")) return I8_ERR_CUDA;
   if (word & i8::kErrWaitTimeout) return I8_ERR_TIMEOUT;
   return I8_ERR_DEVICE;
 }

@@ -259,4 +259,15 @@ __device__ __forceinline__ int quant_code(float x, float s) {
   return (m ^ sgn) - sgn;
 }
 
+// The same code as a byte: the low byte of the result is quant_code(x, s) in two's
+// complement (the upper bytes are not part of it).  The pattern of 1.5 * 2^23 ends in a zero
+// byte and |code| <= 127, so the low byte of r's pattern is |code|; negating the whole word
+// negates its low byte modulo 256.
+__device__ __forceinline__ uint32_t quant_code_byte(float x, float s) {
+  const float v = __fmul_rn(x, s);
+  const float r = __fadd_rz(__fadd_rz(fabsf(v), 0.5f), 12582912.0f);
+  const uint32_t sgn = static_cast<uint32_t>(__float_as_int(v) >> 31);  // 0 or all ones
+  return (__float_as_uint(r) ^ sgn) - sgn;
+}
+
 }  // namespace i8

@@ -50,6 +50,8 @@ constexpr uint32_t IDESC_I8 = idesc_s8_s32(TM, TN);
 constexpr uint32_t IDESC_F16 = idesc_f16_f32(TM, TN);
 constexpr uint32_t IDESC_E4M3 = idesc_e4m3_f32(TM, TN);
 constexpr int INSERT_AT = 8;    // K-blocks of tile i+1 issued before the outlier MMAs of tile i
+                                // (at least; a quarter of the K-blocks in longer K-loops, so
+                                // that tile i's conversion has finished by then)
 constexpr int GROUP_M = 16;     // m-tiles per raster group (L2 reuse of Xq)
 constexpr int COL_BYTES = 2 * 2 * TN * 4;        // SCB/127 and bias as fp32, two buffers
 // fp16 output staging for the TMA stores of C: per epilogue warp two 32 x 32 blocks
@@ -294,7 +296,7 @@ __device__ __forceinline__ void store_row32_f16(__half* crow, int c0, int N, con
 // kind 2 / 3 marking the start / end of a tile's int8 phase (no ring stage).
 template <class F>
 __device__ __forceinline__ bool walk_schedule(int L, int KB, int OC, F&& visit) {
-  const int ins = KB < INSERT_AT ? KB : INSERT_AT;
+  const int ins = KB < INSERT_AT ? KB : (KB / 4 > INSERT_AT ? KB / 4 : INSERT_AT);
   for (int it = 0; it < L; ++it) {
     if (!visit(2, it, 0)) return false;
     for (int kb = 0; kb < KB; ++kb) {

@@ -18,9 +18,9 @@
 //                        the CTA's CB tiles, 32 rows x 512 B per stage (2-D boxes of
 //                        32 rows x 256 B).
 //   compute (8 warps)    the prologue, from the X pieces (every CTA reads all of X when it
-//                        fits two stages; otherwise the CTAs split the scan of X, combine
-//                        mask and row maxima in global memory and meet at two grid
-//                        barriers of a cooperative launch):
+//                        fits eight stages; otherwise the CTAs split the scan of X, combine
+//                        the mask and the block maxima in global memory and meet at one
+//                        grid barrier of a cooperative launch):
 //                          step 1: mask bit k = some row has |x| >= threshold, and the
 //                          largest |x| of every (row, 512-column block);
 //                          SCx[t] = max |x| over the non-outlier columns of row t (a block
@@ -44,9 +44,9 @@
 //
 // The tile counters and the words of the cooperative prologue carry the launch's epoch
 // (1 .. 2^32 - 1) in their upper 32 bits.  The host clears them (one memset) before every
-// launch, so no leftover bytes can carry this launch's epoch; the first update in the
-// launch claims a word, plain atomics follow, and every word is put back to (epoch, 0)
-// before the launch ends.
+// launch, so no leftover bytes can carry this launch's epoch: a counter is claimed by the
+// first update of the launch and plain atomics follow; mask and block-maximum words are
+// tagged and updated by the same OR / max.
 #pragma once
 
 #include "common.cuh"
@@ -165,13 +165,12 @@ struct Args {
   unsigned long long* cnt;   // [n_tiles] arrival counters (epoch << 32 | arrivals)
   unsigned long long epoch;  // this launch's epoch, 1 .. 2^32 - 1
   uint64_t lim;              // bound of every wait, ns
-  // cooperative prologue (larger X): the CTAs split the scan of X and meet at two grid
-  // barriers; the words carry the epoch in their upper 32 bits
+  // cooperative prologue (larger X): the CTAs split the scan of X and meet at one grid
+  // barrier; the words carry the epoch in their upper 32 bits and start at zero
   bool coop;
   unsigned long long* gmask;  // [ceil(K/32)] outlier mask words
-  unsigned long long* gscx;   // [T] row maxima (fp32 bit patterns)
-  unsigned long long* gbar;   // [3] barrier counters (epoch << 32 | arrivals)
-  int8_t* xq;                 // [T, K] codes, written in shares and read back per slice
+  unsigned long long* gbm;    // [T][ceil(K/512)] block maxima (fp16 |x| bit patterns)
+  unsigned long long* gbar;   // [1] barrier counter (epoch << 32 | arrivals)
 };
 
 __device__ __forceinline__ void mma_s8_16816(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -305,7 +304,6 @@ __device__ __forceinline__ bool forward_prologue(
 
   bool ok = true;
   const uint32_t e = static_cast<uint32_t>(a.epoch);
-  uint32_t goal3 = 0;  // cooperative path: third barrier, waited for after the tables below
   // One row: a column is an outlier column exactly when its one element reaches the
   // threshold, so the row maximum over the other columns is the largest |x| below the
   // threshold, taken in the same pass as the mask (no block maxima, no re-read).
@@ -383,65 +381,42 @@ __device__ __forceinline__ bool forward_prologue(
     compute_sync();
 
   } else {
-    // (a') the CTAs split X into shares of 16-byte groups.  Step 1: each ORs the outlier
-    // bits of its share into the global mask; grid barrier; each takes the masked maxima
-    // of its share into the global row maxima; grid barrier; step 2 on its share into the
-    // global codes; grid barrier; then this CTA's slice of the codes is copied into xs.
+    // (a') the CTAs split X into shares of 16-byte groups.  Each ORs the outlier bits of its
+    // share into the global mask and takes the maxima of its share into the global block
+    // maxima (words that start at zero: an OR or max with the epoch in the upper half both
+    // tags and updates them); one grid barrier; then every CTA copies the final mask and
+    // block maxima into shared memory, where they stand exactly as if the CTA had scanned
+    // all of X itself, and the rest of the prologue is the same for both paths.
     const int64_t TG = static_cast<int64_t>(T) * G;
     const int64_t f_lo = TG * blockIdx.x / gridDim.x, f_hi = TG * (blockIdx.x + 1) / gridDim.x;
-    // claim the barrier counters and the row-maximum words for this epoch now, while the
-    // scan's loads are in flight (every CTA does; all but the first claim of a word fail)
-    if (ct < 3)
-      tag_claim(a.gbar + ct, e);
-    else if (ct < 3 + T)
-      tag_claim(a.gscx + (ct - 3), e);
-    for (int64_t f = f_lo + ct; f < f_hi; f += CW * 32) {
-      const int64_t t = f / G, g = f - t * G;
-      const uint4 v = ldg_v4(X + t * K + g * 8);
-      if (half_bits_to_float(absmax8_bits(v)) >= thr) {
-        const uint32_t bits = outlier_bits8(v, thr);
-        if (bits) {
-          tag_claim(a.gmask + (g >> 2), e);
-          atomicOr(a.gmask + (g >> 2), static_cast<unsigned long long>(bits << (8 * (g & 3))));
+    const unsigned long long eh = static_cast<unsigned long long>(e) << 32;
+    if (ct == 0) tag_claim(a.gbar, e);   // while the scan's loads are in flight
+    for (int64_t f0 = f_lo + w * 32; f0 < f_hi; f0 += CW * 32) {
+      const int64_t f = f0 + lane;
+      const bool valid = f < f_hi;
+      uint32_t m = 0u, key = 0xffffffffu;
+      if (valid) {
+        const int64_t t = f / G, g = f - t * G;
+        const uint4 v = ldg_v4(X + t * K + g * 8);
+        m = absmax8_bits(v);
+        if (half_bits_to_float(m) >= thr) {
+          const uint32_t bits = outlier_bits8(v, thr);
+          if (bits) atomicOr(a.gmask + (g >> 2), eh | (bits << (8 * (g & 3))));
         }
+        key = static_cast<uint32_t>(t * NBK + g / GPB);
       }
+      const uint32_t peers = __match_any_sync(0xffffffffu, key);
+      const uint32_t mx = __reduce_max_sync(peers, m);
+      if (valid && lane == __ffs(peers) - 1) atomicMax(a.gbm + key, eh | mx);
     }
     compute_sync();
     if (ct == 0 && !grid_sync(a.gbar, e, gridDim.x, a.lim, true)) *abort_flag = 1;
     compute_sync();
     ok = *abort_flag == 0;
     for (int64_t x = ct; x < KW; x += CW * 32) maskall[x] = ok ? tagged_get(a.gmask + x, e) : 0u;
+    for (int64_t i = ct; i < static_cast<int64_t>(T) * NBK; i += CW * 32)
+      bm[i] = ok ? tagged_get(a.gbm + i, e) : 0u;
     compute_sync();
-    for (int64_t f = f_lo + ct; f < f_hi && ok; f += CW * 32) {
-      const int64_t t = f / G, g = f - t * G;
-      const uint4 v = ldg_v4(X + t * K + g * 8);
-      const uint32_t skip = (maskall[g >> 2] >> (8 * (g & 3))) & 0xffu;
-      atomicMax(&rmx[t], __float_as_uint(absmax8(v, skip)));
-    }
-    compute_sync();
-    for (int t = ct; t < T && ok; t += CW * 32) {
-      if (rmx[t] != 0u) atomicMax(a.gscx + t, (static_cast<unsigned long long>(e) << 32) | rmx[t]);
-    }
-    compute_sync();
-    if (ct == 0 && ok && !grid_sync(a.gbar + 1, e, gridDim.x, a.lim, true)) *abort_flag = 1;
-    compute_sync();
-    ok = *abort_flag == 0;
-    for (int t = ct; t < T; t += CW * 32) {
-      const float m = ok ? __uint_as_float(tagged_get(a.gscx + t, e)) : 0.0f;
-      scx[t] = m;
-      scale[t] = m > 0.0f ? __fdiv_rn(127.0f, m) : 0.0f;
-    }
-    compute_sync();
-    for (int64_t f = f_lo + ct; f < f_hi && ok; f += CW * 32) {
-      const int64_t t = f / G, g = f - t * G;
-      const uint4 v = ldg_v4(X + t * K + g * 8);
-      const uint32_t skip = (maskall[g >> 2] >> (8 * (g & 3))) & 0xffu;
-      *reinterpret_cast<uint2*>(a.xq + t * K + g * 8) = codes8(v, skip, scale[t]);
-    }
-    // the codes are read back by TMA (the async proxy) in other CTAs
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-    compute_sync();
-    if (ct == 0 && ok) goal3 = grid_arrive(a.gbar + 2, e, gridDim.x, true);
   }
 
   // (b) ranks: the compute threads take contiguous runs of mask words, and one block-wide
@@ -505,27 +480,7 @@ __device__ __forceinline__ bool forward_prologue(
     const int t = i / nf, j = i - t * nf;
     xo_s[t * MAXO + j] = X[static_cast<int64_t>(t) * K + idx_s[j]];
   }
-  if (a.coop) {
-    // the third barrier: every CTA's codes are in global memory
-    if (ct == 0 && ok && !grid_wait(a.gbar + 2, e, goal3, a.lim)) *abort_flag = 1;
-    if (ct == 0 && *abort_flag == 0) {
-      asm volatile("fence.proxy.async.global;" ::: "memory");
-      const int64_t k0 = static_cast<int64_t>(slice) * KS;
-      const int64_t klen = KS < K - k0 ? KS : K - k0;
-      mbar_arrive_expect_tx(smem_u32(xq_bar), static_cast<uint32_t>(T * klen));
-      for (int t = 0; t < T; ++t)
-        bulk_load(smem_u32(xs + t * pitch), a.xq + static_cast<int64_t>(t) * K + k0,
-                  static_cast<uint32_t>(klen), smem_u32(xq_bar));
-      // every CTA has read the mask and row maxima: CTA 0 puts them back to (epoch, 0)
-      if (blockIdx.x == 0) {
-        for (int64_t x = 0; x < KW; ++x) a.gmask[x] = static_cast<unsigned long long>(e) << 32;
-        for (int t = 0; t < T; ++t) a.gscx[t] = static_cast<unsigned long long>(e) << 32;
-      }
-    }
-    compute_sync();
-    ok = *abort_flag == 0;
-  }
-  if (!a.coop && !one_row) {
+  if (!one_row) {
     // blocks holding outlier columns (warp 1 lists them); the other blocks give their
     // maxima from (a)
     if (w == 1) {
@@ -602,18 +557,15 @@ __device__ __forceinline__ bool forward_prologue(
     }
   }
   compute_sync();
-  if (!a.coop) {  // (the cooperative path has SCx from (a'))
-    for (int t = ct; t < T; t += CW * 32) {
-      const float m = __uint_as_float(rmx[t]);
-      scx[t] = m;
-      scale[t] = m > 0.0f ? __fdiv_rn(127.0f, m) : 0.0f;
-    }
+  for (int t = ct; t < T; t += CW * 32) {
+    const float m = __uint_as_float(rmx[t]);
+    scx[t] = m;
+    scale[t] = m > 0.0f ? __fdiv_rn(127.0f, m) : 0.0f;
   }
   compute_sync();
 
-  // (d) step 2 on this slice: one ring stage per row of X (the cooperative path has its
-  // codes from (a') already)
-  if (!a.coop) {
+  // (d) step 2 on this slice: one ring stage per row of X
+  {
     const int64_t k0 = static_cast<int64_t>(slice) * KS;
     const int64_t klen = KS < K - k0 ? KS : K - k0;
     const int64_t gl = klen / 8;
@@ -851,7 +803,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           bulk_load(ring + s * STAGE_BYTES, xb + off, bytes, fb);
           advance();
         }
-        for (int tt = 0; tt < T && ok && !a.coop; ++tt) {
+        for (int tt = 0; tt < T && ok; ++tt) {
           const int t = (tt + cta_in_slice) % T;
           const uint32_t fb = acquire(static_cast<uint32_t>(klen * 2));
           if (!fb) {
@@ -926,10 +878,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         ok = forward_prologue<NT>(a, threadIdx.x, slice, KS, S, rg, ring_p, xs, pitch, maskall,
                                   spre, bm, dl, rmx, idx_s, jinfo, xo_s, scx, scale, jbase, misc,
                                   xq_bar, abort_flag);
-        if (a.coop && ok) {
-          const bool got = mbar_wait(smem_u32(xq_bar), 0u, abort_flag, a.lim);
-          ok = __all_sync(0xffffffffu, got);
-        }
       }
     }
     all_sync();

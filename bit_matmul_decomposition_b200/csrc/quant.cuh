@@ -53,6 +53,22 @@ __device__ __forceinline__ uint32_t outlier_bits8(const uint4 v, float thr) {
   return b;
 }
 
+// Largest |x| of 8 fp16 values, as a float (exact: the fp16 maximum of the absolute values).
+__device__ __forceinline__ float group_absmax(const uint4 v) {
+  const __half2 a = __habs2(*reinterpret_cast<const __half2*>(&v.x));
+  const __half2 b = __habs2(*reinterpret_cast<const __half2*>(&v.y));
+  const __half2 c = __habs2(*reinterpret_cast<const __half2*>(&v.z));
+  const __half2 d = __habs2(*reinterpret_cast<const __half2*>(&v.w));
+  const __half2 m = __hmax2(__hmax2(a, b), __hmax2(c, d));
+  return fmaxf(__low2float(m), __high2float(m));
+}
+
+// outlier_bits8 through the group's maximum first: most groups hold no value at the
+// threshold and cost a few packed fp16 instructions.
+__device__ __forceinline__ uint32_t outlier_bits8_fast(const uint4 v, float thr) {
+  return group_absmax(v) >= thr ? outlier_bits8(v, thr) : 0u;
+}
+
 // ------------------------------------------------------------------ step 1: scan
 constexpr int kScanThreads = 256;
 
@@ -73,9 +89,9 @@ __global__ void __launch_bounds__(kScanThreads)
 #pragma unroll
       for (int u = 0; u < 4; ++u) v[u] = ldg_v4(base + (r + u) * groups);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) bits |= outlier_bits8(v[u], thr);
+      for (int u = 0; u < 4; ++u) bits |= outlier_bits8_fast(v[u], thr);
     }
-    for (; r < r1; ++r) bits |= outlier_bits8(ldg_v4(base + r * groups), thr);
+    for (; r < r1; ++r) bits |= outlier_bits8_fast(ldg_v4(base + r * groups), thr);
   }
   // four consecutive threads hold the 32 bits of one mask word
   uint32_t word = bits << (8 * (threadIdx.x & 3));
@@ -146,18 +162,22 @@ __device__ __forceinline__ float absmax8(const uint4 v, uint32_t skip) {
   return m;
 }
 
+// int8 codes of 8 fp16 values (element i at the i-th lowest address) at scale s; excluded
+// columns (skip bit i) give code 0.  Byte permutes gather the codes' low bytes.
 __device__ __forceinline__ uint2 codes8(const uint4 v, uint32_t skip, float s) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t out[2] = {0u, 0u};
+  uint32_t c[8];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    float2 f = h2f2(w[i]);
-    int c0 = ((skip >> (2 * i)) & 1u) ? 0 : quant_code(f.x, s);
-    int c1 = ((skip >> (2 * i + 1)) & 1u) ? 0 : quant_code(f.y, s);
-    uint32_t pair = (static_cast<uint32_t>(c0) & 0xffu) | ((static_cast<uint32_t>(c1) & 0xffu) << 8);
-    out[i >> 1] |= pair << (16 * (i & 1));
+    const float2 f = h2f2(w[i]);
+    c[2 * i] = ((skip >> (2 * i)) & 1u) ? 0u : quant_code_byte(f.x, s);
+    c[2 * i + 1] = ((skip >> (2 * i + 1)) & 1u) ? 0u : quant_code_byte(f.y, s);
   }
-  return make_uint2(out[0], out[1]);
+  const uint32_t lo = __byte_perm(__byte_perm(c[0], c[1], 0x0040), __byte_perm(c[2], c[3], 0x0040),
+                                  0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(c[4], c[5], 0x0040), __byte_perm(c[6], c[7], 0x0040),
+                                  0x5410);
+  return make_uint2(lo, hi);
 }
 
 // e4m3 variant: the codes of 8 fp16 values are the e4m3 roundings (nearest, ties to even;
@@ -308,7 +328,6 @@ struct PrepArgs {
   __half* ocache_CB_o;    // chunk-major slice [ocache_cols / 64][N][64]
   int64_t ocache_cols;    // capacity in columns, a multiple of 64
   int32_t* cbo_sel;       // out (may be NULL): 1 when this call's CB_o is the cache's slice
-  bool e4m3;              // codes in e4m3 (scale 448 / absmax) instead of int8
   int64_t rows_per_cta;
   int64_t cache_rows;     // rows of its block each CTA keeps in shared memory
   int64_t cache_bytes_all; // size of the row-cache region (reused by phase 4)
@@ -425,6 +444,9 @@ __device__ __forceinline__ int32_t nth_outlier(const uint32_t* smask, const int3
   return static_cast<int32_t>(lo * 32 + (__ffs(m) - 1));
 }
 
+// kE4M3: e4m3 codes (scale 448 / absmax) instead of int8 (the layer's code format, fixed at
+// compile time so that each variant carries only its own code path).
+template <bool kE4M3>
 __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs p) {
   extern __shared__ __align__(128) uint8_t psm[];
   const int64_t K = p.K;
@@ -486,7 +508,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
       for (int u = 0; u < 4; ++u) x[u] = ldg_v4(src + v + u * kPrepThreads);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const uint32_t f = outlier_bits8(x[u], p.thr);
+        const uint32_t f = outlier_bits8_fast(x[u], p.thr);
         if (f) {
           const int64_t g = (v + u * kPrepThreads) % gpr;
           atomicOr(smask + (g >> 2), f << (8 * (g & 3)));
@@ -494,7 +516,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
       }
     }
     for (; v < nvec; v += kPrepThreads) {
-      const uint32_t f = outlier_bits8(ldg_v4(src + v), p.thr);
+      const uint32_t f = outlier_bits8_fast(ldg_v4(src + v), p.thr);
       if (f) {
         const int64_t g = v % gpr;
         atomicOr(smask + (g >> 2), f << (8 * (g & 3)));
@@ -533,9 +555,12 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
         float m = 0.0f;
         if (g < g32) {
           const uint4 x = lds_v4(rbase + static_cast<uint32_t>(g) * 16u);
-          const uint32_t f = outlier_bits8(x, p.thr);
-          if (f) atomicOr(smask + (g >> 2), f << (8 * (g & 3)));
-          m = f ? absmax8(x, f) : absmax8_all(x);
+          m = group_absmax(x);
+          if (m >= p.thr) {   // rare: a value at the threshold in this group
+            const uint32_t f = outlier_bits8(x, p.thr);
+            atomicOr(smask + (g >> 2), f << (8 * (g & 3)));
+            m = absmax8(x, f);
+          }
         }
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
@@ -548,9 +573,9 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
       __syncwarp();  // every lane sees the row's own outlier bits in the mask
       // codes at the speculative scale; columns already in the CTA's mask (the row's own
       // outliers among them) get code 0, as every column of the final mask must
-      const float sc = mrow > 0.0f ? __fdiv_rn(code_max(p.e4m3), mrow) : 0.0f;
+      const float sc = mrow > 0.0f ? __fdiv_rn(code_max(kE4M3), mrow) : 0.0f;
       row_codes<true>(rbase, nullptr, reinterpret_cast<uint2*>(p.Xq + (r0 + i) * K), g32, lane,
-                      32, smask, sc, p.e4m3);
+                      32, smask, sc, kE4M3);
       if (lane == 0) samax[i] = mrow;
     }
   } else {
@@ -561,7 +586,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
       const int64_t v0 = static_cast<int64_t>(c) * (kPrepChunk / 16);
       const int64_t v1 = min(v0 + static_cast<int64_t>(kPrepChunk / 16), cbytes / 16);
       for (int64_t v = v0 + tid; v < v1; v += kPrepThreads) {
-        const uint32_t f = got ? outlier_bits8(cache[v], p.thr) : 0u;
+        const uint32_t f = got ? outlier_bits8_fast(cache[v], p.thr) : 0u;
         if (f) {
           const int64_t g = v % gpr;
           atomicOr(smask + (g >> 2), f << (8 * (g & 3)));
@@ -718,7 +743,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
       if (it < items4) {
         const int64_t c = it / p.N, n = it - c * p.N;
         reinterpret_cast<__half2*>(cbo + (c * p.N + n) * 64)[lane] =
-            __halves2half2(code_to_half(v0[u], p.e4m3), code_to_half(v1[u], p.e4m3));
+            __halves2half2(code_to_half(v0[u], kE4M3), code_to_half(v1[u], kE4M3));
       }
     }
   };
@@ -779,16 +804,16 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
         for (int w2 = 0; w2 < wpr; ++w2) amax = fmaxf(amax, s_red[rr * wpr + w2]);
       }
       if (!have) continue;
-      const float sc = amax > 0.0f ? __fdiv_rn(code_max(p.e4m3), amax) : 0.0f;
+      const float sc = amax > 0.0f ? __fdiv_rn(code_max(kE4M3), amax) : 0.0f;
       uint2* qrow = reinterpret_cast<uint2*>(p.Xq + t * K);
       if (specrow && amax == samax[i] && static_cast<int64_t>(n_o) * 8 <= K) {
         // the speculative codes stand: clear those of the outlier columns
         int8_t* qb = p.Xq + t * K;
         for (int j = start; j < n_o; j += step) qb[idx_at(j)] = 0;
       } else if (cached) {
-        row_codes<true>(sbase, gbase, qrow, g32, start, step, smask, sc, p.e4m3);
+        row_codes<true>(sbase, gbase, qrow, g32, start, step, smask, sc, kE4M3);
       } else {
-        row_codes<false>(sbase, gbase, qrow, g32, start, step, smask, sc, p.e4m3);
+        row_codes<false>(sbase, gbase, qrow, g32, start, step, smask, sc, kE4M3);
       }
       if (sub == 0 && lane == 0) p.SCx[t] = amax;
       // the row's outlier values into X_o, eight loads in flight before their stores
@@ -850,7 +875,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
             for (int u = 0; u < 4; ++u)
               if (c0 + u < chunks)
                 reinterpret_cast<__half2*>(cbo + ((c0 + u) * p.N + n) * 64)[lane] =
-                    __halves2half2(code_to_half(v0[u], p.e4m3), code_to_half(v1[u], p.e4m3));
+                    __halves2half2(code_to_half(v0[u], kE4M3), code_to_half(v1[u], kE4M3));
           }
           __syncwarp();
         }
@@ -906,14 +931,15 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
 // shared-memory slots with one bulk (TMA) copy, so that several stages per SM are always
 // in flight; 8 consumer warps take each row's absmax and write its codes and scale from
 // shared memory: a warp per row when R >= 8, else 8 / R warps per row, combining their
-// maxima through shared memory.  Codes and scales are those of quantize_rows_kernel with no
+// maxima through shared memory.  Two CTAs share an SM, so that one CTA's barriers and
+// latencies overlap the other's work.  Codes and scales are those of quantize_rows_kernel with no
 // excluded column.
 constexpr int kWqWarps = 8;                            // consumer warps
 constexpr int kWqThreads = (kWqWarps + 1) * 32;        // + the producer warp
 constexpr int64_t kWqStageTarget = 32768;              // bytes per stage (at most)
-constexpr int64_t kWqRingBytes = 196608;               // shared-memory ring (at most)
+constexpr int64_t kWqRingBytes = 98304;                // shared-memory ring (at most)
 constexpr int kWqMaxSlots = 8;
-constexpr int64_t kWqMaxRowBytes = 65536;              // longer rows: quantize_rows_kernel
+constexpr int64_t kWqMaxRowBytes = 32768;              // longer rows: quantize_rows_kernel
 
 struct WqArgs {
   const __half* W;
@@ -957,7 +983,7 @@ __device__ __forceinline__ bool wq_consumers_all(bool v) {
   return r != 0;
 }
 
-__global__ void __launch_bounds__(kWqThreads, 1) quantize_weight_kernel(const WqArgs a) {
+__global__ void __launch_bounds__(kWqThreads, 2) quantize_weight_kernel(const WqArgs a) {
   extern __shared__ __align__(128) uint8_t wsm[];
   __shared__ __align__(8) uint64_t full[kWqMaxSlots];
   __shared__ __align__(8) uint64_t empty[kWqMaxSlots];

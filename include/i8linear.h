@@ -55,6 +55,12 @@ typedef enum i8_status {
 /* Human-readable name of a status code (static storage). */
 const char* i8_status_string(i8_status s);
 
+/* After a call returned I8_ERR_CUDA to this host thread: which CUDA runtime or driver call
+ * failed and with which error, e.g. "kernel launch failed: cudaErrorInvalidValue (1)".
+ * Empty before any such failure; kept until the next one in the same thread.  Thread-local
+ * storage owned by the library: valid until this thread's next library call. */
+const char* i8_last_error(void);
+
 /*
  * Step 3 -- per-output-channel weight quantisation, run once per weight.
  * Source: "用法" (usage) section -- the weight is quantised when the module moves to the

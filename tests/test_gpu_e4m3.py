@@ -106,6 +106,8 @@ FORWARD_CASES = [
     (64, 208, 256, (9,), 0.0, 0.0, True),           # thr 0: only the fp16 product
     (200, 128, 100, (1, 2, 3), 0.0, 6.0, False),
     (40, 9216, 96, (), 0.0, 0.0, True),             # n_o = 9216 (> 8192 kept indices)
+    (300, 1040, 700, (0, 1, 2, 3, 4, 5, 6, 1039), 0.0, 6.0, True),     # n_o = 8
+    (300, 1040, 700, (0, 1, 2, 3, 4, 5, 6, 7, 1039), 0.0, 6.0, True),  # n_o = 9
 ]
 
 

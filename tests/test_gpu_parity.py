@@ -169,6 +169,9 @@ FORWARD_CASES = [
     (300, 1040, 700, (0, 1, 2, 3, 4, 5, 6, 1039), 0.0, 6.0, True),      # n_o = 8
     (300, 1040, 700, (0, 1, 2, 3, 4, 5, 6, 7, 1039), 0.0, 6.0, True),   # n_o = 9
     (513, 4096, 1000, (77,), 0.0, 6.0, False),      # n_o = 1
+    # few outlier columns with N not a multiple of 8 (stores from registers instead of
+    # TMA), with bias
+    (257, 512, 1001, (3, 400), 0.0, 6.0, True),
     (1500, 1040, 300, (7, 1039), 5e-5, 6.0, True),  # rows quantised before the grid barrier
 ]
 

@@ -1,9 +1,11 @@
 """The kernels round an absmax code without a float-to-int conversion: with
 v = fl32(x * fl32(127 / absmax)) and a = |v|, the code's magnitude is
 floor(fl_rz(a + 0.5)), read from the bit pattern of fl_rz(fl_rz(a + 0.5) + 1.5 * 2^23).
-These checks show, on the CPU with IEEE round-toward-zero additions, that this equals the
-oracle's roundf (round half away from zero) for every fp32 value the product can take, and
-that no code needs a clamp."""
+The byte form the kernels store applies the sign by negating the whole 32-bit pattern:
+the low byte of (pattern ^ s) - s, s = 0 or all ones by the sign of v, is the code in two's
+complement.  These checks show, on the CPU with IEEE round-toward-zero additions, that both
+equal the oracle's roundf (round half away from zero) for every fp32 value the product can
+take, of either sign, and that no code needs a clamp."""
 import subprocess
 
 import numpy as np
@@ -31,6 +33,14 @@ int main(void) {
         uint32_t tb;
         memcpy(&tb, &tt, 4);
         if ((int)tb - 0x4B400000 != (int)roundf(a)) ++bad;
+        /* the stored byte, for +a and for -a (codes fit a byte for |v| < 127.5; the
+           products stay below 127.0000077) */
+        for (int neg = 0; neg < 2 && a < 127.5f; ++neg) {
+            uint32_t s = neg ? 0xFFFFFFFFu : 0u;
+            uint8_t byte = (uint8_t)((tb ^ s) - s);
+            int want = (int)roundf(neg ? -a : a);
+            if ((int8_t)byte != want) ++bad;
+        }
     }
     printf("%llu\n", bad);
     return bad != 0;
