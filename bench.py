@@ -236,7 +236,7 @@ def traffic_record(kernel, workload):
 
 def source_hash():
     h = hashlib.sha256()
-    for f in ("api.cu", "common.cuh", "quant.cuh", "gemm.cuh", "gemv.cuh", "bwd.cuh"):
+    for f in ("api.cu", "common.cuh", "quant.cuh", "gemm.cuh", "gemm_wide.cuh", "gemv.cuh", "bwd.cuh"):
         with open(os.path.join(ROOT, "bit_matmul_decomposition_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()

@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libi8linear.so")
-SOURCES = ["api.cu", "common.cuh", "quant.cuh", "gemm.cuh", "gemv.cuh", "bwd.cuh"]
+SOURCES = ["api.cu", "common.cuh", "quant.cuh", "gemm.cuh", "gemm_wide.cuh", "gemv.cuh", "bwd.cuh"]
 HEADER = os.path.join(ROOT, "include", "i8linear.h")
 
 NVCC_FLAGS = [

@@ -13,6 +13,7 @@
 #include "bwd.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
+#include "gemm_wide.cuh"
 #include "gemv.cuh"
 #include "quant.cuh"
 
@@ -22,6 +23,7 @@ using namespace i8;
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s for every device-side wait
 constexpr int64_t kDecodeMaxT = 16;               // T <= 16 takes the decode kernel
+constexpr int64_t kWideMinK = 8192;               // K from which the 256 x 512 GEMM is used
 constexpr int kMaxDevices = 64;
 
 // ------------------------------------------------------------------ errors
@@ -46,6 +48,7 @@ struct DeviceInfo {
   int sms = 0;
   bool gemm_attr = false;
   int gemm_clusters = 0;  // co-resident CTA pairs of the GEMM kernel
+  int wide_clusters = 0;  // co-resident CTA pairs of the 256 x 512 GEMM kernel
   int bwd_clusters = 0;   // co-resident CTA pairs of the backward fp16 GEMM
   int prep_smem_max = 0;  // dynamic shared memory granted to prepare_kernel
   int smem_optin = 0;     // largest dynamic shared memory a kernel may opt in to
@@ -98,6 +101,12 @@ i8_status device_info(DeviceInfo** out) {
                  "cudaFuncSetAttribute(gemm e4m3)") ||
         !cuda_ok(cudaFuncSetAttribute(bwd::f16_gemm_kernel<false, true>, smem_attr, bwd_bytes),
                  "cudaFuncSetAttribute(f16 gemm)") ||
+        !cuda_ok(cudaFuncSetAttribute(gemmw::i8_gemm_wide_kernel<false>, smem_attr,
+                                      static_cast<int>(gemmw::SMEM_BYTES)),
+                 "cudaFuncSetAttribute(wide gemm)") ||
+        !cuda_ok(cudaFuncSetAttribute(gemmw::i8_gemm_wide_kernel<true>, smem_attr,
+                                      static_cast<int>(gemmw::SMEM_BYTES)),
+                 "cudaFuncSetAttribute(wide gemm e4m3)") ||
         !cuda_ok(cudaFuncSetAttribute(bwd::f16_gemm_kernel<true, true>, smem_attr, bwd_bytes),
                  "cudaFuncSetAttribute(f16 gemm)"))
       return I8_ERR_CUDA;
@@ -120,6 +129,15 @@ i8_status device_info(DeviceInfo** out) {
       return I8_ERR_CUDA;
     if (clusters < 1) return I8_ERR_UNSUPPORTED;
     d.bwd_clusters = clusters;
+    cfg.dynamicSmemBytes = gemmw::SMEM_BYTES;
+    cfg.blockDim = dim3(gemmw::THREADS, 1, 1);
+    clusters = 0;
+    if (!cuda_ok(cudaOccupancyMaxActiveClusters(&clusters, gemmw::i8_gemm_wide_kernel<false>,
+                                                &cfg),
+                 "cudaOccupancyMaxActiveClusters(wide gemm)"))
+      return I8_ERR_CUDA;
+    if (clusters < 1) return I8_ERR_UNSUPPORTED;
+    d.wide_clusters = clusters;
     cudaFuncAttributes fa;
     if (!cuda_ok(cudaFuncGetAttributes(&fa, prepare_kernel<false>), "cudaFuncGetAttributes"))
       return I8_ERR_CUDA;
@@ -288,24 +306,6 @@ bool map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t i
   cuuint32_t es[2] = {1, 1};
   return encoded(enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE));
-}
-
-// 2-D row-major uint8 tensor without swizzle (box inner extent up to 256 bytes).
-bool map_2d_plain(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
-                  uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) {
-    note_cuda("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", 0, "not found");
-    return false;
-  }
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {row_bytes};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t es[2] = {1, 1};
-  return encoded(enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE));
 }
@@ -505,6 +505,23 @@ i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t
   a.acc_out = acc;
   a.c_tma = c_tma;
   a.wait_limit_ns = kWaitLimitNs;
+  // Long K-loops with enough tiles to fill the GPU several times take the 256 x 512 tiles
+  // (a quarter less operand feed per multiply-add; the epilogue is not overlapped, which
+  // a long K-loop hides).
+  const int64_t m_tiles = a.m_tiles;
+  const int64_t wide_tiles = m_tiles * ((N + gemmw::TN - 1) / gemmw::TN);
+  if (!raw && K >= kWideMinK && wide_tiles >= 4 * static_cast<int64_t>(d.wide_clusters)) {
+    a.n_tiles = static_cast<int>((N + gemmw::TN - 1) / gemmw::TN);
+    const int wc = static_cast<int>(wide_tiles < d.wide_clusters ? wide_tiles : d.wide_clusters);
+    const cudaError_t e =
+        e4m3 ? launch_overlapped(gemmw::i8_gemm_wide_kernel<true>, dim3(2 * wc),
+                                 dim3(gemmw::THREADS), gemmw::SMEM_BYTES, s, tA, tB, tAo, tBo,
+                                 tBc, tC, a)
+             : launch_overlapped(gemmw::i8_gemm_wide_kernel<false>, dim3(2 * wc),
+                                 dim3(gemmw::THREADS), gemmw::SMEM_BYTES, s, tA, tB, tAo, tBo,
+                                 tBc, tC, a);
+    return cuda_ok(e, "kernel launch") ? launch_status() : I8_ERR_CUDA;
+  }
   const int64_t tiles = static_cast<int64_t>(a.m_tiles) * a.n_tiles;
   const int clusters = static_cast<int>(tiles < d.gemm_clusters ? tiles : d.gemm_clusters);
   cudaError_t e;
@@ -580,7 +597,8 @@ i8_status run_decode(bool raw, const void* X, const int8_t* Xq, int64_t T, int64
   const size_t smem = gemv::smem_bytes(nt, K);
   if (smem > static_cast<size_t>(d.smem_optin)) return I8_ERR_INVALID_ARG;
   CUtensorMap tCB;
-  if (!map_2d_plain(&tCB, CB, K, N, K, gemv::BOXW, gemv::ROWS)) return I8_ERR_CUDA;
+  if (!map_2d(&tCB, CU_TENSOR_MAP_DATA_TYPE_UINT8, CB, K, N, K, gemv::BOXW, gemv::ROWS))
+    return I8_ERR_CUDA;
   // the tile counters and the prologue's words (contiguous from cnt) start at zero
   if (!cuda_ok(cudaMemsetAsync(ws + w.cnt, 0, w.total - w.cnt, s), "cudaMemsetAsync")) return I8_ERR_CUDA;
   const int S = static_cast<int>(gemv::num_slices(K));

@@ -16,7 +16,9 @@
 //                        every other load waits in): first (forward only)
 //                        all of X in 16 KB pieces, then this slice of every row of X, then
 //                        the CTA's CB tiles, 32 rows x 512 B per stage (2-D boxes of
-//                        32 rows x 256 B).
+//                        32 rows x 128 B, 128-byte swizzle: chunk j of row r lands in chunk
+//                        j ^ (r % 8), so the eight rows of an ldmatrix phase hit eight
+//                        different bank groups).
 //   compute (8 warps)    the prologue, from the X pieces (every CTA reads all of X when it
 //                        fits eight stages; otherwise the CTAs split the scan of X, combine
 //                        the mask and the block maxima in global memory and meet at one
@@ -29,7 +31,8 @@
 //                          step 2 on the slice rows: Xq = round(x * fl32(127/SCx)) (half
 //                          away from zero), outlier columns 0, into shared memory;
 //                        then per CB stage each warp one 64-byte step of K for all 32 rows
-//                        (mma.sync m16n8k32 s8: two 16-row groups x 8 tokens), copying out
+//                        (ldmatrix of both operands, mma.sync m16n8k32 s8: two 16-row
+//                        groups x 8 tokens), copying out
 //                        the CB bytes of the slice's outlier columns as they pass; at a
 //                        tile's end the partials go into one of EW reduction buffers
 //                        (shared-memory integer adds).
@@ -63,13 +66,13 @@ constexpr int EPI0 = CW + 1;                // first epilogue warp
 constexpr int THREADS = (CW + 1 + EW) * 32;
 constexpr int PRO_THREADS = (CW + EW) * 32;  // the warps that meet at the prologue's end
 constexpr int SLICE_TARGET = 3584;          // bytes of K per slice (before rounding)
-constexpr int BOXW = 256;                   // bytes of K per TMA box
+constexpr int BOXW = 128;                   // bytes of K per TMA box (one swizzle row)
 constexpr int CH = 64 * CW;                 // bytes of K per stage per row
 constexpr int BOXES = CH / BOXW;            // TMA boxes per stage
 constexpr int STAGES = 6;
 constexpr int STAGE_BYTES = ROWS * CH;      // 16 KB
-constexpr int XPAD = 64;                    // xs row pitch = KS + 64: a quarter-warp's B loads
-                                            // (tokens g, g+1 x 4 chunks) hit 8 bank groups
+constexpr int XPAD = 16;                    // xs row pitch = KS + 16 (KS % 512 == 0): the 8
+                                            // token rows of an ldmatrix phase hit 8 bank groups
 constexpr int RP = ROWS + 4;                // token pitch of a reduction buffer (words):
                                             // the fragment adds fall on distinct banks
 constexpr int MAXO = 128;                   // outlier columns kept in shared memory
@@ -78,11 +81,13 @@ constexpr int MAXOS = 32;                   // outlier columns per slice copied 
 constexpr int XB = 512;                     // columns per block of the prologue's maxima
 constexpr int64_t MAX_K = 65536;            // larger K take the GEMM path
 constexpr int MAX_S = 32;                   // slices at MAX_K: 19
+constexpr int PREFETCH = 32;                // CB stages per CTA prefetched into the L2 while
+                                            // the prologue runs (~76 MB over 148 CTAs)
 
 static_assert(CH % BOXW == 0, "whole boxes per stage");
 static_assert(SLICE_TARGET % CH == 0, "slices hold whole stages");
 static_assert(EW == 4, "tile i of a CTA goes to epilogue warp i % 4");
-static_assert(2 * SLICE_TARGET <= STAGE_BYTES, "a slice row of X fits one stage");
+static_assert(4 * SLICE_TARGET <= STAGE_BYTES, "two slice rows of X fit one stage");
 static_assert(XB == 512, "a block is 64 groups of 8 columns: two per lane");
 
 // bytes of K per slice: K split evenly, rounded up to whole stages
@@ -133,7 +138,7 @@ __host__ __device__ inline Smem smem_layout(int NT, int64_t K) {
   s.mask = smem_take(off, static_cast<uint64_t>(mask_words_smem(K)) * 4, 16);
   s.spre = smem_take(off, static_cast<uint64_t>(KS / 32) * 4, 16);
   s.bm = smem_take(off, static_cast<uint64_t>(TP) * ((K + XB - 1) / XB) * 4, 16);
-  s.dl = smem_take(off, static_cast<uint64_t>((K + XB - 1) / XB) * 4, 16);
+  s.dl = smem_take(off, static_cast<uint64_t>(TP) * ((K + XB - 1) / XB) * 4, 16);
   s.rmx = smem_take(off, TP * 4, 16);
   s.idx = smem_take(off, MAXO * 4, 16);
   s.jinfo = smem_take(off, MAXO * 4, 16);
@@ -169,7 +174,8 @@ struct Args {
   // barrier; the words carry the epoch in their upper 32 bits and start at zero
   bool coop;
   unsigned long long* gmask;  // [ceil(K/32)] outlier mask words
-  unsigned long long* gbm;    // [T][ceil(K/512)] block maxima (fp16 |x| bit patterns)
+  unsigned long long* gbm;    // [T][ceil(K/512)] block keys (largest |x| below the
+                              // threshold and its column, as block_key8 packs them)
   unsigned long long* gbar;   // [1] barrier counter (epoch << 32 | arrivals)
 };
 
@@ -180,6 +186,28 @@ __device__ __forceinline__ void mma_s8_16816(int (&c)[4], uint32_t a0, uint32_t 
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Prefetch one box of CB into the L2 (no shared memory, no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
+// Four 8 x 16-byte matrices from shared memory (lane l gives the address of row l % 8 of
+// matrix l / 8); lane l receives bytes 4 (l % 4) .. 4 (l % 4) + 3 of row l / 4 of each.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
 }
 
 __device__ __forceinline__ void all_sync() {   // compute + epilogue warps
@@ -209,6 +237,36 @@ __device__ __forceinline__ uint32_t absmax8_bits(const uint4 v) {
 
 __device__ __forceinline__ float half_bits_to_float(uint32_t b) {
   return __half2float(__ushort_as_half(static_cast<unsigned short>(b)));
+}
+
+// Block key of 8 fp16 values at columns c0 .. c0 + 7 of a 512-column block: the largest
+// |x| among the values not in `skip`, as its fp16 bit pattern, in the upper 16 bits, and its
+// column within the block in the lower ones (the larger column on ties); 0 when every value
+// is skipped.  The unsigned maximum of keys is the key of their union.
+__device__ __forceinline__ uint32_t block_key8(const uint4 v, uint32_t c0, uint32_t skip) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t key = 0u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t k0 = ((w[i] & 0x7fffu) << 16) | (c0 + 2 * i);
+    const uint32_t k1 = (w[i] & 0x7fff0000u) | (c0 + 2 * i + 1);
+    if (!((skip >> (2 * i)) & 1u)) key = max(key, k0);
+    if (!((skip >> (2 * i + 1)) & 1u)) key = max(key, k1);
+  }
+  return key;
+}
+
+// The block key of a group of 8 values over those below the threshold; their outlier bits
+// (|x| >= thr) go to *bits.
+__device__ __forceinline__ uint32_t group_key(const uint4 v, uint32_t c0, float thr,
+                                              uint32_t* bits) {
+  uint32_t key = block_key8(v, c0, 0u);
+  *bits = 0u;
+  if (half_bits_to_float(key >> 16) >= thr) {   // rare: a value at the threshold
+    *bits = outlier_bits8(v, thr);
+    key = block_key8(v, c0, *bits);
+  }
+  return key;
 }
 
 // Epoch-tagged words: the upper 32 bits hold the epoch of the launch that last claimed the
@@ -331,19 +389,16 @@ __device__ __forceinline__ bool forward_prologue(
             const int t = f0 / Gi;
             const int g = f0 - t * Gi + lane;
             const uint4 v = sp[i0 + lane];
-            const uint32_t m = absmax8_bits(v);
-            uint32_t m1 = m;  // (one row) the largest |x| below the threshold
-            if (half_bits_to_float(m) >= thr) {  // rare: an outlier in this group
-              const uint32_t bits = outlier_bits8(v, thr);
-              if (bits) atomicOr(&maskall[g >> 2], bits << (8 * (g & 3)));
-              m1 = __half_as_ushort(__float2half_rn(absmax8(v, bits)));
-            }
-            if (one_row) {
-              const uint32_t mx = __reduce_max_sync(0xffffffffu, m1);
-              if (lane == 0) atomicMax(&rmx[0], __float_as_uint(half_bits_to_float(mx)));
-            } else {
-              const uint32_t mx = __reduce_max_sync(0xffffffffu, m);
-              if (lane == 0) atomicMax(&bm[t * NBK + g / GPB], mx);
+            uint32_t bits;
+            const uint32_t key =
+                group_key(v, static_cast<uint32_t>((g & (GPB - 1)) * 8), thr, &bits);
+            if (bits) atomicOr(&maskall[g >> 2], bits << (8 * (g & 3)));
+            const uint32_t mx = __reduce_max_sync(0xffffffffu, key);
+            if (lane == 0) {
+              if (one_row)   // the largest |x| below the threshold
+                atomicMax(&rmx[0], __float_as_uint(half_bits_to_float(mx >> 16)));
+              else
+                atomicMax(&bm[t * NBK + g / GPB], mx);
             }
           }
         } else {
@@ -355,19 +410,16 @@ __device__ __forceinline__ bool forward_prologue(
               const uint4 v = sp[i];
               const int gf = p * (STAGE_BYTES / 16) + i;  // group index in the flat X
               const int t = gf / Gi, g = gf - t * Gi;
-              m = absmax8_bits(v);
-              if (half_bits_to_float(m) >= thr) {
-                const uint32_t bits = outlier_bits8(v, thr);
-                if (bits) atomicOr(&maskall[g >> 2], bits << (8 * (g & 3)));
-                if (one_row) m = __half_as_ushort(__float2half_rn(absmax8(v, bits)));
-              }
+              uint32_t bits;
+              m = group_key(v, static_cast<uint32_t>((g & (GPB - 1)) * 8), thr, &bits);
+              if (bits) atomicOr(&maskall[g >> 2], bits << (8 * (g & 3)));
               key = one_row ? 0u : static_cast<uint32_t>(t * NBK + g / GPB);
             }
             const uint32_t peers = __match_any_sync(0xffffffffu, key);
             const uint32_t mx = __reduce_max_sync(peers, m);
             if (valid && lane == __ffs(peers) - 1) {
               if (one_row)
-                atomicMax(&rmx[0], __float_as_uint(half_bits_to_float(mx)));
+                atomicMax(&rmx[0], __float_as_uint(half_bits_to_float(mx >> 16)));
               else
                 atomicMax(&bm[key], mx);
             }
@@ -398,11 +450,9 @@ __device__ __forceinline__ bool forward_prologue(
       if (valid) {
         const int64_t t = f / G, g = f - t * G;
         const uint4 v = ldg_v4(X + t * K + g * 8);
-        m = absmax8_bits(v);
-        if (half_bits_to_float(m) >= thr) {
-          const uint32_t bits = outlier_bits8(v, thr);
-          if (bits) atomicOr(a.gmask + (g >> 2), eh | (bits << (8 * (g & 3))));
-        }
+        uint32_t bits;
+        m = group_key(v, static_cast<uint32_t>((g & (GPB - 1)) * 8), thr, &bits);
+        if (bits) atomicOr(a.gmask + (g >> 2), eh | (bits << (8 * (g & 3))));
         key = static_cast<uint32_t>(t * NBK + g / GPB);
       }
       const uint32_t peers = __match_any_sync(0xffffffffu, key);
@@ -481,43 +531,37 @@ __device__ __forceinline__ bool forward_prologue(
     xo_s[t * MAXO + j] = X[static_cast<int64_t>(t) * K + idx_s[j]];
   }
   if (!one_row) {
-    // blocks holding outlier columns (warp 1 lists them); the other blocks give their
-    // maxima from (a)
-    if (w == 1) {
-      int nd = 0;
-      for (int64_t b0 = 0; b0 < NBK; b0 += 32) {
-        const int64_t b = b0 + lane;
-        uint32_t o = 0u;
-        if (b < NBK) {
-#pragma unroll
-          for (int i = 0; i < XB / 32; ++i) o |= maskall[b * (XB / 32) + i];
-        }
-        const uint32_t db = __ballot_sync(0xffffffffu, o != 0u);
-        if (o != 0u) dl[nd + __popc(db & ((1u << lane) - 1u))] = static_cast<int32_t>(b);
-        nd += __popc(db);
-      }
-      if (lane == 0) misc[2] = nd;
-    }
+    // Row maxima from the block keys: a block free of outlier columns, or one whose largest
+    // value below the threshold lies in a column that is not an outlier column, gives that
+    // value; the remaining (row, block) pairs are listed and re-read from X without the
+    // outlier columns.  (With systematic outlier columns -- large in every row -- the list
+    // stays empty.)
+    if (ct == 0) misc[2] = 0;
+    compute_sync();
     for (int t = w; t < T; t += CW) {
-      float m = 0.0f;
+      uint32_t m = 0u;
       for (int64_t b0 = 0; b0 < NBK; b0 += 32) {
         const int64_t b = b0 + lane;
         if (b < NBK) {
           uint32_t o = 0u;
 #pragma unroll
           for (int i = 0; i < XB / 32; ++i) o |= maskall[b * (XB / 32) + i];
-          if (o == 0u) m = fmaxf(m, half_bits_to_float(bm[t * NBK + b]));
+          const uint32_t key = bm[t * NBK + b];
+          const int64_t col = b * XB + (key & 0xffffu);
+          if (o == 0u || !((maskall[col >> 5] >> (col & 31)) & 1u))
+            m = max(m, key >> 16);
+          else
+            dl[atomicAdd(&misc[2], 1)] = static_cast<int32_t>(t * NBK + b);
         }
       }
-      m = warp_max(m);
-      if (lane == 0) rmx[t] = __float_as_uint(m);
+      m = __reduce_max_sync(0xffffffffu, m);
+      if (lane == 0) rmx[t] = __float_as_uint(half_bits_to_float(m));
     }
     compute_sync();
-    // the blocks holding outlier columns, re-read from X without them: a warp takes
-    // (row, block) pairs, two groups of 8 columns per lane, four pairs' loads in flight
+    // the listed pairs, re-read without the outlier columns: a warp takes pairs, two groups
+    // of 8 columns per lane, four pairs' loads in flight
     {
-      const int nd = misc[2];
-      const int pairs = T * nd;
+      const int pairs = misc[2];
       constexpr int U = 4;
       for (int q0 = w; q0 < pairs; q0 += CW * U) {
         uint4 v[U][2];
@@ -533,11 +577,12 @@ __device__ __forceinline__ bool forward_prologue(
             sk[u][h] = 0xffu;
           }
           if (q < pairs) {
-            const int t = q / nd, d = q - t * nd;
+            const int pr = dl[q];
+            const int t = static_cast<int>(pr / NBK), d = static_cast<int>(pr - t * NBK);
             tt[u] = t;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const int64_t g = static_cast<int64_t>(dl[d]) * GPB + h * 32 + lane;
+              const int64_t g = static_cast<int64_t>(d) * GPB + h * 32 + lane;
               if (g < G) {
                 v[u][h] = ldg_v4(X + static_cast<int64_t>(t) * K + g * 8);
                 sk[u][h] = (maskall[g >> 2] >> (8 * (g & 3))) & 0xffu;
@@ -564,24 +609,27 @@ __device__ __forceinline__ bool forward_prologue(
   }
   compute_sync();
 
-  // (d) step 2 on this slice: one ring stage per row of X
+  // (d) step 2 on this slice: two rows of X per ring stage, in the producer's order
   {
     const int64_t k0 = static_cast<int64_t>(slice) * KS;
     const int64_t klen = KS < K - k0 ? KS : K - k0;
     const int64_t gl = klen / 8;
-    for (int tt = 0; tt < T; ++tt) {
-      const int t = static_cast<int>((tt + blockIdx.x / S) % T);
+    for (int i = 0; i < T; i += 2) {
       if (ok) {
         const bool got = mbar_wait(rg.full_bar(), rg.ph, abort_flag, a.lim);
         ok = __all_sync(0xffffffffu, got);
       }
       if (ok) {
-        const uint4* sp = reinterpret_cast<const uint4*>(ring_p + rg.s * STAGE_BYTES);
-        const float sc = scale[t];
-        for (int64_t i = ct; i < gl; i += CW * 32) {
-          const int64_t g = k0 / 8 + i;
-          const uint32_t skip = (maskall[g >> 2] >> (8 * (g & 3))) & 0xffu;
-          *reinterpret_cast<uint2*>(xs + t * pitch + i * 8) = codes8(sp[i], skip, sc);
+        for (int h = 0; h < 2 && i + h < T; ++h) {
+          const int t = static_cast<int>((i + h + blockIdx.x / S) % T);
+          const uint4* sp =
+              reinterpret_cast<const uint4*>(ring_p + rg.s * STAGE_BYTES + h * klen * 2);
+          const float sc = scale[t];
+          for (int64_t q = ct; q < gl; q += CW * 32) {
+            const int64_t g = k0 / 8 + q;
+            const uint32_t skip = (maskall[g >> 2] >> (8 * (g & 3))) & 0xffu;
+            *reinterpret_cast<uint2*>(xs + t * pitch + q * 8) = codes8(sp[q], skip, sc);
+          }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(rg.empty_bar());
@@ -803,17 +851,41 @@ __global__ void __launch_bounds__(THREADS, 1)
           bulk_load(ring + s * STAGE_BYTES, xb + off, bytes, fb);
           advance();
         }
-        for (int tt = 0; tt < T && ok; ++tt) {
-          const int t = (tt + cta_in_slice) % T;
-          const uint32_t fb = acquire(static_cast<uint32_t>(klen * 2));
+        // this slice of the rows of X, two rows per stage (rows (i + cta_in_slice) % T in
+        // order of i); once the ring is full, the CTA's first CB stages are prefetched into
+        // the L2, so that HBM streams CB while the prologue runs
+        bool prefetched = false;
+        auto prefetch_cb = [&]() {
+          prefetched = true;
+          int n = 0;
+          for (int64_t tile = cta_in_slice; tile < n_tiles && n < PREFETCH;
+               tile += ctas_in_slice) {
+            for (int st = 0; st < spt && n < PREFETCH; ++st, ++n) {
+              const int x = static_cast<int>(k0 + static_cast<int64_t>(st) * CH);
+#pragma unroll
+              for (int c = 0; c < BOXES; ++c)
+                tma_prefetch_l2_2d(&tmCB, x + c * BOXW, static_cast<int>(tile * ROWS));
+            }
+          }
+        };
+        const uint32_t rb = static_cast<uint32_t>(klen * 2);
+        for (int i = 0; i < T && ok; i += 2) {
+          if (!prefetched && issued >= static_cast<uint32_t>(STAGES)) prefetch_cb();
+          const int ta = (i + cta_in_slice) % T;
+          const int tb = (i + 1 + cta_in_slice) % T;
+          const bool two = i + 1 < T;
+          const uint32_t fb = acquire(two ? 2 * rb : rb);
           if (!fb) {
             ok = false;
             break;
           }
-          bulk_load(ring + s * STAGE_BYTES, xb + (static_cast<int64_t>(t) * K + k0) * 2,
-                    static_cast<uint32_t>(klen * 2), fb);
+          bulk_load(ring + s * STAGE_BYTES, xb + (static_cast<int64_t>(ta) * K + k0) * 2, rb, fb);
+          if (two)
+            bulk_load(ring + s * STAGE_BYTES + rb, xb + (static_cast<int64_t>(tb) * K + k0) * 2,
+                      rb, fb);
           advance();
         }
+        if (!prefetched && ok) prefetch_cb();
       }
       for (int64_t tile = cta_in_slice; tile < n_tiles && ok; tile += ctas_in_slice) {
         const int y = static_cast<int>(tile * ROWS);
@@ -907,46 +979,55 @@ __global__ void __launch_bounds__(THREADS, 1)
             ok = __all_sync(0xffffffffu, got);
           }
           if (ok) {
-            // this warp's 64-byte step of the stage: box warp / 4, bytes 64 * (warp % 4) of
-            // each 256-byte row; k offset within the slice = stage * CH + 64 * warp
-            const uint32_t rowbase = ring + rg.s * STAGE_BYTES + (warp >> 2) * (ROWS * BOXW) +
-                                     (warp & 3) * 64 + q * 16;
-            const int64_t kx = static_cast<int64_t>(st) * CH + 64 * warp + 16 * q;
-            const uint4 A0 = lds_v4(rowbase + g * BOXW);
-            const uint4 A1 = lds_v4(rowbase + (g + 8) * BOXW);
-            const uint4 A2 = lds_v4(rowbase + (g + 16) * BOXW);
-            const uint4 A3 = lds_v4(rowbase + (g + 24) * BOXW);
+            // this warp's 64-byte step of the stage: box warp / 2, chunks cw .. cw + 3 of each
+            // (swizzled) 128-byte row; k offset within the slice = stage * CH + 64 * warp.
+            // ldmatrix.x4 lane l addresses row l % 8 of matrix l / 8; A matrices are (rows
+            // 0-7 | 8-15 of a 16-row group) x (first | second 16 bytes of a 32-byte k step),
+            // B matrices the four 16-byte chunks of the step for 8 tokens.
+            const uint32_t boxb = ring + rg.s * STAGE_BYTES + (warp >> 1) * (ROWS * BOXW);
+            const int cw = (warp & 1) * 4;
+            const int mi = lane >> 3, rr = lane & 7;
+            uint32_t fa[2][2][4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int ks = 0; ks < 2; ++ks) {
+                const int row = 16 * h + 8 * (mi & 1) + rr;
+                const int chunk = cw + 2 * ks + (mi >> 1);
+                ldsm_x4(fa[h][ks], boxb + row * BOXW + ((chunk ^ rr) << 4));
+              }
+            const int64_t kx = static_cast<int64_t>(st) * CH + 64 * warp + 16 * mi;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-              const uint4 B = *reinterpret_cast<const uint4*>(xs + (nt * 8 + g) * pitch + kx);
-              mma_s8_16816(c[0][nt], A0.x, A1.x, A0.y, A1.y, B.x, B.y);
-              mma_s8_16816(c[1][nt], A2.x, A3.x, A2.y, A3.y, B.x, B.y);
-              mma_s8_16816(c[0][nt], A0.z, A1.z, A0.w, A1.w, B.z, B.w);
-              mma_s8_16816(c[1][nt], A2.z, A3.z, A2.w, A3.w, B.z, B.w);
+              uint32_t fb[4];
+              ldsm_x4(fb, smem_u32(xs + (nt * 8 + rr) * pitch + kx));
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks)
+                  mma_s8_16816(c[h][nt], fa[h][ks][0], fa[h][ks][1], fa[h][ks][2], fa[h][ks][3],
+                               fb[2 * ks], fb[2 * ks + 1]);
             }
             if constexpr (!kRaw) {
-              // copy out the bytes of outlier columns in this step (lane q holds columns
-              // 16q .. 16q+15 of rows g, g + 8, g + 16, g + 24)
+              // copy out the bytes of outlier columns in this step: for each one, lane r
+              // reads row r's byte from the stage
               const int wl = st * (CH / 32) + 2 * warp;  // slice-local mask word
-              if ((maskall[w0 + wl] | maskall[w0 + wl + 1]) != 0u) {
-                const int wq = wl + (q >> 1), sh = (q & 1) * 16;
-                const uint32_t mw = maskall[w0 + wq];
-                uint32_t bits = (mw >> sh) & 0xffffu;
-                while (bits) {
-                  const int bp = __ffs(bits) - 1;
-                  bits &= bits - 1u;
-                  const int jl = spre[wq] + __popc(mw & ((1u << (sh + bp)) - 1u)) - jb;
-                  if (jl < MAXOS && jl + jb < MAXO) {
-                    const int wi = bp >> 2, bs = 8 * (bp & 3);
-                    const uint32_t u0 = wi == 0 ? A0.x : wi == 1 ? A0.y : wi == 2 ? A0.z : A0.w;
-                    const uint32_t u1 = wi == 0 ? A1.x : wi == 1 ? A1.y : wi == 2 ? A1.z : A1.w;
-                    const uint32_t u2 = wi == 0 ? A2.x : wi == 1 ? A2.y : wi == 2 ? A2.z : A2.w;
-                    const uint32_t u3 = wi == 0 ? A3.x : wi == 1 ? A3.y : wi == 2 ? A3.z : A3.w;
-                    uint8_t* d = cb_b + jl * ROWS + g;
-                    d[0] = static_cast<uint8_t>(u0 >> bs);
-                    d[8] = static_cast<uint8_t>(u1 >> bs);
-                    d[16] = static_cast<uint8_t>(u2 >> bs);
-                    d[24] = static_cast<uint8_t>(u3 >> bs);
+              const uint32_t mw2[2] = {maskall[w0 + wl], maskall[w0 + wl + 1]};
+              if ((mw2[0] | mw2[1]) != 0u) {
+#pragma unroll
+                for (int hw = 0; hw < 2; ++hw) {
+                  const uint32_t mw = mw2[hw];
+                  uint32_t bits = mw;
+                  while (bits) {
+                    const int bp = __ffs(bits) - 1;
+                    bits &= bits - 1u;
+                    const int jl = spre[wl + hw] + __popc(mw & ((1u << bp) - 1u)) - jb;
+                    if (jl < MAXOS && jl + jb < MAXO) {
+                      const int col = 32 * hw + bp;  // byte of the warp's 64-byte step
+                      const int chunk = cw + (col >> 4);
+                      cb_b[jl * ROWS + lane] = lds_u8(boxb + lane * BOXW +
+                                                      (((chunk ^ (lane & 7)) << 4) | (col & 15)));
+                    }
                   }
                 }
               }

@@ -353,6 +353,64 @@ int64_t oracle_linear_forward_rows_e4m3(const uint16_t *X, int64_t T, int64_t K,
     return 0;
 }
 
+/* Backward of the fp16-weight training mode (the blog's "用法" names it for int8/fp16
+ * mixed-precision training and gives no gradient formulas): the backward of
+ * y = x W^T + b passed straight through the quantisation, in fp64 --
+ *   dX[t,k] = sum_n dY[t,n] W[n,k],   dW[n,k] = sum_t dY[t,n] X[t,k],   db[n] = sum_t dY[t,n].
+ * X [T,K], W [N,K], dY [T,N] fp16 (bits); outputs fp64, any of them NULL to skip. */
+void oracle_linear_backward(const uint16_t *X, const uint16_t *W, const uint16_t *dY,
+                            int64_t T, int64_t N, int64_t K, double *dX, double *dW,
+                            double *db)
+{
+    if (dX) {
+        #pragma omp parallel for schedule(static)
+        for (int64_t t = 0; t < T; ++t)
+            for (int64_t k = 0; k < K; ++k) {
+                double s = 0.0;
+                for (int64_t n = 0; n < N; ++n)
+                    s += (double)oracle_half_to_float(dY[t * N + n]) *
+                         (double)oracle_half_to_float(W[n * K + k]);
+                dX[t * K + k] = s;
+            }
+    }
+    if (dW) {
+        #pragma omp parallel for schedule(static)
+        for (int64_t n = 0; n < N; ++n)
+            for (int64_t k = 0; k < K; ++k) {
+                double s = 0.0;
+                for (int64_t t = 0; t < T; ++t)
+                    s += (double)oracle_half_to_float(dY[t * N + n]) *
+                         (double)oracle_half_to_float(X[t * K + k]);
+                dW[n * K + k] = s;
+            }
+    }
+    if (db) {
+        for (int64_t n = 0; n < N; ++n) {
+            double s = 0.0;
+            for (int64_t t = 0; t < T; ++t)
+                s += (double)oracle_half_to_float(dY[t * N + n]);
+            db[n] = s;
+        }
+    }
+}
+
+/* The weight the int8 forward computes with ("用法": CB * SCB / 127 recovers it), in the
+ * fp32 arithmetic the library's dequantisation states: W'[n,k] = fl32(CB[n,k] *
+ * fl32(SCB[n] / 127)); with e4m3 codes (e4m3 != 0) their exact values times
+ * fl32(SCB[n] / 448). */
+void oracle_dequantize_weight(const uint8_t *CB, const float *SCB, int64_t N, int64_t K,
+                              int32_t e4m3, float *W)
+{
+    for (int64_t n = 0; n < N; ++n) {
+        const float s = SCB[n] / (e4m3 ? 448.0f : 127.0f);
+        for (int64_t k = 0; k < K; ++k) {
+            const float c = e4m3 ? (float)oracle_e4m3_to_double(CB[n * K + k])
+                                 : (float)(int8_t)CB[n * K + k];
+            W[n * K + k] = c * s;
+        }
+    }
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -58,6 +58,10 @@ def _load(path):
     L.oracle_linear_forward_rows.argtypes = [P, i64, i64, P, P, P, i64, ctypes.c_float,
                                              P, i64, P, P, P, P, P, P, P]
     L.oracle_linear_forward_rows.restype = i64
+    L.oracle_linear_backward.argtypes = [P, P, P, i64, i64, i64, P, P, P]
+    L.oracle_linear_backward.restype = None
+    L.oracle_dequantize_weight.argtypes = [P, P, i64, i64, ctypes.c_int32, P]
+    L.oracle_dequantize_weight.restype = None
     L.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
     L.oracle_e4m3_to_double.restype = ctypes.c_double
     L.oracle_e4m3_from_float.argtypes = [ctypes.c_float]
@@ -244,3 +248,31 @@ def linear_forward_e4m3(X, CB, SCB, bias, threshold, rows=None):
         raise MemoryError("oracle allocation failed")
     n = int(n_o[0])
     return dict(mask_words=words, idx=idx[:n].copy(), n_o=n, Xq=Xq, SCx=SCx, acc=acc, C=C)
+
+
+def linear_backward(X, W, dY):
+    """Backward of y = x W^T + b straight through the quantisation, fp64: returns
+    (dX [T,K], dW [N,K], db [N]).  X may be None (no dW) and W may be None (no dX)."""
+    dY = np.ascontiguousarray(_bits(dY))
+    T, N = dY.shape
+    Xb = None if X is None else np.ascontiguousarray(_bits(X))
+    Wb = None if W is None else np.ascontiguousarray(_bits(W))
+    K = Xb.shape[1] if Xb is not None else (Wb.shape[1] if Wb is not None else 0)
+    assert Xb is None or Xb.shape == (T, K)
+    assert Wb is None or Wb.shape == (N, K)
+    dX = None if Wb is None else np.empty((T, K), np.float64)
+    dW = None if Xb is None else np.empty((N, K), np.float64)
+    db = np.empty((N,), np.float64)
+    lib().oracle_linear_backward(_ptr(Xb), _ptr(Wb), _ptr(dY), T, N, K, _ptr(dX), _ptr(dW),
+                                 _ptr(db))
+    return dX, dW, db
+
+
+def dequantize_weight(CB, SCB, e4m3=False):
+    """The recovered weight in fp32 (CB * fl32(SCB / 127), or e4m3 values * fl32(SCB / 448))."""
+    CB = np.ascontiguousarray(CB).view(np.uint8)
+    SCB = np.ascontiguousarray(SCB, np.float32)
+    N, K = CB.shape
+    W = np.empty((N, K), np.float32)
+    lib().oracle_dequantize_weight(_ptr(CB), _ptr(SCB), N, K, 1 if e4m3 else 0, _ptr(W))
+    return W

@@ -518,4 +518,73 @@ def pin_e4m3_row_subset_matches_full():
     assert np.array_equal(rs["acc"], r["acc"][rows])
     assert np.array_equal(rs["C"], r["C"][rows])
 
+# ---------------------------------------------------------------- training-mode backward
+# ("用法": has_fp16_weights=True keeps fp16 weights for int8/fp16 mixed-precision training;
+# the gradients pass straight through the quantisation, i.e. they are those of the linear
+# map y = x W^T + b.)
+
+def _grad_case():
+    X = synth.random_fp16((3, 5), seed=61, sigma=1.0)
+    W = synth.random_fp16((4, 5), seed=62, sigma=0.5)
+    dY = synth.random_fp16((3, 4), seed=63, sigma=1.0)
+    b = synth.random_fp16((4,), seed=64, sigma=0.5)
+    return X, W, dY, b
+
+
+def pin_backward_matches_finite_differences_of_the_linear_map():
+    """Each gradient entry equals the central difference of f = sum(dY * (X W^T + b)) along
+    that entry (f is linear, so the difference is exact up to fp64 rounding); the forward
+    map here is numpy's matmul, never the product dY W the oracle forms."""
+    X, W, dY, b = _grad_case()
+    x, w, g, bb = (a.astype(np.float64) for a in (X, W, dY, b))
+
+    def f(x_, w_, b_):
+        return float((g * (x_ @ w_.T + b_)).sum())
+
+    dX, dW, db = O.linear_backward(X, W, dY)
+    h = 2.0 ** -8
+    for arr, grad, fn in ((x, dX, lambda a: f(a, w, bb)), (w, dW, lambda a: f(x, a, bb)),
+                          (bb, db, lambda a: f(x, w, a))):
+        for idx in np.ndindex(arr.shape):
+            up, dn = arr.copy(), arr.copy()
+            up[idx] += h
+            dn[idx] -= h
+            fd = (fn(up) - fn(dn)) / (2 * h)
+            assert abs(fd - grad[idx]) <= 1e-9 * (1.0 + abs(fd)), (idx, fd, grad[idx])
+
+
+def pin_backward_one_hot_output_gradient_selects_rows_and_columns():
+    """dY with a single 1 at (t, n): dX is row n of W in row t, dW is row t of X in row n,
+    db is the unit vector at n."""
+    X, W, _, _ = _grad_case()
+    dY = np.zeros((3, 4), np.float16)
+    dY[2, 1] = 1.0
+    dX, dW, db = O.linear_backward(X, W, dY)
+    assert np.array_equal(dX[2], W[1].astype(np.float64)) and not dX[:2].any()
+    assert np.array_equal(dW[1], X[2].astype(np.float64)) and not np.delete(dW, 1, 0).any()
+    assert np.array_equal(db, np.eye(4)[1])
+
+
+def pin_dequantized_weight_within_half_a_code_step():
+    """The recovered weight CB * SCB / 127 lies within half a code step (SCB / 254, plus the
+    fp32 product's rounding) of the weight it was quantised from; a row's absmax entry is
+    recovered as +-SCB up to that rounding; e4m3 codes within the e4m3 half step (2^-4
+    relative, SCB / 448 * 2^-10 absolute)."""
+    W = synth.random_fp16((6, 40), seed=65, sigma=0.02)
+    W[2] = 0
+    w = W.astype(np.float64)
+    CB, SCB = O.quantize_weight(W)
+    Wd = O.dequantize_weight(CB, SCB).astype(np.float64)
+    s = SCB.astype(np.float64)[:, None]
+    assert (np.abs(Wd - w) <= s / 254.0 * (1 + 1e-6) + 1e-12).all()
+    assert not Wd[2].any()
+    k = np.abs(w).argmax(axis=1)
+    rows = np.arange(6)
+    assert np.allclose(np.abs(Wd[rows, k]), SCB.astype(np.float64), rtol=1e-6)
+    C8, S8 = O.quantize_weight_e4m3(W)
+    W8 = O.dequantize_weight(C8, S8, e4m3=True).astype(np.float64)
+    s8 = S8.astype(np.float64)[:, None]
+    assert (np.abs(W8 - w) <= 2.0 ** -4 * np.abs(w) + s8 / 448.0 * 2.0 ** -10 + 1e-12).all()
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

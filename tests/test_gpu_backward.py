@@ -1,5 +1,5 @@
-"""The backward of the fp16-weight training mode, through the C ABI, against fp64
-definitions ("用法": has_fp16_weights=True for int8/fp16 mixed-precision training; the
+"""The backward of the fp16-weight training mode, through the C ABI, against the oracle's
+fp64 backward ("用法": has_fp16_weights=True for int8/fp16 mixed-precision training; the
 gradients pass straight through the quantisation):
 
     dX = dY W,   dW = dY^T X,   db = sum_t dY[t, :]
@@ -10,7 +10,7 @@ operands; each output row is held to the forward's tolerance,
 which covers the final fp16 rounding (2^-11 relative) and fp32 summation.  The cases span
 several 256 x 256 tiles with ragged edges on every dimension, a reduction shorter than
 one 64-element stage, and a single row.  The dequantised weight W' = CB * SCB / 127 (e4m3:
-values * SCB / 448) is compared bit for bit with the same fp32 arithmetic in numpy.
+values * SCB / 448) is compared bit for bit with the oracle's fp32 recovery rounded to fp16.
 """
 import numpy as np
 import pytest
@@ -48,7 +48,7 @@ def test_backward_input_product(T, N, K):
     dX = torch.full((T, K), float("nan"), dtype=torch.float16, device=DEV)
     abi.i8_linear_backward_input(dev(dY), dev(W), dX)
     sync_ok()
-    _rows_close(host(dX), dY.astype(np.float64) @ W.astype(np.float64))
+    _rows_close(host(dX), O.linear_backward(None, W, dY)[0])
 
 
 @pytest.mark.parametrize("T,N,K", [(1, 8, 16), (7, 264, 272), (300, 1000, 1040),
@@ -59,7 +59,7 @@ def test_backward_weight_product(T, N, K):
     dW = torch.full((N, K), float("nan"), dtype=torch.float16, device=DEV)
     abi.i8_linear_backward_weight(dev(dY), dev(X), dW)
     sync_ok()
-    _rows_close(host(dW), dY.astype(np.float64).T @ X.astype(np.float64))
+    _rows_close(host(dW), O.linear_backward(X, None, dY)[1])
 
 
 @pytest.mark.parametrize("T,N", [(1, 8), (37, 264), (4096, 1000), (5, 16392)])
@@ -68,10 +68,11 @@ def test_bias_grad(T, N):
     db = torch.full((N,), float("nan"), dtype=torch.float16, device=DEV)
     abi.i8_bias_grad(dev(dY), db)
     sync_ok()
-    ref = dY.astype(np.float64).sum(0)
+    ref = O.linear_backward(None, None, dY)[2]
     got = host(db).astype(np.float64)
     # fp16 rounding of the result plus fp32 summation of T terms
-    bound = 2.0 ** -11 * np.abs(ref) + T * 2.0 ** -24 * np.abs(dY.astype(np.float64)).sum(0) + 1e-7
+    bound = (2.0 ** -11 * np.abs(ref) + T * 2.0 ** -24 * np.abs(dY.astype(np.float64)).sum(0)
+             + 1e-7)
     assert (np.abs(got - ref) <= bound).all()
     db2 = torch.empty_like(db)
     abi.i8_bias_grad(dev(dY), db2)
@@ -87,14 +88,13 @@ def test_dequantize_weight_bitexact(N, K):
     out = torch.full((N, K), float("nan"), dtype=torch.float16, device=DEV)
     abi.i8_dequantize_weight(dev(CB), dev(SCB), out)
     sync_ok()
-    want = (CB.astype(np.float32) * (SCB / np.float32(127.0)).astype(np.float32)[:, None])
-    assert np.array_equal(host(out).view(np.uint16), want.astype(np.float16).view(np.uint16))
+    want = O.dequantize_weight(CB, SCB).astype(np.float16)
+    assert np.array_equal(host(out).view(np.uint16), want.view(np.uint16))
     CB8, SCB8 = O.quantize_weight_e4m3(W)
     abi.i8_dequantize_weight(dev(CB8), dev(SCB8), out)
     sync_ok()
-    vals = O.e4m3_decode(CB8).astype(np.float32)            # exact in fp32
-    want8 = vals * (SCB8 / np.float32(448.0)).astype(np.float32)[:, None]
-    assert np.array_equal(host(out).view(np.uint16), want8.astype(np.float16).view(np.uint16))
+    want8 = O.dequantize_weight(CB8, SCB8, e4m3=True).astype(np.float16)
+    assert np.array_equal(host(out).view(np.uint16), want8.view(np.uint16))
 
 
 def test_backward_rejects_unaligned_rows():

@@ -140,9 +140,8 @@ def test_replaced_layer_stack_layer_by_layer():
 
 
 def _ref_grads(X, W, gy):
-    """Backward of y = x W^T + b in fp64: dx = dy W, dW = dy^T x, db = sum(dy)."""
-    x64, w64, g64 = X.astype(np.float64), W.astype(np.float64), gy.astype(np.float64)
-    return g64 @ w64, g64.T @ x64, g64.sum(0)
+    """Backward of y = x W^T + b (the oracle, fp64): dx = dy W, dW = dy^T x, db = sum(dy)."""
+    return O.linear_backward(X, W, gy)
 
 
 def _close(a, ref, rel=1e-2):
@@ -189,6 +188,6 @@ def test_inference_mode_passes_input_gradients():
     gy = synth.random_fp16((T, N), seed=29, sigma=0.5)
     m(x).backward(torch.from_numpy(gy.view(np.int16)).view(torch.float16).cuda())
     sync_ok()
-    Wd = host(m.CB).astype(np.float64) * (host(m.SCB).astype(np.float64) / 127.0)[:, None]
-    _close(host(x.grad), gy.astype(np.float64) @ Wd)
+    Wd = O.dequantize_weight(host(m.CB), host(m.SCB)).astype(np.float16)
+    _close(host(x.grad), O.linear_backward(None, Wd, gy)[0])
     assert all(p.grad is None for p in m.parameters())

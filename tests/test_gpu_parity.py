@@ -68,6 +68,9 @@ SCAN_CASES = [
     (33, 96, (1, 2), 0.0, math.inf),
     (4100, 1040, (7, 1039), 1e-4, 6.0),
     (3000, 16384, (0, 9000, 16383), 0.0, 6.0),    # rows beyond the per-CTA cache
+    # rows beyond the cache quantised early from global memory, some of them coded again
+    # (a random outlier elsewhere flags the column of their largest value)
+    (3000, 16384, (7, 12000), 3e-5, 6.0),
     (16, 14336, (100, 14000), 0.0, 6.0),
     (20, 10000, (), 0.0, 0.0),      # n_o = 10000: indices past the 8192 kept in shared memory
     # >= 8 cached rows per CTA: rows quantised before the grid barrier.  Random outliers

@@ -101,6 +101,20 @@ MUTATIONS = [
      "            C[i * N + n] = int_part"),
     ("dequant_single_127", "                              / (127.0 * 127.0);",
      "                              / (127.0);"),
+    # training-mode backward and the recovered weight
+    ("backward_dx_wrong_weight_entry",
+     "(double)oracle_half_to_float(W[n * K + k]);\n                dX[t * K + k] = s;",
+     "(double)oracle_half_to_float(W[(k * N + n) % (N * K)]);\n                dX[t * K + k] = s;"),
+    ("backward_dw_drops_last_row",
+     "                for (int64_t t = 0; t < T; ++t)\n                    s += (double)oracle_half_to_float(dY[t * N + n]) *\n"
+     "                         (double)oracle_half_to_float(X[t * K + k]);",
+     "                for (int64_t t = 0; t + 1 < T; ++t)\n                    s += (double)oracle_half_to_float(dY[t * N + n]) *\n"
+     "                         (double)oracle_half_to_float(X[t * K + k]);"),
+    ("bias_grad_every_other_row",
+     "            for (int64_t t = 0; t < T; ++t)\n                s += (double)oracle_half_to_float(dY[t * N + n]);",
+     "            for (int64_t t = 0; t < T; t += 2)\n                s += (double)oracle_half_to_float(dY[t * N + n]);"),
+    ("recovered_weight_over_128", "const float s = SCB[n] / (e4m3 ? 448.0f : 127.0f);",
+     "const float s = SCB[n] / (e4m3 ? 448.0f : 128.0f);"),
     ("bias_index_row",
      "double b = bias ? (double)oracle_half_to_float(bias[n]) : 0.0;\n"
      "            C[i * N + n] = int_part",
