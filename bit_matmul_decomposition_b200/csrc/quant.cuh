@@ -220,6 +220,23 @@ __device__ __forceinline__ __half code_to_half(int c, bool e4m3) {
   return __ushort_as_half(static_cast<unsigned short>(h & 0xffffu));
 }
 
+// fp16 values of two weight codes (bytes b0, b1; only their low bytes count) as a half2
+// (b0 in the low half).  int8: with u = c + 128 = (byte ^ 0x80), the fp16 pattern
+// 0x6400 | u is 1024 + u exactly (a 10-bit mantissa at exponent 10), and subtracting
+// 1152 leaves c exactly -- integer operations and one packed subtraction instead of two
+// conversions.  e4m3: the packed hardware conversion.
+__device__ __forceinline__ __half2 codes_to_half2(uint32_t b0, uint32_t b1, bool e4m3) {
+  const uint32_t pair = __byte_perm(b0, b1, 0x0040);  // b0 in byte 0, b1 in byte 1
+  if (e4m3) {
+    uint32_t h;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(pair)));
+    return *reinterpret_cast<__half2*>(&h);
+  }
+  uint32_t w = __byte_perm(pair, 0x64646464u, 0x5140) ^ 0x00800080u;
+  const __half2 biased = *reinterpret_cast<__half2*>(&w);
+  return __hsub2(biased, __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480)));
+}
+
 __device__ __forceinline__ uint32_t skip_bits8(const uint32_t* mask, int64_t v) {
   return mask ? ((__ldg(mask + (v >> 2)) >> (8 * (v & 3))) & 0xffu) : 0u;
 }
@@ -407,24 +424,58 @@ __device__ __forceinline__ float row_absmax(uint32_t base, const uint4* gbase, i
   return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 }
 
-// codes (int8, or e4m3) of groups start, start+step, ... of one row.
+// The outlier values of one 16-byte group v of a row (its mask bits k != 0) into the
+// row's fp16 outlier slice: the column of bit b has rank spre[v/4] + (mask bits below it),
+// and rank j goes to xo[(j / 64) * cstride + j % 64].
+__device__ __forceinline__ void group_outliers(const uint4 x, int v, uint32_t k,
+                                               const uint32_t* smask, const int32_t* spre,
+                                               __half* xo, int64_t cstride) {
+  const uint32_t w = smask[v >> 2];
+  const int sh = (v & 3) * 8;
+  int j = spre[v >> 2] + __popc(w & ((1u << sh) - 1u));
+  while (k) {
+    const int b = __ffs(k) - 1;
+    k &= k - 1u;
+    const uint32_t pr = (b & 4) ? ((b & 2) ? x.w : x.z) : ((b & 2) ? x.y : x.x);
+    const uint32_t hw = pr >> (16 * (b & 1));
+    xo[static_cast<int64_t>(j >> 6) * cstride + (j & 63)] =
+        __ushort_as_half(static_cast<unsigned short>(hw & 0xffffu));
+    ++j;
+  }
+}
+
+// codes (int8, or e4m3) of groups start, start+step, ... of one row; with xo non-NULL, the
+// row's outlier values also go into its fp16 outlier slice (group_outliers).
 template <bool kShared>
 __device__ __forceinline__ void row_codes(uint32_t base, const uint4* gbase, uint2* q, int gpr,
                                           int start, int step, const uint32_t* smask, float s,
-                                          bool e4m3) {
+                                          bool e4m3, const int32_t* spre = nullptr,
+                                          __half* xo = nullptr, int64_t cstride = 0) {
   int v = start;
   for (; v + 3 * step < gpr; v += 4 * step) {
     const uint4 x0 = row_vec<kShared>(base, gbase, v);
     const uint4 x1 = row_vec<kShared>(base, gbase, v + step);
     const uint4 x2 = row_vec<kShared>(base, gbase, v + 2 * step);
     const uint4 x3 = row_vec<kShared>(base, gbase, v + 3 * step);
-    q[v] = codes8_fmt(x0, scan_bits(smask, v), s, e4m3);
-    q[v + step] = codes8_fmt(x1, scan_bits(smask, v + step), s, e4m3);
-    q[v + 2 * step] = codes8_fmt(x2, scan_bits(smask, v + 2 * step), s, e4m3);
-    q[v + 3 * step] = codes8_fmt(x3, scan_bits(smask, v + 3 * step), s, e4m3);
+    const uint32_t k0 = scan_bits(smask, v), k1 = scan_bits(smask, v + step);
+    const uint32_t k2 = scan_bits(smask, v + 2 * step), k3 = scan_bits(smask, v + 3 * step);
+    q[v] = codes8_fmt(x0, k0, s, e4m3);
+    q[v + step] = codes8_fmt(x1, k1, s, e4m3);
+    q[v + 2 * step] = codes8_fmt(x2, k2, s, e4m3);
+    q[v + 3 * step] = codes8_fmt(x3, k3, s, e4m3);
+    if (xo != nullptr && (k0 | k1 | k2 | k3) != 0u) {
+      if (k0) group_outliers(x0, v, k0, smask, spre, xo, cstride);
+      if (k1) group_outliers(x1, v + step, k1, smask, spre, xo, cstride);
+      if (k2) group_outliers(x2, v + 2 * step, k2, smask, spre, xo, cstride);
+      if (k3) group_outliers(x3, v + 3 * step, k3, smask, spre, xo, cstride);
+    }
   }
-  for (; v < gpr; v += step)
-    q[v] = codes8_fmt(row_vec<kShared>(base, gbase, v), scan_bits(smask, v), s, e4m3);
+  for (; v < gpr; v += step) {
+    const uint4 x = row_vec<kShared>(base, gbase, v);
+    const uint32_t k = scan_bits(smask, v);
+    q[v] = codes8_fmt(x, k, s, e4m3);
+    if (xo != nullptr && k != 0u) group_outliers(x, v, k, smask, spre, xo, cstride);
+  }
 }
 
 // Column of the j-th outlier (j < n_o) from the mask words and their exclusive popcount
@@ -459,7 +510,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
   uint4* cache = reinterpret_cast<uint4*>(psm);
   uint32_t* smask = reinterpret_cast<uint32_t*>(psm + cache_bytes);
   int32_t* spre = reinterpret_cast<int32_t*>(smask + words);
-  int32_t* sidx = spre + words + 1;
+  int32_t* sidx = spre + words + 2;  // 8-byte aligned: pairs of indices load as one word
   float* samax = reinterpret_cast<float*>(sidx + kPrepMaxIdx);   // [rows_per_cta]
   float* sbm = samax + p.rows_per_cta;                           // [cache_rows][nblk]
   __shared__ __align__(8) uint64_t s_bar[kPrepMaxChunks];
@@ -731,8 +782,8 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
       if (it < items4) {
         const int64_t c = it / p.N, n = it - c * p.N;
         const int64_t j0 = c * 64 + 2 * lane;
-        if (j0 < n_o) v0[u] = p.CB[n * K + idx_at(j0)];
-        if (j0 + 1 < n_o) v1[u] = p.CB[n * K + idx_at(j0 + 1)];
+        if (j0 < n_o) v0[u] = reinterpret_cast<const uint8_t*>(p.CB)[n * K + idx_at(j0)];
+        if (j0 + 1 < n_o) v1[u] = reinterpret_cast<const uint8_t*>(p.CB)[n * K + idx_at(j0 + 1)];
       }
     }
   };
@@ -743,7 +794,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
       if (it < items4) {
         const int64_t c = it / p.N, n = it - c * p.N;
         reinterpret_cast<__half2*>(cbo + (c * p.N + n) * 64)[lane] =
-            __halves2half2(code_to_half(v0[u], kE4M3), code_to_half(v1[u], kE4M3));
+            codes_to_half2(static_cast<uint32_t>(v0[u]), static_cast<uint32_t>(v1[u]), kE4M3);
       }
     }
   };
@@ -806,32 +857,43 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
       if (!have) continue;
       const float sc = amax > 0.0f ? __fdiv_rn(code_max(kE4M3), amax) : 0.0f;
       uint2* qrow = reinterpret_cast<uint2*>(p.Xq + t * K);
-      if (specrow && amax == samax[i] && static_cast<int64_t>(n_o) * 8 <= K) {
+      __half* xo_row = p.X_o + t * 64;
+      const int64_t cstride = p.T * 64;
+      const bool stand = specrow && amax == samax[i] && static_cast<int64_t>(n_o) * 8 <= K;
+      if (stand) {
         // the speculative codes stand: clear those of the outlier columns
         int8_t* qb = p.Xq + t * K;
         for (int j = start; j < n_o; j += step) qb[idx_at(j)] = 0;
       } else if (cached) {
-        row_codes<true>(sbase, gbase, qrow, g32, start, step, smask, sc, kE4M3);
+        row_codes<true>(sbase, gbase, qrow, g32, start, step, smask, sc, kE4M3, spre, xo_row,
+                        cstride);
       } else {
-        row_codes<false>(sbase, gbase, qrow, g32, start, step, smask, sc, kE4M3);
+        row_codes<false>(sbase, gbase, qrow, g32, start, step, smask, sc, kE4M3, spre, xo_row,
+                         cstride);
       }
       if (sub == 0 && lane == 0) p.SCx[t] = amax;
-      // the row's outlier values into X_o, eight loads in flight before their stores
-      const __half* xrow = cached ? reinterpret_cast<const __half*>(cache + i * gpr) : p.X + t * K;
-      for (int j0 = start; j0 < padded; j0 += 8 * step) {
-        __half v[8];
+      // the row's outlier values into X_o (the codes pass above wrote them unless the
+      // speculative codes stood; a cached row reads them from shared memory), and zeros up
+      // to the next multiple of 64
+      if (stand) {
+        const __half* xrow = reinterpret_cast<const __half*>(cache + i * gpr);
+        for (int j0 = start; j0 < n_o; j0 += 8 * step) {
+          __half v[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int j = j0 + u * step;
-          v[u] = __float2half_rn(0.0f);
-          if (j < n_o) v[u] = xrow[idx_at(j)];
-        }
+          for (int u = 0; u < 8; ++u) {
+            const int j = j0 + u * step;
+            v[u] = __float2half_rn(0.0f);
+            if (j < n_o) v[u] = xrow[idx_at(j)];
+          }
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int j = j0 + u * step;
-          if (j < padded) p.X_o[(static_cast<int64_t>(j >> 6) * p.T + t) * 64 + (j & 63)] = v[u];
+          for (int u = 0; u < 8; ++u) {
+            const int j = j0 + u * step;
+            if (j < n_o) xo_row[static_cast<int64_t>(j >> 6) * cstride + (j & 63)] = v[u];
+          }
         }
       }
+      for (int j = n_o + start; j < padded; j += step)
+        xo_row[static_cast<int64_t>(j >> 6) * cstride + (j & 63)] = __float2half_rn(0.0f);
     }
   }
   __syncthreads();   // the row cache is free from here on (phase 4 may reuse it)
@@ -841,43 +903,77 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
     const int64_t chunks = (n_o + 63) >> 6;
     const int64_t nbuf = min(static_cast<int64_t>(kPrepWarps), p.cache_bytes_all / K);
     if (static_cast<int64_t>(n_o) * 32 >= K && nbuf > 0) {
-      // Many outlier columns: whole CB rows come by bulk copy into a per-warp buffer in the
-      // freed row cache (one round trip per row), and the warp picks the outlier columns
-      // there, four chunks' picks in flight at a time.
-      if (warp < nbuf) {
-        uint8_t* rowbuf = psm + static_cast<size_t>(warp) * static_cast<size_t>(K);
-        const uint32_t bar = smem_u32(&s_rbar[warp]);
-        const int64_t nw = static_cast<int64_t>(gridDim.x) * nbuf;
-        uint32_t ph = 0;
+      // Many outlier columns: whole CB rows come by bulk copy into per-warp buffers in the
+      // freed row cache -- two per warp when there is room, so that the next row's copy is
+      // in flight while the warp picks this row's outlier columns -- and the warp picks the
+      // columns there, lane l taking ranks 2l and 2l+1 of each chunk of 64 (one 8-byte load
+      // of their indices), four chunks in flight at a time.
+      const int nbw = nbuf >= 2 ? 2 : 1;            // buffers per warp
+      const int nwarps = static_cast<int>(nbuf) / nbw;
+      if (warp < nwarps) {
+        // buffer i of this warp: shared memory at buf0 + i * boff, barrier bar0 + 8 i
+        const uint32_t buf0 = smem_u32(psm) + static_cast<uint32_t>(warp * nbw * K);
+        const uint32_t boff = nbw == 2 ? static_cast<uint32_t>(K) : 0u;
+        const uint32_t bar0 = smem_u32(&s_rbar[warp * nbw]);
+        const uint32_t boff8 = nbw == 2 ? 8u : 0u;
+        uint32_t phs = 0u;  // bit i: the phase of buffer i's barrier
+        const int64_t nw = static_cast<int64_t>(gridDim.x) * nwarps;
         int no_abort = 0;
-        for (int64_t n = static_cast<int64_t>(blockIdx.x) * nbuf + warp; n < p.N; n += nw) {
+        auto issue = [&](int i, int64_t row) {
           if (lane == 0) {
             // the buffer's previous reads (generic proxy) come before the copy into it
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(K));
-            bulk_load(smem_u32(rowbuf), p.CB + n * K, static_cast<uint32_t>(K), bar);
+            mbar_arrive_expect_tx(bar0 + i * boff8, static_cast<uint32_t>(K));
+            bulk_load(buf0 + i * boff, p.CB + row * K, static_cast<uint32_t>(K),
+                      bar0 + i * boff8);
           }
-          const bool got = mbar_wait(bar, ph, &no_abort, p.wait_limit_ns);
-          ph ^= 1u;
+        };
+        int cur = 0;
+        int64_t n = static_cast<int64_t>(blockIdx.x) * nwarps + warp;
+        if (n < p.N) issue(0, n);
+        const bool direct = n_o <= kPrepMaxIdx;  // every index in sidx
+        for (; n < p.N; n += nw) {
+          const bool more = n + nw < p.N;
+          if (more && nbw == 2) issue(cur ^ 1, n + nw);
+          const bool got =
+              mbar_wait(bar0 + cur * boff8, (phs >> cur) & 1u, &no_abort, p.wait_limit_ns);
+          phs ^= 1u << cur;
           if (!__all_sync(0xffffffffu, got)) {
             if (lane == 0) s_gfail = 1;
+            if (more && nbw == 2)  // let the other copy land (bounded) before moving on
+              mbar_wait(bar0 + (cur ^ 1) * boff8, (phs >> (cur ^ 1)) & 1u, &no_abort,
+                        p.wait_limit_ns);
             break;
           }
+          const uint8_t* rb = psm + warp * nbw * K + cur * boff;
           for (int64_t c0 = 0; c0 < chunks; c0 += 4) {
-            int v0[4], v1[4];
+            uint32_t v0[4], v1[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const int64_t j0 = (c0 + u) * 64 + 2 * lane;
-              v0[u] = j0 < n_o ? static_cast<int8_t>(rowbuf[idx_at(j0)]) : 0;
-              v1[u] = j0 + 1 < n_o ? static_cast<int8_t>(rowbuf[idx_at(j0 + 1)]) : 0;
+              int2 jj = make_int2(0, 0);
+              if (direct) {
+                if (j0 < n_o) jj = *reinterpret_cast<const int2*>(sidx + j0);
+              } else {
+                if (j0 < n_o) jj.x = static_cast<int>(idx_at(j0));
+                if (j0 + 1 < n_o) jj.y = static_cast<int>(idx_at(j0 + 1));
+              }
+              v0[u] = 0u;
+              v1[u] = 0u;
+              if (j0 < n_o) v0[u] = rb[jj.x];
+              if (j0 + 1 < n_o) v1[u] = rb[jj.y];
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u)
               if (c0 + u < chunks)
                 reinterpret_cast<__half2*>(cbo + ((c0 + u) * p.N + n) * 64)[lane] =
-                    __halves2half2(code_to_half(v0[u], kE4M3), code_to_half(v1[u], kE4M3));
+                    codes_to_half2(v0[u], v1[u], kE4M3);
           }
           __syncwarp();
+          if (nbw == 2)
+            cur ^= 1;
+          else if (more)
+            issue(0, n + nw);
         }
       }
     } else {
@@ -1102,7 +1198,7 @@ __host__ inline size_t prepare_row_bytes(int64_t K) {
 __host__ inline size_t prepare_smem_bytes(int64_t K, int64_t cache_rows, int64_t rows_per_cta) {
   const int64_t words = (K + 31) / 32;
   return static_cast<size_t>(cache_rows) * prepare_row_bytes(K) +
-         static_cast<size_t>(2 * words + 1 + kPrepMaxIdx + rows_per_cta) * 4;
+         static_cast<size_t>(2 * words + 2 + kPrepMaxIdx + rows_per_cta) * 4;
 }
 
 }  // namespace i8
