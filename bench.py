@@ -420,7 +420,7 @@ def time_forward(abi, forward, steps, warmup, flush_l2, stream, uuid, barrier=la
     return step_ms, kern_ms, clk
 
 
-def roofline(L, kern_per, clk, pk, sms):
+def roofline(abi, L, kern_per, clk, pk, sms):
     """The dominant kernel against its roofline: the decode kernel (the whole forward of a
     decode batch, one stream of CB) against HBM bandwidth, else the tcgen05 GEMM against
     the 8-bit tensor peak.  `peak` is the measured figure; the pipe instruction rate at the
@@ -442,8 +442,13 @@ def roofline(L, kern_per, clk, pk, sms):
     peak_i8, basis = tensor_peak(pk, clk, L.e4m3)
     mhz = clk.get("sm_mhz") if clk else None
     pipe = pipe_peak_tops(sms, mhz)
+    # the GEMM variant the library picks for these sizes on this device (the e4m3 forward
+    # runs a GEMM at every T)
+    kernel = abi.i8_forward_kernel(T, N, K)
+    if kernel == "decode_kernel":
+        kernel = "i8_gemm_tcgen05_kernel"
     return {"bound": "tensor", "achieved": achieved, "peak": peak_i8, "unit": "TOPS",
-            "frac": achieved / peak_i8, "kernel": "i8_gemm_tcgen05_kernel",
+            "frac": achieved / peak_i8, "kernel": kernel,
             "peak_basis": basis,
             "frac_of_burst_peak": achieved / (2.0 * pk["bf16"]),
             "frac_of_sustained_peak": achieved / (2.0 * pk["bf16_sus"]),
@@ -472,7 +477,7 @@ def measure_layer(abi, L, steps, warmup, l2_mode, stream, uuid, pk, sms, forward
     step_ms, kern_ms, clk = time_forward(abi, forward, steps, warmup, flush_l2, stream, uuid)
     ms = step_ms / steps
     _, _, eff, nbytes = work_counts(L.T, L.N, L.K, L.n_o)
-    roof = roofline(L, kern_ms / steps, clk, pk, sms)
+    roof = roofline(abi, L, kern_ms / steps, clk, pk, sms)
     return {"workload": L.w.name, "T": L.T, "N": L.N, "K": L.K,
             "threshold": json_threshold(L.w.threshold),
             "n_outliers": L.n_o, "steps": steps, "ms_per_step": ms,
@@ -668,7 +673,7 @@ def run_gpu(args, w0):
 
     decode = T <= 16 and not e4m3   # (the e4m3 forward runs the GEMM for every T)
     pk = peaks()
-    roof = roofline(L, kern_ms / K_steps, clk, pk, sms)
+    roof = roofline(abi, L, kern_ms / K_steps, clk, pk, sms)
     tr = traffic_record(roof["kernel"], w0.name) if not e4m3 else None
     roof["traffic"] = None if tr is None else tr["dram_bytes_per_launch"]
     if tr is not None:

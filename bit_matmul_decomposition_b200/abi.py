@@ -32,6 +32,7 @@ SIGNATURES = {
     "i8_quantize_act": (_ST, [_P, _I64, _I64, _P, _P, _P, _P, _P, _P, _P]),
     "i8_prepare_act": (_ST, [_P, _I64, _I64, _F, _P, _P, _P, _P, _P, _P, _P]),
     "i8_linear_workspace_size": (_SZ, [_I64, _I64, _I64]),
+    "i8_forward_kernel": (_ST, [_I64, _I64, _I64, _P]),
     "i8_linear_forward": (_ST, [_P, _I64, _I64, _P, _P, _P, _I64, _F, _P, _P, _SZ, _P]),
     "i8_igemm_s32": (_ST, [_P, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
     "i8_linear_forward_noalloc": (_ST, [_P, _I64, _I64, _P, _P, _P, _I64, _F, _P, _P]),
@@ -218,6 +219,16 @@ def i8_prepare_act(X, threshold, col_mask, outlier_idx, n_outliers, Xq, SCx, X_o
 
 def i8_linear_workspace_size(T, N, K) -> int:
     return int(load().i8_linear_workspace_size(T, N, K))
+
+
+FORWARD_KERNELS = {0: "decode_kernel", 1: "i8_gemm_tcgen05_kernel", 2: "i8_gemm_wide_kernel"}
+
+
+def i8_forward_kernel(T, N, K) -> str:
+    """Name of the product kernel i8_linear_forward runs for these sizes on this device."""
+    kind = ctypes.c_int32(-1)
+    _check("i8_forward_kernel", load().i8_forward_kernel(T, N, K, ctypes.addressof(kind)))
+    return FORWARD_KERNELS[kind.value]
 
 
 def i8_linear_forward(X, CB, SCB, bias, threshold, C, workspace, stream=None):

@@ -463,6 +463,15 @@ i8_status run_prepare(const void* X, int64_t T, int64_t K, float thr, uint32_t* 
 // tcgen05 GEMM (pairs of CTAs, 256 x 256 tiles); raw=true writes the int32 accumulator.
 // B_c (ocols columns) is the outlier cache's CB_o slice, read instead of B_o when the
 // device word *cbo_sel is nonzero.
+// Long K-loops with enough tiles to fill the GPU several times take the 256 x 512 tiles
+// (a quarter less operand feed per multiply-add; the epilogue is not overlapped, which a
+// long K-loop hides).
+bool use_wide(int64_t T, int64_t N, int64_t K, const DeviceInfo& d) {
+  const int64_t m_tiles = (T + gemm::TM - 1) / gemm::TM;
+  const int64_t wide_tiles = m_tiles * ((N + gemmw::TN - 1) / gemmw::TN);
+  return K >= kWideMinK && wide_tiles >= 4 * static_cast<int64_t>(d.wide_clusters);
+}
+
 i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t* B, int64_t N,
                    const void* A_o, const void* B_o, const int32_t* n_o, const float* SCx,
                    const float* SCB, const void* bias, void* C, int32_t* acc,
@@ -505,12 +514,8 @@ i8_status run_gemm(bool raw, const int8_t* A, int64_t T, int64_t K, const int8_t
   a.acc_out = acc;
   a.c_tma = c_tma;
   a.wait_limit_ns = kWaitLimitNs;
-  // Long K-loops with enough tiles to fill the GPU several times take the 256 x 512 tiles
-  // (a quarter less operand feed per multiply-add; the epilogue is not overlapped, which
-  // a long K-loop hides).
-  const int64_t m_tiles = a.m_tiles;
-  const int64_t wide_tiles = m_tiles * ((N + gemmw::TN - 1) / gemmw::TN);
-  if (!raw && K >= kWideMinK && wide_tiles >= 4 * static_cast<int64_t>(d.wide_clusters)) {
+  const int64_t wide_tiles = static_cast<int64_t>(a.m_tiles) * ((N + gemmw::TN - 1) / gemmw::TN);
+  if (!raw && use_wide(T, N, K, d)) {
     a.n_tiles = static_cast<int>((N + gemmw::TN - 1) / gemmw::TN);
     const int wc = static_cast<int>(wide_tiles < d.wide_clusters ? wide_tiles : d.wide_clusters);
     const cudaError_t e =
@@ -770,6 +775,19 @@ size_t i8_outlier_slice_elems(int64_t rows, int64_t K) {
 size_t i8_linear_workspace_size(int64_t T, int64_t N, int64_t K) {
   if (!shape_ok(T, K) || N <= 0 || N > 0x7fffffffLL) return 0;
   return layout(T, N, K).total;
+}
+
+i8_status i8_forward_kernel(int64_t T, int64_t N, int64_t K, int32_t* kind) {
+  if (!kind || !shape_ok(T, K) || N <= 0 || N > 0x7fffffffLL) return I8_ERR_INVALID_ARG;
+  if (use_decode(T, K)) {
+    *kind = I8_KERNEL_DECODE;
+    return I8_OK;
+  }
+  DeviceInfo* d;
+  const i8_status st = device_info(&d);
+  if (st != I8_OK) return st;
+  *kind = use_wide(T, N, K, *d) ? I8_KERNEL_GEMM_WIDE : I8_KERNEL_GEMM;
+  return I8_OK;
 }
 
 i8_status i8_quantize_weight(const void* W, int64_t N, int64_t K, int8_t* CB, float* SCB,

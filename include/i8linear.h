@@ -138,6 +138,17 @@ i8_status i8_prepare_act(const void* X, int64_t T, int64_t K, float threshold,
  * is invalid. */
 size_t i8_linear_workspace_size(int64_t T, int64_t N, int64_t K);
 
+/* The product kernel i8_linear_forward runs for these sizes on the current device (the
+ * GEMM variant depends on how many CTA pairs the device holds at once).  Writes one of
+ * I8_KERNEL_* to *kind.  I8_ERR_INVALID_ARG for a NULL kind or an invalid size; the
+ * device query's error (I8_ERR_CUDA) when the GEMM path needs it and no device answers. */
+enum {
+  I8_KERNEL_DECODE = 0,     /* decode_kernel: T <= 16 and K <= 65536                  */
+  I8_KERNEL_GEMM = 1,       /* i8_gemm_tcgen05_kernel: 256 x 256 tiles per CTA pair   */
+  I8_KERNEL_GEMM_WIDE = 2   /* i8_gemm_wide_kernel: 256 x 512 tiles per CTA pair      */
+};
+i8_status i8_forward_kernel(int64_t T, int64_t N, int64_t K, int32_t* kind);
+
 /*
  * Steps 1, 2, 4, 5 and 6 -- the whole forward of the decomposed linear layer.
  * Sources: "LLM.int8() 的总结" (three steps), "内部的 MatMul" (threshold 6, fp16 outlier

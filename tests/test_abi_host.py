@@ -62,6 +62,18 @@ def test_workspace_size_host_logic(lib):
     assert lib.i8_outlier_slice_elems(10, 64) == 10 * 64
 
 
+def test_forward_kernel_query_host_logic(lib):
+    # decode sizes are decided without a device; invalid sizes and a NULL result are refused
+    assert abi.i8_forward_kernel(1, 64, 64) == "decode_kernel"
+    assert abi.i8_forward_kernel(16, 57344, 14336) == "decode_kernel"
+    assert abi.i8_forward_kernel(4, 33, 65536) == "decode_kernel"
+    for T, N, K in [(0, 64, 64), (16, 0, 64), (16, 64, 72)]:
+        with pytest.raises(abi.I8Error) as e:
+            abi.i8_forward_kernel(T, N, K)
+        assert e.value.code == 1
+    assert lib.i8_forward_kernel(1, 64, 64, None) == 1
+
+
 FAKE = 0x10000  # aligned, never dereferenced: validation rejects before any launch
 
 

@@ -57,6 +57,13 @@ def _sample(n, extra, count, seed):
     return np.array(sorted(s), np.int64)
 
 
+def test_forward_kernel_query_names_the_wide_tiles():
+    assert abi.i8_forward_kernel(T, N, K) == "i8_gemm_wide_kernel"
+    assert abi.i8_forward_kernel(T, N, 4096) == "i8_gemm_tcgen05_kernel"   # K below 8192
+    assert abi.i8_forward_kernel(300, 1000, K) == "i8_gemm_tcgen05_kernel"  # too few tiles
+    assert abi.i8_forward_kernel(16, N, K) == "decode_kernel"
+
+
 @pytest.mark.parametrize("n_cols,thr", [(0, math.inf), (8, 6.0), (80, 6.0), (0, 0.0)])
 def test_wide_tiles_match_the_oracle(weights, n_cols, thr):
     CB, SCB, CBr, SCBr, b = weights
