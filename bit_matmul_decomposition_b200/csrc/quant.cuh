@@ -515,6 +515,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
   float* sbm = samax + p.rows_per_cta;                           // [cache_rows][nblk]
   __shared__ __align__(8) uint64_t s_bar[kPrepMaxChunks];
   __shared__ __align__(8) uint64_t s_rbar[kPrepWarps];  // phase 4 row buffers
+  __shared__ __align__(8) uint64_t s_sbar[kPrepWarps];  // phase 3 row slots
   __shared__ int s_fail;
   __shared__ int s_gfail;  // phase 4 gave up on a wait: the cache is left invalid
   __shared__ int s_last;
@@ -535,6 +536,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
     s_gfail = 0;
     for (int c = 0; c < nchunks; ++c) mbar_init(smem_u32(&s_bar[c]), 1);
     for (int c = 0; c < kPrepWarps; ++c) mbar_init(smem_u32(&s_rbar[c]), 1);
+    for (int c = 0; c < kPrepWarps; ++c) mbar_init(smem_u32(&s_sbar[c]), 1);
     fence_mbar_init();
   }
   for (int64_t w = tid; w < words; w += kPrepThreads) smask[w] = 0u;
@@ -802,27 +804,63 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
   if (few4) gather_load(first4, pv0, pv1);
 
   // ------------------------------------------------ phase 3: quantise
-  // Rows go in rounds of (16 / wpr) rows with wpr warps per row (wpr = 1 when the CTA owns
-  // 16 rows or more; up to 16 when it owns one, as in decode batches).  Every warp walks
-  // the same rounds, so the block barriers of the cross-warp reduction are uniform.
+  // Rows go in rounds of (16 / wpr) rows with wpr warps per row (wpr = 1 for 16 rows or
+  // more; up to 16 for one row, as in decode batches).  Every warp walks the same rounds,
+  // so the block barriers of the cross-warp reduction are uniform.  First the cached rows,
+  // from shared memory; then the others.  Those come into the freed row cache by bulk copy,
+  // one row per slot and round (each row is then read from shared memory for both its
+  // maximum and its codes, instead of twice from global memory with a few loads in flight
+  // per lane); without room for one row they are read from global memory.
+  const int padded = (n_o + 63) & ~63;
+  const int g32 = static_cast<int>(gpr);
+  const uint32_t cache_s = smem_u32(cache);
+  const int64_t row_bytes = gpr * 16;
+  int nsl = 0;  // row slots for the uncached rows: a power of two, at most kPrepWarps
   {
-    const int padded = (n_o + 63) & ~63;
+    const int64_t cap = row_bytes > 0 ? p.cache_bytes_all / row_bytes : 0;
+    while (nsl < kPrepWarps && 2 * (nsl > 0 ? nsl : 1) <= cap) nsl = nsl > 0 ? 2 * nsl : 2;
+    if (nsl == 0 && cap >= 1) nsl = 1;
+  }
+  auto quantise_rows = [&](int64_t lo, int64_t hi, bool staged) {
+    const int64_t n = hi - lo;
     int wpr = 1;
-    while (wpr < kPrepWarps && wpr * 2 * nrows <= kPrepWarps) wpr *= 2;
+    while (wpr < kPrepWarps && wpr * 2 * n <= kPrepWarps) wpr *= 2;
+    if (staged)
+      while (kPrepWarps / wpr > nsl) wpr *= 2;
     const int rows_per_round = kPrepWarps / wpr;
     const int sub = warp % wpr;
     const int rr = warp / wpr;
     const int start = sub * 32 + lane, step = 32 * wpr;
-    const int g32 = static_cast<int>(gpr);
-    const uint32_t cache_s = smem_u32(cache);
-    const int64_t rounds = (nrows + rows_per_round - 1) / rows_per_round;
+    const int64_t rounds = (n + rows_per_round - 1) / rows_per_round;
     for (int64_t round = 0; round < rounds; ++round) {
-      const int64_t i = round * rows_per_round + rr;
-      const bool have = i < nrows;
+      const int64_t i = lo + round * rows_per_round + rr;
+      const bool have = i < hi;
       const bool cached = have && i < ncached;
       const int64_t t = r0 + i;
-      const uint32_t sbase = cache_s + static_cast<uint32_t>(i * gpr * 16);
+      uint32_t sbase = cache_s + static_cast<uint32_t>(i * row_bytes);
       const uint4* gbase = reinterpret_cast<const uint4*>(p.X + t * K);
+      if (staged) {
+        // the previous round's reads of the slots are done before they are written again
+        __syncthreads();
+        if (warp == 0 && lane < rows_per_round) {
+          const int64_t il = lo + round * rows_per_round + lane;
+          if (il < hi) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            const uint32_t bar = smem_u32(&s_sbar[lane]);
+            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(row_bytes));
+            bulk_load(cache_s + static_cast<uint32_t>(lane * row_bytes), p.X + (r0 + il) * K,
+                      static_cast<uint32_t>(row_bytes), bar);
+          }
+        }
+        sbase = cache_s + static_cast<uint32_t>(rr * row_bytes);
+        if (have) {
+          int no_abort = 0;
+          const bool got = mbar_wait(smem_u32(&s_sbar[rr]), static_cast<uint32_t>(round & 1),
+                                     &no_abort, p.wait_limit_ns);
+          if (!__all_sync(0xffffffffu, got) && lane == 0) s_gfail = 1;
+        }
+      }
+      const bool in_smem = cached || (staged && have);
       const bool specrow = spec && cached;
       float amax = 0.0f;
       if (specrow) {
@@ -842,7 +880,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
             }
           }
         }
-      } else if (cached) {
+      } else if (in_smem) {
         amax = row_absmax<true>(sbase, gbase, g32, start, step, smask);
       } else if (have) {
         amax = row_absmax<false>(sbase, gbase, g32, start, step, smask);
@@ -864,7 +902,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
         // the speculative codes stand: clear those of the outlier columns
         int8_t* qb = p.Xq + t * K;
         for (int j = start; j < n_o; j += step) qb[idx_at(j)] = 0;
-      } else if (cached) {
+      } else if (in_smem) {
         row_codes<true>(sbase, gbase, qrow, g32, start, step, smask, sc, kE4M3, spre, xo_row,
                         cstride);
       } else {
@@ -895,6 +933,11 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prepare_kernel(const PrepArgs
       for (int j = n_o + start; j < padded; j += step)
         xo_row[static_cast<int64_t>(j >> 6) * cstride + (j & 63)] = __float2half_rn(0.0f);
     }
+  };
+  quantise_rows(0, ncached, false);
+  if (nrows > ncached) {
+    __syncthreads();  // the cached rows are done: their shared memory becomes the slots
+    quantise_rows(ncached, nrows, nsl > 0);
   }
   __syncthreads();   // the row cache is free from here on (phase 4 may reuse it)
 

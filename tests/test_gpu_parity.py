@@ -80,6 +80,10 @@ SCAN_CASES = [
     (2000, 2064, (5, 100, 2063), 5e-5, 6.0),
     (1500, 1040, (), 0.0, math.inf),
     (1400, 256, (3,), 0.0, 0.0),
+    # one row per CTA fits in shared memory: the other rows of a CTA pass through that one
+    # slot, all 16 warps on each; and rows too long for any slot, read from global memory
+    (300, 57344, (5, 30000, 57343), 1e-5, 6.0),
+    (300, 131072, (0, 131071), 0.0, 6.0),
 ]
 
 
