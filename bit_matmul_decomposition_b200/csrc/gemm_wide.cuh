@@ -295,14 +295,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           continue;
         }
         tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < TN / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>(c * 32), r);
-          tmem_ld_wait();
+        // two chunks of 32 columns in flight: chunk c + 1 loads while chunk c converts
+        auto convert = [&](int c, uint32_t (&r)[32]) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(gemm::acc_value<kE4M3>(r[j]) * sx);
           gemm::tmem_st_32x32b_x32(lane_base + static_cast<uint32_t>(c * 32), r);
+        };
+        uint32_t ra[32], rb[32];
+        tmem_ld_32x32b_x32(lane_base, ra);
+#pragma unroll 1
+        for (int c = 0; c < TN / 32; c += 2) {
+          tmem_ld_wait_regs(ra);
+          tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>((c + 1) * 32), rb);
+          convert(c, ra);
+          tmem_ld_wait_regs(rb);
+          if (c + 2 < TN / 32)
+            tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>((c + 2) * 32), ra);
+          convert(c + 1, rb);
         }
         gemm::tmem_st_wait();
         tc_fence_before();
@@ -317,13 +326,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
       }
       tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < TN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>(c * 32), r);
-        tmem_ld_wait();
+      // one chunk of 32 columns: scale, bias, fp16, out through shared memory by TMA
+      auto store_chunk = [&](int c, const uint32_t (&r)[32]) {
         const int c0 = n0 + c * 32;
-        if (c0 >= a.N || trow0 >= a.T) continue;
+        if (c0 >= a.N || trow0 >= a.T) return;
         float v[32];
         gemm::epilogue_values<kE4M3>(r, OC, sx, ws + c * 32, bs + c * 32, v);
         if (a.c_tma) {
@@ -350,10 +356,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         } else if (row_ok) {
           gemm::store_row32_f16(a.C + static_cast<int64_t>(t) * a.N, c0, a.N, v, vec_ok);
         }
+      };
+      // two chunks in flight: chunk c + 1 loads while chunk c is stored; the accumulator
+      // is released as soon as its last chunk is in registers, so the next tile's MMAs
+      // start while this tile's last chunk is still being written out
+      uint32_t ra[32], rb[32];
+      tmem_ld_32x32b_x32(lane_base, ra);
+#pragma unroll 1
+      for (int c = 0; c < TN / 32; c += 2) {
+        tmem_ld_wait_regs(ra);
+        tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>((c + 1) * 32), rb);
+        store_chunk(c, ra);
+        tmem_ld_wait_regs(rb);
+        if (c + 2 < TN / 32) {
+          tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>((c + 2) * 32), ra);
+        } else {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0)
+            gemm::mbar_arrive_remote(gemm::map_to_rank(smem_u32(&bars->tmem_empty), 0));
+        }
+        store_chunk(c + 1, rb);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) gemm::mbar_arrive_remote(gemm::map_to_rank(smem_u32(&bars->tmem_empty), 0));
     }
     if (lane == 0) gemm::bulk_wait_all();
   }
