@@ -43,7 +43,6 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -152,56 +151,85 @@ def rank_workload(w, rank, world):
 
 
 # ----------------------------------------------------------------------------- clocks
+NVML_REASONS = (("sw_power_cap", 0x4), ("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+                ("hw_thermal_slowdown", 0x40))
+
+
+def summarise_clock_samples(samples, t0, t1):
+    """Clock record of the samples taken inside [t0, t1]: samples are (time, sm_mhz,
+    max_mhz, reason_bits, power_w).  None when no sample falls inside."""
+    inside = [x for x in samples if t0 <= x[0] <= t1]
+    if not inside:
+        return None
+    reasons = sorted({name for x in inside for name, bit in NVML_REASONS if x[3] & bit})
+    return {"sm_mhz": statistics.median(x[1] for x in inside),
+            "sm_max_mhz": inside[0][2], "reasons": reasons, "samples": len(inside),
+            "power_w_max": max(x[4] for x in inside),
+            "source": "NVML every ~2 ms, timed region only"}
+
+
 class ClockSampler:
-    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, throttle reasons and power of the GPU, read through NVML by a background
+    thread every ~2 ms; begin() / end() delimit the timed region, and stop() summarises
+    the samples inside it (NVML reads only: nothing is set)."""
 
     def __init__(self, uuid=None):
         self.uuid = uuid
-        self.proc = None
-        self.path = os.path.join("/tmp", "i8bench_clocks_%d.csv" % os.getpid())
+        self.samples = []
+        self.t0 = self.t1 = None
+        self.thread = None
+        self.running = False
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        if self.uuid:
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                if (u.decode() if isinstance(u, bytes) else u) == self.uuid:
+                    return pynvml, h
+        import torch
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(torch.cuda.current_device())
 
     def start(self):
+        import threading
         try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
-                 "-lms", "20"], stdout=self.f, stderr=subprocess.DEVNULL)
+            nv, h = self._handle()
+            max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
         except Exception:
-            self.proc = None
+            return
+
+        def run():
+            while self.running:
+                try:
+                    self.samples.append((time.monotonic(),
+                                         float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                         max_mhz,
+                                         int(nv.nvmlDeviceGetCurrentClocksEventReasons(h)),
+                                         nv.nvmlDeviceGetPowerUsage(h) / 1000.0))
+                except Exception:
+                    return
+                time.sleep(0.002)
+
+        self.running = True
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
+
+    def begin(self):
+        self.t0 = time.monotonic()
+
+    def end(self):
+        self.t1 = time.monotonic()
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.f.close()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 10:
-                    continue
-                if self.uuid and parts[1] != self.uuid:
-                    continue
-                rows.append(parts)
-        try:
-            os.remove(self.path)
-        except OSError:
-            pass
-        if not rows:
+        self.running = False
+        self.thread.join(timeout=5)
+        if self.t0 is None or self.t1 is None:
             return None
-        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[6:10]) if v == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": float(rows[0][3]) if rows[0][3].replace(".", "").isdigit() else None,
-                "reasons": reasons, "samples": len(rows),
-                "power_w_max": max(float(r[4]) for r in rows if r[4].replace(".", "").isdigit())}
+        return summarise_clock_samples(self.samples, self.t0, self.t1)
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -392,13 +420,15 @@ def time_forward(abi, forward, steps, warmup, flush_l2, stream, uuid, barrier=la
     barrier()
     torch.cuda.synchronize()
     clocks.start()
-    time.sleep(0.3)
+    time.sleep(0.05)
+    clocks.begin()
     for i in range(steps):
         flush_l2()
         ev_s[i].record(stream)
         forward()
         ev_e[i].record(stream)
     torch.cuda.synchronize()
+    clocks.end()
     barrier()
     clk = clocks.stop()
     st = abi.i8_sync_status()
@@ -780,13 +810,15 @@ def run_train(args, w):
           for _ in range(args.steps)]
     clocks = ClockSampler()
     clocks.start()
-    time.sleep(0.3)
+    time.sleep(0.05)
+    clocks.begin()
     for e0, e1 in ev:
         flush.zero_()
         e0.record()
         step()
         e1.record()
     torch.cuda.synchronize()
+    clocks.end()
     clk = clocks.stop()
     ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
     flops = 3.0 * 2.0 * T * N * K

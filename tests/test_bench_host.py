@@ -205,3 +205,29 @@ def test_tensor_peak_follows_the_power_cap_seen_while_timing():
     assert capped == 2 * 1418.9 and "sustained" in why
     unknown, why = bench.tensor_peak(pk, None, e4m3=True)
     assert unknown == 2 * 1679.9 and "fp8" in why and "no clock record" in why
+
+
+def test_clock_record_keeps_only_samples_inside_the_timed_region():
+    # (time, sm_mhz, max_mhz, NVML reason bits, power_w): idle samples before and after,
+    # power-capped samples at 1620 MHz inside
+    samples = [(0.00, 1965.0, 1965.0, 0x1, 120.0), (0.10, 1965.0, 1965.0, 0x0, 130.0),
+               (0.20, 1620.0, 1965.0, 0x4, 990.0), (0.21, 1605.0, 1965.0, 0x4, 1001.0),
+               (0.22, 1650.0, 1965.0, 0x0, 950.0), (0.50, 1965.0, 1965.0, 0x1, 140.0)]
+    rec = bench.summarise_clock_samples(samples, 0.15, 0.30)
+    assert rec["samples"] == 3
+    assert rec["sm_mhz"] == 1620.0
+    assert rec["sm_max_mhz"] == 1965.0
+    assert rec["reasons"] == ["sw_power_cap"]
+    assert rec["power_w_max"] == 1001.0
+    hot = [(0.2, 1400.0, 1965.0, 0x8 | 0x40 | 0x20, 700.0)]
+    assert bench.summarise_clock_samples(hot, 0.0, 1.0)["reasons"] == [
+        "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"]
+    assert bench.summarise_clock_samples(samples, 0.6, 0.7) is None
+
+
+def test_clock_sampler_without_a_gpu_reports_nothing():
+    c = bench.ClockSampler()
+    c.start()
+    c.begin()
+    c.end()
+    assert c.stop() is None
