@@ -400,8 +400,10 @@ class Layer:
 
 
 def time_forward(abi, forward, steps, warmup, flush_l2, stream, uuid, barrier=lambda: None):
-    """Region 1: `steps` whole steps, each bracketed by events (clocks sampled meanwhile).
-    Region 2: the same steps with events around the dominant kernel alone.  Returns
+    """`steps` whole steps, each bracketed by events, with events around the dominant kernel
+    inside each step as well (clocks sampled meanwhile), so that the kernel's time and the
+    step's come from the same loop in the same power and thermal state.  (The kernel events
+    cost the step the launch overlap of its two kernels: a few microseconds.)  Returns
     (summed step ms, summed kernel ms, clock record)."""
     import torch
     for _ in range(warmup):
@@ -425,8 +427,10 @@ def time_forward(abi, forward, steps, warmup, flush_l2, stream, uuid, barrier=la
     for i in range(steps):
         flush_l2()
         ev_s[i].record(stream)
+        abi.i8_set_profile_events(kv_s[i], kv_e[i])
         forward()
         ev_e[i].record(stream)
+    abi.i8_set_profile_events(None, None)
     torch.cuda.synchronize()
     clocks.end()
     barrier()
@@ -434,17 +438,6 @@ def time_forward(abi, forward, steps, warmup, flush_l2, stream, uuid, barrier=la
     st = abi.i8_sync_status()
     if st != 0:
         raise RuntimeError("device error in the timed loop: %s" % abi.STATUS.get(st, st))
-    # (recording events between kernels costs the launch overlap, so region 1 runs without)
-    for i in range(steps):
-        flush_l2()
-        abi.i8_set_profile_events(kv_s[i], kv_e[i])
-        forward()
-    abi.i8_set_profile_events(None, None)
-    torch.cuda.synchronize()
-    barrier()
-    st = abi.i8_sync_status()
-    if st != 0:
-        raise RuntimeError("device error in the kernel-timing loop: %s" % abi.STATUS.get(st, st))
     step_ms = sum(ev_s[i].elapsed_time(ev_e[i]) for i in range(steps))
     kern_ms = sum(kv_s[i].elapsed_time(kv_e[i]) for i in range(steps))
     return step_ms, kern_ms, clk
