@@ -247,7 +247,7 @@ def work_counts(T, N, K, n_o):
 
 def traffic_record(kernel, workload):
     """DRAM bytes per launch from the committed ncu summary (profiles/dram_traffic.txt), if
-    it was taken on this workload and on the current CUDA sources (else None)."""
+    it was taken on this workload and on the kernel's current sources (else None)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     try:
         with open(path) as f:
@@ -255,16 +255,29 @@ def traffic_record(kernel, workload):
     except OSError:
         return None
     for parts in lines:
-        if (len(parts) >= 4 and parts[0] == kernel and parts[2] == source_hash()
+        if (len(parts) >= 4 and parts[0] == kernel and parts[2] == source_hash(kernel)
                 and parts[3] == workload):
             return {"dram_bytes_per_launch": int(parts[1]),
                     "note": parts[4].strip() if len(parts) > 4 else ""}
     return None
 
 
-def source_hash():
+# The CUDA sources that decide a kernel's code and launch: its own header, the headers it
+# includes, and the host code that sizes its launch.
+CUDA_SOURCES = ("api.cu", "common.cuh", "quant.cuh", "gemm.cuh", "gemm_wide.cuh", "gemv.cuh",
+                "bwd.cuh")
+KERNEL_SOURCES = {
+    "decode_kernel": ("api.cu", "common.cuh", "quant.cuh", "gemv.cuh"),
+    "prepare_kernel": ("api.cu", "common.cuh", "quant.cuh"),
+    "i8_gemm_tcgen05_kernel": ("api.cu", "common.cuh", "gemm.cuh"),
+    "i8_gemm_wide_kernel": ("api.cu", "common.cuh", "gemm.cuh", "gemm_wide.cuh"),
+}
+
+
+def source_hash(kernel=None):
+    """sha256 over the sources of `kernel` (all CUDA sources for an unknown kernel)."""
     h = hashlib.sha256()
-    for f in ("api.cu", "common.cuh", "quant.cuh", "gemm.cuh", "gemm_wide.cuh", "gemv.cuh", "bwd.cuh"):
+    for f in KERNEL_SOURCES.get(kernel, CUDA_SOURCES):
         with open(os.path.join(ROOT, "bit_matmul_decomposition_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()

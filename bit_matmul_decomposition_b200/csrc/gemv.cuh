@@ -43,7 +43,9 @@
 //                        (the exact int32 acc_s for the raw product), and counts the
 //                        arrival on the tile's counter; the CTA that completes a tile sums
 //                        the S records in slice order and writes
-//                          C[t,n] = fp16((sum_s P_s[t,n]) * SCB[n]/127 + bias[n]).
+//                          C[t,n] = fp16((sum_s P_s[t,n]) * SCB[n]/127 + bias[n]),
+//                        then drops the records' lines from the L2 (discard: the records
+//                        never reach DRAM; the workspace is scratch after the call).
 //
 // The tile counters and the words of the cooperative prologue carry the launch's epoch
 // (1 .. 2^32 - 1) in their upper 32 bits.  The host clears them (one memset) before every
@@ -738,6 +740,15 @@ __device__ __forceinline__ void finish_tile(const Args& a, const int64_t tile, c
         if (t < T) a.C[static_cast<int64_t>(t) * N + n] = __float2half_rn(fmaf(part[t], ws, bn));
     }
   }
+  // The S records are summed (every loaded value has reached the stores above): drop their
+  // L2 lines so they are never written back to DRAM.  Only whole 128-byte lines inside
+  // this tile's records are dropped.
+  __syncwarp();
+  const uintptr_t lo = reinterpret_cast<uintptr_t>(a.rec + tile * S * rb);
+  const uintptr_t hi = lo + static_cast<uintptr_t>(S) * static_cast<uintptr_t>(rb);
+  for (uintptr_t p = ((lo + 127u) & ~static_cast<uintptr_t>(127u)) + lane * 128u; p + 128u <= hi;
+       p += 32u * 128u)
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
 }
 
 // ---------------------------------------------------------------------- the kernel

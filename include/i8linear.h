@@ -164,7 +164,9 @@ i8_status i8_forward_kernel(int64_t T, int64_t N, int64_t K, int32_t* kind);
  *     operands with fp32 accumulation, and the epilogue runs in fp32.
  *   workspace  device buffer of at least i8_linear_workspace_size(T, N, K) bytes, owned by
  *              the caller; its contents need no initialisation and are scratch after the
- *              call (calls sharing one workspace must be ordered on one stream).
+ *              call: the decode path drops part of it from the L2 without write-back, so
+ *              those bytes may read back as any earlier contents of the memory (calls
+ *              sharing one workspace must be ordered on one stream).
  * T <= 16 with K <= 65536 runs the decode path: one kernel (one CTA per SM, each on a
  * K-slice; CB streamed once by TMA into warp-level int8 tensor-core MMAs; steps 1 and 2
  * in its prologue, a cooperative launch when 2*T*K > 128 KB; the outlier sum per K-slice,

@@ -4,6 +4,7 @@ ranks running the oracle on their shards reproduce the unsharded layer bit for b
 the JSON contract of the reference arm (the CPU oracle timed on this host)."""
 import json
 import os
+import re
 import socket
 import subprocess
 import sys
@@ -191,10 +192,35 @@ def test_traffic_is_reported_only_for_the_sources_it_was_measured_on(monkeypatch
     rec = bench.traffic_record("i8_gemm_tcgen05_kernel", "opt6.7b_ffn_up_prefill_2048x4096x16384")
     if rec is not None:   # the committed capture matches the current CUDA sources
         assert rec["dram_bytes_per_launch"] > 0
-    monkeypatch.setattr(bench, "source_hash", lambda: "0" * 64)
+    monkeypatch.setattr(bench, "source_hash", lambda kernel=None: "0" * 64)
     assert bench.traffic_record("i8_gemm_tcgen05_kernel",
                                 "opt6.7b_ffn_up_prefill_2048x4096x16384") is None
     assert bench.traffic_record("decode_kernel", "no_such_workload") is None
+
+
+def test_kernel_source_hash_covers_its_headers_and_the_launch_code():
+    # every kernel's hash reads api.cu (launch sizing) and common.cuh, and its own header
+    for k, files in bench.KERNEL_SOURCES.items():
+        assert {"api.cu", "common.cuh"} <= set(files), k
+        assert set(files) <= set(bench.CUDA_SOURCES), k
+    assert "gemv.cuh" in bench.KERNEL_SOURCES["decode_kernel"]
+    assert "gemm_wide.cuh" in bench.KERNEL_SOURCES["i8_gemm_wide_kernel"]
+    # headers a kernel's header includes are in its list
+    csrc = os.path.join(bench.ROOT, "bit_matmul_decomposition_b200", "csrc")
+    own = {"decode_kernel": "gemv.cuh", "prepare_kernel": "quant.cuh",
+           "i8_gemm_tcgen05_kernel": "gemm.cuh", "i8_gemm_wide_kernel": "gemm_wide.cuh"}
+    for k, hdr in own.items():
+        todo, seen = [hdr], set()
+        while todo:
+            f = todo.pop()
+            if f in seen:
+                continue
+            seen.add(f)
+            with open(os.path.join(csrc, f)) as fh:
+                todo += re.findall(r'#include "([a-z_]+\.cuh)"', fh.read())
+        assert seen <= set(bench.KERNEL_SOURCES[k]), (k, seen)
+    assert bench.source_hash("decode_kernel") != bench.source_hash("i8_gemm_tcgen05_kernel")
+    assert bench.source_hash("no_such_kernel") == bench.source_hash()
 
 
 def test_tensor_peak_follows_the_power_cap_seen_while_timing():
